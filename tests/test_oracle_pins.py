@@ -1,0 +1,263 @@
+"""Pins for the fp64 oracle: hand-derived values, closed forms, invariants, library
+routines and brute force. Each check is chosen so that a plausible slip in the
+oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong
+count for a partial block) fails at least one of them."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import block_sparse_attention as O
+from free_block_sparse_kv_b200 import workloads as W
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# --- hand-derived worked examples --------------------------------------------
+
+def test_golden_single_block(golden_dir):
+    g = _load(golden_dir, "single_block_d2.json")
+    q, k, v = (np.array(g[x], float) for x in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(g["d"])
+    kbar, vsum, counts, mats = O.pool_keys_values(k, v, g["block"], 1)
+    np.testing.assert_allclose(kbar, g["kbar"], atol=1e-15)
+    np.testing.assert_allclose(vsum, g["vsum"], atol=1e-15)
+    np.testing.assert_allclose(mats, g["M"], atol=1e-15)
+    assert counts.tolist() == [2]
+    skipped = [np.zeros(0, int)]
+    o0 = O.forward_head(q, k, v, skipped, g["block"], 0, scale)
+    o1 = O.forward_head(q, k, v, skipped, g["block"], 1, scale)
+    ok = O.forward_head(q, k, v, [np.array([0])], g["block"], 1, scale)
+    np.testing.assert_allclose(o0, g["out_order0_skipped"], atol=1e-14)
+    np.testing.assert_allclose(o1, g["out_order1_skipped"], atol=1e-14)
+    np.testing.assert_allclose(ok, g["out_kept"], atol=1e-14)
+
+
+def test_golden_routing(golden_dir):
+    g = _load(golden_dir, "routing_d4.json")
+    q, k = np.array(g["q"], float), np.array(g["k"], float)
+    scale = 1.0 / math.sqrt(g["d"])
+    qbar = O.pool_queries(q, g["block"])
+    kbar = O.pool_keys_values(k, np.zeros((k.shape[0], 1)), g["block"], 0)[0]
+    s = O.routing_scores(qbar, kbar, scale)
+    np.testing.assert_allclose(s, g["scores"], atol=1e-15)
+    for kk, want in g["topk"].items():
+        assert O.route_topk(s, int(kk))[0].tolist() == want
+    for tau, want in g["mass"].items():
+        kept, cnt = O.route_mass(s, float(tau))
+        assert kept[0].tolist() == want and cnt[0] == len(want)
+    gaps, _, _ = O.gate_diagnostics(s, [2])
+    assert gaps[0] == pytest.approx(g["gap_top2"], abs=1e-15)
+    gaps, _, _ = O.gate_diagnostics(s, [1])
+    assert gaps[0] == 0.0
+
+
+def test_golden_structured(golden_dir):
+    g = _load(golden_dir, "structured_small.json")
+    kept = O.structured_kept(g["Nq"], g["Nk"], g["block"], g["frame_tokens"], g["n_frames"],
+                             g["window"], g["n_anchors"], g["period"], g["step"])
+    assert [x.tolist() for x in kept] == g["kept"]
+
+
+# --- rho = 1 is dense attention ----------------------------------------------
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_all_kept_equals_dense_loops(order):
+    rng = np.random.default_rng(1)
+    n, d, b = 100, 8, 32                  # partial last block (4 tokens)
+    q, k, v = _rand(rng, n, d), _rand(rng, n, d), _rand(rng, n, d)
+    scale = 1 / math.sqrt(d)
+    nb = -(-n // b)
+    kept = [np.arange(nb)] * nb
+    got = O.forward_head(q, k, v, kept, b, order, scale)
+    want = O.dense_attention_loops(q, k, v, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_all_kept_equals_sdpa_at_small_workload_size():
+    w = W.WORKLOADS["uniform-4k"]
+    q, k, v = W.head_inputs(w, 0, 1)
+    kept = [np.arange(w.nkb)] * w.nqb
+    rows = np.arange(0, w.Nq, 37)
+    got = O.forward_head(q, k, v, kept, w.block, 0, w.scale, rows=rows)
+    qt, kt, vt = (torch.from_numpy(x.astype(np.float64)) for x in (q[rows], k, v))
+    want = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None]).numpy()[0]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# --- order-0 exactness and first-order convergence ----------------------------
+
+def test_order0_exact_for_identical_keys_in_block():
+    rng = np.random.default_rng(2)
+    n, d, b = 200, 16, 32                 # 7 blocks, last holds 8 tokens
+    nb = -(-n // b)
+    centers = _rand(rng, nb, d)
+    k = centers[np.arange(n) // b]
+    q, v = _rand(rng, n, d), _rand(rng, n, d)
+    scale = 1 / math.sqrt(d)
+    _, _, counts, mats = O.pool_keys_values(k, v, b, 1)
+    assert np.abs(mats).max() < 1e-12
+    assert counts[-1] == n - (nb - 1) * b
+    kept = [rng.choice(nb, size=2, replace=False) for _ in range(nb)]
+    for order in (0, 1):
+        got = O.forward_head(q, k, v, kept, b, order, scale)
+        want = O.dense_attention_loops(q, k, v, scale)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_taylor_orders_converge_at_rate_one_and_two():
+    rng = np.random.default_rng(3)
+    n, d, b = 192, 16, 64
+    nb = n // b
+    centers = 0.5 * _rand(rng, nb, d)
+    delta = _rand(rng, n, d)
+    q, v = _rand(rng, n, d), _rand(rng, n, d)
+    scale = 1 / math.sqrt(d)
+    kept = [np.array([i]) for i in range(nb)]    # each query block keeps only itself
+    errs = {0: [], 1: []}
+    eps_list = [1e-1, 1e-2, 1e-3]
+    for eps in eps_list:
+        k = centers[np.arange(n) // b] + eps * delta
+        dense = O.dense_attention_loops(q, k, v, scale)
+        for order in (0, 1):
+            errs[order].append(np.abs(O.forward_head(q, k, v, kept, b, order, scale) - dense).max())
+    for order, want in ((0, 1.0), (1, 2.0)):
+        slope = np.polyfit(np.log(eps_list), np.log(errs[order]), 1)[0]
+        assert abs(slope - want) < 0.15, (order, slope, errs[order])
+    assert errs[1][-1] < 1e-2 * errs[0][-1]
+
+
+# --- pooled-table algebra vs the per-pair twin ---------------------------------
+
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("rho", [(1, 4), (1, 2)])
+def test_blockwise_equals_per_pair_twin(order, rho):
+    rng = np.random.default_rng(10 + order)
+    n, d, b = 300, 8, 32                  # 10 blocks, the last has 12 tokens
+    q, k, v = _rand(rng, n, d), 0.5 * _rand(rng, n, d), _rand(rng, n, d)
+    scale = 1 / math.sqrt(d)
+    keep = O.keep_count(-(-n // b), *rho)
+    kept, _, _ = O.route_head(q, k, b, "topk", scale, keep=keep)
+    got = O.forward_head(q, k, v, kept, b, order, scale)
+    want = O.brute_force_pairs(q, k, v, kept, b, order, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_all_skipped_order0_is_attention_over_pseudo_tokens():
+    """With nothing kept, order 0 is attention over one pseudo-token per block: key
+    kbar_j, value S_j / n_j and logit bias ln n_j (torch SDPA in fp64)."""
+    rng = np.random.default_rng(4)
+    n, d, b = 500, 32, 64                 # last block 52 tokens
+    q, k, v = _rand(rng, n, d), _rand(rng, n, d), _rand(rng, n, d)
+    scale = 1 / math.sqrt(d)
+    nb = -(-n // b)
+    got = O.forward_head(q, k, v, [np.zeros(0, int)] * nb, b, 0, scale)
+    kb = np.stack([k[s:s + b].mean(0) for s in range(0, n, b)])
+    vm = np.stack([v[s:s + b].mean(0) for s in range(0, n, b)])
+    cnt = np.array([min(b, n - s) for s in range(0, n, b)], float)
+    bias = torch.from_numpy(np.log(cnt))[None, :].expand(n, nb)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(kb)[None], torch.from_numpy(vm)[None],
+        attn_mask=bias[None]).numpy()[0]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# --- routing -----------------------------------------------------------------
+
+def test_topk_matches_rank_counting():
+    rng = np.random.default_rng(5)
+    s = np.round(rng.standard_normal((40, 37)), 1)     # many exact ties
+    keep = 9
+    kept = O.route_topk(s, keep)
+    for i, row in enumerate(s):
+        rank = [sum(1 for jj in range(len(row)) if row[jj] > row[j] or (row[jj] == row[j] and jj < j))
+                for j in range(len(row))]
+        assert kept[i].tolist() == [j for j in range(len(row)) if rank[j] < keep]
+
+
+def test_mass_prefix_is_shortest_covering():
+    rng = np.random.default_rng(6)
+    s = 2.0 * rng.standard_normal((50, 60))
+    for tau in (0.5, 0.9, 0.99):
+        kept, counts = O.route_mass(s, tau)
+        for i, row in enumerate(s):
+            z = [math.exp(x) for x in row]
+            total = math.fsum(z)
+            ranked = sorted(range(len(row)), key=lambda j: (-row[j], j))
+            k = counts[i]
+            assert math.fsum(z[j] for j in ranked[:k]) / total >= tau - 1e-12
+            assert math.fsum(z[j] for j in ranked[:k - 1]) / total < tau
+            assert kept[i].tolist() == sorted(ranked[:k])
+
+
+def test_keep_count_is_integer_ceiling():
+    assert O.keep_count(64, 1, 4) == 16
+    assert O.keep_count(256, 1, 5) == 52
+    assert O.keep_count(591, 1, 10) == 60
+    assert O.keep_count(10, 1, 1) == 10
+
+
+# --- structured mask ---------------------------------------------------------
+
+def test_rotating_anchors_cover_each_frame_once():
+    period, n_anchors, n_frames = 10, 4, 41
+    seen = {}
+    for s in range(period):
+        for f in O.anchor_frames(s, period, n_anchors, n_frames):
+            seen[f] = seen.get(f, 0) + 1
+    assert sorted(seen) == list(range(40)) and set(seen.values()) == {1}
+    assert O.anchor_frames(3, period, n_anchors, n_frames) == O.anchor_frames(13, period, n_anchors, n_frames)
+
+
+def test_structured_mask_against_token_pairs():
+    """Brute force over every (query token, key token) pair on a geometry whose
+    blocks straddle frame boundaries."""
+    ft, T, b, win, na, per = 7, 9, 5, 1, 2, 4
+    n = ft * T
+    for step in range(per):
+        kept = O.structured_kept(n, n, b, ft, T, win, na, per, step)
+        anchors = {(step % per) + per * m for m in range(na)}
+        for i in range(-(-n // b)):
+            want = []
+            for j in range(-(-n // b)):
+                hit = False
+                for tq in range(i * b, min(n, (i + 1) * b)):
+                    for tk in range(j * b, min(n, (j + 1) * b)):
+                        fq, fk = tq // ft, tk // ft
+                        if abs(fq - fk) <= win or fk in anchors:
+                            hit = True
+                want.append(hit)
+            assert kept[i].tolist() == [j for j, h in enumerate(want) if h]
+
+
+def test_structured_kept_fraction_at_long_video_size():
+    """At 41 frames x 1560 tokens, blocks of 128, window 3, 4 anchors: a query frame
+    sees its clipped window plus the anchors outside it; block granularity adds
+    the straddling blocks. The kept fraction lies between the frame-level pair
+    fraction and that fraction plus two boundary blocks per row."""
+    w = W.WORKLOADS["longvideo-41x30x52"]
+    T = w.n_frames
+    for step in (0, 7):
+        kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, T, w.window,
+                                 w.n_anchors, w.period, step)
+        frac = sum(len(x) for x in kept) / (w.nqb * w.nkb)
+        g = {(step % w.period) + w.period * m for m in range(w.n_anchors)}
+        pairs = sum(len(g | {f for f in range(t - 3, t + 4) if 0 <= f < T}) for t in range(T))
+        lo = pairs / T ** 2
+        assert lo <= frac <= lo + 2 * (1 + len(g)) * 2 / w.nkb + 2 / w.nkb
+
+
+def test_mass_boundary_is_inclusive(golden_dir):
+    g = _load(golden_dir, "routing_d4.json")
+    kept, cnt = O.route_mass(np.array(g["equal_scores"]), g["equal_scores_tau"])
+    assert kept[0].tolist() == g["equal_scores_kept"] and cnt[0] == 2
