@@ -1,0 +1,382 @@
+"""Benchmark: one step = pool -> route (or structured mask) -> forward over one
+synthetic workload, on each GPU (weak scaling: every rank runs its own copy of
+the workload, seeded by its rank; no collective on the data path).
+
+Prints one JSON line on rank 0. `value` is dense-equivalent attention TFLOPS
+(4 * B * H * Nq * Nk * d per call) summed over ranks, timed with CUDA events
+on the launching stream (max over ranks), inputs resident in HBM. `e2e` is the
+same metric through the public API with pinned host buffers, including the
+host-to-device copy of Q, K, V and the device-to-host copy of the output.
+
+--impl reference times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from free_block_sparse_kv_b200 import workloads as W  # noqa: E402
+
+METRIC = "dense-equiv attention TFLOPS & ms/call at N=75,600 d=128; % of bf16 TC peak"
+UNIT = "TFLOPS"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.METRIC_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    hbm=d["hbm_gbs"], source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# work model
+# ---------------------------------------------------------------------------
+
+def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dict:
+    """MMA flops the forward executes for the given kept lists (per launch).
+
+    exact kept block j, query block i:     4 * nq_i * n_j * d
+    skipped block, order 0 (logit + value): 4 * nq_i * d
+    skipped block, order 1 (q M_j):         2 * nq_i * d * d
+    """
+    nq = np.array([min(w.block, w.Nq - i * w.block) for i in range(w.nqb)], np.float64)
+    nk = np.array([min(w.block, w.Nk - j * w.block) for j in range(w.nkb)], np.float64)
+    exact = order0 = order1 = 0.0
+    for b in range(kv_cnt.shape[0]):
+        for h in range(kv_cnt.shape[1]):
+            for i in range(w.nqb):
+                c = int(kv_cnt[b, h, i])
+                kept = kv_idx[b, h, i, :c]
+                tok = nk[kept].sum()
+                exact += 4.0 * nq[i] * tok * w.d
+                skipped = w.nkb - c
+                order0 += 4.0 * nq[i] * w.d * skipped
+                if w.order == 1:
+                    order1 += 2.0 * nq[i] * w.d * w.d * skipped
+    return dict(exact=exact, order0=order0, order1=order1, total=exact + order0 + order1)
+
+
+def pool_bytes(w: W.Workload, with_q: bool) -> float:
+    """Algorithmic HBM bytes of one pool launch: read K, V (and Q), write the tables."""
+    bh = w.B * w.H
+    rd = bh * w.Nk * w.d * 2 * 2 + (bh * w.Nq * w.d * 2 if with_q else 0)
+    wr = bh * w.nkb * w.d * (4 + 4 + 2 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
+    if w.order == 1:
+        wr += bh * w.nkb * w.d * w.d * 2
+    return float(rd + wr)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.device_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline key)
+# ---------------------------------------------------------------------------
+
+def time_oracle(w: W.Workload, seconds: float) -> dict:
+    """Time the fp64 oracle on a bounded sample: one head's pooling and routing, then
+    query rows (spread over the head) until `seconds` have passed. Scaled to
+    dense-equivalent TFLOPS: rows * Nk * d * 4 per second of the oracle's time."""
+    from oracle import block_sparse_attention as O
+    q, k, v = W.head_inputs(w, 0, 0)
+    t0 = time.perf_counter()
+    if w.mode == "structured":
+        kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
+                                 w.n_anchors, w.period, 0, w.q_frame0)
+    else:
+        kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau)[0]
+    kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, w.order)
+    t_setup = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    order = rng.permutation(w.Nq)
+    done = 0
+    t1 = time.perf_counter()
+    q64 = q.astype(np.float64)
+    while done < w.Nq and time.perf_counter() - t1 < seconds:
+        rows = order[done:done + 16]
+        O.forward_rows(q64[rows], rows // w.block, k, v, kbar, vsum, counts, mats, kept, w.block,
+                       w.order, w.scale)
+        done += len(rows)
+    t_rows = time.perf_counter() - t1
+    # one head's setup is amortised over its Nq rows
+    per_row = t_rows / done + t_setup / w.Nq
+    tflops = 4.0 * w.Nk * w.d / per_row / 1e12
+    cores = len(os.sched_getaffinity(0))
+    return dict(value=tflops, unit=UNIT, cores=cores, kind="oracle",
+                sample=f"{w.name}: head (0,0) pooled and routed ({t_setup:.1f} s), then {done} of "
+                       f"{w.Nq} query rows forwarded ({t_rows:.1f} s); scaled per row to the "
+                       f"dense-equivalent flops of one call",
+                seconds=t_setup + t_rows, ms_per_call_est=per_row * w.Nq * w.B * w.H * 1e3)
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    res = time_oracle(w, args.cpu_seconds)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": res["value"], "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": res["ms_per_call_est"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "block": w.block, "order": w.order, "mode": w.mode},
+        "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from free_block_sparse_kv_b200 import attention as A
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wr = W.shrink(w, seed=w.seed + rank)   # weak scaling: each rank its own problem
+    qb, kb, vb = W.full_inputs_bits(wr)
+    as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    q_h, k_h, v_h = (as_t(x).pin_memory() for x in (qb, kb, vb))
+    del qb, kb, vb
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    p = A.Problem(w.B, w.H, w.Nq, w.Nk, w.d, w.block, w.order)
+    geometry = dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
+                    n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0)
+    op = A.BlockSparseAttention(p, w.mode, rho=w.rho, tau=w.tau,
+                                geometry=geometry if w.mode == "structured" else None,
+                                out_dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps_cycle = w.steps if w.mode == "structured" else (0,)
+
+    def stage_step(s, ev):
+        """One step with events around each stage (pool, mask/route, forward)."""
+        use_q = w.mode != "structured"
+        ev[0].record(stream)
+        A.pool(q if use_q else None, k, v, p, op.tables)
+        ev[1].record(stream)
+        if w.mode == "structured":
+            A.structured_mask(p, op.kv_idx, op.kv_cnt, w.frame_tokens, w.n_frames, w.window,
+                              w.n_anchors, w.period, s, w.q_frame0)
+        else:
+            A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
+        ev[2].record(stream)
+        A.forward(q, k, v, p, op.tables, op.kv_idx, op.kv_cnt, op.out)
+        ev[3].record(stream)
+
+    for i in range(args.warmup):
+        op(q, k, v, step=steps_cycle[i % len(steps_cycle)])
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    dev_id = str(getattr(props, "uuid", local))
+    if dev_id and not dev_id.startswith("GPU-") and len(dev_id) == 36:
+        dev_id = "GPU-" + dev_id
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev_id) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            stage_step(steps_cycle[i % len(steps_cycle)], evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms_step = start.elapsed_time(end) / args.steps
+    ms_step_max = max_over_ranks(ms_step)
+    stage_ms = [float(np.mean([e[s].elapsed_time(e[s + 1]) for e in evs])) for s in range(3)]
+
+    # per-launch forward work for the lists of the last step
+    kv_idx, kv_cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
+    fl = executed_flops(w, kv_idx, kv_cnt)
+    pk = peaks()
+    fwd_s = stage_ms[2] / 1e3
+    achieved = fl["total"] / fwd_s / 1e12
+    value = world * w.dense_flops() / (ms_step_max / 1e3) / 1e12
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty(op.out.shape, dtype=op.out.dtype, pin_memory=True)
+        q.copy_(q_h, non_blocking=True)
+        op(q, k, v, step=0)
+        out_h.copy_(op.out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(args.e2e_steps):
+            q.copy_(q_h, non_blocking=True)
+            k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            op(q, k, v, step=steps_cycle[i % len(steps_cycle)])
+            out_h.copy_(op.out, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps)
+        h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
+        d2h = out_h.numel() * out_h.element_size()
+        e2e = {"value": world * w.dense_flops() / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res = time_oracle(w, args.cpu_seconds)
+        cpu = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        peak = pk["bf16_sustained"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                       "block": w.block, "order": w.order, "mode": w.mode,
+                       "keep": (f"top {w.rho[0]}/{w.rho[1]}" if w.mode == "topk" else
+                                f"mass {w.tau}" if w.mode == "mass" else "window+anchors"),
+                       "output": "fp32",
+                       "l2": "inputs exceed L2 (Q+K+V %.2f GB per GPU)" % (
+                           (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2) / 1e9),
+                       "parallelism": f"weak: {world} independent problems, one per GPU"},
+            "pct_of_bf16_peak_dense_equiv": 100.0 * value / world / pk["bf16"],
+            "stages_ms": {"pool": stage_ms[0], "route" if w.mode != "structured" else "mask":
+                          stage_ms[1], "forward": stage_ms[2]},
+            "roofline": {"kernel": "sparse_attn_forward", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": f"bf16 sustained ({pk['source']})",
+                         "flops_per_launch": fl},
+            "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")
+                              / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
+            "clocks": clocks.summary(),
+            "gpu_launches": 3 * args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        line["pool_roofline"]["frac"] = line["pool_roofline"]["achieved"] / pk["hbm"]
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,134 @@
+"""Torch-side plumbing around the C ABI: table and list allocation, and the
+three-stage call (pool -> route or structured mask -> forward) on one stream.
+
+Torch only provides device memory and the stream; each stage is one call into
+``libsparse_attn.so``.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+from . import sparse_attn as C
+
+
+@dataclasses.dataclass
+class Tables:
+    """Pooled tables of one problem (layouts as in include/sparse_attn.h)."""
+    qbar: torch.Tensor      # [B,H,nqb,d] fp32
+    kbar_t: torch.Tensor    # [B,H,d,nkb] fp32
+    vsum: torch.Tensor      # [B,H,nkb,d] fp32
+    kbar16: torch.Tensor    # [B,H,nkb,d] bf16
+    vsum16: torch.Tensor    # [B,H,nkb,d] bf16
+    M: Optional[torch.Tensor]  # [B,H,nkb,d,d] bf16 (order 1)
+
+
+@dataclasses.dataclass
+class Problem:
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    block: int
+    order: int
+
+    @property
+    def nqb(self) -> int:
+        return -(-self.Nq // self.block)
+
+    @property
+    def nkb(self) -> int:
+        return -(-self.Nk // self.block)
+
+
+def allocate_tables(p: Problem, device) -> Tables:
+    f32 = dict(dtype=torch.float32, device=device)
+    b16 = dict(dtype=torch.bfloat16, device=device)
+    return Tables(
+        qbar=torch.empty(p.B, p.H, p.nqb, p.d, **f32),
+        kbar_t=torch.empty(p.B, p.H, p.d, p.nkb, **f32),
+        vsum=torch.empty(p.B, p.H, p.nkb, p.d, **f32),
+        kbar16=torch.empty(p.B, p.H, p.nkb, p.d, **b16),
+        vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **b16),
+        M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **b16) if p.order == 1 else None,
+    )
+
+
+def allocate_lists(p: Problem, cap: int, device):
+    return (torch.zeros(p.B, p.H, p.nqb, max(cap, 1), dtype=torch.int32, device=device),
+            torch.zeros(p.B, p.H, p.nqb, dtype=torch.int32, device=device))
+
+
+def _check_inputs(q, k, v):
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        if not (x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 4):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor [B,H,N,d]")
+
+
+def pool(q, k, v, p: Problem, t: Tables, stream=None):
+    C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar, t.kbar_t,
+                       t.vsum, t.kbar16, t.vsum16, t.M, stream)
+
+
+def route(p: Problem, t: Tables, kv_idx, kv_cnt, mode: str, rho=(1, 4), tau=0.9, scale=None,
+          stream=None):
+    scale = 1.0 / math.sqrt(p.d) if scale is None else scale
+    m = C.SA_ROUTE_TOPK if mode == "topk" else C.SA_ROUTE_MASS
+    C.sparse_attn_route(t.qbar, t.kbar_t, p.B, p.H, p.nqb, p.nkb, p.d, m, rho[0], rho[1], tau,
+                        scale, kv_idx, kv_cnt, kv_idx.shape[-1], stream)
+
+
+def structured_mask(p: Problem, kv_idx, kv_cnt, frame_tokens, n_frames, window, n_anchors, period,
+                    step, q_frame0=0, stream=None):
+    C.sparse_attn_structured_mask(p.B, p.H, p.Nq, p.Nk, p.block, frame_tokens, n_frames, window,
+                                  n_anchors, period, step, q_frame0, kv_idx, kv_cnt,
+                                  kv_idx.shape[-1], stream)
+
+
+def forward(q, k, v, p: Problem, t: Tables, kv_idx, kv_cnt, out, scale=None, err_flag=None,
+            stream=None):
+    scale = 1.0 / math.sqrt(p.d) if scale is None else scale
+    dt = C.SA_OUT_F32 if out.dtype == torch.float32 else C.SA_OUT_BF16
+    C.sparse_attn_forward(q, k, v, t.kbar16, t.vsum16, t.M, kv_idx, kv_cnt, kv_idx.shape[-1],
+                          p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, scale, out, dt, err_flag,
+                          stream)
+
+
+class BlockSparseAttention:
+    """Reusable buffers plus the three-stage call for one problem shape.
+
+    mode "topk" keeps ceil(rho * nkb) blocks per query block, "mass" the shortest
+    prefix covering tau of the pooled softmax, "structured" the window + rotating
+    anchor geometry given in ``geometry`` (frame_tokens, n_frames, window,
+    n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
+    """
+
+    def __init__(self, p: Problem, mode: str, rho=(1, 4), tau=0.9, geometry=None,
+                 out_dtype=torch.float32, device="cuda"):
+        self.p, self.mode, self.rho, self.tau, self.geometry = p, mode, rho, tau, geometry
+        if mode == "topk":
+            cap = -(-rho[0] * p.nkb // rho[1])
+        else:
+            cap = p.nkb
+        self.tables = allocate_tables(p, device)
+        self.kv_idx, self.kv_cnt = allocate_lists(p, cap, device)
+        self.out = torch.empty(p.B, p.H, p.Nq, p.d, dtype=out_dtype, device=device)
+
+    def __call__(self, q, k, v, step: int = 0, stream=None) -> torch.Tensor:
+        _check_inputs(q, k, v)
+        p = self.p
+        pool(q if self.mode != "structured" else None, k, v, p, self.tables, stream)
+        if self.mode == "structured":
+            g = self.geometry
+            structured_mask(p, self.kv_idx, self.kv_cnt, g["frame_tokens"], g["n_frames"],
+                            g["window"], g["n_anchors"], g["period"], step, g.get("q_frame0", 0),
+                            stream)
+        else:
+            route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
+                  stream=stream)
+        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out, stream=stream)
+        return self.out

@@ -1,0 +1,206 @@
+// C ABI of the library: argument checks on the host, then one kernel launch per
+// entry point on the caller's stream. No allocation, no synchronisation.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/sparse_attn.h"
+#include "launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return SA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define SA_REQUIRE(cond, ...) \
+  do {                        \
+    if (!(cond)) return fail(SA_ERR_INVALID, __VA_ARGS__); \
+  } while (0)
+
+#define SA_REQUIRE_PTR(ptr) \
+  SA_REQUIRE((ptr) != nullptr && aligned16(ptr), "%s must be a non-null 16-byte aligned pointer", #ptr)
+
+int check_device() {
+  static int cache[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SA_ERR_LAUNCH, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64 && cache[dev] == 1) return SA_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  const bool good = major == 10 && minor == 0;
+  if (dev >= 0 && dev < 64) cache[dev] = good ? 1 : 2;
+  if (!good)
+    return fail(SA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                major, minor);
+  return SA_OK;
+}
+
+int launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(SA_ERR_LAUNCH, "%s: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+int check_shape(int B, int H, int Nq, int Nk, int d, int block) {
+  SA_REQUIRE(B >= 0 && H >= 0 && Nq >= 0 && Nk >= 0, "B, H, Nq, Nk must be >= 0");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(block == 64 || block == 128, "block must be 64 or 128 (got %d)", block);
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535 (got %lld)", (long long)B * H);
+  return SA_OK;
+}
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sparse_attn_last_error(void) { return g_last_error.c_str(); }
+
+int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
+                            size_t sizes[6]) {
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  SA_REQUIRE(sizes != nullptr, "sizes must not be NULL");
+  const size_t bh = (size_t)B * H, nqb = cdiv(Nq, block), nkb = cdiv(Nk, block);
+  sizes[0] = bh * nqb * d * sizeof(float);
+  sizes[1] = bh * nkb * d * sizeof(float);
+  sizes[2] = bh * nkb * d * sizeof(float);
+  sizes[3] = bh * nkb * d * 2;
+  sizes[4] = bh * nkb * d * 2;
+  sizes[5] = order == 1 ? bh * nkb * d * d * 2 : 0;
+  return ok();
+}
+
+int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Nq,
+                     int Nk, int d, int block, int order, float* qbar, float* kbar_t, float* vsum,
+                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, void* stream) {
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  const bool do_q = q != nullptr && Nq > 0;
+  if ((long long)B * H == 0 || (Nk == 0 && !do_q)) return ok();
+  if (Nk > 0) {
+    SA_REQUIRE_PTR(k);
+    SA_REQUIRE_PTR(v);
+    SA_REQUIRE_PTR(kbar_t);
+    SA_REQUIRE_PTR(vsum);
+    SA_REQUIRE_PTR(kbar16);
+    SA_REQUIRE_PTR(vsum16);
+    if (order == 1) SA_REQUIRE_PTR(M);
+  }
+  if (do_q) {
+    SA_REQUIRE_PTR(q);
+    SA_REQUIRE_PTR(qbar);
+  }
+  if (int rc = check_device()) return rc;
+  sa::PoolArgs p{do_q ? q : nullptr, k, v, B, H, Nq, Nk, d, block, order,
+                 cdiv(Nq, block), cdiv(Nk, block), qbar, kbar_t, vsum, kbar16, vsum16, M};
+  return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
+}
+
+int sparse_attn_route(const float* qbar, const float* kbar_t, int B, int H, int nqb, int nkb, int d,
+                      int mode, int rho_num, int rho_den, float tau, float scale, int32_t* kv_idx,
+                      int32_t* kv_cnt, int cap, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && nqb >= 0 && nkb >= 0, "B, H, nqb, nkb must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(mode == SA_ROUTE_TOPK || mode == SA_ROUTE_MASS, "mode must be TOPK or MASS");
+  SA_REQUIRE(std::isfinite(scale), "scale must be finite");
+  if ((long long)B * H * nqb == 0) return ok();
+  SA_REQUIRE(nkb >= 1 && nkb <= SA_MAX_KV_BLOCKS, "nkb must be in [1, %d] (got %d)",
+             SA_MAX_KV_BLOCKS, nkb);
+  int keep = nkb;
+  if (mode == SA_ROUTE_TOPK) {
+    SA_REQUIRE(rho_num > 0 && rho_den > 0 && rho_num <= rho_den,
+               "top-k needs 0 < rho_num <= rho_den (got %d/%d)", rho_num, rho_den);
+    keep = (int)(((long long)rho_num * nkb + rho_den - 1) / rho_den);
+    SA_REQUIRE(cap >= keep, "cap %d is below the keep count %d", cap, keep);
+  } else {
+    SA_REQUIRE(tau > 0.f && tau <= 1.f, "tau must be in (0, 1] (got %g)", (double)tau);
+    SA_REQUIRE(cap >= nkb, "mass routing needs cap >= nkb (cap %d, nkb %d)", cap, nkb);
+  }
+  SA_REQUIRE_PTR(qbar);
+  SA_REQUIRE_PTR(kbar_t);
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  if (int rc = check_device()) return rc;
+  sa::RouteArgs p{qbar, kbar_t, B, H, nqb, nkb, d, mode, keep, tau, scale, kv_idx, kv_cnt, cap};
+  return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
+}
+
+int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block, int frame_tokens,
+                                int n_frames, int window, int n_anchors, int period, int step,
+                                int q_frame0, int32_t* kv_idx, int32_t* kv_cnt, int cap,
+                                void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && Nq >= 0 && Nk >= 0, "B, H, Nq, Nk must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(block == 64 || block == 128, "block must be 64 or 128 (got %d)", block);
+  SA_REQUIRE(frame_tokens >= 1 && n_frames >= 1, "frame_tokens and n_frames must be >= 1");
+  SA_REQUIRE(window >= 0 && n_anchors >= 0 && period >= 1 && step >= 0 && q_frame0 >= 0,
+             "window, n_anchors, step, q_frame0 must be >= 0 and period >= 1");
+  SA_REQUIRE((long long)Nk <= (long long)n_frames * frame_tokens,
+             "Nk exceeds n_frames * frame_tokens");
+  SA_REQUIRE((long long)q_frame0 * frame_tokens + Nq <= (long long)n_frames * frame_tokens,
+             "the query tokens run past the last frame");
+  if ((long long)B * H * Nq == 0) return ok();
+  const int nkb = cdiv(Nk, block);
+  SA_REQUIRE(nkb >= 1, "Nk must be >= 1");
+  SA_REQUIRE(cap >= nkb, "structured mask needs cap >= nkb (cap %d, nkb %d)", cap, nkb);
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  if (int rc = check_device()) return rc;
+  sa::MaskArgs p{B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors, period, step,
+                 q_frame0, cdiv(Nq, block), nkb, kv_idx, kv_cnt, cap};
+  return launched(sa::launch_structured_mask(p, static_cast<cudaStream_t>(stream)), "mask launch");
+}
+
+int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
+                        const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H, int Nq,
+                        int Nk, int d, int block, int order, float scale, void* out, int out_dtype,
+                        int32_t* err_flag, void* stream) {
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  SA_REQUIRE(out_dtype == SA_OUT_F32 || out_dtype == SA_OUT_BF16, "out_dtype must be F32 or BF16");
+  SA_REQUIRE(std::isfinite(scale), "scale must be finite");
+  if ((long long)B * H * Nq == 0) return ok();
+  SA_REQUIRE(Nk >= 1, "Nk must be >= 1 when there are queries");
+  const int nkb = cdiv(Nk, block);
+  SA_REQUIRE(nkb <= SA_MAX_KV_BLOCKS, "nkb must be <= %d (got %d)", SA_MAX_KV_BLOCKS, nkb);
+  SA_REQUIRE(cap >= 0, "cap must be >= 0");
+  SA_REQUIRE_PTR(q);
+  SA_REQUIRE_PTR(k);
+  SA_REQUIRE_PTR(v);
+  SA_REQUIRE_PTR(kbar16);
+  SA_REQUIRE_PTR(vsum16);
+  if (order == 1) SA_REQUIRE_PTR(M);
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  SA_REQUIRE_PTR(out);
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
+  if (int rc = check_device()) return rc;
+  sa::ForwardArgs p{q, k, v, kbar16, vsum16, order == 1 ? M : nullptr, kv_idx, kv_cnt, cap,
+                    B, H, Nq, Nk, d, block, order, cdiv(Nq, block), nkb, scale, out, out_dtype,
+                    err_flag};
+  return launched(sa::launch_forward(p, static_cast<cudaStream_t>(stream)), "forward launch");
+}
+
+}  // extern "C"

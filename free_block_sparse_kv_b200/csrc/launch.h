@@ -1,0 +1,46 @@
+// Host-side launch interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sa {
+
+struct PoolArgs {
+  const uint16_t *q, *k, *v;
+  int B, H, Nq, Nk, d, block, order, nqb, nkb;
+  float *qbar, *kbar_t, *vsum;
+  uint16_t *kbar16, *vsum16, *M;
+};
+
+struct RouteArgs {
+  const float *qbar, *kbar_t;
+  int B, H, nqb, nkb, d, mode, keep;
+  float tau, scale;
+  int32_t *kv_idx, *kv_cnt;
+  int cap;
+};
+
+struct MaskArgs {
+  int B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors, period, step, q_frame0;
+  int nqb, nkb;
+  int32_t *kv_idx, *kv_cnt;
+  int cap;
+};
+
+struct ForwardArgs {
+  const uint16_t *q, *k, *v, *kbar16, *vsum16, *M;
+  const int32_t *kv_idx, *kv_cnt;
+  int cap, B, H, Nq, Nk, d, block, order, nqb, nkb;
+  float scale;
+  void* out;
+  int out_dtype;
+  int32_t* err_flag;
+};
+
+cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
+cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
+cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);
+cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st);
+
+}  // namespace sa

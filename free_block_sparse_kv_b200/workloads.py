@@ -181,12 +181,8 @@ def _clustered(w: Workload, rng: np.random.Generator, first_token: int, n_tokens
     raise ValueError(f"unknown recipe {w.recipe!r}")
 
 
-def head_inputs(w: Workload, b: int, h: int):
-    """Q [Nq, d], K [Nk, d], V [Nk, d] of one (batch, head), bf16-rounded, as fp32 arrays.
-
-    Draw order within the head: Q centers, Q noise, K centers, K noise, outlier
-    mask, V. Q and K draw independent centers from the same distribution.
-    """
+def _head_f32(w: Workload, b: int, h: int):
+    """Unrounded fp32 draws of one head (see :func:`head_inputs` for the order)."""
     q_first = w.q_frame0 * w.frame_tokens
     q = _clustered(w, _rng(w, _Q, b, h), q_first, w.Nq)
     rk = _rng(w, _K, b, h)
@@ -195,27 +191,49 @@ def head_inputs(w: Workload, b: int, h: int):
         rows = rk.random(w.Nk) < w.outlier_p
         k[rows] *= np.float32(w.outlier_scale)
     v = _rng(w, _V, b, h).standard_normal((w.Nk, w.d), dtype=np.float32)
-    return bf16_round(q)[0], bf16_round(k)[0], bf16_round(v)[0]
+    return q, k, v
 
 
 def head_inputs_bits(w: Workload, b: int, h: int):
-    """Same draws as :func:`head_inputs`, as uint16 bf16 bit patterns."""
-    q, k, v = head_inputs(w, b, h)
-    return tuple(bf16_round(x)[1] for x in (q, k, v))
+    """bf16 bit patterns (uint16) of Q [Nq, d], K [Nk, d], V [Nk, d] of one head."""
+    return tuple(bf16_round(x)[1] for x in _head_f32(w, b, h))
 
 
-def full_inputs_bits(w: Workload, heads=None):
+def bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact fp32 values of bf16 bit patterns."""
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def head_inputs(w: Workload, b: int, h: int):
+    """Q [Nq, d], K [Nk, d], V [Nk, d] of one (batch, head), bf16-rounded, as fp32 arrays.
+
+    Draw order within the head: Q centers, Q noise, K centers, K noise, outlier
+    mask, V. Q and K draw independent centers from the same distribution.
+    """
+    return tuple(bits_to_f32(x) for x in head_inputs_bits(w, b, h))
+
+
+def full_inputs_bits(w: Workload, heads=None, threads: int = 0):
     """bf16 bits of Q [B,H,Nq,d], K and V [B,H,Nk,d] for the whole workload.
 
     ``heads`` optionally limits the draw to a list of (b, h) pairs; the other heads
-    are left zero.
+    are left zero. Heads are drawn on ``threads`` threads (default: the usable
+    cores); each head's stream is independent, so the result does not depend on it.
     """
+    import concurrent.futures
+    import os
     q = np.zeros((w.B, w.H, w.Nq, w.d), dtype=np.uint16)
     k = np.zeros((w.B, w.H, w.Nk, w.d), dtype=np.uint16)
     v = np.zeros((w.B, w.H, w.Nk, w.d), dtype=np.uint16)
     todo = heads if heads is not None else [(b, h) for b in range(w.B) for h in range(w.H)]
-    for b, h in todo:
+
+    def one(bh):
+        b, h = bh
         q[b, h], k[b, h], v[b, h] = head_inputs_bits(w, b, h)
+
+    n = threads or max(1, min(32, len(os.sched_getaffinity(0))))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(one, todo))
     return q, k, v
 
 

@@ -1,0 +1,160 @@
+/*
+ * sparse_attn.h - C ABI of the block-sparse attention library with compensation
+ * for skipped blocks, for NVIDIA B200 (sm_100a).
+ *
+ * The operation. Per (batch b, head h), with Q [Nq, d] and K, V [Nk, d] split into
+ * blocks of `block` tokens (the last block may be partial, holding n_j tokens):
+ *   - every KV block j is pooled into its centroid kbar_j = mean K, its value sum
+ *     S_j = sum V and (first order) M_j = sum_r (k_r - kbar_j) v_r^T;
+ *   - every query block i keeps a set of KV blocks, chosen from the pooled scores
+ *     scale * qbar_i . kbar_j (top-rho or covering mass tau), or from a frame
+ *     geometry (local window plus rotating anchor frames);
+ *   - the output o_t = N_t / D_t sums exact softmax terms over the tokens of kept
+ *     blocks and, for every skipped block j, alpha_tj * (S_j + [order 1] scale *
+ *     q_t M_j) in the numerator and alpha_tj * n_j in the denominator, with
+ *     alpha_tj = exp(scale * q_t . kbar_j): all inside one softmax.
+ * Sources: "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion
+ * Transformers" §2 (Algorithme Central: o_t = N_t / D_t, the numerator N_t,
+ * alpha_{t,j}; Cohérence de Normalisation; Implémentation Matérielle);
+ * "LVSA: Training-Free Sparse Attention for Long Video Diffusion" §2 (Mécanisme
+ * Central: A(t) = G u W(t), rotating anchors); "SVG-EAR: Parameter-Free Linear
+ * Compensation for Sparse Video Generation via Error-aware Routing" §2 (centroid
+ * substitution; query centroids as routing proxies).
+ *
+ * Conventions for every entry point.
+ *   - bf16 tensors are passed as pointers to their 16-bit patterns (uint16_t).
+ *   - Tensors are dense and contiguous in the layout stated for each argument,
+ *     d innermost. Every device pointer must be 16-byte aligned.
+ *   - The caller allocates and owns every buffer. The library never allocates,
+ *     frees or synchronises; all work is enqueued on `stream` (a cudaStream_t,
+ *     NULL for the legacy default stream) in call order.
+ *   - Supported shapes: d in {64, 128}; block in {64, 128}; B, H >= 0; Nq, Nk >= 0.
+ *     A call with an empty problem (B*H*Nq == 0) returns SA_OK and does nothing.
+ *     Nq = 0 with Nk > 0 and the reverse are both empty for the forward.
+ *   - Return value: SA_OK, or an error code below; the calling thread's last
+ *     error message is then available from sparse_attn_last_error(). Argument
+ *     errors are found on the host before anything is enqueued.
+ */
+#ifndef SPARSE_ATTN_H_
+#define SPARSE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SA_OK = 0,
+  SA_ERR_INVALID = 1,      /* bad shape, null or misaligned pointer, capacity too small */
+  SA_ERR_LAUNCH = 2,       /* a CUDA launch or runtime call failed */
+  SA_ERR_TIMEOUT = 3,      /* a bounded device wait gave up (reported through err_flag) */
+  SA_ERR_UNSUPPORTED = 4   /* the current device is not sm_100 */
+};
+
+enum { SA_ROUTE_TOPK = 0, SA_ROUTE_MASS = 1 };
+enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
+
+/* Largest number of KV blocks per head that routing and the forward accept. */
+#define SA_MAX_KV_BLOCKS 2048
+
+/*
+ * Byte sizes of the pooled tables for a problem, written to sizes[0..5] in the
+ * order qbar, kbar_t, vsum, kbar16, vsum16, M (M is 0 when order == 0).
+ * nqb = ceil(Nq / block), nkb = ceil(Nk / block).
+ */
+int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
+                            size_t sizes[6]);
+
+/*
+ * Pooling (PISA §2 Implémentation Matérielle, pre-computation step; the per-block
+ * first-order matrix of the Taylor expansion about kbar_j; SVG-EAR §2 B query
+ * centroids). One pass over Q, K and V.
+ *   q       [B,H,Nq,d] bf16, may be NULL (then qbar is not written and may be NULL)
+ *   k, v    [B,H,Nk,d] bf16
+ *   order   0 or 1; with 1, M is written and must not be NULL
+ *   qbar    [B,H,nqb,d]  fp32   mean of each query block's rows
+ *   kbar_t  [B,H,d,nkb]  fp32   block centroids, dim-major (routing reads it)
+ *   vsum    [B,H,nkb,d]  fp32   value sums S_j
+ *   kbar16  [B,H,nkb,d]  bf16   centroids, rounded to nearest (forward reads it)
+ *   vsum16  [B,H,nkb,d]  bf16   value sums, rounded to nearest (forward reads it)
+ *   M       [B,H,nkb,d,d] bf16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
+ *                               a = key dim (rows), c = value dim; fp32 accumulate
+ * Means of a partial last block use its true token count.
+ */
+int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     int B, int H, int Nq, int Nk, int d, int block, int order,
+                     float* qbar, float* kbar_t, float* vsum,
+                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, void* stream);
+
+/*
+ * Routing (PISA §2 top-k choice of the critical blocks; SVG-EAR §2 B pooled
+ * proxies). Scores s_ij = scale * qbar_i . kbar_j in fp32; blocks are ordered by
+ * (s descending, j ascending).
+ *   qbar    [B,H,nqb,d] fp32;  kbar_t [B,H,d,nkb] fp32 (as written by the pool)
+ *   mode    SA_ROUTE_TOPK: keep the first ceil(rho_num * nkb / rho_den) blocks
+ *                          (integer arithmetic; 0 < rho_num <= rho_den)
+ *           SA_ROUTE_MASS: keep the shortest prefix whose softmax(s_i.) mass is
+ *                          >= tau (0 < tau <= 1)
+ *   kv_idx  [B,H,nqb,cap] int32  kept block indices of each query block, ascending;
+ *                                entries past kv_cnt are left untouched
+ *   kv_cnt  [B,H,nqb]     int32  number of kept blocks
+ *   cap     >= the keep count for TOPK, >= nkb for MASS
+ * nkb <= SA_MAX_KV_BLOCKS.
+ */
+int sparse_attn_route(const float* qbar, const float* kbar_t,
+                      int B, int H, int nqb, int nkb, int d,
+                      int mode, int rho_num, int rho_den, float tau, float scale,
+                      int32_t* kv_idx, int32_t* kv_cnt, int cap, void* stream);
+
+/*
+ * Structured mask (LVSA §2 Mécanisme Central). Tokens are frame-major with
+ * frame_tokens tokens per frame; query token t lies in frame
+ * q_frame0 + t / frame_tokens and key token r in frame r / frame_tokens.
+ * At denoising step `step` the anchor frames are
+ *   G = { (step mod period) + period * m : m = 0 .. n_anchors-1 } (those < n_frames),
+ * and query frame f attends A(f) = G u { f-window .. f+window } (inside the video).
+ * KV block j is kept for query block i when some query token of i and some key
+ * token of j have frames (f, g) with g in A(f). Same list format as routing;
+ * cap >= nkb. Every (b, h) gets the same lists.
+ */
+int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
+                                int frame_tokens, int n_frames, int window,
+                                int n_anchors, int period, int step, int q_frame0,
+                                int32_t* kv_idx, int32_t* kv_cnt, int cap, void* stream);
+
+/*
+ * Forward (PISA §2 Algorithme Central and Implémentation Matérielle, phases 1-3,
+ * with the first-order term per block). For each query row t of query block i:
+ *   exact logits    scale * q_t . k_r   for the tokens r of the kept blocks of i
+ *   centroid logits scale * q_t . kbar_j for the other blocks j
+ *   N_t = sum_r e^(l_r - m) v_r + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j)
+ *   D_t = sum_r e^(l_r - m)     + sum_j e^(c_j - m) n_j
+ *   o_t = N_t / D_t
+ *   q, k, v           as for the pool
+ *   kbar16, vsum16, M as written by the pool (M NULL when order == 0)
+ *   kv_idx, kv_cnt    as written by routing or the structured mask: indices of
+ *                     each row must be distinct and < nkb; entries outside
+ *                     [0, nkb) are ignored; kv_cnt is clamped to [0, cap]
+ *   scale             logit scale, normally 1/sqrt(d)
+ *   out               [B,H,Nq,d], fp32 (SA_OUT_F32) or bf16 (SA_OUT_BF16)
+ *   err_flag          optional device int32: set non-zero if a bounded device
+ *                     wait gives up (the call then returns normally; the caller
+ *                     reads the flag and sees SA_ERR_TIMEOUT semantics)
+ */
+int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
+                        const int32_t* kv_idx, const int32_t* kv_cnt, int cap,
+                        int B, int H, int Nq, int Nk, int d, int block, int order,
+                        float scale, void* out, int out_dtype, int32_t* err_flag,
+                        void* stream);
+
+/* Message for the last error returned on the calling thread ("" if none). */
+const char* sparse_attn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H_ */

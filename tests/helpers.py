@@ -1,0 +1,63 @@
+"""Shared helpers for the parity tests: run the CUDA path on seeded inputs and
+compare with the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+from free_block_sparse_kv_b200 import workloads as W
+from oracle import block_sparse_attention as O
+
+# Output tolerance for floating point: max abs error and mean relative (L1 ratio) error.
+MAX_ABS = 1e-2
+MEAN_REL = 2e-3
+# A kept-set decision is pinned (must match bit for bit) when the oracle's logit gap at
+# the cutoff, and for mass routing both cumulative-mass margins, exceed this.
+GATE = 1e-4
+
+# Reduced workloads the oracle finishes in seconds. They keep each full workload's
+# recipe and span several 64-wide tiles plus a ragged last block.
+SMALL = {
+    "uniform-4k": W.WORKLOADS["uniform-4k"],
+    "dit-small": W.shrink(W.WORKLOADS["dit-21x30x52"], name="dit-small", H=2, Nq=9000, Nk=9000,
+                          grid=(9, 20, 50)),
+    "dit720p-small": W.shrink(W.WORKLOADS["dit720p-21x45x80"], name="dit720p-small", H=2, Nq=9480,
+                              Nk=9480, grid=(6, 20, 79)),
+    "longvideo-small": W.shrink(W.WORKLOADS["longvideo-41x30x52"], name="longvideo-small", H=2,
+                                Nq=9500, Nk=9500, grid=(19, 10, 50), window=2, n_anchors=3,
+                                period=6, steps=(0, 5)),
+    "worldmodel-small": W.shrink(W.WORKLOADS["worldmodel-chunk"], name="worldmodel-small", B=2, H=2,
+                                 Nq=500, Nk=6500, grid=(13, 10, 50), q_frame0=12),
+}
+
+
+def err_stats(got: np.ndarray, want: np.ndarray):
+    diff = np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64))
+    return float(diff.max()), float(diff.sum() / np.abs(want).sum())
+
+
+def oracle_kept(w: W.Workload, q, k, step: int = 0):
+    """Oracle kept lists of one head and the per-row gate flags (True = pinned)."""
+    if w.mode == "structured":
+        kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
+                                 w.n_anchors, w.period, step, w.q_frame0)
+        return kept, np.ones(len(kept), bool)
+    if w.mode == "topk":
+        kept, s, counts = O.route_head(q, k, w.block, "topk", w.scale, keep=w.keep())
+        gaps, _, _ = O.gate_diagnostics(s, counts)
+        return kept, gaps > GATE
+    kept, s, counts = O.route_head(q, k, w.block, "mass", w.scale, tau=w.tau)
+    gaps, lo, hi = O.gate_diagnostics(s, counts, tau=w.tau)
+    return kept, (gaps > GATE) & (lo > GATE) & (hi > GATE)
+
+
+def lists_to_sets(kv_idx: np.ndarray, kv_cnt: np.ndarray):
+    return [sorted(int(x) for x in kv_idx[i, :kv_cnt[i]]) for i in range(kv_cnt.shape[0])]
+
+
+def sample_rows(w: W.Workload, n: int, seed: int = 0):
+    """Query rows to check at full size: first and last rows, both ends of the last
+    (possibly partial) block, and a seeded spread in between."""
+    rng = np.random.default_rng(seed)
+    fixed = {0, 1, w.Nq - 1, w.Nq - 2, (w.nqb - 1) * w.block, min(w.Nq - 1, w.block)}
+    rest = rng.choice(w.Nq, size=max(0, n - len(fixed)), replace=False)
+    return np.array(sorted(fixed | set(int(x) for x in rest)))

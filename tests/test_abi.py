@@ -1,0 +1,86 @@
+"""The C ABI library loads, exports every entry point the header declares, and
+rejects bad arguments on the host (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from free_block_sparse_kv_b200 import build
+from free_block_sparse_kv_b200 import sparse_attn as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(sparse_attn_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return C.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared >= set(C.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_table_sizes():
+    assert C.sparse_attn_table_sizes(1, 40, 75600, 75600, 128, 128, 1) == (
+        40 * 591 * 128 * 4, 40 * 591 * 128 * 4, 40 * 591 * 128 * 4,
+        40 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2)
+    assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[5] == 0
+    assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[0] == 4 * 16 * 25 * 128 * 4
+
+
+def test_host_argument_checks(lib):
+    buf = (ctypes.c_char * 4096)()
+    base = ctypes.addressof(buf)
+    p = base + (-base) % 16
+    cases = [
+        lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 96, 64, 0),
+        lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 64, 32, 0),
+        lambda: C.sparse_attn_table_sizes(-1, 1, 64, 64, 64, 64, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, p, 0),
+        lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_route(p, p, 1, 1, 4, 3000, 64, 0, 1, 4, 0.9, 0.1, p, p, 750, 0),
+        lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 0, 3, 2, 0.9, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 1, 1, 4, 1.5, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 7, 1, 4, 0.9, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_structured_mask(1, 1, 64, 6400, 64, 10, 10, 1, 1, 1, 0, 0, p, p, 100, 0),
+        lambda: C.sparse_attn_structured_mask(1, 1, 64, 64, 64, 8, 8, 1, 1, 0, 0, 0, p, p, 1, 0),
+        lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 0, 64, 64, 0, 0.1, p, 0,
+                                      None, 0),
+        lambda: C.sparse_attn_forward(p, p, p, p, p, None, p, p, 1, 1, 1, 64, 64, 64, 64, 1, 0.1, p,
+                                      0, None, 0),
+        lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 64, 64, 0, 0.1, p, 5,
+                                      None, 0),
+        lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64 * 4096, 64, 64, 0, 0.1,
+                                      p, 0, None, 0),
+    ]
+    for i, call in enumerate(cases):
+        with pytest.raises(C.SparseAttnError) as e:
+            call()
+        assert e.value.code == C.SA_ERR_INVALID, (i, str(e.value))
+        assert C.sparse_attn_last_error(), i
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = C._lib
+    C._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="missing"):
+            C.load_library(str(tmp_path / "absent.so"))
+    finally:
+        C._lib = saved

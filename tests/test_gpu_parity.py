@@ -1,0 +1,339 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on seeded inputs.
+
+Masks: bit-exact wherever the oracle's cutoff gap exceeds the gate. Outputs: max
+abs error and mean relative error within the stated tolerance, on fp32 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+from free_block_sparse_kv_b200 import attention as A
+from free_block_sparse_kv_b200 import sparse_attn as C
+from free_block_sparse_kv_b200 import workloads as W
+from oracle import block_sparse_attention as O
+from tests.helpers import (GATE, MAX_ABS, MEAN_REL, SMALL, err_stats, lists_to_sets, oracle_kept,
+                           sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _problem(w):
+    return A.Problem(w.B, w.H, w.Nq, w.Nk, w.d, w.block, w.order)
+
+
+def _geometry(w):
+    return dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
+                n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0)
+
+
+def _run(w, q, k, v, step=0, out_dtype=torch.float32):
+    op = A.BlockSparseAttention(_problem(w), w.mode, rho=w.rho, tau=w.tau,
+                                geometry=_geometry(w) if w.mode == "structured" else None,
+                                out_dtype=out_dtype)
+    out = op(q, k, v, step=step)
+    torch.cuda.synchronize()
+    return op, out
+
+
+def _sample_rows_small(w, per_tile=3, seed=1):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for s in range(0, w.Nq, 64):
+        e = min(w.Nq, s + 64)
+        rows |= {s, e - 1}
+        rows |= set(int(x) for x in rng.integers(s, e, size=per_tile))
+    return np.array(sorted(rows))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    C.load_library()
+
+
+@pytest.fixture(scope="module")
+def small_inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            w = SMALL[name]
+            cache[name] = (w,) + W.full_inputs_bits(w)
+        return cache[name]
+    return get
+
+
+# --- pooling -------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_pool_matches_oracle(name, small_inputs):
+    w, qb, kb, vb = small_inputs(name)
+    p = _problem(w)
+    t = A.allocate_tables(p, "cuda")
+    A.pool(_dev(qb), _dev(kb), _dev(vb), p, t)
+    torch.cuda.synchronize()
+    for b in range(w.B):
+        for h in range(w.H):
+            q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+            kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, w.order)
+            qbar = O.pool_queries(q, w.block)
+            np.testing.assert_allclose(t.qbar[b, h].cpu().numpy(), qbar, rtol=0, atol=2e-6)
+            np.testing.assert_allclose(t.kbar_t[b, h].cpu().numpy().T, kbar, rtol=0, atol=2e-6)
+            np.testing.assert_allclose(t.vsum[b, h].cpu().numpy(), vsum, rtol=0, atol=2e-5)
+            k16 = t.kbar16[b, h].float().cpu().numpy()
+            np.testing.assert_allclose(k16, kbar, rtol=2 ** -8, atol=1e-6)
+            v16 = t.vsum16[b, h].float().cpu().numpy()
+            np.testing.assert_allclose(v16, vsum, rtol=2 ** -8, atol=1e-5)
+            if w.order == 1:
+                mg = t.M[b, h].float().cpu().numpy()
+                tol = 2 ** -8 * np.abs(mats) + 1e-3
+                assert np.all(np.abs(mg - mats) <= tol), float(np.abs(mg - mats).max())
+
+
+# --- routing and structured masks ----------------------------------------------
+
+@pytest.mark.parametrize("name", [n for n, w in SMALL.items() if w.mode != "structured"])
+def test_route_masks_bit_exact_above_gate(name, small_inputs):
+    w, qb, kb, vb = small_inputs(name)
+    op, _ = _run(w, _dev(qb), _dev(kb), _dev(vb))
+    idx, cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
+    pinned = total = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            q, k = W.bits_to_f32(qb[b, h]), W.bits_to_f32(kb[b, h])
+            kept, gate = oracle_kept(w, q, k)
+            got = lists_to_sets(idx[b, h], cnt[b, h])
+            for i in range(w.nqb):
+                total += 1
+                if w.mode == "topk":
+                    assert len(got[i]) == w.keep()
+                if gate[i]:
+                    pinned += 1
+                    assert got[i] == kept[i].tolist(), (b, h, i)
+    assert pinned >= 0.5 * total, (pinned, total)
+
+
+@pytest.mark.parametrize("name", ["longvideo-small", "longvideo-41x30x52", "worldmodel-chunk"])
+def test_structured_mask_bit_exact(name):
+    w = SMALL.get(name) or W.WORKLOADS[name]
+    p = A.Problem(1, 2, w.Nq, w.Nk, w.d, w.block, w.order)
+    steps = range(w.period) if w.mode == "structured" else (0, 3)
+    for step in steps:
+        idx, cnt = A.allocate_lists(p, p.nkb, "cuda")
+        A.structured_mask(p, idx, cnt, w.frame_tokens, w.n_frames, w.window, w.n_anchors,
+                          w.period, step, w.q_frame0)
+        torch.cuda.synchronize()
+        want = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
+                                 w.n_anchors, w.period, step, w.q_frame0)
+        for h in range(2):
+            got = lists_to_sets(idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy())
+            assert got == [x.tolist() for x in want], (name, step)
+
+
+# --- forward ------------------------------------------------------------------
+
+def _oracle_lists_to_device(w, kept_per_head, cap):
+    idx = np.zeros((w.B, w.H, w.nqb, max(cap, 1)), np.int32)
+    cnt = np.zeros((w.B, w.H, w.nqb), np.int32)
+    for (b, h), kept in kept_per_head.items():
+        for i, row in enumerate(kept):
+            idx[b, h, i, :len(row)] = row
+            cnt[b, h, i] = len(row)
+    return torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_matches_oracle_on_oracle_masks(name, out_dtype, small_inputs):
+    """Forward alone: the GPU forward consumes the oracle's kept lists."""
+    w, qb, kb, vb = small_inputs(name)
+    step = w.steps[-1] if w.mode == "structured" else 0
+    kept_all = {}
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    for b, h in heads:
+        q, k = W.bits_to_f32(qb[b, h]), W.bits_to_f32(kb[b, h])
+        kept_all[(b, h)] = oracle_kept(w, q, k, step)[0]
+    cap = max(len(r) for kept in kept_all.values() for r in kept)
+    idx, cnt = _oracle_lists_to_device(w, kept_all, cap)
+    p = _problem(w)
+    t = A.allocate_tables(p, "cuda")
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    A.pool(q_d, k_d, v_d, p, t)
+    out = torch.empty(w.B, w.H, w.Nq, w.d, dtype=out_dtype, device="cuda")
+    A.forward(q_d, k_d, v_d, p, t, idx, cnt, out)
+    torch.cuda.synchronize()
+    rows = _sample_rows_small(w)
+    got_all, want_all = [], []
+    for b, h in heads:
+        q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+        want_all.append(O.forward_head(q, k, v, kept_all[(b, h)], w.block, w.order, w.scale,
+                                       rows=rows))
+        got_all.append(out[b, h, rows].float().cpu().numpy())
+    got, want = np.concatenate(got_all), np.concatenate(want_all)
+    mx, mr = err_stats(got, want)
+    if out_dtype == torch.float32:
+        assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+    else:
+        want16 = torch.from_numpy(want).to(torch.bfloat16).double().numpy()
+        floor = err_stats(want16, want)[1]
+        assert mx <= MAX_ABS and mr <= MEAN_REL + floor, (mx, mr, floor)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_pipeline_matches_oracle(name, small_inputs):
+    """pool -> route (or mask) -> forward on the GPU against the oracle's own pipeline."""
+    w, qb, kb, vb = small_inputs(name)
+    steps = w.steps if w.mode == "structured" else (0,)
+    rows = _sample_rows_small(w, per_tile=2, seed=2)
+    for step in steps:
+        _, out = _run(w, _dev(qb), _dev(kb), _dev(vb), step=step)
+        got_all, want_all = [], []
+        for b in range(w.B):
+            for h in range(w.H):
+                q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+                kept, _ = oracle_kept(w, q, k, step)
+                want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=rows))
+                got_all.append(out[b, h, rows].cpu().numpy())
+        mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
+        assert mx <= MAX_ABS and mr <= MEAN_REL, (name, step, mx, mr)
+
+
+# --- full-size workloads (sampled heads and rows) -------------------------------
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_full_size_sampled(name):
+    w = W.WORKLOADS[name]
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    qb, kb, vb = W.full_inputs_bits(w)
+    step = 7 if w.mode == "structured" else 0
+    op, out = _run(w, _dev(qb), _dev(kb), _dev(vb), step=step)
+    idx, cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
+    rows = sample_rows(w, 40)
+    got_all, want_all = [], []
+    pinned = total = 0
+    for b, h in heads:
+        q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+        kept, gate = oracle_kept(w, q, k, step)
+        got = lists_to_sets(idx[b, h], cnt[b, h])
+        for i in range(w.nqb):
+            total += 1
+            if gate[i]:
+                pinned += 1
+                assert got[i] == kept[i].tolist(), (name, b, h, i)
+        want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=rows))
+        got_all.append(out[b, h, rows].cpu().numpy())
+    assert pinned >= 0.5 * total, (pinned, total)
+    mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (name, mx, mr)
+
+
+# --- edge cases -----------------------------------------------------------------
+
+def _rand_bits(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return W.bf16_round(scale * rng.standard_normal(shape).astype(np.float32))[1]
+
+
+@pytest.mark.parametrize("d,block,order", [(64, 64, 0), (64, 128, 1), (128, 64, 1), (128, 128, 0)])
+def test_all_kept_is_dense_attention(d, block, order):
+    B, H, N = 1, 2, 700
+    qb, kb, vb = (_rand_bits((B, H, N, d), s) for s in (1, 2, 3))
+    p = A.Problem(B, H, N, N, d, block, order)
+    t = A.allocate_tables(p, "cuda")
+    idx = torch.arange(p.nkb, dtype=torch.int32, device="cuda").expand(B, H, p.nqb, p.nkb).contiguous()
+    cnt = torch.full((B, H, p.nqb), p.nkb, dtype=torch.int32, device="cuda")
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    A.pool(q_d, k_d, v_d, p, t)
+    out = torch.empty(B, H, N, d, device="cuda")
+    A.forward(q_d, k_d, v_d, p, t, idx, cnt, out)
+    torch.cuda.synchronize()
+    rows = np.arange(0, N, 7)
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        want = torch.nn.functional.scaled_dot_product_attention(
+            *(torch.from_numpy(x.astype(np.float64))[None] for x in (q[rows], k, v)))[0].numpy()
+        mx, mr = err_stats(out[0, h, rows].cpu().numpy(), want)
+        assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_nothing_kept_and_bad_list_entries(order):
+    """cap 0 (every block compensated) and lists holding out-of-range entries, which
+    the forward ignores, against the oracle with nothing kept / the valid entries."""
+    B, H, N, d, block = 1, 1, 1000, 128, 128
+    qb, kb, vb = _rand_bits((B, H, N, d), 4), _rand_bits((B, H, N, d), 5, 0.3), _rand_bits((B, H, N, d), 6)
+    p = A.Problem(B, H, N, N, d, block, order)
+    t = A.allocate_tables(p, "cuda")
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    A.pool(q_d, k_d, v_d, p, t)
+    q, k, v = (W.bits_to_f32(x[0, 0]) for x in (qb, kb, vb))
+    # nothing kept
+    idx = torch.zeros(B, H, p.nqb, 1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, H, p.nqb, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, H, N, d, device="cuda")
+    C.sparse_attn_forward(q_d, k_d, v_d, t.kbar16, t.vsum16, t.M, idx, cnt, 0, B, H, N, N, d, block,
+                          order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
+    torch.cuda.synchronize()
+    want = O.forward_head(q, k, v, [np.zeros(0, int)] * p.nqb, block, order, 1 / np.sqrt(d))
+    mx, mr = err_stats(out[0, 0].cpu().numpy(), want)
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+    # lists with entries outside [0, nkb) and a count above cap
+    lists = [[i, (i + 3) % p.nkb] for i in range(p.nqb)]
+    raw = np.full((B, H, p.nqb, 4), -5, np.int32)
+    for i, r in enumerate(lists):
+        raw[0, 0, i, :3] = [r[0], p.nkb + 2, r[1]]
+    idx = torch.from_numpy(raw).cuda()
+    cnt = torch.full((B, H, p.nqb), 9, dtype=torch.int32, device="cuda")
+    C.sparse_attn_forward(q_d, k_d, v_d, t.kbar16, t.vsum16, t.M, idx, cnt, 4, B, H, N, N, d, block,
+                          order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
+    torch.cuda.synchronize()
+    want = O.forward_head(q, k, v, [np.array(sorted(r)) for r in lists], block, order, 1 / np.sqrt(d))
+    mx, mr = err_stats(out[0, 0].cpu().numpy(), want)
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+
+
+def test_empty_problems_are_no_ops():
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(16, dtype=torch.float32, device="cuda")
+    i = torch.zeros(16, dtype=torch.int32, device="cuda")
+    C.sparse_attn_pool(x, x, x, 0, 4, 100, 100, 128, 128, 1, f, f, f, x, x, x)
+    C.sparse_attn_route(f, f, 1, 1, 0, 10, 128, 0, 1, 4, 0.9, 0.1, i, i, 3)
+    C.sparse_attn_structured_mask(1, 1, 0, 100, 64, 10, 10, 1, 1, 1, 0, 0, i, i, 2)
+    C.sparse_attn_forward(x, x, x, x, x, x, i, i, 1, 1, 1, 0, 100, 128, 128, 1, 0.1, f, 0)
+    torch.cuda.synchronize()
+    assert int(i.abs().sum()) == 0
+
+
+def test_invalid_arguments_raise():
+    x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(64, dtype=torch.float32, device="cuda")
+    i = torch.zeros(64, dtype=torch.int32, device="cuda")
+    with pytest.raises(C.SparseAttnError) as e:
+        C.sparse_attn_forward(x, x, x, x, x, x, i, i, 1, 1, 1, 64, 64, 96, 64, 0, 0.1, f, 0)
+    assert e.value.code == C.SA_ERR_INVALID and "d must be" in str(e.value)
+    with pytest.raises(C.SparseAttnError) as e:
+        C.sparse_attn_forward(x.data_ptr() + 2, x, x, x, x, x, i, i, 1, 1, 1, 64, 64, 64, 64, 0,
+                              0.1, f, 0)
+    assert e.value.code == C.SA_ERR_INVALID and "aligned" in str(e.value)
+    with pytest.raises(C.SparseAttnError) as e:   # cap below the keep count
+        C.sparse_attn_route(f, f, 1, 1, 4, 10, 64, 0, 1, 2, 0.9, 0.1, i, i, 4)
+    assert e.value.code == C.SA_ERR_INVALID
+    with pytest.raises(C.SparseAttnError) as e:   # mass routing needs cap >= nkb
+        C.sparse_attn_route(f, f, 1, 1, 4, 10, 64, 1, 1, 2, 0.9, 0.1, i, i, 9)
+    assert e.value.code == C.SA_ERR_INVALID
+    with pytest.raises(C.SparseAttnError):        # order 1 without M
+        C.sparse_attn_pool(x, x, x, 1, 1, 64, 64, 64, 64, 1, f, f, f, x, x, None)
+
+
+def test_repeat_calls_are_bitwise_deterministic(small_inputs):
+    w, qb, kb, vb = small_inputs("dit-small")
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    _, a = _run(w, q, k, v)
+    a = a.clone()
+    _, b = _run(w, q, k, v)
+    assert torch.equal(a, b)
