@@ -21,9 +21,9 @@ class Tables:
     qbar: torch.Tensor      # [B,H,nqb,d] fp32
     kbar_t: torch.Tensor    # [B,H,d,nkb] fp32
     vsum: torch.Tensor      # [B,H,nkb,d] fp32
-    kbar16: torch.Tensor    # [B,H,nkb,d] bf16
-    vsum16: torch.Tensor    # [B,H,nkb,d] bf16
-    M: Optional[torch.Tensor]  # [B,H,nkb,d,d] bf16 (order 1)
+    kbar16: torch.Tensor    # [B,H,nkb,d] fp16
+    vsum16: torch.Tensor    # [B,H,nkb,d] fp16
+    M: Optional[torch.Tensor]  # [B,H,nkb,d,d] fp16 (order 1)
 
 
 @dataclasses.dataclass
@@ -47,14 +47,14 @@ class Problem:
 
 def allocate_tables(p: Problem, device) -> Tables:
     f32 = dict(dtype=torch.float32, device=device)
-    b16 = dict(dtype=torch.bfloat16, device=device)
+    h16 = dict(dtype=torch.float16, device=device)
     return Tables(
         qbar=torch.empty(p.B, p.H, p.nqb, p.d, **f32),
         kbar_t=torch.empty(p.B, p.H, p.d, p.nkb, **f32),
         vsum=torch.empty(p.B, p.H, p.nkb, p.d, **f32),
-        kbar16=torch.empty(p.B, p.H, p.nkb, p.d, **b16),
-        vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **b16),
-        M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **b16) if p.order == 1 else None,
+        kbar16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
+        vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
+        M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **h16) if p.order == 1 else None,
     )
 
 

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #define SA_DEVI __device__ __forceinline__
@@ -42,12 +43,28 @@ SA_DEVI void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A(16x16 f16, row) * B(16x8 f16, col) + D, fp32 accumulate.
+SA_DEVI void mma_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+SA_DEVI uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 SA_DEVI uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 SA_DEVI float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 SA_DEVI float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// Two packed bf16 -> two packed f16 (exact for magnitudes in the f16 normal range).
+SA_DEVI uint32_t bf16x2_to_f16x2(uint32_t v) { return pack_f16(bf16_lo(v), bf16_hi(v)); }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
 // `row_bytes` long (a multiple of 128). The chunk index is XOR-swizzled with the

@@ -23,6 +23,8 @@
 #include "common.cuh"
 #include "launch.h"
 
+#include <type_traits>
+
 namespace sa {
 
 namespace fwd {
@@ -228,21 +230,32 @@ forward_kernel(ForwardArgs p) {
     }
   };
 
-  // S(16 x KT) = Q K^T for this warp's rows; keys at `kb` (KT rows, swizzled).
-  auto qk = [&](uint32_t kb, float (&s)[NT_S][4]) {
+  // S(16 x KT) = Q K^T for this warp's rows; keys at `kb` (KT rows, swizzled). With
+  // HALF, the keys are the fp16 centroid table and Q is converted to fp16 (exact).
+  auto qk = [&](uint32_t kb, float (&s)[NT_S][4], auto half_tag) {
+    constexpr bool HALF = decltype(half_tag)::value;
 #pragma unroll
     for (int nt = 0; nt < NT_S; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk)
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t a[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = HALF ? bf16x2_to_f16x2(qf[kk][e]) : qf[kk][e];
 #pragma unroll
       for (int np = 0; np < NT_S / 2; ++np) {
         const int r = np * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
         const int col = kk * 16 + ((lane >> 3) & 1) * 8;
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kb + swz(r, col / 8, ROWB), b0, b1, b2, b3);
-        mma_bf16(s[2 * np], qf[kk], b0, b1);
-        mma_bf16(s[2 * np + 1], qf[kk], b2, b3);
+        if (HALF) {
+          mma_f16(s[2 * np], a, b0, b1);
+          mma_f16(s[2 * np + 1], a, b2, b3);
+        } else {
+          mma_bf16(s[2 * np], a, b0, b1);
+          mma_bf16(s[2 * np + 1], a, b2, b3);
+        }
       }
+    }
   };
 
   // Online-softmax update with masked base-2 logits already in s; turns s into P.
@@ -272,26 +285,36 @@ forward_kernel(ForwardArgs p) {
     }
   };
 
-  // O += P(16 x KT) V(KT x D); values at `vb` (KT rows, swizzled).
-  auto pv = [&](const float (&s)[NT_S][4], uint32_t vb) {
+  // O += P(16 x KT) V(KT x D); values at `vb` (KT rows, swizzled). With HALF, P and
+  // the values (the fp16 value-sum table) are fp16.
+  auto pv = [&](const float (&s)[NT_S][4], uint32_t vb, auto half_tag) {
+    constexpr bool HALF = decltype(half_tag)::value;
+    auto pk = [&](float x, float y) { return HALF ? pack_f16(x, y) : pack_bf16(x, y); };
 #pragma unroll
     for (int kk = 0; kk < KT / 16; ++kk) {
       uint32_t a[4];
-      a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      a[0] = pk(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = pk(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = pk(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = pk(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int np = 0; np < NT_O / 2; ++np) {
         const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
         const int col = np * 16 + ((lane >> 4) & 1) * 8;
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(vb + swz(r, col / 8, ROWB), b0, b1, b2, b3);
-        mma_bf16(o[2 * np], a, b0, b1);
-        mma_bf16(o[2 * np + 1], a, b2, b3);
+        if (HALF) {
+          mma_f16(o[2 * np], a, b0, b1);
+          mma_f16(o[2 * np + 1], a, b2, b3);
+        } else {
+          mma_bf16(o[2 * np], a, b0, b1);
+          mma_bf16(o[2 * np + 1], a, b2, b3);
+        }
       }
     }
   };
+  using kHalf = std::true_type;
+  using kBf16 = std::false_type;
 
   Walk wk{0, 0, -1, 0, 0};
   Item cur = walk_next<BLK, ORDER>(wk, skip, list, cnt, ntiles, nkb);
@@ -310,7 +333,7 @@ forward_kernel(ForwardArgs p) {
     if (cur.kind == kTile) {
       cur_tile = cur.a;
       float s[NT_S][4];
-      qk(sb, s);
+      qk(sb, s, kHalf{});
       float wn[NT_S][2];  // token count n_j of each column (0 where masked)
 #pragma unroll
       for (int nt = 0; nt < NT_S; ++nt)
@@ -337,7 +360,7 @@ forward_kernel(ForwardArgs p) {
               make_float2(s[nt][2], s[nt][3]);
         }
       }
-      pv(s, sb + KT * ROWB);
+      pv(s, sb + KT * ROWB, kHalf{});
     } else if (cur.kind == kMat) {
       if constexpr (ORDER == 1) {
         __syncwarp();
@@ -348,16 +371,20 @@ forward_kernel(ForwardArgs p) {
 #pragma unroll
         for (int nt = 0; nt < NT_O; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk)
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          uint32_t a[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a[e] = bf16x2_to_f16x2(qf[kk][e]);
 #pragma unroll
           for (int np = 0; np < NT_O / 2; ++np) {
             const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
             const int cc = np * 16 + ((lane >> 4) & 1) * 8;
             uint32_t b0, b1, b2, b3;
             ldsm_x4_t(sb + swz(r, cc / 8, ROWB), b0, b1, b2, b3);
-            mma_bf16(u[2 * np], qf[kk], b0, b1);
-            mma_bf16(u[2 * np + 1], qf[kk], b2, b3);
+            mma_f16(u[2 * np], a, b0, b1);
+            mma_f16(u[2 * np + 1], a, b2, b3);
           }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT_O; ++nt) {
           o[nt][0] = fmaf(a0, u[nt][0], o[nt][0]);
@@ -368,7 +395,7 @@ forward_kernel(ForwardArgs p) {
       }
     } else {
       float s[NT_S][4];
-      qk(sb, s);
+      qk(sb, s, kBf16{});
       const int tok0 = cur.a * BLK + cur.b * KT;
 #pragma unroll
       for (int nt = 0; nt < NT_S; ++nt)
@@ -384,7 +411,7 @@ forward_kernel(ForwardArgs p) {
         lrow[0] += s[nt][0] + s[nt][1];
         lrow[1] += s[nt][2] + s[nt][3];
       }
-      pv(s, sb + KT * ROWB);
+      pv(s, sb + KT * ROWB, kBf16{});
     }
     __syncthreads();
     cur = nxt;

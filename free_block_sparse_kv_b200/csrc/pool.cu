@@ -9,7 +9,7 @@
 // One CTA per block. KV CTAs stage the block's K and V tiles in shared memory
 // with 16-byte cp.async (rows past the end zero-filled), reduce the column sums,
 // and for order 1 compute K^T V on the tensor cores (mma.sync m16n8k16, fp32
-// accumulate), subtract kbar S^T in fp32, and store M as bf16 through a
+// accumulate), subtract kbar S^T in fp32, and store M as fp16 through a
 // swizzled shared-memory stage so that the global stores are 16-byte coalesced.
 // The pass is HBM-bound: it reads Q, K, V once and writes M once.
 #include "common.cuh"
@@ -117,12 +117,12 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
       const float mean = s / (float)n;
       ks[c] = mean;
       kbar_t[((size_t)bh * D + c) * nkb + j] = mean;
-      __nv_bfloat16 h = __float2bfloat16_rn(mean);
+      __half h = __float2half_rn(mean);
       kbar16[row] = *reinterpret_cast<uint16_t*>(&h);
     } else {
       vs[c] = s;
       vsum[row] = s;
-      __nv_bfloat16 h = __float2bfloat16_rn(s);
+      __half h = __float2half_rn(s);
       vsum16[row] = *reinterpret_cast<uint16_t*>(&h);
     }
   }
@@ -174,7 +174,7 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
           const int c = c0 + nt * 8 + 2 * t;
           const float x0 = acc[mt][nt][2 * hf] - ks[a] * vs[c];
           const float x1 = acc[mt][nt][2 * hf + 1] - ks[a] * vs[c + 1];
-          *reinterpret_cast<uint32_t*>(sk + swz(a, c / 8, ROWB) + (c % 8) * 2) = pack_bf16(x0, x1);
+          *reinterpret_cast<uint32_t*>(sk + swz(a, c / 8, ROWB) + (c % 8) * 2) = pack_f16(x0, x1);
         }
     __syncthreads();
     uint16_t* mg = M + ((size_t)bh * nkb + j) * D * D;

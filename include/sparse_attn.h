@@ -22,7 +22,7 @@
  * substitution; query centroids as routing proxies).
  *
  * Conventions for every entry point.
- *   - bf16 tensors are passed as pointers to their 16-bit patterns (uint16_t).
+ *   - bf16 and fp16 tensors are passed as pointers to their 16-bit patterns (uint16_t).
  *   - Tensors are dense and contiguous in the layout stated for each argument,
  *     d innermost. Every device pointer must be 16-byte aligned.
  *   - The caller allocates and owns every buffer. The library never allocates,
@@ -77,10 +77,13 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
  *   qbar    [B,H,nqb,d]  fp32   mean of each query block's rows
  *   kbar_t  [B,H,d,nkb]  fp32   block centroids, dim-major (routing reads it)
  *   vsum    [B,H,nkb,d]  fp32   value sums S_j
- *   kbar16  [B,H,nkb,d]  bf16   centroids, rounded to nearest (forward reads it)
- *   vsum16  [B,H,nkb,d]  bf16   value sums, rounded to nearest (forward reads it)
- *   M       [B,H,nkb,d,d] bf16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
+ *   kbar16  [B,H,nkb,d]  fp16   centroids, rounded to nearest (forward reads it)
+ *   vsum16  [B,H,nkb,d]  fp16   value sums, rounded to nearest (forward reads it)
+ *   M       [B,H,nkb,d,d] fp16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
  *                               a = key dim (rows), c = value dim; fp32 accumulate
+ * The three 16-bit tables are IEEE fp16 (11-bit significand): the forward runs
+ * the compensation products in fp16 with fp32 accumulation, while the exact
+ * products use the bf16 inputs.
  * Means of a partial last block use its true token count.
  */
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -86,12 +86,12 @@ def test_pool_matches_oracle(name, small_inputs):
             np.testing.assert_allclose(t.kbar_t[b, h].cpu().numpy().T, kbar, rtol=0, atol=2e-6)
             np.testing.assert_allclose(t.vsum[b, h].cpu().numpy(), vsum, rtol=0, atol=2e-5)
             k16 = t.kbar16[b, h].float().cpu().numpy()
-            np.testing.assert_allclose(k16, kbar, rtol=2 ** -8, atol=1e-6)
+            np.testing.assert_allclose(k16, kbar, rtol=2 ** -10, atol=1e-6)
             v16 = t.vsum16[b, h].float().cpu().numpy()
-            np.testing.assert_allclose(v16, vsum, rtol=2 ** -8, atol=1e-5)
+            np.testing.assert_allclose(v16, vsum, rtol=2 ** -10, atol=1e-5)
             if w.order == 1:
                 mg = t.M[b, h].float().cpu().numpy()
-                tol = 2 ** -8 * np.abs(mats) + 1e-3
+                tol = 2 ** -10 * np.abs(mats) + 1e-3
                 assert np.all(np.abs(mg - mats) <= tol), float(np.abs(mg - mats).max())
 
 
