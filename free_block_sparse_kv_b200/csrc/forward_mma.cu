@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "launch.h"
 
+#include <cstdlib>
 #include <type_traits>
 
 namespace sa {
@@ -454,13 +455,23 @@ static cudaError_t launch_forward_t(const ForwardArgs& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st) {
+cudaError_t launch_forward_mma(const ForwardArgs& p, cudaStream_t st) {
 #define SA_FWD_CASE(D_, B_, O_) \
   if (p.d == D_ && p.block == B_ && p.order == O_) return launch_forward_t<D_, B_, O_>(p, st);
   SA_FWD_CASE(64, 64, 0) SA_FWD_CASE(64, 64, 1) SA_FWD_CASE(64, 128, 0) SA_FWD_CASE(64, 128, 1)
   SA_FWD_CASE(128, 64, 0) SA_FWD_CASE(128, 64, 1) SA_FWD_CASE(128, 128, 0) SA_FWD_CASE(128, 128, 1)
 #undef SA_FWD_CASE
   return cudaErrorInvalidValue;
+}
+
+// The tcgen05 kernel is the forward; the register-tile kernel stays selectable with
+// SPARSE_ATTN_FORWARD=mma for side-by-side measurements.
+cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st) {
+  static const int use_mma = [] {
+    const char* e = getenv("SPARSE_ATTN_FORWARD");
+    return e && e[0] == 'm' ? 1 : 0;
+  }();
+  return use_mma ? launch_forward_mma(p, st) : launch_forward_tc(p, st);
 }
 
 }  // namespace sa

@@ -1,0 +1,684 @@
+// Forward pass on the 5th-generation tensor cores: tcgen05.mma with accumulators in
+// tensor memory, operands staged by TMA, one warp-specialised CTA per 128 query rows.
+//
+// Follows "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion
+// Transformers" §2: Algorithme Central (o_t = N_t / D_t; exact terms for the kept
+// blocks; alpha_{t,j} (sum_n v_{j,n}) for the others; the first-order term, here per
+// block: alpha_{t,j} * scale * q_t M_j) and Implémentation Matérielle (phase 1 exact
+// tiles in on-chip memory, phase 2 a sweep over the aggregated block vectors, phase 3
+// the first-order correction), all merged into one online softmax.
+//
+// Roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r of the tile = TMEM lane r. Reads
+//              logits from TMEM, keeps the running max (rescaling O lazily, only when
+//              the max grows by more than 2^8) and the denominator, writes P back to
+//              TMEM as the A operand of the next product, and builds the order-1
+//              operand A_j = (scale * alpha_tj) q_t in TMEM.
+//   warp 4     TMA producer: Q once, then every operand tile through a 4 x 32 KB ring.
+//   warp 5     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
+// Work items, in order (the same walk runs in all three roles):
+//   TILE t   64 centroids (fp16) and value sums (fp16): S = Q16 Kbar^T, P, O += P S
+//   MAT j    each skipped block of the current tile (order 1): O += A_j M_j (fp16)
+//   EXACT j  each kept block: S = Q K_j^T, P, O += P V_j (bf16)
+// The MMA warp issues the logits of the next TILE/EXACT item before the value
+// product of the current one, so logits overlap the softmax of the previous item.
+// TMEM columns: O [0, D), S/P buffers at 128 and 256, A buffers at 384 and 448.
+// Every mbarrier wait is bounded: on timeout the CTA sets err_flag, abandons its work,
+// drains its own TMA loads and MMAs, frees TMEM and exits.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+
+namespace sa {
+namespace tcf {
+
+constexpr int TQ = 128;        // query rows per CTA
+constexpr int KC = 64;         // centroids per TILE item
+constexpr int NU = 4;          // ring units
+constexpr int UNIT = 32768;    // bytes per ring unit
+constexpr int MAXW = 64;       // bitmap words (2048 blocks)
+constexpr int NTHREADS = 192;
+constexpr float kThresh = 8.0f;  // lazy-rescale threshold, base-2 units
+constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
+
+constexpr uint32_t COL_O = 0, COL_R0 = 128, COL_A0 = 384;
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr int OFF_Q = 0;
+constexpr int OFF_Q16 = 32768;
+constexpr int OFF_U = 65536;
+constexpr int OFF_CTL = OFF_U + NU * UNIT;
+constexpr int SMEM_BYTES = OFF_CTL + 2048 + 1024;
+
+struct Params {
+  CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmM;
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  void* out;
+  int32_t* err_flag;
+  int cap, Nq, Nk, nqb, nkb, out_dtype;
+  float scale;
+};
+
+struct Ctl {  // control block in shared memory
+  uint64_t full[NU], empty[NU];
+  uint64_t s_full[2], p_full[2], pv_done[2], s_free[2], a_full[2], a_done[2];
+  uint64_t q_full, init_done, drain;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t kept[2][MAXW];   // kept blocks of each query block in the tile (half)
+  uint32_t keptU[MAXW];     // union: EXACT items
+  uint32_t skipU[MAXW];     // union of skipped blocks: TILE / MAT items
+};
+
+enum : int { kTile = 0, kMat = 1, kExact = 2, kNone = 3 };
+struct Item {
+  int kind, j;  // TILE: j = tile index; MAT / EXACT: j = block index
+};
+
+// The walk over work items; identical in every role.
+struct Walk {
+  int phase = 0, tile = 0, j = -1;
+  template <int ORDER>
+  SA_DEVI Item next(const Ctl& c, int nkb) {
+    const int ntiles = (nkb + KC - 1) / KC;
+    while (true) {
+      if (phase == 0) {
+        if (tile >= ntiles) {
+          phase = 1;
+          j = 0;
+          continue;
+        }
+        if (j < 0) {
+          j = tile * KC;
+          if (c.skipU[2 * tile] | c.skipU[2 * tile + 1]) return Item{kTile, tile};
+          ++tile;
+          j = -1;
+          continue;
+        }
+        if (ORDER == 1) {
+          const int end = min(nkb, (tile + 1) * KC);
+          j = next_bit(c.skipU, j, end);
+          if (j < end) return Item{kMat, j++};
+        }
+        ++tile;
+        j = -1;
+        continue;
+      }
+      j = next_bit(c.keptU, j, nkb);
+      if (j < nkb) return Item{kExact, j++};
+      return Item{kNone, 0};
+    }
+  }
+  // First set bit at index >= from (and < end), else end.
+  static SA_DEVI int next_bit(const uint32_t* bits, int from, int end) {
+    while (from < end) {
+      const uint32_t w = bits[from >> 5] >> (from & 31);
+      if (w) return min(end, from + __ffs(w) - 1);
+      from = (from | 31) + 1;
+    }
+    return end;
+  }
+};
+
+// MMA-side event stream: S(next TILE/EXACT) is issued before PV(current).
+enum : int { eS = 0, ePV = 1, eMat = 2, eNone = 3 };
+struct Event {
+  int kind;   // eS, ePV, eMat, eNone
+  Item item;
+  int buf, use;
+};
+struct EventGen {
+  Walk cur, ahead;
+  int ns_ahead = 0, ns_cur = 0, nmat = 0;
+  bool started = false;
+  Event pend;
+  bool has_pend = false;
+
+  template <int ORDER>
+  SA_DEVI Item next_s(const Ctl& c, int nkb) {
+    while (true) {
+      Item it = ahead.template next<ORDER>(c, nkb);
+      if (it.kind != kMat) return it;
+    }
+  }
+  template <int ORDER>
+  SA_DEVI Event next(const Ctl& c, int nkb) {
+    if (has_pend) {
+      has_pend = false;
+      return pend;
+    }
+    if (!started) {
+      started = true;
+      Item s = next_s<ORDER>(c, nkb);
+      if (s.kind == kNone) return Event{eNone, s, 0, 0};
+      const int n = ns_ahead++;
+      return Event{eS, s, n & 1, n >> 1};
+    }
+    Item it = cur.template next<ORDER>(c, nkb);
+    if (it.kind == kNone) return Event{eNone, it, 0, 0};
+    if (it.kind == kMat) {
+      const int n = nmat++;
+      return Event{eMat, it, n & 1, n >> 1};
+    }
+    const int n = ns_cur++;
+    const Event pv{ePV, it, n & 1, n >> 1};
+    Item s = next_s<ORDER>(c, nkb);
+    if (s.kind == kNone) return pv;
+    const int m = ns_ahead++;
+    pend = pv;
+    has_pend = true;
+    return Event{eS, s, m & 1, m >> 1};
+  }
+};
+
+template <int D, int BLK>
+struct Bytes {
+  static constexpr int SUB = D / 64;                    // 64-column sub-tiles per row
+  static constexpr uint32_t KB = SUB * KC * 128;        // centroid tile
+  static constexpr uint32_t VS = SUB * KC * 128;        // value-sum tile
+  static constexpr uint32_t M = SUB * D * 128;          // one M_j
+  static constexpr uint32_t KV = SUB * BLK * 128;       // one K or V block
+  static constexpr uint32_t Q = SUB * TQ * 128;         // query tile
+};
+
+template <int D, int BLK, int ORDER>
+__global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_constant__ Params p) {
+  using By = Bytes<D, BLK>;
+  constexpr int SUB = By::SUB;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  Ctl& c = *reinterpret_cast<Ctl*>(gbase + OFF_CTL);
+  auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int bh = blockIdx.y;
+  const int q0 = blockIdx.x * TQ;
+  const int nkb = p.nkb;
+
+  // A failure reported by an earlier CTA (or call) makes the rest of the grid skip
+  // its work, so a fault costs one wave, not the whole grid.
+  if (tid == 0) c.abort = (p.err_flag && *reinterpret_cast<volatile int32_t*>(p.err_flag)) ? 1 : 0;
+  __syncthreads();
+  if (c.abort) return;
+
+  // ---- setup: barriers (producer warp), TMEM (MMA warp), kept bitmaps (softmax) ----
+  if (warp == 4 && lane == 0) {
+    for (int u = 0; u < NU; ++u) {
+      tc::mbar_init(bar(c.full[u]), 1);
+      tc::mbar_init(bar(c.empty[u]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(bar(c.s_full[b]), 1);
+      tc::mbar_init(bar(c.pv_done[b]), 1);
+      tc::mbar_init(bar(c.a_done[b]), 1);
+      tc::mbar_init(bar(c.p_full[b]), TQ);
+      tc::mbar_init(bar(c.s_free[b]), TQ);
+      tc::mbar_init(bar(c.a_full[b]), TQ);
+    }
+    tc::mbar_init(bar(c.q_full), 1);
+    tc::mbar_init(bar(c.init_done), TQ);
+    tc::mbar_init(bar(c.drain), 1);
+    tc::fence_mbar_init();
+    tc::fence_proxy_async();
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(smem_u32(&c.tmem_base), 512);
+    tc::tmem_relinquish();
+  }
+  if (warp < 4) {
+    // Kept bitmaps of the one (block 128) or two (block 64) query blocks of the tile.
+    const int nh = BLK == 128 ? 1 : 2;
+    for (int w = tid; w < 2 * MAXW; w += 128) (&c.kept[0][0])[w] = 0u;
+    __syncwarp();
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    for (int h = 0; h < nh; ++h) {
+      const int qb = q0 / BLK + h;
+      if (qb >= p.nqb) continue;
+      const size_t row = (size_t)bh * p.nqb + qb;
+      const int n = min(max(p.kv_cnt[row], 0), p.cap);
+      const int32_t* src = p.kv_idx + row * p.cap;
+      for (int x = tid; x < n; x += 128) {
+        const int j = src[x];
+        if (j >= 0 && j < nkb) atomicOr(&c.kept[h][j >> 5], 1u << (j & 31));
+      }
+    }
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    const bool has1 = BLK == 64 && (q0 / BLK + 1) < p.nqb;
+    for (int w = tid; w < MAXW; w += 128) {
+      const int lo = w * 32;
+      const uint32_t valid = lo + 32 <= nkb ? 0xffffffffu : (lo < nkb ? (1u << (nkb - lo)) - 1u : 0u);
+      const uint32_t k0 = c.kept[0][w];
+      const uint32_t k1 = BLK == 128 ? k0 : (has1 ? c.kept[1][w] : k0);
+      if (BLK == 128 || !has1) c.kept[1][w] = k0;
+      c.keptU[w] = (k0 | k1) & valid;
+      c.skipU[w] = (~k0 | ~k1) & valid;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = c.tmem_base;
+  tc::Waiter wt{&c.abort, p.err_flag, kWaitLimit};
+
+  if (warp == 4) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      tc::prefetch_tmap(&p.tmQ);
+      tc::mbar_arrive_expect_tx(bar(c.q_full), By::Q);
+      for (int s = 0; s < SUB; ++s)
+        tc::tma_load_3d(base + OFF_Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s, q0, bh);
+      EventGen gen;
+      int u = 0;
+      bool ok = true;
+      while (ok) {
+        const Event e = gen.next<ORDER>(c, nkb);
+        if (e.kind == eNone) break;
+        const int slot = u % NU;
+        if (u >= NU) ok = wt.wait(bar(c.empty[slot]), ((u / NU) - 1) & 1, 1);
+        if (!ok) break;
+        const uint32_t dst = base + OFF_U + slot * UNIT;
+        const uint32_t fb = bar(c.full[slot]);
+        const Item& it = e.item;
+        if (e.kind == eS && it.kind == kTile) {
+          tc::mbar_arrive_expect_tx(fb, By::KB);
+          for (int s = 0; s < SUB; ++s)
+            tc::tma_load_3d(dst + s * KC * 128, &p.tmKb, fb, 64 * s, it.j * KC, bh);
+        } else if (e.kind == ePV && it.kind == kTile) {
+          tc::mbar_arrive_expect_tx(fb, By::VS);
+          for (int s = 0; s < SUB; ++s)
+            tc::tma_load_3d(dst + s * KC * 128, &p.tmVs, fb, 64 * s, it.j * KC, bh);
+        } else if (e.kind == eMat) {
+          tc::mbar_arrive_expect_tx(fb, By::M);
+          for (int s = 0; s < SUB; ++s)
+            tc::tma_load_3d(dst + s * D * 128, &p.tmM, fb, 64 * s, 0, bh * nkb + it.j);
+        } else {
+          const CUtensorMap* m = e.kind == eS ? &p.tmK : &p.tmV;
+          tc::mbar_arrive_expect_tx(fb, By::KV);
+          for (int s = 0; s < SUB; ++s)
+            tc::tma_load_3d(dst + s * BLK * 128, m, fb, 64 * s, it.j * BLK, bh);
+        }
+        ++u;
+      }
+      // Drain: every load issued must land before the CTA exits.
+      tc::wait_drain(bar(c.q_full), 0, kWaitLimit);
+      for (int v = max(0, u - NU); v < u; ++v)
+        tc::wait_drain(bar(c.full[v % NU]), (v / NU) & 1, kWaitLimit);
+    }
+  } else if (warp == 5) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      constexpr uint32_t I_S_TILE = tc::idesc_f16(0, 0, 0, KC);
+      constexpr uint32_t I_PV_TILE = tc::idesc_f16(0, 0, 1, D);
+      constexpr uint32_t I_S_EX = tc::idesc_f16(1, 1, 0, BLK);
+      constexpr uint32_t I_PV_EX = tc::idesc_f16(1, 1, 1, D);
+      constexpr uint32_t I_MAT = tc::idesc_f16(0, 0, 1, D);
+      bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
+      tc::fence_after_sync();
+      EventGen gen;
+      int u = 0;
+      while (ok) {
+        const Event e = gen.next<ORDER>(c, nkb);
+        if (e.kind == eNone) break;
+        const int slot = u % NU;
+        const uint32_t src = base + OFF_U + slot * UNIT;
+        ok = wt.wait(bar(c.full[slot]), (u / NU) & 1, 4);
+        if (!ok) break;
+        const Item& it = e.item;
+        if (e.kind == eS) {
+          if (e.use >= 1) ok = wt.wait(bar(c.s_free[e.buf]), (e.use - 1) & 1, 5);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t dt = tmem + COL_R0 + 128 * e.buf;
+          const bool tile = it.kind == kTile;
+          const uint32_t qa = base + (tile ? OFF_Q16 : OFF_Q);
+          const int rows = tile ? KC : BLK;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk % 4) * 32;
+            const uint64_t ad = tc::sdesc(qa + (kk / 4) * TQ * 128 + off, 16, 1024);
+            const uint64_t bd = tc::sdesc(src + (kk / 4) * rows * 128 + off, 16, 1024);
+            tc::mma_ss(dt, ad, bd, tile ? I_S_TILE : I_S_EX, kk > 0);
+          }
+          tc::mma_commit(bar(c.s_full[e.buf]));
+        } else if (e.kind == ePV) {
+          ok = wt.wait(bar(c.p_full[e.buf]), e.use & 1, 6);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t pa = tmem + COL_R0 + 128 * e.buf;
+          const bool tile = it.kind == kTile;
+          const int rows = tile ? KC : BLK;
+          for (int kk = 0; kk < rows / 16; ++kk) {
+            const uint64_t bd = tc::sdesc(src + kk * 2048, rows * 128, 1024);
+            tc::mma_ts(tmem + COL_O, pa + kk * 8, bd, tile ? I_PV_TILE : I_PV_EX, 1);
+          }
+          tc::mma_commit(bar(c.pv_done[e.buf]));
+        } else {
+          ok = wt.wait(bar(c.a_full[e.buf]), e.use & 1, 7);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t aa = tmem + COL_A0 + 64 * e.buf;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t bd = tc::sdesc(src + kk * 2048, D * 128, 1024);
+            tc::mma_ts(tmem + COL_O, aa + kk * 8, bd, I_MAT, 1);
+          }
+          tc::mma_commit(bar(c.a_done[e.buf]));
+        }
+        tc::mma_commit(bar(c.empty[slot]));
+        ++u;
+      }
+      // Drain: wait for every MMA issued so far before TMEM is released.
+      tc::mma_commit(bar(c.drain));
+      tc::wait_drain(bar(c.drain), 0, kWaitLimit);
+    }
+  } else {
+    // =========================== softmax (rows) ===========================
+    const int r = tid;                       // query row within the tile, TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int h = BLK == 64 ? (r >> 6) : 0;  // which query block of the tile
+    const float sl2 = p.scale * kLog2e;
+    // tcgen05.ld / st are warp-collective: every decision that guards them is made
+    // uniform across the warp.
+    auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
+    bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
+    // fp16 copy of this row of Q (registers and the swizzled Q16 tile) and O = 0
+    uint32_t q16[D / 2];
+#pragma unroll
+    for (int s = 0; s < SUB; ++s)
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = s * TQ * 128 + r * 128 + ((ch ^ (r & 7)) << 4);
+        const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
+        uint4 y;
+        y.x = bf16x2_to_f16x2(x.x);
+        y.y = bf16x2_to_f16x2(x.y);
+        y.z = bf16x2_to_f16x2(x.z);
+        y.w = bf16x2_to_f16x2(x.w);
+        *reinterpret_cast<uint4*>(gbase + OFF_Q16 + off) = y;
+        q16[s * 32 + ch * 4 + 0] = y.x;
+        q16[s * 32 + ch * 4 + 1] = y.y;
+        q16[s * 32 + ch * 4 + 2] = y.z;
+        q16[s * 32 + ch * 4 + 3] = y.w;
+      }
+    tc::fence_proxy_async();
+    {
+      uint32_t z[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tc::tmem_st32(tmem + lane_off + COL_O + 32 * cc, z);
+      tc::tmem_wait_st();
+    }
+    tc::fence_before_sync();
+    tc::mbar_arrive(bar(c.init_done));
+
+    float m_ref = -INFINITY, l = 0.f;
+    // last O-writing MMA the MMA warp will issue before our next value product
+    int lw_kind = -1, lw_buf = 0, lw_use = 0;
+    auto wait_last_writer = [&](int where) {
+      if (lw_kind < 0) return true;
+      const uint32_t b = lw_kind == 0 ? bar(c.pv_done[lw_buf]) : bar(c.a_done[lw_buf]);
+      const bool r2 = uni(wt.wait(b, lw_use & 1, where));
+      tc::fence_after_sync();
+      return r2;
+    };
+
+    Walk wk;
+    int ns = 0, nmat = 0, cur_buf = 0, cur_tile = 0, prev_buf = -1;
+    while (ok) {
+      const Item it = wk.next<ORDER>(c, nkb);
+      if (it.kind == kNone) break;
+      if (it.kind == kMat) {
+        if constexpr (ORDER == 1) {
+          const int n = nmat++;
+          const int ab = n & 1, use = n >> 1;
+          if (use >= 1) ok = uni(wt.wait(bar(c.a_done[ab]), (use - 1) & 1, 10));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const int cl = it.j - cur_tile * KC;
+          const uint32_t w = tc::tmem_ld1(tmem + lane_off + COL_R0 + 128 * cur_buf + (cl >> 1));
+          tc::tmem_wait_ld();
+          const __half ph = __ushort_as_half((unsigned short)((cl & 1) ? (w >> 16) : (w & 0xFFFFu)));
+          const __half2 al = __float2half2_rn(__half2float(ph) * p.scale);
+          uint32_t a[32];
+#pragma unroll
+          for (int s = 0; s < D / 64; ++s) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              __half2 x = *reinterpret_cast<const __half2*>(&q16[32 * s + i]);
+              __half2 y = __hmul2(x, al);
+              a[i] = *reinterpret_cast<uint32_t*>(&y);
+            }
+            tc::tmem_st32(tmem + lane_off + COL_A0 + 64 * ab + 32 * s, a);
+          }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          tc::mbar_arrive(bar(c.a_full[ab]));
+          lw_kind = 1;
+          lw_buf = ab;
+          lw_use = use;
+        }
+        continue;
+      }
+      // ---- TILE or EXACT: logits in S buffer ----
+      if (prev_buf >= 0) {
+        tc::fence_before_sync();
+        tc::mbar_arrive(bar(c.s_free[prev_buf]));
+      }
+      const int n = ns++;
+      const int sb = n & 1, use = n >> 1;
+      cur_buf = sb;
+      prev_buf = sb;
+      const bool tile = it.kind == kTile;
+      if (tile) cur_tile = it.j;
+      ok = uni(wt.wait(bar(c.s_full[sb]), use & 1, 11));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t sa = tmem + lane_off + COL_R0 + 128 * sb;
+      const int ncols = tile ? KC : BLK;
+      const int col0 = tile ? it.j * KC : it.j * BLK;  // first block (tile) or token (exact)
+      // pass 1: masked row max
+      float mx = -INFINITY;
+      for (int ck = 0; ck < ncols / 32; ++ck) {
+        uint32_t v[32];
+        tc::tmem_ld32(sa + 32 * ck, v);
+        tc::tmem_wait_ld();
+        uint32_t mbits;
+        if (tile) {
+          const int j0 = col0 + 32 * ck;
+          mbits = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
+        } else {
+          const int t0 = col0 + 32 * ck;
+          mbits = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
+          if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if ((mbits >> i) & 1u) mx = fmaxf(mx, __uint_as_float(v[i]) * sl2);
+      }
+      // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
+      // reference; rows that had no reference yet just take one (O is still zero).
+      const bool grow = mx > m_ref + kThresh;
+      const bool need_o = grow && m_ref != -INFINITY;
+      const float f = need_o ? tc::ex2(m_ref - mx) : 1.f;
+      if (grow) m_ref = mx;
+      l *= f;
+      if (__any_sync(0xffffffffu, need_o)) {
+        if (!wait_last_writer(12)) {
+          ok = false;
+          break;
+        }
+        for (int ck = 0; ck < D / 32; ++ck) {
+          uint32_t v[32];
+          tc::tmem_ld32(tmem + lane_off + COL_O + 32 * ck, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+          tc::tmem_st32(tmem + lane_off + COL_O + 32 * ck, v);
+        }
+        tc::tmem_wait_st();
+      }
+      // P overwrites logits this thread has already read. The value product that read
+      // this buffer's previous P was issued before these logits, so it has finished.
+      // pass 2: P = 2^(x - m_ref), written back as 16-bit pairs
+      for (int ck = 0; ck < ncols / 32; ++ck) {
+        uint32_t v[32];
+        tc::tmem_ld32(sa + 32 * ck, v);
+        tc::tmem_wait_ld();
+        uint32_t mbits;
+        float wlast = 1.f;
+        int jlast = -1;
+        if (tile) {
+          const int j0 = col0 + 32 * ck;
+          mbits = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
+          jlast = nkb - 1 - j0;  // column of the possibly partial last block
+          wlast = (float)(p.Nk - (nkb - 1) * BLK);
+        } else {
+          const int t0 = col0 + 32 * ck;
+          mbits = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
+          if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float x0 = ((mbits >> i) & 1u) ? tc::ex2(__uint_as_float(v[i]) * sl2 - m_ref) : 0.f;
+          const float x1 =
+              ((mbits >> (i + 1)) & 1u) ? tc::ex2(__uint_as_float(v[i + 1]) * sl2 - m_ref) : 0.f;
+          if (tile) {
+            const float w0 = (i == jlast) ? wlast : (float)BLK;
+            const float w1 = (i + 1 == jlast) ? wlast : (float)BLK;
+            l += x0 * w0 + x1 * w1;
+            pk[i / 2] = pack_f16(x0, x1);
+          } else {
+            l += x0 + x1;
+            pk[i / 2] = pack_bf16(x0, x1);
+          }
+        }
+        tc::tmem_st16(sa + 16 * ck, pk);
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar(c.p_full[sb]));
+      lw_kind = 0;
+      lw_buf = sb;
+      lw_use = use;
+    }
+    // ---- epilogue: O / l ----
+    if (ok) ok = wait_last_writer(13);
+    if (ok) {
+      const bool store = q0 + r < p.Nq;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const size_t rowoff = ((size_t)bh * p.Nq + q0 + (store ? r : 0)) * D;
+      for (int ck = 0; ck < D / 32; ++ck) {
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + lane_off + COL_O + 32 * ck, v);
+        tc::tmem_wait_ld();
+        if (!store) continue;
+        if (p.out_dtype == 0) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff + 32 * ck);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            o[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                               __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
+        } else {
+          uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff + 32 * ck);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 y;
+            y.x = pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv);
+            y.y = pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv);
+            y.z = pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv);
+            y.w = pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv);
+            o[i] = y;
+          }
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 5) tc::tmem_dealloc(tmem, 512);
+}
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over a dense [d2][d1][d0] tensor of 16-bit elements, 128-byte swizzle,
+// box {64, rows, 1}; reads past the end of d1 return zeros.
+bool map3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+           uint64_t d2, uint32_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+template <int D, int BLK, int ORDER>
+static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
+  Params p;
+  const uint64_t bh = (uint64_t)a.B * a.H;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  bool ok = map3d(&p.tmQ, BF, a.q, D, a.Nq, bh, TQ) && map3d(&p.tmK, BF, a.k, D, a.Nk, bh, BLK) &&
+            map3d(&p.tmV, BF, a.v, D, a.Nk, bh, BLK) &&
+            map3d(&p.tmKb, HF, a.kbar16, D, a.nkb, bh, KC) &&
+            map3d(&p.tmVs, HF, a.vsum16, D, a.nkb, bh, KC);
+  if (ORDER == 1) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh * a.nkb, D);
+  else p.tmM = p.tmVs;
+  if (!ok) return cudaErrorInvalidValue;
+  p.kv_idx = a.kv_idx;
+  p.kv_cnt = a.kv_cnt;
+  p.out = a.out;
+  p.err_flag = a.err_flag;
+  p.cap = a.cap;
+  p.Nq = a.Nq;
+  p.Nk = a.Nk;
+  p.nqb = a.nqb;
+  p.nkb = a.nkb;
+  p.out_dtype = a.out_dtype;
+  p.scale = a.scale;
+  auto kern = forward_tc_kernel<D, BLK, ORDER>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.Nq + TQ - 1) / TQ, a.B * a.H);
+  kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace tcf
+
+cudaError_t launch_forward_tc(const ForwardArgs& p, cudaStream_t st) {
+#define SA_TC_CASE(D_, B_, O_) \
+  if (p.d == D_ && p.block == B_ && p.order == O_) return tcf::launch_t<D_, B_, O_>(p, st);
+  SA_TC_CASE(64, 64, 0) SA_TC_CASE(64, 64, 1) SA_TC_CASE(64, 128, 0) SA_TC_CASE(64, 128, 1)
+  SA_TC_CASE(128, 64, 0) SA_TC_CASE(128, 64, 1) SA_TC_CASE(128, 128, 0) SA_TC_CASE(128, 128, 1)
+#undef SA_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sa

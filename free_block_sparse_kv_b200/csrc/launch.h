@@ -42,5 +42,7 @@ cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);
 cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st);
+cudaError_t launch_forward_tc(const ForwardArgs& p, cudaStream_t st);
+cudaError_t launch_forward_mma(const ForwardArgs& p, cudaStream_t st);
 
 }  // namespace sa

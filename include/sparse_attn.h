@@ -142,9 +142,14 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
  *                     [0, nkb) are ignored; kv_cnt is clamped to [0, cap]
  *   scale             logit scale, normally 1/sqrt(d)
  *   out               [B,H,Nq,d], fp32 (SA_OUT_F32) or bf16 (SA_OUT_BF16)
- *   err_flag          optional device int32: set non-zero if a bounded device
- *                     wait gives up (the call then returns normally; the caller
- *                     reads the flag and sees SA_ERR_TIMEOUT semantics)
+ *   err_flag          optional device int32, zero on entry. A CTA whose bounded
+ *                     device wait gives up sets bits in it, drains its own copies
+ *                     and MMAs, frees its tensor memory and exits; CTAs that start
+ *                     after that find the flag set and skip their work. The call
+ *                     itself still returns SA_OK (the kernel runs asynchronously):
+ *                     a non-zero flag after the stream completes means
+ *                     SA_ERR_TIMEOUT and the output is not valid. The flag is
+ *                     sticky: clear it before the next call.
  */
 int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
