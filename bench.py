@@ -87,10 +87,12 @@ def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dic
 
 
 def pool_bytes(w: W.Workload, with_q: bool) -> float:
-    """Algorithmic HBM bytes of one pool launch: read K, V (and Q), write the tables."""
+    """Algorithmic HBM bytes of one pool launch: read K, V (and Q), write the tables
+    and the fp16 copy of V."""
     bh = w.B * w.H
     rd = bh * w.Nk * w.d * 2 * 2 + (bh * w.Nq * w.d * 2 if with_q else 0)
     wr = bh * w.nkb * w.d * (4 + 4 + 2 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
+    wr += bh * w.Nk * w.d * 2   # fp16 copy of V
     if w.order == 1:
         wr += bh * w.nkb * w.d * w.d * 2
     return float(rd + wr)
@@ -300,6 +302,7 @@ def main():
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
+    op.check()
     ms_step = start.elapsed_time(end) / args.steps
     ms_step_max = max_over_ranks(ms_step)
     stage_ms = [float(np.mean([e[s].elapsed_time(e[s + 1]) for e in evs])) for s in range(3)]

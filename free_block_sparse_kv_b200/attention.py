@@ -24,6 +24,7 @@ class Tables:
     kbar16: torch.Tensor    # [B,H,nkb,d] fp16
     vsum16: torch.Tensor    # [B,H,nkb,d] fp16
     M: Optional[torch.Tensor]  # [B,H,nkb,d,d] fp16 (order 1)
+    v16: torch.Tensor       # [B,H,Nk,d] fp16 copy of V
 
 
 @dataclasses.dataclass
@@ -55,6 +56,7 @@ def allocate_tables(p: Problem, device) -> Tables:
         kbar16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
         vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
         M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **h16) if p.order == 1 else None,
+        v16=torch.empty(p.B, p.H, p.Nk, p.d, **h16),
     )
 
 
@@ -71,7 +73,7 @@ def _check_inputs(q, k, v):
 
 def pool(q, k, v, p: Problem, t: Tables, stream=None):
     C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar, t.kbar_t,
-                       t.vsum, t.kbar16, t.vsum16, t.M, stream)
+                       t.vsum, t.kbar16, t.vsum16, t.M, t.v16, stream)
 
 
 def route(p: Problem, t: Tables, kv_idx, kv_cnt, mode: str, rho=(1, 4), tau=0.9, scale=None,
@@ -93,7 +95,7 @@ def forward(q, k, v, p: Problem, t: Tables, kv_idx, kv_cnt, out, scale=None, err
             stream=None):
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
     dt = C.SA_OUT_F32 if out.dtype == torch.float32 else C.SA_OUT_BF16
-    C.sparse_attn_forward(q, k, v, t.kbar16, t.vsum16, t.M, kv_idx, kv_cnt, kv_idx.shape[-1],
+    C.sparse_attn_forward(q, k, t.v16, t.kbar16, t.vsum16, t.M, kv_idx, kv_cnt, kv_idx.shape[-1],
                           p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, scale, out, dt, err_flag,
                           stream)
 
@@ -117,6 +119,7 @@ class BlockSparseAttention:
         self.tables = allocate_tables(p, device)
         self.kv_idx, self.kv_cnt = allocate_lists(p, cap, device)
         self.out = torch.empty(p.B, p.H, p.Nq, p.d, dtype=out_dtype, device=device)
+        self.err_flag = torch.zeros(1, dtype=torch.int32, device=device)
 
     def __call__(self, q, k, v, step: int = 0, stream=None) -> torch.Tensor:
         _check_inputs(q, k, v)
@@ -130,5 +133,12 @@ class BlockSparseAttention:
         else:
             route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
                   stream=stream)
-        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out, stream=stream)
+        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out,
+                err_flag=self.err_flag, stream=stream)
         return self.out
+
+    def check(self):
+        """Raise if a bounded device wait of an earlier call gave up (synchronises)."""
+        flag = int(self.err_flag.item())
+        if flag:
+            raise C.SparseAttnError(C.SA_ERR_TIMEOUT, f"device wait timed out (flag {flag:#x})")

@@ -76,7 +76,7 @@ extern "C" {
 const char* sparse_attn_last_error(void) { return g_last_error.c_str(); }
 
 int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
-                            size_t sizes[6]) {
+                            size_t sizes[7]) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
   SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
   SA_REQUIRE(sizes != nullptr, "sizes must not be NULL");
@@ -87,12 +87,14 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
   sizes[3] = bh * nkb * d * 2;
   sizes[4] = bh * nkb * d * 2;
   sizes[5] = order == 1 ? bh * nkb * d * d * 2 : 0;
+  sizes[6] = bh * (size_t)Nk * d * 2;
   return ok();
 }
 
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Nq,
                      int Nk, int d, int block, int order, float* qbar, float* kbar_t, float* vsum,
-                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, void* stream) {
+                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
+                     void* stream) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
   SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
   const bool do_q = q != nullptr && Nq > 0;
@@ -104,6 +106,7 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
     SA_REQUIRE_PTR(vsum);
     SA_REQUIRE_PTR(kbar16);
     SA_REQUIRE_PTR(vsum16);
+    SA_REQUIRE_PTR(v16);
     if (order == 1) SA_REQUIRE_PTR(M);
   }
   if (do_q) {
@@ -112,7 +115,7 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
   }
   if (int rc = check_device()) return rc;
   sa::PoolArgs p{do_q ? q : nullptr, k, v, B, H, Nq, Nk, d, block, order,
-                 cdiv(Nq, block), cdiv(Nk, block), qbar, kbar_t, vsum, kbar16, vsum16, M};
+                 cdiv(Nq, block), cdiv(Nk, block), qbar, kbar_t, vsum, kbar16, vsum16, M, v16};
   return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
 }
 
@@ -172,7 +175,7 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block, int fra
   return launched(sa::launch_structured_mask(p, static_cast<cudaStream_t>(stream)), "mask launch");
 }
 
-int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
                         const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H, int Nq,
                         int Nk, int d, int block, int order, float scale, void* out, int out_dtype,
@@ -188,7 +191,7 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   SA_REQUIRE(cap >= 0, "cap must be >= 0");
   SA_REQUIRE_PTR(q);
   SA_REQUIRE_PTR(k);
-  SA_REQUIRE_PTR(v);
+  SA_REQUIRE_PTR(v16);
   SA_REQUIRE_PTR(kbar16);
   SA_REQUIRE_PTR(vsum16);
   if (order == 1) SA_REQUIRE_PTR(M);
@@ -197,7 +200,7 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   SA_REQUIRE_PTR(out);
   if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
   if (int rc = check_device()) return rc;
-  sa::ForwardArgs p{q, k, v, kbar16, vsum16, order == 1 ? M : nullptr, kv_idx, kv_cnt, cap,
+  sa::ForwardArgs p{q, k, v16, kbar16, vsum16, order == 1 ? M : nullptr, kv_idx, kv_cnt, cap,
                     B, H, Nq, Nk, d, block, order, cdiv(Nq, block), nkb, scale, out, out_dtype,
                     err_flag};
   return launched(sa::launch_forward(p, static_cast<cudaStream_t>(stream)), "forward launch");

@@ -19,7 +19,7 @@
 // Work items, in order (the same walk runs in all three roles):
 //   TILE t   64 centroids (fp16) and value sums (fp16): S = Q16 Kbar^T, P, O += P S
 //   MAT j    each skipped block of the current tile (order 1): O += A_j M_j (fp16)
-//   EXACT j  each kept block: S = Q K_j^T, P, O += P V_j (bf16)
+//   EXACT j  each kept block: S = Q K_j^T (bf16), P, O += P V_j (fp16 P and V)
 // The MMA warp issues the logits of the next TILE/EXACT item before the value
 // product of the current one, so logits overlap the softmax of the previous item.
 // TMEM columns: O [0, D), S/P buffers at 128 and 256, A buffers at 384 and 448.
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       constexpr uint32_t I_S_TILE = tc::idesc_f16(0, 0, 0, KC);
       constexpr uint32_t I_PV_TILE = tc::idesc_f16(0, 0, 1, D);
       constexpr uint32_t I_S_EX = tc::idesc_f16(1, 1, 0, BLK);
-      constexpr uint32_t I_PV_EX = tc::idesc_f16(1, 1, 1, D);
+      constexpr uint32_t I_PV_EX = tc::idesc_f16(0, 0, 1, D);
       constexpr uint32_t I_MAT = tc::idesc_f16(0, 0, 1, D);
       bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
       tc::fence_after_sync();
@@ -553,11 +553,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
             const float w0 = (i == jlast) ? wlast : (float)BLK;
             const float w1 = (i + 1 == jlast) ? wlast : (float)BLK;
             l += x0 * w0 + x1 * w1;
-            pk[i / 2] = pack_f16(x0, x1);
           } else {
             l += x0 + x1;
-            pk[i / 2] = pack_bf16(x0, x1);
           }
+          pk[i / 2] = pack_f16(x0, x1);
         }
         tc::tmem_st16(sa + 16 * ck, pk);
       }
@@ -645,7 +644,7 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   const uint64_t bh = (uint64_t)a.B * a.H;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   bool ok = map3d(&p.tmQ, BF, a.q, D, a.Nq, bh, TQ) && map3d(&p.tmK, BF, a.k, D, a.Nk, bh, BLK) &&
-            map3d(&p.tmV, BF, a.v, D, a.Nk, bh, BLK) &&
+            map3d(&p.tmV, HF, a.v, D, a.Nk, bh, BLK) &&
             map3d(&p.tmKb, HF, a.kbar16, D, a.nkb, bh, KC) &&
             map3d(&p.tmVs, HF, a.vsum16, D, a.nkb, bh, KC);
   if (ORDER == 1) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh * a.nkb, D);
@@ -672,7 +671,7 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
 
 }  // namespace tcf
 
-cudaError_t launch_forward_tc(const ForwardArgs& p, cudaStream_t st) {
+cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st) {
 #define SA_TC_CASE(D_, B_, O_) \
   if (p.d == D_ && p.block == B_ && p.order == O_) return tcf::launch_t<D_, B_, O_>(p, st);
   SA_TC_CASE(64, 64, 0) SA_TC_CASE(64, 64, 1) SA_TC_CASE(64, 128, 0) SA_TC_CASE(64, 128, 1)

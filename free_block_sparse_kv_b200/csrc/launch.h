@@ -10,7 +10,7 @@ struct PoolArgs {
   const uint16_t *q, *k, *v;
   int B, H, Nq, Nk, d, block, order, nqb, nkb;
   float *qbar, *kbar_t, *vsum;
-  uint16_t *kbar16, *vsum16, *M;
+  uint16_t *kbar16, *vsum16, *M, *v16;
 };
 
 struct RouteArgs {
@@ -42,7 +42,5 @@ cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);
 cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st);
-cudaError_t launch_forward_tc(const ForwardArgs& p, cudaStream_t st);
-cudaError_t launch_forward_mma(const ForwardArgs& p, cudaStream_t st);
 
 }  // namespace sa

@@ -11,7 +11,8 @@
 // and for order 1 compute K^T V on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate), subtract kbar S^T in fp32, and store M as fp16 through a
 // swizzled shared-memory stage so that the global stores are 16-byte coalesced.
-// The pass is HBM-bound: it reads Q, K, V once and writes M once.
+// It also writes an fp16 copy of V, the value operand of the forward's exact
+// products. The pass is HBM-bound: it reads Q, K, V once and writes M and V16 once.
 #include "common.cuh"
 #include "launch.h"
 
@@ -25,7 +26,7 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
             const uint16_t* __restrict__ v, int Nq, int Nk, int nqb, int nkb,
             float* __restrict__ qbar, float* __restrict__ kbar_t, float* __restrict__ vsum,
             uint16_t* __restrict__ kbar16, uint16_t* __restrict__ vsum16,
-            uint16_t* __restrict__ M) {
+            uint16_t* __restrict__ M, uint16_t* __restrict__ v16) {
   constexpr int ROWB = D * 2;             // bytes per bf16 row
   constexpr int CPR = D / 8;              // 16-byte chunks per row
   constexpr int RPP = kPoolThreads / CPR; // rows covered per pass
@@ -88,10 +89,14 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
 
   {
     float ak[8] = {0, 0, 0, 0, 0, 0, 0, 0}, av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint16_t* v16g = v16 + ((size_t)bh * Nk + start) * D;
     for (int r = r0; r < n; r += RPP) {
       const uint4 xk = *reinterpret_cast<const uint4*>(sk + swz(r, ch, ROWB));
       const uint4 xv = *reinterpret_cast<const uint4*>(sv + swz(r, ch, ROWB));
       const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
+      *reinterpret_cast<uint4*>(v16g + (size_t)r * D + ch * 8) =
+          make_uint4(bf16x2_to_f16x2(xv.x), bf16x2_to_f16x2(xv.y), bf16x2_to_f16x2(xv.z),
+                     bf16x2_to_f16x2(xv.w));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         ak[2 * e] += bf16_lo(wk[e]);
@@ -195,7 +200,7 @@ static cudaError_t launch_pool_t(const PoolArgs& p, cudaStream_t st) {
   const int nq_blocks = p.q ? p.nqb : 0;
   dim3 grid(p.nkb + nq_blocks, p.B * p.H);
   kern<<<grid, kPoolThreads, smem, st>>>(p.q, p.k, p.v, p.Nq, p.Nk, p.nqb, p.nkb, p.qbar,
-                                         p.kbar_t, p.vsum, p.kbar16, p.vsum16, p.M);
+                                         p.kbar_t, p.vsum, p.kbar16, p.vsum16, p.M, p.v16);
   return cudaGetLastError();
 }
 

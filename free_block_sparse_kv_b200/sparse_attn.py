@@ -45,7 +45,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_last_error.restype = ctypes.c_char_p
     lib.sparse_attn_last_error.argtypes = []
     lib.sparse_attn_table_sizes.argtypes = [_I] * 7 + [ctypes.POINTER(ctypes.c_size_t)]
-    lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 6 + [_P]
+    lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 7 + [_P]
     lib.sparse_attn_route.argtypes = [_P, _P] + [_I] * 8 + [_F, _F, _P, _P, _I, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
@@ -78,17 +78,17 @@ def _check(rc: int):
 
 
 def sparse_attn_table_sizes(B, H, Nq, Nk, d, block, order):
-    """Byte sizes (qbar, kbar_t, vsum, kbar16, vsum16, M) of the pooled tables."""
-    out = (ctypes.c_size_t * 6)()
+    """Byte sizes (qbar, kbar_t, vsum, kbar16, vsum16, M, v16) of the pooled tables."""
+    out = (ctypes.c_size_t * 7)()
     _check(load_library().sparse_attn_table_sizes(B, H, Nq, Nk, d, block, order, out))
     return tuple(int(x) for x in out)
 
 
 def sparse_attn_pool(q, k, v, B, H, Nq, Nk, d, block, order, qbar, kbar_t, vsum, kbar16, vsum16, M,
-                     stream=None):
+                     v16, stream=None):
     _check(load_library().sparse_attn_pool(
         _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, block, order, _ptr(qbar), _ptr(kbar_t),
-        _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _stream(stream)))
+        _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _stream(stream)))
 
 
 def sparse_attn_route(qbar, kbar_t, B, H, nqb, nkb, d, mode, rho_num, rho_den, tau, scale, kv_idx,
@@ -105,10 +105,10 @@ def sparse_attn_structured_mask(B, H, Nq, Nk, block, frame_tokens, n_frames, win
         _ptr(kv_idx), _ptr(kv_cnt), cap, _stream(stream)))
 
 
-def sparse_attn_forward(q, k, v, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H, Nq, Nk, d, block,
+def sparse_attn_forward(q, k, v16, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H, Nq, Nk, d, block,
                         order, scale, out, out_dtype, err_flag=None, stream=None):
     _check(load_library().sparse_attn_forward(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(kv_idx),
+        _ptr(q), _ptr(k), _ptr(v16), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(kv_idx),
         _ptr(kv_cnt), cap, B, H, Nq, Nk, d, block, order, scale, _ptr(out), out_dtype,
         _ptr(err_flag), _stream(stream)))
 

@@ -60,12 +60,12 @@ enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
 #define SA_MAX_KV_BLOCKS 2048
 
 /*
- * Byte sizes of the pooled tables for a problem, written to sizes[0..5] in the
- * order qbar, kbar_t, vsum, kbar16, vsum16, M (M is 0 when order == 0).
+ * Byte sizes of the pooled tables for a problem, written to sizes[0..6] in the
+ * order qbar, kbar_t, vsum, kbar16, vsum16, M (0 when order == 0), v16.
  * nqb = ceil(Nq / block), nkb = ceil(Nk / block).
  */
 int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
-                            size_t sizes[6]);
+                            size_t sizes[7]);
 
 /*
  * Pooling (PISA §2 Implémentation Matérielle, pre-computation step; the per-block
@@ -81,15 +81,18 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
  *   vsum16  [B,H,nkb,d]  fp16   value sums, rounded to nearest (forward reads it)
  *   M       [B,H,nkb,d,d] fp16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
  *                               a = key dim (rows), c = value dim; fp32 accumulate
- * The three 16-bit tables are IEEE fp16 (11-bit significand): the forward runs
- * the compensation products in fp16 with fp32 accumulation, while the exact
- * products use the bf16 inputs.
+ *   v16     [B,H,Nk,d]   fp16   V converted to fp16 (exact for |v| in the fp16
+ *                               normal range; |v| must stay below 65504)
+ * The 16-bit tables are IEEE fp16 (11-bit significand): the forward runs every
+ * product that involves probabilities in fp16 with fp32 accumulation; the
+ * logits of kept tokens use the bf16 Q and K as given.
  * Means of a partial last block use its true token count.
  */
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int B, int H, int Nq, int Nk, int d, int block, int order,
                      float* qbar, float* kbar_t, float* vsum,
-                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, void* stream);
+                     uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
+                     void* stream);
 
 /*
  * Routing (PISA §2 top-k choice of the critical blocks; SVG-EAR §2 B pooled
@@ -135,8 +138,8 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
  *   N_t = sum_r e^(l_r - m) v_r + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j)
  *   D_t = sum_r e^(l_r - m)     + sum_j e^(c_j - m) n_j
  *   o_t = N_t / D_t
- *   q, k, v           as for the pool
- *   kbar16, vsum16, M as written by the pool (M NULL when order == 0)
+ *   q, k              [B,H,Nq,d] / [B,H,Nk,d] bf16, as for the pool
+ *   v16, kbar16, vsum16, M  as written by the pool (M NULL when order == 0)
  *   kv_idx, kv_cnt    as written by routing or the structured mask: indices of
  *                     each row must be distinct and < nkb; entries outside
  *                     [0, nkb) are ignored; kv_cnt is clamped to [0, cap]
@@ -151,7 +154,7 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
  *                     SA_ERR_TIMEOUT and the output is not valid. The flag is
  *                     sticky: clear it before the next call.
  */
-int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
                         const int32_t* kv_idx, const int32_t* kv_cnt, int cap,
                         int B, int H, int Nq, int Nk, int d, int block, int order,

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 def test_table_sizes():
     assert C.sparse_attn_table_sizes(1, 40, 75600, 75600, 128, 128, 1) == (
         40 * 591 * 128 * 4, 40 * 591 * 128 * 4, 40 * 591 * 128 * 4,
-        40 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2)
+        40 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2, 40 * 75600 * 128 * 2)
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[5] == 0
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[0] == 4 * 16 * 25 * 128 * 4
 
@@ -51,9 +51,10 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 96, 64, 0),
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 64, 32, 0),
         lambda: C.sparse_attn_table_sizes(-1, 1, 64, 64, 64, 64, 0),
-        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, p, 0),
-        lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, 0),
-        lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, p, p, 0),
+        lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
+        lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, None, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 3000, 64, 0, 1, 4, 0.9, 0.1, p, p, 750, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 0, 3, 2, 0.9, 0.1, p, p, 10, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 1, 1, 4, 1.5, 0.1, p, p, 10, 0),

@@ -36,6 +36,7 @@ def _run(w, q, k, v, step=0, out_dtype=torch.float32):
                                 out_dtype=out_dtype)
     out = op(q, k, v, step=step)
     torch.cuda.synchronize()
+    op.check()
     return op, out
 
 
@@ -89,6 +90,8 @@ def test_pool_matches_oracle(name, small_inputs):
             np.testing.assert_allclose(k16, kbar, rtol=2 ** -10, atol=1e-6)
             v16 = t.vsum16[b, h].float().cpu().numpy()
             np.testing.assert_allclose(v16, vsum, rtol=2 ** -10, atol=1e-5)
+            v16 = t.v16[b, h].float().cpu().numpy()
+            assert np.array_equal(v16, v), "fp16 copy of V must be exact"
             if w.order == 1:
                 mg = t.M[b, h].float().cpu().numpy()
                 tol = 2 ** -10 * np.abs(mats) + 1e-3
@@ -276,8 +279,8 @@ def test_nothing_kept_and_bad_list_entries(order):
     idx = torch.zeros(B, H, p.nqb, 1, dtype=torch.int32, device="cuda")
     cnt = torch.zeros(B, H, p.nqb, dtype=torch.int32, device="cuda")
     out = torch.empty(B, H, N, d, device="cuda")
-    C.sparse_attn_forward(q_d, k_d, v_d, t.kbar16, t.vsum16, t.M, idx, cnt, 0, B, H, N, N, d, block,
-                          order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
+    C.sparse_attn_forward(q_d, k_d, t.v16, t.kbar16, t.vsum16, t.M, idx, cnt, 0, B, H, N, N, d,
+                          block, order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
     torch.cuda.synchronize()
     want = O.forward_head(q, k, v, [np.zeros(0, int)] * p.nqb, block, order, 1 / np.sqrt(d))
     mx, mr = err_stats(out[0, 0].cpu().numpy(), want)
@@ -289,8 +292,8 @@ def test_nothing_kept_and_bad_list_entries(order):
         raw[0, 0, i, :3] = [r[0], p.nkb + 2, r[1]]
     idx = torch.from_numpy(raw).cuda()
     cnt = torch.full((B, H, p.nqb), 9, dtype=torch.int32, device="cuda")
-    C.sparse_attn_forward(q_d, k_d, v_d, t.kbar16, t.vsum16, t.M, idx, cnt, 4, B, H, N, N, d, block,
-                          order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
+    C.sparse_attn_forward(q_d, k_d, t.v16, t.kbar16, t.vsum16, t.M, idx, cnt, 4, B, H, N, N, d,
+                          block, order, 1 / np.sqrt(d), out, C.SA_OUT_F32)
     torch.cuda.synchronize()
     want = O.forward_head(q, k, v, [np.array(sorted(r)) for r in lists], block, order, 1 / np.sqrt(d))
     mx, mr = err_stats(out[0, 0].cpu().numpy(), want)
@@ -301,7 +304,7 @@ def test_empty_problems_are_no_ops():
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     f = torch.zeros(16, dtype=torch.float32, device="cuda")
     i = torch.zeros(16, dtype=torch.int32, device="cuda")
-    C.sparse_attn_pool(x, x, x, 0, 4, 100, 100, 128, 128, 1, f, f, f, x, x, x)
+    C.sparse_attn_pool(x, x, x, 0, 4, 100, 100, 128, 128, 1, f, f, f, x, x, x, x)
     C.sparse_attn_route(f, f, 1, 1, 0, 10, 128, 0, 1, 4, 0.9, 0.1, i, i, 3)
     C.sparse_attn_structured_mask(1, 1, 0, 100, 64, 10, 10, 1, 1, 1, 0, 0, i, i, 2)
     C.sparse_attn_forward(x, x, x, x, x, x, i, i, 1, 1, 1, 0, 100, 128, 128, 1, 0.1, f, 0)
@@ -327,7 +330,7 @@ def test_invalid_arguments_raise():
         C.sparse_attn_route(f, f, 1, 1, 4, 10, 64, 1, 1, 2, 0.9, 0.1, i, i, 9)
     assert e.value.code == C.SA_ERR_INVALID
     with pytest.raises(C.SparseAttnError):        # order 1 without M
-        C.sparse_attn_pool(x, x, x, 1, 1, 64, 64, 64, 64, 1, f, f, f, x, x, None)
+        C.sparse_attn_pool(x, x, x, 1, 1, 64, 64, 64, 64, 1, f, f, f, x, x, None, x)
 
 
 def test_repeat_calls_are_bitwise_deterministic(small_inputs):
