@@ -91,7 +91,8 @@ def test_pool_matches_oracle(name, small_inputs):
             v16 = t.vsum16[b, h].float().cpu().numpy()
             np.testing.assert_allclose(v16, vsum, rtol=2 ** -10, atol=1e-5)
             v16 = t.v16[b, h].float().cpu().numpy()
-            assert np.array_equal(v16, v), "fp16 copy of V must be exact"
+            # fp16 rounding of V (round to nearest even; exact except for subnormals)
+            assert np.array_equal(v16, v.astype(np.float16).astype(np.float32))
             if w.order == 1:
                 mg = t.M[b, h].float().cpu().numpy()
                 tol = 2 ** -10 * np.abs(mats) + 1e-3
