@@ -8,24 +8,32 @@
 // tiles in on-chip memory, phase 2 a sweep over the aggregated block vectors, phase 3
 // the first-order correction), all merged into one online softmax.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r of the tile = TMEM lane r. Reads
-//              logits from TMEM, keeps the running max (rescaling O lazily, only when
-//              the max grows by more than 2^8) and the denominator, writes P back to
-//              TMEM as the A operand of the next product, and builds the order-1
-//              operand A_j = (scale * alpha_tj) q_t in TMEM.
-//   warp 4     TMA producer: Q once, then every operand tile through a 4 x 32 KB ring.
-//   warp 5     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
+// Roles (384 threads):
+//   warps 0-7  softmax. Warps w and w+4 share TMEM lanes 32*(w%4).. (query rows) and
+//              split each row's columns in halves; they exchange row maxima and row
+//              sums through shared memory. They read logits from TMEM, keep the running
+//              max (rescaling O lazily, only when a row's max grows by more than 2^8),
+//              write P back to TMEM as the A operand of the value product, and build the
+//              order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
+//   warp 8     TMA producer: Q once, then every operand tile through a 4 x 32 KB ring.
+//   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
+//   warps 10-11 idle (they complete the control warpgroup for the register split).
 // Work items, in order (the same walk runs in all three roles):
 //   TILE t   64 centroids (fp16) and value sums (fp16): S = Q16 Kbar^T, P, O += P S
 //   MAT j    each skipped block of the current tile (order 1): O += A_j M_j (fp16)
 //   EXACT j  each kept block: S = Q K_j^T (bf16), P, O += P V_j (fp16 P and V)
 // The MMA warp issues the logits of the next TILE/EXACT item before the value
 // product of the current one, so logits overlap the softmax of the previous item.
-// TMEM columns: O [0, D), S/P buffers at 128 and 256, A buffers at 384 and 448.
+// TMEM columns: O [0, D); S/P buffers R0 = [128, 256), R1 = [256, 384); A slots 0, 1
+// at 384 and 448. During a tile's MAT items the tile's S/P buffer is free once its
+// value product has run (the tile's P is also kept in shared memory for alpha), and
+// it holds A slots 2 and 3: four A operands in flight hide the hand-off latency
+// between the softmax warps and the MMA thread.
 // Every mbarrier wait is bounded: on timeout the CTA sets err_flag, abandons its work,
 // drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -39,18 +47,26 @@ constexpr int KC = 64;         // centroids per TILE item
 constexpr int NU = 4;          // ring units
 constexpr int UNIT = 32768;    // bytes per ring unit
 constexpr int MAXW = 64;       // bitmap words (2048 blocks)
-constexpr int NTHREADS = 192;
+constexpr int NSOFT = 256;     // softmax threads (8 warps, 2 warpgroups)
+constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA, 2 idle)
+// Register split after launch (168 per thread at launch = 64,512 per CTA): the
+// control warpgroup gives registers back, the softmax warpgroups take them.
+constexpr int kRegCtl = 72, kRegSoft = 208;
+static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
+constexpr int NA = 4;          // A-operand slots for the order-1 products
 constexpr float kThresh = 8.0f;  // lazy-rescale threshold, base-2 units
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
 constexpr uint32_t COL_O = 0, COL_R0 = 128, COL_A0 = 384;
 
 // shared-memory map (offsets from a 1024-aligned base)
-constexpr int OFF_Q = 0;
-constexpr int OFF_Q16 = 32768;
-constexpr int OFF_U = 65536;
-constexpr int OFF_CTL = OFF_U + NU * UNIT;
-constexpr int SMEM_BYTES = OFF_CTL + 2048 + 1024;
+constexpr int OFF_Q = 0;                       // Q tile, bf16, swizzled (32 KB)
+constexpr int OFF_Q16 = 32768;                 // Q tile, fp16, swizzled (32 KB)
+constexpr int OFF_U = 65536;                   // ring
+constexpr int OFF_CTL = OFF_U + NU * UNIT;     // control block (2 KB)
+constexpr int OFF_STASH = OFF_CTL + 2048;      // P of the current tile, fp16 [KC][TQ]
+constexpr int OFF_RED = OFF_STASH + KC * TQ * 2;  // row max (2 x 2 x TQ) and sum (2 x TQ), f32
+constexpr int SMEM_BYTES = OFF_RED + 6 * TQ * 4 + 1024;
 
 struct Params {
   CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmM;
@@ -64,14 +80,17 @@ struct Params {
 
 struct Ctl {  // control block in shared memory
   uint64_t full[NU], empty[NU];
-  uint64_t s_full[2], p_full[2], pv_done[2], s_free[2], a_full[2], a_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2], s_free[2];
+  uint64_t a_full[NA], a_done[NA];
   uint64_t q_full, init_done, drain;
+  uint64_t pair[4];         // the two softmax warps sharing 32 rows
   uint32_t tmem_base;
   int abort;
   uint32_t kept[2][MAXW];   // kept blocks of each query block in the tile (half)
   uint32_t keptU[MAXW];     // union: EXACT items
   uint32_t skipU[MAXW];     // union of skipped blocks: TILE / MAT items
 };
+static_assert(sizeof(Ctl) <= 2048, "control block");
 
 enum : int { kTile = 0, kMat = 1, kExact = 2, kNone = 3 };
 struct Item {
@@ -128,11 +147,12 @@ enum : int { eS = 0, ePV = 1, eMat = 2, eNone = 3 };
 struct Event {
   int kind;   // eS, ePV, eMat, eNone
   Item item;
-  int buf, use;
+  int buf, use;   // S / PV: S-buffer and its use count; MAT: A slot and its use count
+  int tbuf;       // MAT: S-buffer of the tile the block belongs to
 };
 struct EventGen {
   Walk cur, ahead;
-  int ns_ahead = 0, ns_cur = 0, nmat = 0;
+  int ns_ahead = 0, ns_cur = 0, nmat = 0, tile_buf = 0;
   bool started = false;
   Event pend;
   bool has_pend = false;
@@ -153,26 +173,32 @@ struct EventGen {
     if (!started) {
       started = true;
       Item s = next_s<ORDER>(c, nkb);
-      if (s.kind == kNone) return Event{eNone, s, 0, 0};
+      if (s.kind == kNone) return Event{eNone, s, 0, 0, 0};
       const int n = ns_ahead++;
-      return Event{eS, s, n & 1, n >> 1};
+      return Event{eS, s, n & 1, n >> 1, 0};
     }
     Item it = cur.template next<ORDER>(c, nkb);
-    if (it.kind == kNone) return Event{eNone, it, 0, 0};
+    if (it.kind == kNone) return Event{eNone, it, 0, 0, 0};
     if (it.kind == kMat) {
       const int n = nmat++;
-      return Event{eMat, it, n & 1, n >> 1};
+      return Event{eMat, it, n % NA, n / NA, tile_buf};
     }
     const int n = ns_cur++;
-    const Event pv{ePV, it, n & 1, n >> 1};
+    if (it.kind == kTile) tile_buf = n & 1;
+    const Event pv{ePV, it, n & 1, n >> 1, 0};
     Item s = next_s<ORDER>(c, nkb);
     if (s.kind == kNone) return pv;
     const int m = ns_ahead++;
     pend = pv;
     has_pend = true;
-    return Event{eS, s, m & 1, m >> 1};
+    return Event{eS, s, m & 1, m >> 1, 0};
   }
 };
+
+// TMEM column of A slot `slot` for a tile whose S/P buffer is `tbuf`.
+SA_DEVI uint32_t a_col(int slot, int tbuf) {
+  return slot < 2 ? COL_A0 + 64 * slot : COL_R0 + 128 * tbuf + 64 * (slot - 2);
+}
 
 template <int D, int BLK>
 struct Bytes {
@@ -183,6 +209,267 @@ struct Bytes {
   static constexpr uint32_t KV = SUB * BLK * 128;       // one K or V block
   static constexpr uint32_t Q = SUB * TQ * 128;         // query tile
 };
+
+// TMEM store of W consecutive 32-bit columns (W = 16 or 32).
+template <int W>
+SA_DEVI void tmem_st_w(uint32_t taddr, const uint32_t* r) {
+  if constexpr (W == 32) {
+    tc::tmem_st32(taddr, r);
+  } else {
+    static_assert(W == 16, "width");
+    tc::tmem_st16(taddr, r);
+  }
+}
+
+// Softmax warps. Thread (warp w, lane l) owns query row r = 32*(w%4) + l and the
+// column half w/4 of every logit tile; the two threads of a row meet through an
+// mbarrier of their warp pair (bounded waits, so an abort never strands a partner).
+template <int D, int BLK, int ORDER>
+SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem, tc::Waiter& wt,
+                          int warp, int lane) {
+  constexpr int SUB = D / 64;
+  constexpr int DH = D / 2;  // O columns per thread
+  constexpr int AW = D / 4;  // A-operand columns (fp16 pairs) per thread
+  const int qw = warp & 3, ch = warp >> 2;
+  const int r = 32 * qw + lane;
+  const uint32_t lane_off = (uint32_t)(32 * qw) << 16;
+  const int h = BLK == 64 ? (r >> 6) : 0;  // which query block of the tile
+  const float sl2 = p.scale * kLog2e;
+  const int nkb = p.nkb;
+  const int bh = blockIdx.y, q0 = blockIdx.x * TQ;
+  auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
+  auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
+  float* red = reinterpret_cast<float*>(gbase + OFF_RED);       // max [2][2][TQ], sum [2][TQ]
+  __half* stash = reinterpret_cast<__half*>(gbase + OFF_STASH);  // [KC][TQ]
+  const uint32_t pbar = bar(c.pair[qw]);
+  int pair_phase = 0;
+  auto pair_sync = [&]() {
+    tc::mbar_arrive(pbar);
+    const bool r2 = uni(wt.wait(pbar, pair_phase & 1, 14));
+    ++pair_phase;
+    return r2;
+  };
+
+  bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
+  // fp16 copy of this thread's half of its Q row: registers and the swizzled Q16 tile
+  uint32_t q16[AW];
+#pragma unroll
+  for (int i = 0; i < 4 * SUB; ++i) {
+    const int cc = ch * 4 * SUB + i;
+    const int s = cc / 8, cw = cc % 8;
+    const uint32_t off = s * TQ * 128 + r * 128 + ((cw ^ (r & 7)) << 4);
+    const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
+    const uint4 y = make_uint4(bf16x2_to_f16x2(x.x), bf16x2_to_f16x2(x.y), bf16x2_to_f16x2(x.z),
+                               bf16x2_to_f16x2(x.w));
+    *reinterpret_cast<uint4*>(gbase + OFF_Q16 + off) = y;
+    q16[4 * i + 0] = y.x;
+    q16[4 * i + 1] = y.y;
+    q16[4 * i + 2] = y.z;
+    q16[4 * i + 3] = y.w;
+  }
+  tc::fence_proxy_async();
+  {
+    uint32_t z[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll
+    for (int k = 0; k < DH / 32; ++k) tc::tmem_st32(tmem + lane_off + COL_O + ch * DH + 32 * k, z);
+    tc::tmem_wait_st();
+  }
+  tc::fence_before_sync();
+  tc::mbar_arrive(bar(c.init_done));
+
+  float m_ref = -INFINITY, l = 0.f;
+  // The last O-writing MMA issued before our next value product: kind 0 = value
+  // product of S-buffer lw_buf, kind 1 = order-1 product of A slot lw_buf.
+  int lw_kind = -1, lw_buf = 0, lw_use = 0;
+  auto wait_last_writer = [&](int where) {
+    if (lw_kind < 0) return true;
+    const uint32_t b = lw_kind == 0 ? bar(c.pv_done[lw_buf]) : bar(c.a_done[lw_buf]);
+    const bool r2 = uni(wt.wait(b, lw_use & 1, where));
+    tc::fence_after_sync();
+    return r2;
+  };
+
+  Walk wk;
+  int ns = 0, nmat = 0, cur_buf = 0, cur_use = 0, cur_tile = 0, prev_buf = -1;
+  bool r_slots_free = false;  // this tile's value product has read its P
+
+  // One TILE (IS_TILE, NH = 32) or EXACT (NH = BLK / 2) item: this thread's NH logits.
+  auto s_item = [&](const Item& it, int sb, int n, auto nh_tag, auto tile_tag) -> bool {
+    constexpr int NH = decltype(nh_tag)::value;
+    constexpr bool TILE = decltype(tile_tag)::value;
+    constexpr int NK = NH / 32;
+    const uint32_t sa = tmem + lane_off + COL_R0 + 128 * sb;
+    const int col0 = ch * NH;
+    uint32_t sv[NH];
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+      tc::tmem_ld32(sa + col0 + 32 * k, sv + 32 * k);
+    tc::tmem_wait_ld();
+    uint32_t mbits[NK];
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+      if (TILE) {
+        const int j0 = it.j * KC + col0 + 32 * k;
+        mbits[k] = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
+      } else {
+        const int t0 = it.j * BLK + col0 + 32 * k;
+        mbits[k] = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
+        if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits[k] = 0u;
+      }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if ((mbits[k] >> i) & 1u) mx = fmaxf(mx, __uint_as_float(sv[32 * k + i]) * sl2);
+    float* rmax = red + (n & 1) * 2 * TQ;
+    rmax[ch * TQ + r] = mx;
+    if (!pair_sync()) return false;
+    mx = fmaxf(mx, rmax[(1 - ch) * TQ + r]);
+    // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
+    // reference; rows that had no reference yet just take one (O is still zero).
+    const bool grow = mx > m_ref + kThresh;
+    const bool need_o = grow && m_ref != -INFINITY;
+    const float f = need_o ? tc::ex2(m_ref - mx) : 1.f;
+    if (grow) m_ref = mx;
+    l *= f;
+    if (__any_sync(0xffffffffu, need_o)) {
+      if (!wait_last_writer(12)) return false;
+#pragma unroll
+      for (int k = 0; k < DH / 32; ++k) {
+        uint32_t v[32];
+        const uint32_t oa = tmem + lane_off + COL_O + ch * DH + 32 * k;
+        tc::tmem_ld32(oa, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+        tc::tmem_st32(oa, v);
+      }
+      tc::tmem_wait_st();
+    }
+    // P = 2^(x - m_ref) as fp16 pairs over the logits of both halves (all of them were
+    // read before the pair met, so the writes cannot overtake a partner's read).
+    const float wlast = (float)(p.Nk - (nkb - 1) * BLK);
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float x0 = ((mbits[k] >> i) & 1u) ? tc::ex2(__uint_as_float(sv[32 * k + i]) * sl2 - m_ref) : 0.f;
+        const float x1 =
+            ((mbits[k] >> (i + 1)) & 1u) ? tc::ex2(__uint_as_float(sv[32 * k + i + 1]) * sl2 - m_ref) : 0.f;
+        if (TILE) {
+          const int j = it.j * KC + col0 + 32 * k + i;
+          l += x0 * (j == nkb - 1 ? wlast : (float)BLK) + x1 * (j + 1 == nkb - 1 ? wlast : (float)BLK);
+          stash[(col0 + 32 * k + i) * TQ + r] = __float2half_rn(x0);
+          stash[(col0 + 32 * k + i + 1) * TQ + r] = __float2half_rn(x1);
+        } else {
+          l += x0 + x1;
+        }
+        pk[i / 2] = pack_f16(x0, x1);
+      }
+      tc::tmem_st16(sa + col0 / 2 + 16 * k, pk);
+    }
+    tc::tmem_wait_st();
+    tc::fence_before_sync();
+    tc::mbar_arrive(bar(c.p_full[sb]));
+    if (TILE && !pair_sync()) return false;  // the partner's half of the stash is visible
+    return true;
+  };
+
+  while (ok) {
+    const Item it = wk.next<ORDER>(c, nkb);
+    if (it.kind == kNone) break;
+    if (it.kind == kMat) {
+      if constexpr (ORDER == 1) {
+        const int n = nmat++;
+        const int slot = n % NA, use = n / NA;
+        if (use >= 1) ok = uni(wt.wait(bar(c.a_done[slot]), (use - 1) & 1, 10));
+        if (ok && slot >= 2 && !r_slots_free) {
+          ok = uni(wt.wait(bar(c.pv_done[cur_buf]), cur_use & 1, 15));
+          r_slots_free = true;
+        }
+        if (!ok) break;
+        tc::fence_after_sync();
+        const float pj = __half2float(stash[(it.j - cur_tile * KC) * TQ + r]);
+        const __half2 al = __float2half2_rn(pj * p.scale);
+        uint32_t a[AW];
+#pragma unroll
+        for (int i = 0; i < AW; ++i) {
+          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
+          a[i] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+        tmem_st_w<AW>(tmem + lane_off + a_col(slot, cur_buf) + ch * AW, a);
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        tc::mbar_arrive(bar(c.a_full[slot]));
+        lw_kind = 1;
+        lw_buf = slot;
+        lw_use = use;
+      }
+      continue;
+    }
+    // ---- TILE or EXACT: logits in an S buffer ----
+    if (prev_buf >= 0) {
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar(c.s_free[prev_buf]));
+    }
+    const int n = ns++;
+    const int sb = n & 1, use = n >> 1;
+    prev_buf = sb;
+    ok = uni(wt.wait(bar(c.s_full[sb]), use & 1, 11));
+    if (!ok) break;
+    tc::fence_after_sync();
+    if (it.kind == kTile) {
+      cur_buf = sb;
+      cur_use = use;
+      cur_tile = it.j;
+      r_slots_free = false;
+      ok = s_item(it, sb, n, std::integral_constant<int, KC / 2>{}, std::true_type{});
+    } else {
+      ok = s_item(it, sb, n, std::integral_constant<int, BLK / 2>{}, std::false_type{});
+    }
+    lw_kind = 0;
+    lw_buf = sb;
+    lw_use = use;
+  }
+
+  // ---- epilogue: O / l over both column halves ----
+  if (ok) ok = wait_last_writer(13);
+  float* rsum = red + 4 * TQ;
+  rsum[ch * TQ + r] = l;
+  if (ok) ok = pair_sync();
+  if (!ok) return;
+  const float lt = l + rsum[(1 - ch) * TQ + r];
+  const bool store = q0 + r < p.Nq;
+  const float inv = lt > 0.f ? 1.f / lt : 0.f;
+  const size_t rowoff = ((size_t)bh * p.Nq + q0 + (store ? r : 0)) * D + ch * DH;
+#pragma unroll
+  for (int k = 0; k < DH / 32; ++k) {
+    uint32_t v[32];
+    tc::tmem_ld32(tmem + lane_off + COL_O + ch * DH + 32 * k, v);
+    tc::tmem_wait_ld();
+    if (!store) continue;
+    if (p.out_dtype == 0) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff + 32 * k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        o[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                           __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff + 32 * k);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = make_uint4(pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv),
+                          pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv),
+                          pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv),
+                          pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv));
+    }
+  }
+}
 
 template <int D, int BLK, int ORDER>
 __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_constant__ Params p) {
@@ -207,7 +494,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   if (c.abort) return;
 
   // ---- setup: barriers (producer warp), TMEM (MMA warp), kept bitmaps (softmax) ----
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     for (int u = 0; u < NU; ++u) {
       tc::mbar_init(bar(c.full[u]), 1);
       tc::mbar_init(bar(c.empty[u]), 1);
@@ -215,41 +502,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(c.s_full[b]), 1);
       tc::mbar_init(bar(c.pv_done[b]), 1);
-      tc::mbar_init(bar(c.a_done[b]), 1);
-      tc::mbar_init(bar(c.p_full[b]), TQ);
-      tc::mbar_init(bar(c.s_free[b]), TQ);
-      tc::mbar_init(bar(c.a_full[b]), TQ);
+      tc::mbar_init(bar(c.p_full[b]), NSOFT);
+      tc::mbar_init(bar(c.s_free[b]), NSOFT);
+    }
+    for (int a = 0; a < NA; ++a) {
+      tc::mbar_init(bar(c.a_done[a]), 1);
+      tc::mbar_init(bar(c.a_full[a]), NSOFT);
     }
     tc::mbar_init(bar(c.q_full), 1);
-    tc::mbar_init(bar(c.init_done), TQ);
+    tc::mbar_init(bar(c.init_done), NSOFT);
     tc::mbar_init(bar(c.drain), 1);
+    for (int w = 0; w < 4; ++w) tc::mbar_init(bar(c.pair[w]), 64);
     tc::fence_mbar_init();
     tc::fence_proxy_async();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tc::tmem_alloc(smem_u32(&c.tmem_base), 512);
     tc::tmem_relinquish();
   }
-  if (warp < 4) {
+  if (warp < 8) {
     // Kept bitmaps of the one (block 128) or two (block 64) query blocks of the tile.
     const int nh = BLK == 128 ? 1 : 2;
-    for (int w = tid; w < 2 * MAXW; w += 128) (&c.kept[0][0])[w] = 0u;
-    __syncwarp();
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    for (int w = tid; w < 2 * MAXW; w += NSOFT) (&c.kept[0][0])[w] = 0u;
+    asm volatile("bar.sync 1, %0;\n" ::"n"(NSOFT) : "memory");
     for (int h = 0; h < nh; ++h) {
       const int qb = q0 / BLK + h;
       if (qb >= p.nqb) continue;
       const size_t row = (size_t)bh * p.nqb + qb;
       const int n = min(max(p.kv_cnt[row], 0), p.cap);
       const int32_t* src = p.kv_idx + row * p.cap;
-      for (int x = tid; x < n; x += 128) {
+      for (int x = tid; x < n; x += NSOFT) {
         const int j = src[x];
         if (j >= 0 && j < nkb) atomicOr(&c.kept[h][j >> 5], 1u << (j & 31));
       }
     }
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+    asm volatile("bar.sync 1, %0;\n" ::"n"(NSOFT) : "memory");
     const bool has1 = BLK == 64 && (q0 / BLK + 1) < p.nqb;
-    for (int w = tid; w < MAXW; w += 128) {
+    for (int w = tid; w < MAXW; w += NSOFT) {
       const int lo = w * 32;
       const uint32_t valid = lo + 32 <= nkb ? 0xffffffffu : (lo < nkb ? (1u << (nkb - lo)) - 1u : 0u);
       const uint32_t k0 = c.kept[0][w];
@@ -265,7 +554,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   const uint32_t tmem = c.tmem_base;
   tc::Waiter wt{&c.abort, p.err_flag, kWaitLimit};
 
-  if (warp == 4) {
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegSoft));
+    softmax_role<D, BLK, ORDER>(p, c, gbase, tmem, wt, warp, lane);
+  } else {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegCtl));
+  if (warp == 8) {
     // =========================== TMA producer ===========================
     if (lane == 0) {
       tc::prefetch_tmap(&p.tmQ);
@@ -309,7 +603,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       for (int v = max(0, u - NU); v < u; ++v)
         tc::wait_drain(bar(c.full[v % NU]), (v / NU) & 1, kWaitLimit);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // =========================== MMA issuer ===========================
     if (lane == 0) {
       constexpr uint32_t I_S_TILE = tc::idesc_f16(0, 0, 0, KC);
@@ -361,7 +655,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
           ok = wt.wait(bar(c.a_full[e.buf]), e.use & 1, 7);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t aa = tmem + COL_A0 + 64 * e.buf;
+          const uint32_t aa = tmem + a_col(e.buf, e.tbuf);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t bd = tc::sdesc(src + kk * 2048, D * 128, 1024);
@@ -376,234 +670,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       tc::mma_commit(bar(c.drain));
       tc::wait_drain(bar(c.drain), 0, kWaitLimit);
     }
-  } else {
-    // =========================== softmax (rows) ===========================
-    const int r = tid;                       // query row within the tile, TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    const int h = BLK == 64 ? (r >> 6) : 0;  // which query block of the tile
-    const float sl2 = p.scale * kLog2e;
-    // tcgen05.ld / st are warp-collective: every decision that guards them is made
-    // uniform across the warp.
-    auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
-    bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
-    // fp16 copy of this row of Q (registers and the swizzled Q16 tile) and O = 0
-    uint32_t q16[D / 2];
-#pragma unroll
-    for (int s = 0; s < SUB; ++s)
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = s * TQ * 128 + r * 128 + ((ch ^ (r & 7)) << 4);
-        const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
-        uint4 y;
-        y.x = bf16x2_to_f16x2(x.x);
-        y.y = bf16x2_to_f16x2(x.y);
-        y.z = bf16x2_to_f16x2(x.z);
-        y.w = bf16x2_to_f16x2(x.w);
-        *reinterpret_cast<uint4*>(gbase + OFF_Q16 + off) = y;
-        q16[s * 32 + ch * 4 + 0] = y.x;
-        q16[s * 32 + ch * 4 + 1] = y.y;
-        q16[s * 32 + ch * 4 + 2] = y.z;
-        q16[s * 32 + ch * 4 + 3] = y.w;
-      }
-    tc::fence_proxy_async();
-    {
-      uint32_t z[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) z[i] = 0u;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tc::tmem_st32(tmem + lane_off + COL_O + 32 * cc, z);
-      tc::tmem_wait_st();
-    }
-    tc::fence_before_sync();
-    tc::mbar_arrive(bar(c.init_done));
-
-    float m_ref = -INFINITY, l = 0.f;
-    // last O-writing MMA the MMA warp will issue before our next value product
-    int lw_kind = -1, lw_buf = 0, lw_use = 0;
-    auto wait_last_writer = [&](int where) {
-      if (lw_kind < 0) return true;
-      const uint32_t b = lw_kind == 0 ? bar(c.pv_done[lw_buf]) : bar(c.a_done[lw_buf]);
-      const bool r2 = uni(wt.wait(b, lw_use & 1, where));
-      tc::fence_after_sync();
-      return r2;
-    };
-
-    Walk wk;
-    int ns = 0, nmat = 0, cur_buf = 0, cur_tile = 0, prev_buf = -1;
-    while (ok) {
-      const Item it = wk.next<ORDER>(c, nkb);
-      if (it.kind == kNone) break;
-      if (it.kind == kMat) {
-        if constexpr (ORDER == 1) {
-          const int n = nmat++;
-          const int ab = n & 1, use = n >> 1;
-          if (use >= 1) ok = uni(wt.wait(bar(c.a_done[ab]), (use - 1) & 1, 10));
-          if (!ok) break;
-          tc::fence_after_sync();
-          const int cl = it.j - cur_tile * KC;
-          const uint32_t w = tc::tmem_ld1(tmem + lane_off + COL_R0 + 128 * cur_buf + (cl >> 1));
-          tc::tmem_wait_ld();
-          const __half ph = __ushort_as_half((unsigned short)((cl & 1) ? (w >> 16) : (w & 0xFFFFu)));
-          const __half2 al = __float2half2_rn(__half2float(ph) * p.scale);
-          uint32_t a[32];
-#pragma unroll
-          for (int s = 0; s < D / 64; ++s) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              __half2 x = *reinterpret_cast<const __half2*>(&q16[32 * s + i]);
-              __half2 y = __hmul2(x, al);
-              a[i] = *reinterpret_cast<uint32_t*>(&y);
-            }
-            tc::tmem_st32(tmem + lane_off + COL_A0 + 64 * ab + 32 * s, a);
-          }
-          tc::tmem_wait_st();
-          tc::fence_before_sync();
-          tc::mbar_arrive(bar(c.a_full[ab]));
-          lw_kind = 1;
-          lw_buf = ab;
-          lw_use = use;
-        }
-        continue;
-      }
-      // ---- TILE or EXACT: logits in S buffer ----
-      if (prev_buf >= 0) {
-        tc::fence_before_sync();
-        tc::mbar_arrive(bar(c.s_free[prev_buf]));
-      }
-      const int n = ns++;
-      const int sb = n & 1, use = n >> 1;
-      cur_buf = sb;
-      prev_buf = sb;
-      const bool tile = it.kind == kTile;
-      if (tile) cur_tile = it.j;
-      ok = uni(wt.wait(bar(c.s_full[sb]), use & 1, 11));
-      if (!ok) break;
-      tc::fence_after_sync();
-      const uint32_t sa = tmem + lane_off + COL_R0 + 128 * sb;
-      const int ncols = tile ? KC : BLK;
-      const int col0 = tile ? it.j * KC : it.j * BLK;  // first block (tile) or token (exact)
-      // pass 1: masked row max
-      float mx = -INFINITY;
-      for (int ck = 0; ck < ncols / 32; ++ck) {
-        uint32_t v[32];
-        tc::tmem_ld32(sa + 32 * ck, v);
-        tc::tmem_wait_ld();
-        uint32_t mbits;
-        if (tile) {
-          const int j0 = col0 + 32 * ck;
-          mbits = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
-        } else {
-          const int t0 = col0 + 32 * ck;
-          mbits = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
-          if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits = 0u;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((mbits >> i) & 1u) mx = fmaxf(mx, __uint_as_float(v[i]) * sl2);
-      }
-      // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
-      // reference; rows that had no reference yet just take one (O is still zero).
-      const bool grow = mx > m_ref + kThresh;
-      const bool need_o = grow && m_ref != -INFINITY;
-      const float f = need_o ? tc::ex2(m_ref - mx) : 1.f;
-      if (grow) m_ref = mx;
-      l *= f;
-      if (__any_sync(0xffffffffu, need_o)) {
-        if (!wait_last_writer(12)) {
-          ok = false;
-          break;
-        }
-        for (int ck = 0; ck < D / 32; ++ck) {
-          uint32_t v[32];
-          tc::tmem_ld32(tmem + lane_off + COL_O + 32 * ck, v);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-          tc::tmem_st32(tmem + lane_off + COL_O + 32 * ck, v);
-        }
-        tc::tmem_wait_st();
-      }
-      // P overwrites logits this thread has already read. The value product that read
-      // this buffer's previous P was issued before these logits, so it has finished.
-      // pass 2: P = 2^(x - m_ref), written back as 16-bit pairs
-      for (int ck = 0; ck < ncols / 32; ++ck) {
-        uint32_t v[32];
-        tc::tmem_ld32(sa + 32 * ck, v);
-        tc::tmem_wait_ld();
-        uint32_t mbits;
-        float wlast = 1.f;
-        int jlast = -1;
-        if (tile) {
-          const int j0 = col0 + 32 * ck;
-          mbits = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
-          jlast = nkb - 1 - j0;  // column of the possibly partial last block
-          wlast = (float)(p.Nk - (nkb - 1) * BLK);
-        } else {
-          const int t0 = col0 + 32 * ck;
-          mbits = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
-          if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits = 0u;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float x0 = ((mbits >> i) & 1u) ? tc::ex2(__uint_as_float(v[i]) * sl2 - m_ref) : 0.f;
-          const float x1 =
-              ((mbits >> (i + 1)) & 1u) ? tc::ex2(__uint_as_float(v[i + 1]) * sl2 - m_ref) : 0.f;
-          if (tile) {
-            const float w0 = (i == jlast) ? wlast : (float)BLK;
-            const float w1 = (i + 1 == jlast) ? wlast : (float)BLK;
-            l += x0 * w0 + x1 * w1;
-          } else {
-            l += x0 + x1;
-          }
-          pk[i / 2] = pack_f16(x0, x1);
-        }
-        tc::tmem_st16(sa + 16 * ck, pk);
-      }
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      tc::mbar_arrive(bar(c.p_full[sb]));
-      lw_kind = 0;
-      lw_buf = sb;
-      lw_use = use;
-    }
-    // ---- epilogue: O / l ----
-    if (ok) ok = wait_last_writer(13);
-    if (ok) {
-      const bool store = q0 + r < p.Nq;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const size_t rowoff = ((size_t)bh * p.Nq + q0 + (store ? r : 0)) * D;
-      for (int ck = 0; ck < D / 32; ++ck) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + lane_off + COL_O + 32 * ck, v);
-        tc::tmem_wait_ld();
-        if (!store) continue;
-        if (p.out_dtype == 0) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff + 32 * ck);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
-                               __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
-        } else {
-          uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff + 32 * ck);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 y;
-            y.x = pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv);
-            y.y = pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv);
-            y.z = pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv);
-            y.w = pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv);
-            o[i] = y;
-          }
-        }
-      }
-    }
+  }
   }
 
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 5) tc::tmem_dealloc(tmem, 512);
+  if (warp == 9) tc::tmem_dealloc(tmem, 512);
 }
 
 namespace {
