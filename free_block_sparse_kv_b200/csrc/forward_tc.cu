@@ -84,6 +84,7 @@ struct Ctl {  // control block in shared memory
   uint64_t a_full[NA], a_done[NA];
   uint64_t q_full, init_done, drain;
   uint64_t pair[4];         // the two softmax warps sharing 32 rows
+  int4 evq[NU];             // event of each ring unit: {kind | item kind << 4, j, buf | tbuf << 4, use}
   uint32_t tmem_base;
   int abort;
   uint32_t kept[2][MAXW];   // kept blocks of each query block in the tile (half)
@@ -245,7 +246,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   int pair_phase = 0;
   auto pair_sync = [&]() {
     tc::mbar_arrive(pbar);
-    const bool r2 = uni(wt.wait(pbar, pair_phase & 1, 14));
+    const bool r2 = uni(wt.fast(pbar, pair_phase & 1, 14));
     ++pair_phase;
     return r2;
   };
@@ -387,7 +388,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       if constexpr (ORDER == 1) {
         const int n = nmat++;
         const int slot = n % NA, use = n / NA;
-        if (use >= 1) ok = uni(wt.wait(bar(c.a_done[slot]), (use - 1) & 1, 10));
+        if (use >= 1) ok = uni(wt.fast(bar(c.a_done[slot]), (use - 1) & 1, 10));
         if (ok && slot >= 2 && !r_slots_free) {
           ok = uni(wt.wait(bar(c.pv_done[cur_buf]), cur_use & 1, 15));
           r_slots_free = true;
@@ -420,7 +421,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     const int n = ns++;
     const int sb = n & 1, use = n >> 1;
     prev_buf = sb;
-    ok = uni(wt.wait(bar(c.s_full[sb]), use & 1, 11));
+    ok = uni(wt.fast(bar(c.s_full[sb]), use & 1, 11));
     if (!ok) break;
     tc::fence_after_sync();
     if (it.kind == kTile) {
@@ -571,13 +572,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       bool ok = true;
       while (ok) {
         const Event e = gen.next<ORDER>(c, nkb);
-        if (e.kind == eNone) break;
         const int slot = u % NU;
-        if (u >= NU) ok = wt.wait(bar(c.empty[slot]), ((u / NU) - 1) & 1, 1);
+        if (u >= NU) ok = wt.fast(bar(c.empty[slot]), ((u / NU) - 1) & 1, 1);
         if (!ok) break;
         const uint32_t dst = base + OFF_U + slot * UNIT;
         const uint32_t fb = bar(c.full[slot]);
         const Item& it = e.item;
+        // The MMA thread reads the event of a unit after the unit's full barrier.
+        c.evq[slot] =
+            make_int4(e.kind | (it.kind << 4), it.j, e.buf | (e.tbuf << 4), e.use);
+        if (e.kind == eNone) {
+          tc::mbar_arrive(fb);  // terminal record, no data
+          ++u;
+          break;
+        }
         if (e.kind == eS && it.kind == kTile) {
           tc::mbar_arrive_expect_tx(fb, By::KB);
           for (int s = 0; s < SUB; ++s)
@@ -613,58 +621,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       constexpr uint32_t I_MAT = tc::idesc_f16(0, 0, 1, D);
       bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
       tc::fence_after_sync();
-      EventGen gen;
-      int u = 0;
-      while (ok) {
-        const Event e = gen.next<ORDER>(c, nkb);
-        if (e.kind == eNone) break;
+      // Descriptor bases; per k-step only the start-address field (low bits) moves.
+      const uint64_t dQ = tc::sdesc(base + OFF_Q, 16, 1024), dQ16 = tc::sdesc(base + OFF_Q16, 16, 1024);
+      for (int u = 0; ok; ++u) {
         const int slot = u % NU;
-        const uint32_t src = base + OFF_U + slot * UNIT;
-        ok = wt.wait(bar(c.full[slot]), (u / NU) & 1, 4);
+        ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
         if (!ok) break;
-        const Item& it = e.item;
-        if (e.kind == eS) {
-          if (e.use >= 1) ok = wt.wait(bar(c.s_free[e.buf]), (e.use - 1) & 1, 5);
+        const int4 rec = c.evq[slot];  // ordered by the full-barrier wait (asm with memory clobber)
+        const int kind = rec.x & 15, ikind = rec.x >> 4, buf = rec.z & 15, tbuf = rec.z >> 4;
+        const int use = rec.w;
+        if (kind == eNone) break;
+        const uint32_t src = base + OFF_U + slot * UNIT;
+        if (kind == eS) {
+          if (use >= 1) ok = wt.fast(bar(c.s_free[buf]), (use - 1) & 1, 5);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t dt = tmem + COL_R0 + 128 * e.buf;
-          const bool tile = it.kind == kTile;
-          const uint32_t qa = base + (tile ? OFF_Q16 : OFF_Q);
+          const uint32_t dt = tmem + COL_R0 + 128 * buf;
+          const bool tile = ikind == kTile;
+          const uint64_t ad0 = tile ? dQ16 : dQ;
           const int rows = tile ? KC : BLK;
+          const uint64_t bd0 = tc::sdesc(src, 16, 1024);
+          const uint32_t idesc = tile ? I_S_TILE : I_S_EX;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk % 4) * 32;
-            const uint64_t ad = tc::sdesc(qa + (kk / 4) * TQ * 128 + off, 16, 1024);
-            const uint64_t bd = tc::sdesc(src + (kk / 4) * rows * 128 + off, 16, 1024);
-            tc::mma_ss(dt, ad, bd, tile ? I_S_TILE : I_S_EX, kk > 0);
+            const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
+            const uint32_t boff = ((kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
+            tc::mma_ss(dt, ad0 + aoff, bd0 + boff, idesc, kk > 0);
           }
-          tc::mma_commit(bar(c.s_full[e.buf]));
-        } else if (e.kind == ePV) {
-          ok = wt.wait(bar(c.p_full[e.buf]), e.use & 1, 6);
+          tc::mma_commit(bar(c.s_full[buf]));
+        } else if (kind == ePV) {
+          ok = wt.fast(bar(c.p_full[buf]), use & 1, 6);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t pa = tmem + COL_R0 + 128 * e.buf;
-          const bool tile = it.kind == kTile;
+          const uint32_t pa = tmem + COL_R0 + 128 * buf;
+          const bool tile = ikind == kTile;
           const int rows = tile ? KC : BLK;
-          for (int kk = 0; kk < rows / 16; ++kk) {
-            const uint64_t bd = tc::sdesc(src + kk * 2048, rows * 128, 1024);
-            tc::mma_ts(tmem + COL_O, pa + kk * 8, bd, tile ? I_PV_TILE : I_PV_EX, 1);
-          }
-          tc::mma_commit(bar(c.pv_done[e.buf]));
+          const uint64_t bd0 = tc::sdesc(src, rows * 128, 1024);
+          const uint32_t idesc = tile ? I_PV_TILE : I_PV_EX;
+          for (int kk = 0; kk < rows / 16; ++kk)
+            tc::mma_ts(tmem + COL_O, pa + kk * 8, bd0 + ((kk * 2048) >> 4), idesc, 1);
+          tc::mma_commit(bar(c.pv_done[buf]));
         } else {
-          ok = wt.wait(bar(c.a_full[e.buf]), e.use & 1, 7);
+          ok = wt.fast(bar(c.a_full[buf]), use & 1, 7);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t aa = tmem + a_col(e.buf, e.tbuf);
+          const uint32_t aa = tmem + a_col(buf, tbuf);
+          const uint64_t bd0 = tc::sdesc(src, D * 128, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t bd = tc::sdesc(src + kk * 2048, D * 128, 1024);
-            tc::mma_ts(tmem + COL_O, aa + kk * 8, bd, I_MAT, 1);
-          }
-          tc::mma_commit(bar(c.a_done[e.buf]));
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc::mma_ts(tmem + COL_O, aa + kk * 8, bd0 + ((kk * 2048) >> 4), I_MAT, 1);
+          tc::mma_commit(bar(c.a_done[buf]));
         }
         tc::mma_commit(bar(c.empty[slot]));
-        ++u;
       }
       // Drain: wait for every MMA issued so far before TMEM is released.
       tc::mma_commit(bar(c.drain));

@@ -58,6 +58,12 @@ struct Waiter {
       }
     }
   }
+  // One try_wait first (about 50 cycles when the phase is already complete), then the
+  // bounded loop.
+  SA_DEVI bool fast(uint32_t bar, uint32_t parity, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait(bar, parity, where);
+  }
 };
 
 // Bounded wait that ignores the abort word: used when draining the CTA's own
