@@ -20,15 +20,16 @@
 //   warps 10-11 idle (they complete the control warpgroup for the register split).
 // Work items, in order (the same walk runs in all three roles):
 //   TILE t   64 centroids (fp16) and value sums (fp16): S = Q16 Kbar^T, P, O += P S
-//   MAT j    each skipped block of the current tile (order 1): O += A_j M_j (fp16)
+//   MAT j    each pair of skipped blocks of the current tile (order 1):
+//            O += [A_j1 | A_j2] [M_j1; M_j2] (fp16)
 //   EXACT j  each kept block: S = Q K_j^T (bf16), P, O += P V_j (fp16 P and V)
 // The MMA warp issues the logits of the next TILE/EXACT item before the value
 // product of the current one, so logits overlap the softmax of the previous item.
-// TMEM columns: O [0, D); S/P buffers R0 = [128, 256), R1 = [256, 384); A slots 0, 1
-// at 384 and 448. During a tile's MAT items the tile's S/P buffer is free once its
-// value product has run (the tile's P is also kept in shared memory for alpha), and
-// it holds A slots 2 and 3: four A operands in flight hide the hand-off latency
-// between the softmax warps and the MMA thread.
+// TMEM columns: O [0, D); S/P buffers R0 = [128, 256), R1 = [256, 384); A slot 0 at
+// [384, 512). Order-1 products go two skipped blocks at a time: A = [a1 q | a2 q]
+// (K = 2d) against [M_j1; M_j2], 16 tensor-core instructions per hand-off. During a
+// tile's MAT items the tile's S/P buffer is free once its value product has run (the
+// tile's P is also kept in shared memory for alpha) and serves as A slot 1.
 // Every mbarrier wait is bounded: on timeout the CTA sets err_flag, abandons its work,
 // drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -53,7 +54,7 @@ constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA
 // control warpgroup gives registers back, the softmax warpgroups take them.
 constexpr int kRegCtl = 72, kRegSoft = 208;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
-constexpr int NA = 4;          // A-operand slots for the order-1 products
+constexpr int NA = 2;          // A-operand slots for the order-1 products (each holds a pair)
 constexpr float kThresh = 8.0f;  // lazy-rescale threshold, base-2 units
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
@@ -96,6 +97,7 @@ static_assert(sizeof(Ctl) <= 2048, "control block");
 enum : int { kTile = 0, kMat = 1, kExact = 2, kNone = 3 };
 struct Item {
   int kind, j;  // TILE: j = tile index; MAT / EXACT: j = block index
+  int j2 = -1;  // MAT: second skipped block of the pair, or -1
 };
 
 // The walk over work items; identical in every role.
@@ -119,9 +121,14 @@ struct Walk {
           continue;
         }
         if (ORDER == 1) {
+          // skipped blocks of this tile, two at a time
           const int end = min(nkb, (tile + 1) * KC);
-          j = next_bit(c.skipU, j, end);
-          if (j < end) return Item{kMat, j++};
+          const int j1 = next_bit(c.skipU, j, end);
+          if (j1 < end) {
+            const int j2 = next_bit(c.skipU, j1 + 1, end);
+            j = j2 < end ? j2 + 1 : end;
+            return Item{kMat, j1, j2 < end ? j2 : -1};
+          }
         }
         ++tile;
         j = -1;
@@ -196,10 +203,9 @@ struct EventGen {
   }
 };
 
-// TMEM column of A slot `slot` for a tile whose S/P buffer is `tbuf`.
-SA_DEVI uint32_t a_col(int slot, int tbuf) {
-  return slot < 2 ? COL_A0 + 64 * slot : COL_R0 + 128 * tbuf + 64 * (slot - 2);
-}
+// TMEM column of A slot `slot` (128 columns: the operands of two skipped blocks) for a
+// tile whose S/P buffer is `tbuf`. Slot 1 reuses that buffer once its P has been read.
+SA_DEVI uint32_t a_col(int slot, int tbuf) { return slot == 0 ? COL_A0 : COL_R0 + 128 * tbuf; }
 
 template <int D, int BLK>
 struct Bytes {
@@ -389,21 +395,27 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
         const int n = nmat++;
         const int slot = n % NA, use = n / NA;
         if (use >= 1) ok = uni(wt.fast(bar(c.a_done[slot]), (use - 1) & 1, 10));
-        if (ok && slot >= 2 && !r_slots_free) {
+        if (ok && slot == 1 && !r_slots_free) {
           ok = uni(wt.wait(bar(c.pv_done[cur_buf]), cur_use & 1, 15));
           r_slots_free = true;
         }
         if (!ok) break;
         tc::fence_after_sync();
-        const float pj = __half2float(stash[(it.j - cur_tile * KC) * TQ + r]);
-        const __half2 al = __float2half2_rn(pj * p.scale);
-        uint32_t a[AW];
+        const uint32_t ab = tmem + lane_off + a_col(slot, cur_buf) + ch * AW;
+        const int jb[2] = {it.j, it.j2};
 #pragma unroll
-        for (int i = 0; i < AW; ++i) {
-          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
-          a[i] = *reinterpret_cast<const uint32_t*>(&y);
+        for (int b = 0; b < 2; ++b) {
+          if (jb[b] < 0) break;
+          const float pj = __half2float(stash[(jb[b] - cur_tile * KC) * TQ + r]);
+          const __half2 al = __float2half2_rn(pj * p.scale);
+          uint32_t a[AW];
+#pragma unroll
+          for (int i = 0; i < AW; ++i) {
+            const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
+            a[i] = *reinterpret_cast<const uint32_t*>(&y);
+          }
+          tmem_st_w<AW>(ab + b * (D / 2), a);
         }
-        tmem_st_w<AW>(tmem + lane_off + a_col(slot, cur_buf) + ch * AW, a);
         tc::tmem_wait_st();
         tc::fence_before_sync();
         tc::mbar_arrive(bar(c.a_full[slot]));
@@ -579,8 +591,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         const uint32_t fb = bar(c.full[slot]);
         const Item& it = e.item;
         // The MMA thread reads the event of a unit after the unit's full barrier.
-        c.evq[slot] =
-            make_int4(e.kind | (it.kind << 4), it.j, e.buf | (e.tbuf << 4), e.use);
+        c.evq[slot] = make_int4(e.kind | (it.kind << 4) | ((it.j2 >= 0) << 8), it.j,
+                                e.buf | (e.tbuf << 4), e.use);
         if (e.kind == eNone) {
           tc::mbar_arrive(fb);  // terminal record, no data
           ++u;
@@ -598,6 +610,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
           tc::mbar_arrive_expect_tx(fb, By::M);
           for (int s = 0; s < SUB; ++s)
             tc::tma_load_3d(dst + s * D * 128, &p.tmM, fb, 64 * s, 0, bh * nkb + it.j);
+          if (it.j2 >= 0) {  // the pair's second block goes to the next unit
+            ++u;
+            const int s2 = u % NU;
+            if (u >= NU) ok = wt.fast(bar(c.empty[s2]), ((u / NU) - 1) & 1, 1);
+            if (!ok) break;
+            const uint32_t fb2 = bar(c.full[s2]);
+            tc::mbar_arrive_expect_tx(fb2, By::M);
+            for (int s = 0; s < SUB; ++s)
+              tc::tma_load_3d(base + OFF_U + s2 * UNIT + s * D * 128, &p.tmM, fb2, 64 * s, 0,
+                              bh * nkb + it.j2);
+          }
         } else {
           const CUtensorMap* m = e.kind == eS ? &p.tmK : &p.tmV;
           tc::mbar_arrive_expect_tx(fb, By::KV);
@@ -628,7 +651,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
         if (!ok) break;
         const int4 rec = c.evq[slot];  // ordered by the full-barrier wait (asm with memory clobber)
-        const int kind = rec.x & 15, ikind = rec.x >> 4, buf = rec.z & 15, tbuf = rec.z >> 4;
+        const int kind = rec.x & 15, ikind = (rec.x >> 4) & 15, buf = rec.z & 15, tbuf = rec.z >> 4;
+        const bool pair = (rec.x >> 8) & 1;
         const int use = rec.w;
         if (kind == eNone) break;
         const uint32_t src = base + OFF_U + slot * UNIT;
@@ -662,7 +686,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
             tc::mma_ts(tmem + COL_O, pa + kk * 8, bd0 + ((kk * 2048) >> 4), idesc, 1);
           tc::mma_commit(bar(c.pv_done[buf]));
         } else {
-          ok = wt.fast(bar(c.a_full[buf]), use & 1, 7);
+          const int slot2 = (u + 1) % NU;
+          if (pair) ok = wt.fast(bar(c.full[slot2]), ((u + 1) / NU) & 1, 4);
+          if (ok) ok = wt.fast(bar(c.a_full[buf]), use & 1, 7);
           if (!ok) break;
           tc::fence_after_sync();
           const uint32_t aa = tmem + a_col(buf, tbuf);
@@ -670,7 +696,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             tc::mma_ts(tmem + COL_O, aa + kk * 8, bd0 + ((kk * 2048) >> 4), I_MAT, 1);
+          if (pair) {
+            const uint64_t bd1 = tc::sdesc(base + OFF_U + slot2 * UNIT, D * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              tc::mma_ts(tmem + COL_O, aa + D / 2 + kk * 8, bd1 + ((kk * 2048) >> 4), I_MAT, 1);
+          }
           tc::mma_commit(bar(c.a_done[buf]));
+          if (pair) {
+            tc::mma_commit(bar(c.empty[slot]));
+            ++u;
+            tc::mma_commit(bar(c.empty[slot2]));
+            continue;
+          }
         }
         tc::mma_commit(bar(c.empty[slot]));
       }
