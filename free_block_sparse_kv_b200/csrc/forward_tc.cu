@@ -100,53 +100,57 @@ struct Item {
   int j2 = -1;  // MAT: second skipped block of the pair, or -1
 };
 
-// The walk over work items; identical in every role.
+// The walk over work items; identical in every role. The skipped blocks of the
+// current tile and the kept blocks of the current 32-block word are held in
+// registers as bit masks, so each step is a few integer instructions.
 struct Walk {
-  int phase = 0, tile = 0, j = -1;
+  int phase = 0, tile = 0, word = 0;
+  uint64_t tmask = 0;  // phase 0: skipped blocks of `tile` not yet walked
+  uint32_t kmask = 0;  // phase 1: kept blocks of `word` not yet walked
+  bool in_tile = false;
   template <int ORDER>
   SA_DEVI Item next(const Ctl& c, int nkb) {
     const int ntiles = (nkb + KC - 1) / KC;
     while (true) {
       if (phase == 0) {
-        if (tile >= ntiles) {
-          phase = 1;
-          j = 0;
-          continue;
-        }
-        if (j < 0) {
-          j = tile * KC;
-          if (c.skipU[2 * tile] | c.skipU[2 * tile + 1]) return Item{kTile, tile};
-          ++tile;
-          j = -1;
-          continue;
-        }
-        if (ORDER == 1) {
-          // skipped blocks of this tile, two at a time
-          const int end = min(nkb, (tile + 1) * KC);
-          const int j1 = next_bit(c.skipU, j, end);
-          if (j1 < end) {
-            const int j2 = next_bit(c.skipU, j1 + 1, end);
-            j = j2 < end ? j2 + 1 : end;
-            return Item{kMat, j1, j2 < end ? j2 : -1};
+        if (!in_tile) {
+          if (tile >= ntiles) {
+            phase = 1;
+            word = 0;
+            kmask = c.keptU[0];
+            continue;
           }
+          tmask = (uint64_t)c.skipU[2 * tile] | ((uint64_t)c.skipU[2 * tile + 1] << 32);
+          if (tmask) {
+            in_tile = true;
+            return Item{kTile, tile};
+          }
+          ++tile;
+          continue;
         }
+        if (ORDER == 1 && tmask) {
+          // skipped blocks of this tile, two at a time
+          const int j1 = tile * KC + __ffsll((long long)tmask) - 1;
+          tmask &= tmask - 1;
+          int j2 = -1;
+          if (tmask) {
+            j2 = tile * KC + __ffsll((long long)tmask) - 1;
+            tmask &= tmask - 1;
+          }
+          return Item{kMat, j1, j2};
+        }
+        in_tile = false;
         ++tile;
-        j = -1;
         continue;
       }
-      j = next_bit(c.keptU, j, nkb);
-      if (j < nkb) return Item{kExact, j++};
-      return Item{kNone, 0};
+      while (!kmask) {
+        if (++word >= (nkb + 31) / 32) return Item{kNone, 0};
+        kmask = c.keptU[word];
+      }
+      const int j = word * 32 + __ffs(kmask) - 1;
+      kmask &= kmask - 1;
+      return Item{kExact, j};
     }
-  }
-  // First set bit at index >= from (and < end), else end.
-  static SA_DEVI int next_bit(const uint32_t* bits, int from, int end) {
-    while (from < end) {
-      const uint32_t w = bits[from >> 5] >> (from & 31);
-      if (w) return min(end, from + __ffs(w) - 1);
-      from = (from | 31) + 1;
-    }
-    return end;
   }
 };
 
@@ -248,10 +252,17 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
   float* red = reinterpret_cast<float*>(gbase + OFF_RED);       // max [2][2][TQ], sum [2][TQ]
   __half* stash = reinterpret_cast<__half*>(gbase + OFF_STASH);  // [KC][TQ]
+  // One arrival per warp: every lane's tensor-memory stores are ordered before the
+  // warp barrier, and lane 0 arrives after it.
+  auto warp_arrive = [&](uint32_t b) {
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(b);
+  };
   const uint32_t pbar = bar(c.pair[qw]);
   int pair_phase = 0;
   auto pair_sync = [&]() {
-    tc::mbar_arrive(pbar);
+    warp_arrive(pbar);
     const bool r2 = uni(wt.fast(pbar, pair_phase & 1, 14));
     ++pair_phase;
     return r2;
@@ -283,8 +294,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     for (int k = 0; k < DH / 32; ++k) tc::tmem_st32(tmem + lane_off + COL_O + ch * DH + 32 * k, z);
     tc::tmem_wait_st();
   }
-  tc::fence_before_sync();
-  tc::mbar_arrive(bar(c.init_done));
+  warp_arrive(bar(c.init_done));
 
   float m_ref = -INFINITY, l = 0.f;
   // The last O-writing MMA issued before our next value product: kind 0 = value
@@ -381,8 +391,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       tc::tmem_st16(sa + col0 / 2 + 16 * k, pk);
     }
     tc::tmem_wait_st();
-    tc::fence_before_sync();
-    tc::mbar_arrive(bar(c.p_full[sb]));
+    warp_arrive(bar(c.p_full[sb]));
     if (TILE && !pair_sync()) return false;  // the partner's half of the stash is visible
     return true;
   };
@@ -417,8 +426,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
           tmem_st_w<AW>(ab + b * (D / 2), a);
         }
         tc::tmem_wait_st();
-        tc::fence_before_sync();
-        tc::mbar_arrive(bar(c.a_full[slot]));
+        warp_arrive(bar(c.a_full[slot]));
         lw_kind = 1;
         lw_buf = slot;
         lw_use = use;
@@ -426,10 +434,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       continue;
     }
     // ---- TILE or EXACT: logits in an S buffer ----
-    if (prev_buf >= 0) {
-      tc::fence_before_sync();
-      tc::mbar_arrive(bar(c.s_free[prev_buf]));
-    }
+    if (prev_buf >= 0) warp_arrive(bar(c.s_free[prev_buf]));
     const int n = ns++;
     const int sb = n & 1, use = n >> 1;
     prev_buf = sb;
@@ -515,17 +520,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(c.s_full[b]), 1);
       tc::mbar_init(bar(c.pv_done[b]), 1);
-      tc::mbar_init(bar(c.p_full[b]), NSOFT);
-      tc::mbar_init(bar(c.s_free[b]), NSOFT);
+      tc::mbar_init(bar(c.p_full[b]), NSOFT / 32);
+      tc::mbar_init(bar(c.s_free[b]), NSOFT / 32);
     }
     for (int a = 0; a < NA; ++a) {
       tc::mbar_init(bar(c.a_done[a]), 1);
-      tc::mbar_init(bar(c.a_full[a]), NSOFT);
+      tc::mbar_init(bar(c.a_full[a]), NSOFT / 32);
     }
     tc::mbar_init(bar(c.q_full), 1);
-    tc::mbar_init(bar(c.init_done), NSOFT);
+    tc::mbar_init(bar(c.init_done), NSOFT / 32);
     tc::mbar_init(bar(c.drain), 1);
-    for (int w = 0; w < 4; ++w) tc::mbar_init(bar(c.pair[w]), 64);
+    for (int w = 0; w < 4; ++w) tc::mbar_init(bar(c.pair[w]), 2);
     tc::fence_mbar_init();
     tc::fence_proxy_async();
   }
