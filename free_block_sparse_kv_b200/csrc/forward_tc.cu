@@ -12,7 +12,7 @@
 //   warps 0-7  softmax. Warps w and w+4 share TMEM lanes 32*(w%4).. (query rows) and
 //              split each row's columns in halves; they exchange row maxima and row
 //              sums through shared memory. They read logits from TMEM, keep the running
-//              max (rescaling O lazily, only when a row's max grows by more than 2^8),
+//              max (rescaling O lazily, only when a row's max grows by more than 2^11),
 //              write P back to TMEM as the A operand of the value product, and build the
 //              order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
 //   warp 8     TMA producer: Q once, then every operand tile through a 4 x 32 KB ring.
@@ -55,7 +55,7 @@ constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA
 constexpr int kRegCtl = 72, kRegSoft = 208;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
 constexpr int NA = 2;          // A-operand slots for the order-1 products (each holds a pair)
-constexpr float kThresh = 8.0f;  // lazy-rescale threshold, base-2 units
+constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
 constexpr uint32_t COL_O = 0, COL_R0 = 128, COL_A0 = 384;
@@ -336,12 +336,24 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
         if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits[k] = 0u;
       }
     }
-    float mx = -INFINITY;
+    // Logits in base-2 units; masked columns become -inf, which the exponential maps
+    // to an exact zero, so the second pass needs no per-column tests.
+    float xv[NH];
 #pragma unroll
     for (int k = 0; k < NK; ++k)
 #pragma unroll
       for (int i = 0; i < 32; ++i)
-        if ((mbits[k] >> i) & 1u) mx = fmaxf(mx, __uint_as_float(sv[32 * k + i]) * sl2);
+        xv[32 * k + i] = ((mbits[k] >> i) & 1u) ? __uint_as_float(sv[32 * k + i]) * sl2 : -INFINITY;
+    float mx;
+    {
+      float m8[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) m8[a] = xv[a];
+#pragma unroll
+      for (int i = 8; i < NH; ++i) m8[i % 8] = fmaxf(m8[i % 8], xv[i]);
+      mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    }
     float* rmax = red + (n & 1) * 2 * TQ;
     rmax[ch * TQ + r] = mx;
     if (!pair_sync()) return false;
@@ -369,26 +381,35 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     }
     // P = 2^(x - m_ref) as fp16 pairs over the logits of both halves (all of them were
     // read before the pair met, so the writes cannot overtake a partner's read).
-    const float wlast = (float)(p.Nk - (nkb - 1) * BLK);
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+    // TILE: column of the possibly partial last block within this half, and its P
+    const int jl = TILE ? nkb - 1 - (it.j * KC + col0) : -1;
+    float plast = 0.f;
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        const float x0 = ((mbits[k] >> i) & 1u) ? tc::ex2(__uint_as_float(sv[32 * k + i]) * sl2 - m_ref) : 0.f;
-        const float x1 =
-            ((mbits[k] >> (i + 1)) & 1u) ? tc::ex2(__uint_as_float(sv[32 * k + i + 1]) * sl2 - m_ref) : 0.f;
+        const float x0 = tc::ex2(xv[32 * k + i] - m_ref);
+        const float x1 = tc::ex2(xv[32 * k + i + 1] - m_ref);
+        l4[(i / 2) & 3] += x0 + x1;
+        pk[i / 2] = pack_f16(x0, x1);
         if (TILE) {
-          const int j = it.j * KC + col0 + 32 * k + i;
-          l += x0 * (j == nkb - 1 ? wlast : (float)BLK) + x1 * (j + 1 == nkb - 1 ? wlast : (float)BLK);
           stash[(col0 + 32 * k + i) * TQ + r] = __float2half_rn(x0);
           stash[(col0 + 32 * k + i + 1) * TQ + r] = __float2half_rn(x1);
-        } else {
-          l += x0 + x1;
+          plast = (32 * k + i == jl) ? x0 : ((32 * k + i + 1 == jl) ? x1 : plast);
         }
-        pk[i / 2] = pack_f16(x0, x1);
       }
       tc::tmem_st16(sa + col0 / 2 + 16 * k, pk);
+    }
+    if (TILE) {
+      // order-0 denominator weight n_j: b for every block but a partial last one
+      float lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      lt *= (float)BLK;
+      lt += plast * (float)(p.Nk - nkb * BLK);
+      l += lt;
+    } else {
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
     }
     tc::tmem_wait_st();
     warp_arrive(bar(c.p_full[sb]));
