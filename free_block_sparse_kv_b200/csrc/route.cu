@@ -11,13 +11,10 @@
 //   1. Scores s_ij = scale * qbar_i . kbar_j in fp32: thread j streams column j of
 //      the dim-major centroid table (coalesced), the 8 qbar rows are broadcast from
 //      shared memory.
-//   2. One warp per query block selects. Each block gets the 48-bit key
-//      (order-preserving bits of s) << 16 | (0xFFFF - j), so that larger keys come
-//      first in the order (s descending, j ascending) and all keys differ. A
-//      most-significant-bit-first search finds the threshold key T:
-//        top-k:  the largest T with #{key >= T} >= k   (the k-th key)
-//        mass:   the largest T with sum_{key >= T} e^(s - max) >= tau * Z
-//      and the kept set is {key >= T}, written in ascending j with ballots.
+//   2. One warp per query block selects (select_row): a 32-step search over
+//      order-preserving score keys held in registers finds the threshold, ties at
+//      the threshold are taken in ascending block index, and the kept indices are
+//      written in ascending order with ballots.
 #include "common.cuh"
 #include "launch.h"
 
@@ -26,11 +23,111 @@ namespace sa {
 constexpr int kRouteRows = 8;      // query blocks per CTA (one warp each)
 constexpr int kRouteThreads = 256;
 
-SA_DEVI uint64_t route_key(float s, int j) {
-  return ((uint64_t)float_key(s) << 16) | (uint64_t)(0xFFFF - j);
+
+// One warp selects the kept blocks of one query block from its scores s[0..nkb).
+// Lane l holds blocks j = l + 32 i (i < SLOTS) as order-preserving 32-bit keys.
+//   1. MSB-first search over 32 key bits for the threshold key T:
+//        top-k: the largest T with #{key >= T} >= k;
+//        mass:  the largest T with sum_{key >= T} e^(s - max) >= tau * Z.
+//   2. Every block with key > T is kept; blocks with key == T (ties) are taken in
+//      ascending j until the count (top-k) or the mass (mass rule) is reached, so the
+//      order is (score descending, index ascending).
+//   3. Kept indices are written in ascending j with ballots.
+template <int SLOTS>
+SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, int32_t* out,
+                        int32_t* cnt_out, int cap, int lane) {
+  uint32_t key[SLOTS];
+  float e[SLOTS];
+#pragma unroll
+  for (int i = 0; i < SLOTS; ++i) {
+    const int j = lane + 32 * i;
+    key[i] = j < nkb ? float_key(s[j]) : 0u;  // 0 sorts below every real score
+  }
+  float goal = 0.f;
+  if (mode == 1) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i)
+      if (lane + 32 * i < nkb) mx = fmaxf(mx, s[lane + 32 * i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float z = 0.f;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) {
+      e[i] = lane + 32 * i < nkb ? expf(s[lane + 32 * i] - mx) : 0.f;
+      z += e[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    goal = tau * z;
+  }
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    if (mode == 0) {
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < SLOTS; ++i) c += key[i] >= cand;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= keep) T = cand;
+    } else {
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < SLOTS; ++i) m += key[i] >= cand ? e[i] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+      if (m >= goal) T = cand;
+    }
+  }
+  // what the strictly larger keys already give
+  int above = 0;
+  float mabove = 0.f;
+#pragma unroll
+  for (int i = 0; i < SLOTS; ++i) {
+    above += key[i] > T;
+    if (mode == 1) mabove += key[i] > T ? e[i] : 0.f;
+  }
+  above = __reduce_add_sync(0xffffffffu, above);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mabove += __shfl_xor_sync(0xffffffffu, mabove, o);
+  // walk the ties in ascending j; write every kept index in ascending j
+  const unsigned lt = (1u << lane) - 1u;
+  int off = 0, ties = 0;
+  float tmass = 0.f;
+  bool done = false;  // the tie quota is filled
+#pragma unroll
+  for (int i = 0; i < SLOTS; ++i) {
+    const bool tie = key[i] == T && lane + 32 * i < nkb;
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    bool take_tie = false;
+    if (mode == 0) {
+      take_tie = tie && (ties + __popc(tb & lt)) < keep - above;
+      ties += __popc(tb);
+    } else {
+      // inclusive prefix of tie masses in j order
+      float x = tie ? e[i] : 0.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const float before = tmass + x - (tie ? e[i] : 0.f);
+      take_tie = tie && !done && (mabove + before < goal);
+      tmass += __shfl_sync(0xffffffffu, x, 31);
+      done = done || (mabove + tmass >= goal);
+    }
+    const bool in = key[i] > T || take_tie;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const int pos = off + __popc(bal & lt);
+      if (pos < cap) out[pos] = lane + 32 * i;
+    }
+    off += __popc(bal);
+  }
+  if (lane == 0) *cnt_out = min(off, cap);
 }
 
-template <int D>
+template <int D, int SLOTS>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, int nqb, int nkb,
              int mode, int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
@@ -38,7 +135,6 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
   extern __shared__ __align__(16) float rsm[];
   float* qs = rsm;                         // [D][kRouteRows]
   float* sc = rsm + D * kRouteRows;        // [kRouteRows][nkb] scores
-  float* ex = sc + kRouteRows * nkb;       // [kRouteRows][nkb] e^(s - max) (mass mode)
   const int tid = threadIdx.x;
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * kRouteRows;
@@ -76,64 +172,15 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
 
   const int warp = tid / 32, lane = tid % 32;
   if (warp >= rows) return;
-  const float* s = sc + warp * nkb;
-  const size_t row = (size_t)bh * nqb + i0 + warp;
-
-  uint64_t prefix = 0;
-  if (mode == 0) {
-    for (int bit = 47; bit >= 0; --bit) {
-      const uint64_t cand = prefix | (1ull << bit);
-      int cnt = 0;
-      for (int j = lane; j < nkb; j += 32) cnt += route_key(s[j], j) >= cand;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= keep) prefix = cand;
-    }
-  } else {
-    float mx = -INFINITY;
-    for (int j = lane; j < nkb; j += 32) mx = fmaxf(mx, s[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float* e = ex + warp * nkb;
-    float z = 0.f;
-    for (int j = lane; j < nkb; j += 32) {
-      const float w = expf(s[j] - mx);
-      e[j] = w;
-      z += w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    const float goal = tau * z;
-    __syncwarp();
-    for (int bit = 47; bit >= 0; --bit) {
-      const uint64_t cand = prefix | (1ull << bit);
-      float m = 0.f;
-      for (int j = lane; j < nkb; j += 32)
-        if (route_key(s[j], j) >= cand) m += e[j];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
-      if (m >= goal) prefix = cand;
-    }
-  }
-
-  int32_t* out = kv_idx + row * cap;
-  int off = 0;
-  for (int base = 0; base < nkb; base += 32) {
-    const int j = base + lane;
-    const bool in = j < nkb && route_key(s[j], j) >= prefix;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (in) {
-      const int pos = off + __popc(bal & ((1u << lane) - 1u));
-      if (pos < cap) out[pos] = j;
-    }
-    off += __popc(bal);
-  }
-  if (lane == 0) kv_cnt[row] = min(off, cap);
+  select_row<SLOTS>(sc + warp * nkb, nkb, mode, keep, tau,
+                    kv_idx + ((size_t)bh * nqb + i0 + warp) * cap, kv_cnt + (size_t)bh * nqb + i0 + warp,
+                    cap, lane);
 }
 
-template <int D>
+template <int D, int SLOTS>
 static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
-  const size_t smem = (size_t)(D * kRouteRows + 2 * kRouteRows * p.nkb) * sizeof(float);
-  auto kern = route_kernel<D>;
+  const size_t smem = (size_t)(D * kRouteRows + kRouteRows * p.nkb) * sizeof(float);
+  auto kern = route_kernel<D, SLOTS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nqb + kRouteRows - 1) / kRouteRows, p.B * p.H);
@@ -142,9 +189,19 @@ static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_route_d(const RouteArgs& p, cudaStream_t st) {
+  if (p.nkb <= 128) return launch_route_t<D, 4>(p, st);
+  if (p.nkb <= 256) return launch_route_t<D, 8>(p, st);
+  if (p.nkb <= 512) return launch_route_t<D, 16>(p, st);
+  if (p.nkb <= 1024) return launch_route_t<D, 32>(p, st);
+  if (p.nkb <= 2048) return launch_route_t<D, 64>(p, st);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st) {
-  if (p.d == 64) return launch_route_t<64>(p, st);
-  if (p.d == 128) return launch_route_t<128>(p, st);
+  if (p.d == 64) return launch_route_d<64>(p, st);
+  if (p.d == 128) return launch_route_d<128>(p, st);
   return cudaErrorInvalidValue;
 }
 

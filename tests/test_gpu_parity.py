@@ -341,3 +341,32 @@ def test_repeat_calls_are_bitwise_deterministic(small_inputs):
     a = a.clone()
     _, b = _run(w, q, k, v)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("mode", ["topk", "mass"])
+def test_route_exact_ties_break_by_lower_index(mode):
+    """Key blocks duplicated pairwise give bit-identical centroids, hence exactly tied
+    scores on both sides; the kept sets must then match the oracle on every row,
+    including rows whose cutoff falls inside a tie."""
+    B, H, d, block, nkb = 1, 2, 64, 64, 40
+    N = nkb * block
+    rng = np.random.default_rng(7)
+    kb = np.empty((B, H, N, d), np.uint16)
+    for h in range(H):
+        base = rng.standard_normal((nkb // 2, block, d)).astype(np.float32)
+        blocks = np.repeat(base, 2, axis=0)          # block 2m and 2m+1 identical
+        kb[0, h] = W.bf16_round(blocks.reshape(N, d))[1]
+    qb = _rand_bits((B, H, N, d), 8)
+    vb = _rand_bits((B, H, N, d), 9)
+    w = W.Workload(name="ties", B=B, H=H, Nq=N, Nk=N, d=d, block=block, order=0, mode=mode,
+                   rho=(7, 40), tau=0.6)
+    op, _ = _run(w, _dev(qb), _dev(kb), _dev(vb))
+    idx, cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
+    for h in range(H):
+        q, k = W.bits_to_f32(qb[0, h]), W.bits_to_f32(kb[0, h])
+        if mode == "topk":
+            kept = O.route_head(q, k, block, "topk", w.scale, keep=w.keep())[0]
+        else:
+            kept = O.route_head(q, k, block, "mass", w.scale, tau=w.tau)[0]
+        got = lists_to_sets(idx[0, h], cnt[0, h])
+        assert got == [x.tolist() for x in kept], (mode, h)
