@@ -91,7 +91,7 @@ def pool_bytes(w: W.Workload, with_q: bool) -> float:
     and the fp16 copy of V."""
     bh = w.B * w.H
     rd = bh * w.Nk * w.d * 2 * 2 + (bh * w.Nq * w.d * 2 if with_q else 0)
-    wr = bh * w.nkb * w.d * (4 + 4 + 2 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
+    wr = bh * w.nkb * w.d * (4 + 4 + 4 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
     wr += bh * w.Nk * w.d * 2   # fp16 copy of V
     if w.order == 1:
         wr += bh * w.nkb * w.d * w.d * 2

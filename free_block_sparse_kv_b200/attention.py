@@ -21,7 +21,7 @@ class Tables:
     qbar: torch.Tensor      # [B,H,nqb,d] fp32
     kbar_t: torch.Tensor    # [B,H,d,nkb] fp32
     vsum: torch.Tensor      # [B,H,nkb,d] fp32
-    kbar16: torch.Tensor    # [B,H,nkb,d] fp16
+    kbar16: torch.Tensor    # [B,H,2,nkb,d] bf16: centroid hi and lo parts
     vsum16: torch.Tensor    # [B,H,nkb,d] fp16
     M: Optional[torch.Tensor]  # [B,H,nkb,d,d] fp16 (order 1)
     v16: torch.Tensor       # [B,H,Nk,d] fp16 copy of V
@@ -53,7 +53,7 @@ def allocate_tables(p: Problem, device) -> Tables:
         qbar=torch.empty(p.B, p.H, p.nqb, p.d, **f32),
         kbar_t=torch.empty(p.B, p.H, p.d, p.nkb, **f32),
         vsum=torch.empty(p.B, p.H, p.nkb, p.d, **f32),
-        kbar16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
+        kbar16=torch.empty(p.B, p.H, 2, p.nkb, p.d, dtype=torch.bfloat16, device=device),
         vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
         M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **h16) if p.order == 1 else None,
         v16=torch.empty(p.B, p.H, p.Nk, p.d, **h16),

@@ -84,7 +84,7 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
   sizes[0] = bh * nqb * d * sizeof(float);
   sizes[1] = bh * nkb * d * sizeof(float);
   sizes[2] = bh * nkb * d * sizeof(float);
-  sizes[3] = bh * nkb * d * 2;
+  sizes[3] = bh * 2 * nkb * d * 2;
   sizes[4] = bh * nkb * d * 2;
   sizes[5] = order == 1 ? bh * nkb * d * d * 2 : 0;
   sizes[6] = bh * (size_t)Nk * d * 2;

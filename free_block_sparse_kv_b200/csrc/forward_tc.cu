@@ -15,11 +15,12 @@
 //              max (rescaling O lazily, only when a row's max grows by more than 2^11),
 //              write P back to TMEM as the A operand of the value product, and build the
 //              order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
-//   warp 8     TMA producer: Q once, then every operand tile through a 4 x 32 KB ring.
+//   warp 8     TMA producer: Q once, then every operand tile through a 5 x 32 KB ring.
 //   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
 //   warps 10-11 idle (they complete the control warpgroup for the register split).
 // Work items, in order (the same walk runs in all three roles):
-//   TILE t   64 centroids (fp16) and value sums (fp16): S = Q16 Kbar^T, P, O += P S
+//   TILE t   64 centroids (bf16 hi + lo) and value sums (fp16):
+//            S = Q Kbar_hi^T + Q Kbar_lo^T, P, O += P S
 //   MAT j    each pair of skipped blocks of the current tile (order 1):
 //            O += [A_j1 | A_j2] [M_j1; M_j2] (fp16)
 //   EXACT j  each kept block: S = Q K_j^T (bf16), P, O += P V_j (fp16 P and V)
@@ -45,7 +46,7 @@ namespace tcf {
 
 constexpr int TQ = 128;        // query rows per CTA
 constexpr int KC = 64;         // centroids per TILE item
-constexpr int NU = 4;          // ring units
+constexpr int NU = 5;          // ring units
 constexpr int UNIT = 32768;    // bytes per ring unit
 constexpr int MAXW = 64;       // bitmap words (2048 blocks)
 constexpr int NSOFT = 256;     // softmax threads (8 warps, 2 warpgroups)
@@ -54,7 +55,7 @@ constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA
 // control warpgroup gives registers back, the softmax warpgroups take them.
 constexpr int kRegCtl = 72, kRegSoft = 208;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
-constexpr int NA = 2;          // A-operand slots for the order-1 products (each holds a pair)
+constexpr int NA = 3;          // A-operand slots for the order-1 products (each holds a pair)
 constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
@@ -62,8 +63,7 @@ constexpr uint32_t COL_O = 0, COL_R0 = 128, COL_A0 = 384;
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr int OFF_Q = 0;                       // Q tile, bf16, swizzled (32 KB)
-constexpr int OFF_Q16 = 32768;                 // Q tile, fp16, swizzled (32 KB)
-constexpr int OFF_U = 65536;                   // ring
+constexpr int OFF_U = 32768;                   // ring
 constexpr int OFF_CTL = OFF_U + NU * UNIT;     // control block (2 KB)
 constexpr int OFF_STASH = OFF_CTL + 2048;      // P of the current tile, fp16 [KC][TQ]
 constexpr int OFF_RED = OFF_STASH + KC * TQ * 2;  // row max (2 x 2 x TQ) and sum (2 x TQ), f32
@@ -154,7 +154,9 @@ struct Walk {
   }
 };
 
-// MMA-side event stream: S(next TILE/EXACT) is issued before PV(current).
+// MMA-side event stream. The logits of the next TILE/EXACT item are issued before
+// the value product of the current one (look-ahead), except after an order-1 TILE:
+// there they follow the tile's order-1 products, which use the other S/P buffer.
 enum : int { eS = 0, ePV = 1, eMat = 2, eNone = 3 };
 struct Event {
   int kind;   // eS, ePV, eMat, eNone
@@ -166,8 +168,8 @@ struct EventGen {
   Walk cur, ahead;
   int ns_ahead = 0, ns_cur = 0, nmat = 0, tile_buf = 0;
   bool started = false;
-  Event pend;
-  bool has_pend = false;
+  Event q0, q1;  // queued events (at most two)
+  int nq = 0;
 
   template <int ORDER>
   SA_DEVI Item next_s(const Ctl& c, int nkb) {
@@ -178,9 +180,11 @@ struct EventGen {
   }
   template <int ORDER>
   SA_DEVI Event next(const Ctl& c, int nkb) {
-    if (has_pend) {
-      has_pend = false;
-      return pend;
+    if (nq) {
+      const Event e = q0;
+      q0 = q1;
+      --nq;
+      return e;
     }
     if (!started) {
       started = true;
@@ -198,18 +202,43 @@ struct EventGen {
     const int n = ns_cur++;
     if (it.kind == kTile) tile_buf = n & 1;
     const Event pv{ePV, it, n & 1, n >> 1, 0};
-    Item s = next_s<ORDER>(c, nkb);
-    if (s.kind == kNone) return pv;
-    const int m = ns_ahead++;
-    pend = pv;
-    has_pend = true;
-    return Event{eS, s, m & 1, m >> 1, 0};
+    Event first = pv;
+    bool have_first = false;
+    if (ns_ahead <= n) {  // this item's logits were deferred
+      const Item s = next_s<ORDER>(c, nkb);
+      const int m = ns_ahead++;
+      first = Event{eS, s, m & 1, m >> 1, 0};
+      have_first = true;
+    }
+    if (!(ORDER == 1 && it.kind == kTile)) {
+      const Item s = next_s<ORDER>(c, nkb);
+      if (s.kind != kNone) {
+        const int m = ns_ahead++;
+        const Event la{eS, s, m & 1, m >> 1, 0};
+        if (have_first) {
+          q0 = la;
+          nq = 1;
+        } else {
+          first = la;
+          have_first = true;
+        }
+      }
+    }
+    if (have_first) {
+      if (nq == 0) q0 = pv; else q1 = pv;
+      ++nq;
+    }
+    return first;
   }
 };
 
 // TMEM column of A slot `slot` (128 columns: the operands of two skipped blocks) for a
-// tile whose S/P buffer is `tbuf`. Slot 1 reuses that buffer once its P has been read.
-SA_DEVI uint32_t a_col(int slot, int tbuf) { return slot == 0 ? COL_A0 : COL_R0 + 128 * tbuf; }
+// tile whose S/P buffer is `tbuf`. Slot 1 reuses that buffer once its P has been read;
+// slot 2 is the other S/P buffer, left free during a tile's order-1 products (the
+// logits of the next item are issued after them).
+SA_DEVI uint32_t a_col(int slot, int tbuf) {
+  return slot == 0 ? COL_A0 : COL_R0 + 128 * (slot == 1 ? tbuf : 1 - tbuf);
+}
 
 template <int D, int BLK>
 struct Bytes {
@@ -269,7 +298,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   };
 
   bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
-  // fp16 copy of this thread's half of its Q row: registers and the swizzled Q16 tile
+  // fp16 copy of this thread's half of its Q row, in registers (order-1 operands)
   uint32_t q16[AW];
 #pragma unroll
   for (int i = 0; i < 4 * SUB; ++i) {
@@ -279,7 +308,6 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
     const uint4 y = make_uint4(bf16x2_to_f16x2(x.x), bf16x2_to_f16x2(x.y), bf16x2_to_f16x2(x.z),
                                bf16x2_to_f16x2(x.w));
-    *reinterpret_cast<uint4*>(gbase + OFF_Q16 + off) = y;
     q16[4 * i + 0] = y.x;
     q16[4 * i + 1] = y.y;
     q16[4 * i + 2] = y.z;
@@ -625,9 +653,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
           break;
         }
         if (e.kind == eS && it.kind == kTile) {
-          tc::mbar_arrive_expect_tx(fb, By::KB);
-          for (int s = 0; s < SUB; ++s)
-            tc::tma_load_3d(dst + s * KC * 128, &p.tmKb, fb, 64 * s, it.j * KC, bh);
+          tc::mbar_arrive_expect_tx(fb, 2 * By::KB);
+          for (int pl = 0; pl < 2; ++pl)
+            for (int s = 0; s < SUB; ++s)
+              tc::tma_load_3d(dst + pl * By::KB + s * KC * 128, &p.tmKb, fb, 64 * s, it.j * KC,
+                              2 * bh + pl);
         } else if (e.kind == ePV && it.kind == kTile) {
           tc::mbar_arrive_expect_tx(fb, By::VS);
           for (int s = 0; s < SUB; ++s)
@@ -663,7 +693,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   } else if (warp == 9) {
     // =========================== MMA issuer ===========================
     if (lane == 0) {
-      constexpr uint32_t I_S_TILE = tc::idesc_f16(0, 0, 0, KC);
+      constexpr uint32_t I_S_TILE = tc::idesc_f16(1, 1, 0, KC);
       constexpr uint32_t I_PV_TILE = tc::idesc_f16(0, 0, 1, D);
       constexpr uint32_t I_S_EX = tc::idesc_f16(1, 1, 0, BLK);
       constexpr uint32_t I_PV_EX = tc::idesc_f16(0, 0, 1, D);
@@ -671,7 +701,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
       tc::fence_after_sync();
       // Descriptor bases; per k-step only the start-address field (low bits) moves.
-      const uint64_t dQ = tc::sdesc(base + OFF_Q, 16, 1024), dQ16 = tc::sdesc(base + OFF_Q16, 16, 1024);
+      const uint64_t dQ = tc::sdesc(base + OFF_Q, 16, 1024);
       for (int u = 0; ok; ++u) {
         const int slot = u % NU;
         ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
@@ -688,16 +718,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
           tc::fence_after_sync();
           const uint32_t dt = tmem + COL_R0 + 128 * buf;
           const bool tile = ikind == kTile;
-          const uint64_t ad0 = tile ? dQ16 : dQ;
           const int rows = tile ? KC : BLK;
           const uint64_t bd0 = tc::sdesc(src, 16, 1024);
           const uint32_t idesc = tile ? I_S_TILE : I_S_EX;
+          // tile: the hi plane, then the lo plane of the centroids, into the same logits
+          const int planes = tile ? 2 : 1;
+          for (int pl = 0; pl < planes; ++pl)
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
-            const uint32_t boff = ((kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
-            tc::mma_ss(dt, ad0 + aoff, bd0 + boff, idesc, kk > 0);
-          }
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
+              const uint32_t boff = (pl * By::KB + (kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
+              tc::mma_ss(dt, dQ + aoff, bd0 + boff, idesc, (pl | kk) > 0);
+            }
           tc::mma_commit(bar(c.s_full[buf]));
         } else if (kind == ePV) {
           ok = wt.fast(bar(c.p_full[buf]), use & 1, 6);
@@ -790,7 +822,7 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   bool ok = map3d(&p.tmQ, BF, a.q, D, a.Nq, bh, TQ) && map3d(&p.tmK, BF, a.k, D, a.Nk, bh, BLK) &&
             map3d(&p.tmV, HF, a.v, D, a.Nk, bh, BLK) &&
-            map3d(&p.tmKb, HF, a.kbar16, D, a.nkb, bh, KC) &&
+            map3d(&p.tmKb, BF, a.kbar16, D, a.nkb, 2 * bh, KC) &&
             map3d(&p.tmVs, HF, a.vsum16, D, a.nkb, bh, KC);
   if (ORDER == 1) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh * a.nkb, D);
   else p.tmM = p.tmVs;

@@ -122,8 +122,11 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
       const float mean = s / (float)n;
       ks[c] = mean;
       kbar_t[((size_t)bh * D + c) * nkb + j] = mean;
-      __half h = __float2half_rn(mean);
-      kbar16[row] = *reinterpret_cast<uint16_t*>(&h);
+      // bf16 hi/lo split: hi = rn(mean), lo = rn(mean - hi); plane 0 then plane 1
+      const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
+      kbar16[((size_t)(2 * bh) * nkb + j) * D + c] = *reinterpret_cast<const uint16_t*>(&hi);
+      kbar16[((size_t)(2 * bh + 1) * nkb + j) * D + c] = *reinterpret_cast<const uint16_t*>(&lo);
     } else {
       vs[c] = s;
       vsum[row] = s;

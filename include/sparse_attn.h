@@ -77,15 +77,18 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
  *   qbar    [B,H,nqb,d]  fp32   mean of each query block's rows
  *   kbar_t  [B,H,d,nkb]  fp32   block centroids, dim-major (routing reads it)
  *   vsum    [B,H,nkb,d]  fp32   value sums S_j
- *   kbar16  [B,H,nkb,d]  fp16   centroids, rounded to nearest (forward reads it)
+ *   kbar16  [B,H,2,nkb,d] bf16  centroids as hi + lo: plane 0 = rn(kbar), plane 1 =
+ *                               rn(kbar - hi); hi + lo carries ~16 significant bits
+ *                               (forward reads it)
  *   vsum16  [B,H,nkb,d]  fp16   value sums, rounded to nearest (forward reads it)
  *   M       [B,H,nkb,d,d] fp16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
  *                               a = key dim (rows), c = value dim; fp32 accumulate
  *   v16     [B,H,Nk,d]   fp16   V converted to fp16 (exact for |v| in the fp16
  *                               normal range; |v| must stay below 65504)
- * The 16-bit tables are IEEE fp16 (11-bit significand): the forward runs every
- * product that involves probabilities in fp16 with fp32 accumulation; the
- * logits of kept tokens use the bf16 Q and K as given.
+ * vsum16, M and v16 are IEEE fp16 (11-bit significand): the forward runs every
+ * product that involves probabilities in fp16 with fp32 accumulation. Logits use
+ * the bf16 Q against the bf16 K as given (kept tokens) or against both centroid
+ * planes (skipped blocks).
  * Means of a partial last block use its true token count.
  */
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,

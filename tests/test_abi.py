@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 def test_table_sizes():
     assert C.sparse_attn_table_sizes(1, 40, 75600, 75600, 128, 128, 1) == (
         40 * 591 * 128 * 4, 40 * 591 * 128 * 4, 40 * 591 * 128 * 4,
-        40 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2, 40 * 75600 * 128 * 2)
+        40 * 2 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2, 40 * 75600 * 128 * 2)
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[5] == 0
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[0] == 4 * 16 * 25 * 128 * 4
 

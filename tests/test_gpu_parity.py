@@ -86,8 +86,10 @@ def test_pool_matches_oracle(name, small_inputs):
             np.testing.assert_allclose(t.qbar[b, h].cpu().numpy(), qbar, rtol=0, atol=2e-6)
             np.testing.assert_allclose(t.kbar_t[b, h].cpu().numpy().T, kbar, rtol=0, atol=2e-6)
             np.testing.assert_allclose(t.vsum[b, h].cpu().numpy(), vsum, rtol=0, atol=2e-5)
-            k16 = t.kbar16[b, h].float().cpu().numpy()
-            np.testing.assert_allclose(k16, kbar, rtol=2 ** -10, atol=1e-6)
+            hi = t.kbar16[b, h, 0].double().cpu().numpy()
+            lo = t.kbar16[b, h, 1].double().cpu().numpy()
+            np.testing.assert_allclose(hi, kbar, rtol=2 ** -8, atol=1e-30)
+            np.testing.assert_allclose(hi + lo, kbar, rtol=2 ** -15, atol=1e-7)
             v16 = t.vsum16[b, h].float().cpu().numpy()
             np.testing.assert_allclose(v16, vsum, rtol=2 ** -10, atol=1e-5)
             v16 = t.v16[b, h].float().cpu().numpy()
