@@ -14,7 +14,6 @@ bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import math
 import os
@@ -230,30 +229,17 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
     from free_block_sparse_kv_b200 import attention as A
+    from free_block_sparse_kv_b200 import dist as D
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = D.env_ranks()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+    D.init("nccl", device=dev)
+    barrier = D.barrier
+    max_over_ranks = lambda x: D.max_over_ranks(x, device=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    wr = W.shrink(w, seed=w.seed + rank)   # weak scaling: each rank its own problem
+    wr = D.rank_workload(w, rank)   # weak scaling: each rank its own problem
     qb, kb, vb = W.full_inputs_bits(wr)
     as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
     q_h, k_h, v_h = (as_t(x).pin_memory() for x in (qb, kb, vb))
@@ -313,7 +299,7 @@ def main():
     pk = peaks()
     fwd_s = stage_ms[2] / 1e3
     achieved = fl["total"] / fwd_s / 1e12
-    value = world * w.dense_flops() / (ms_step_max / 1e3) / 1e12
+    value = D.weak_scaling_value(w.dense_flops(), world, ms_step_max)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -338,7 +324,7 @@ def main():
         e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps)
         h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
         d2h = out_h.numel() * out_h.element_size()
-        e2e = {"value": world * w.dense_flops() / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+        e2e = {"value": D.weak_scaling_value(w.dense_flops(), world, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cpu = None
@@ -378,7 +364,8 @@ def main():
         line["pool_roofline"]["frac"] = line["pool_roofline"]["achieved"] / pk["hbm"]
         print(json.dumps(line), flush=True)
     if world > 1:
-        dist.destroy_process_group()
+        import torch.distributed as tdist
+        tdist.destroy_process_group()
 
 
 if __name__ == "__main__":
