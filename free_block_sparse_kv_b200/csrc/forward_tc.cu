@@ -1,5 +1,6 @@
 // Forward pass on the 5th-generation tensor cores: tcgen05.mma with accumulators in
-// tensor memory, operands staged by TMA, one warp-specialised CTA per 128 query rows.
+// tensor memory, operands staged by TMA, one warp-specialised CTA per two tiles of
+// 128 query rows.
 //
 // Follows "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion
 // Transformers" §2: Algorithme Central (o_t = N_t / D_t; exact terms for the kept
@@ -8,29 +9,38 @@
 // tiles in on-chip memory, phase 2 a sweep over the aggregated block vectors, phase 3
 // the first-order correction), all merged into one online softmax.
 //
+// Two query tiles per CTA. Neighbouring query blocks skip mostly the same key blocks,
+// so every operand tile that TMA brings in (centroids, value sums, M_j, K_j, V_j)
+// serves both tiles: half the L2 traffic per tensor-core flop of one tile per CTA.
+// Each tile takes part only in the work items its own rows need.
+//
 // Roles (384 threads):
-//   warps 0-7  softmax. Warps w and w+4 share TMEM lanes 32*(w%4).. (query rows) and
-//              split each row's columns in halves; they exchange row maxima and row
-//              sums through shared memory. They read logits from TMEM, keep the running
-//              max (rescaling O lazily, only when a row's max grows by more than 2^11),
-//              write P back to TMEM as the A operand of the value product, and build the
-//              order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
-//   warp 8     TMA producer: Q once, then every operand tile through a 5 x 32 KB ring.
-//   warp 9     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
-//   warps 10-11 idle (they complete the control warpgroup for the register split).
-// Work items, in order (the same walk runs in all three roles):
-//   TILE t   64 centroids (bf16 hi + lo) and value sums (fp16):
-//            S = Q Kbar_hi^T + Q Kbar_lo^T, P, O += P S
-//   MAT j    each pair of skipped blocks of the current tile (order 1):
-//            O += [A_j1 | A_j2] [M_j1; M_j2] (fp16)
-//   EXACT j  each kept block: S = Q K_j^T (bf16), P, O += P V_j (fp16 P and V)
-// The MMA warp issues the logits of the next TILE/EXACT item before the value
-// product of the current one, so logits overlap the softmax of the previous item.
-// TMEM columns: O [0, D); S/P buffers R0 = [128, 256), R1 = [256, 384); A slot 0 at
-// [384, 512). Order-1 products go two skipped blocks at a time: A = [a1 q | a2 q]
-// (K = 2d) against [M_j1; M_j2], 16 tensor-core instructions per hand-off. During a
-// tile's MAT items the tile's S/P buffer is free once its value product has run (the
-// tile's P is also kept in shared memory for alpha) and serves as A slot 1.
+//   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: one thread per query
+//              row (TMEM lane 32*(w%4) + lane). They read logits from TMEM, keep the
+//              running max (rescaling O lazily, only when a row's max grows by more
+//              than 2^11), write P back to TMEM as the A operand of the value product,
+//              and build the order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
+//   warp 8     TMA producer: both Q tiles once, then every operand tile through a
+//              5 x 32 KB ring.
+//   warps 9-10 one MMA-issuing thread per tile (warp 9 also allocates TMEM). Issuing
+//              a 128x128x16 tcgen05.mma takes about as long as the tensor core takes to
+//              run it, so one thread cannot also wait and commit without leaving the
+//              pipe idle; two issuers keep it fed.
+//   warp 11    idle (it completes the control warpgroup for the register split).
+// TMEM columns: O_0 [0, 128), O_1 [128, 256); R_t = [256 + 128 t, 384 + 128 t) holds
+// tile t's logits, then its P (fp16), or two order-1 operands (two slots of d/2
+// columns, so that one is built while the other is in use).
+//
+// Work items, in order (the same walk runs in every role):
+//   TILE c   64 centroids (bf16 hi + lo) and value sums (fp16):
+//            S_t = Q_t Kbar_hi^T + Q_t Kbar_lo^T, P_t, O_t += P_t Vsum
+//   MAT j    each skipped block of the current centroid tile (order 1):
+//            O_t += A_t,j M_j (fp16)
+//   EXACT j  each kept block: S_t = Q_t K_j^T (bf16), P_t, O_t += P_t V_j (fp16)
+// For each tile, the value product of its last item and the logits of its next item
+// are issued back to back, so a tile's softmax runs while the other tile's products
+// run. Order-1 TILE items are an exception: their value product follows at once,
+// because R_t then holds A operands.
 // Every mbarrier wait is bounded: on timeout the CTA sets err_flag, abandons its work,
 // drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -44,30 +54,28 @@
 namespace sa {
 namespace tcf {
 
-constexpr int TQ = 128;        // query rows per CTA
+constexpr int TQ = 128;        // query rows per tile
+constexpr int NT = 2;          // tiles per CTA
 constexpr int KC = 64;         // centroids per TILE item
 constexpr int NU = 5;          // ring units
 constexpr int UNIT = 32768;    // bytes per ring unit
 constexpr int MAXW = 64;       // bitmap words (2048 blocks)
-constexpr int NSOFT = 256;     // softmax threads (8 warps, 2 warpgroups)
+constexpr int NSOFT = 256;     // softmax threads (2 warpgroups, one per tile)
 constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA, 2 idle)
 // Register split after launch (168 per thread at launch = 64,512 per CTA): the
 // control warpgroup gives registers back, the softmax warpgroups take them.
-constexpr int kRegCtl = 72, kRegSoft = 208;
+constexpr int kRegCtl = 120, kRegSoft = 192;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
-constexpr int NA = 3;          // A-operand slots for the order-1 products (each holds a pair)
 constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
-constexpr uint32_t COL_O = 0, COL_R0 = 128, COL_A0 = 384;
+constexpr uint32_t COL_O = 0, COL_R = 256;
 
 // shared-memory map (offsets from a 1024-aligned base)
-constexpr int OFF_Q = 0;                       // Q tile, bf16, swizzled (32 KB)
-constexpr int OFF_U = 32768;                   // ring
-constexpr int OFF_CTL = OFF_U + NU * UNIT;     // control block (2 KB)
-constexpr int OFF_STASH = OFF_CTL + 2048;      // P of the current tile, fp16 [KC][TQ]
-constexpr int OFF_RED = OFF_STASH + KC * TQ * 2;  // row max (2 x 2 x TQ) and sum (2 x TQ), f32
-constexpr int SMEM_BYTES = OFF_RED + 6 * TQ * 4 + 1024;
+constexpr int OFF_Q = 0;                        // Q tiles, bf16, swizzled (2 x 32 KB)
+constexpr int OFF_U = 65536;                    // ring
+constexpr int OFF_CTL = OFF_U + NU * UNIT;      // control block (2 KB)
+constexpr int SMEM_BYTES = OFF_CTL + 2048 + 1024;
 
 struct Params {
   CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmM;
@@ -81,33 +89,47 @@ struct Params {
 
 struct Ctl {  // control block in shared memory
   uint64_t full[NU], empty[NU];
-  uint64_t s_full[2], p_full[2], pv_done[2], s_free[2];
-  uint64_t a_full[NA], a_done[NA];
-  uint64_t q_full, init_done, drain;
-  uint64_t pair[4];         // the two softmax warps sharing 32 rows
-  int4 evq[NU];             // event of each ring unit: {kind | item kind << 4, j, buf | tbuf << 4, use}
+  uint64_t s_full[NT], p_full[NT], pv_done[NT], o_final[NT];
+  uint64_t a_full[NT][2], a_done[NT][2];  // order-1 operand slots of each tile
+  uint64_t q_full, init_done;
+  int4 evq[NU];             // step record of the first ring unit of each step
   uint32_t tmem_base;
   int abort;
-  uint32_t kept[2][MAXW];   // kept blocks of each query block in the tile (half)
-  uint32_t keptU[MAXW];     // union: EXACT items
-  uint32_t skipU[MAXW];     // union of skipped blocks: TILE / MAT items
+  int tvalid;               // bit t: tile t has rows below Nq
+  uint32_t kept[NT][2][MAXW];  // kept blocks of each query block (half) of each tile
 };
 static_assert(sizeof(Ctl) <= 2048, "control block");
 
 enum : int { kTile = 0, kMat = 1, kExact = 2, kNone = 3 };
 struct Item {
-  int kind, j;  // TILE: j = tile index; MAT / EXACT: j = block index
-  int j2 = -1;  // MAT: second skipped block of the pair, or -1
+  int kind, j;  // TILE: j = centroid-tile index; MAT / EXACT: j = block index
+  int mask;     // bit t: tile t takes part
 };
 
-// The walk over work items; identical in every role. The skipped blocks of the
-// current tile and the kept blocks of the current 32-block word are held in
-// registers as bit masks, so each step is a few integer instructions.
+SA_DEVI uint32_t valid_bits(int w, int nkb) {
+  const int lo = w * 32;
+  return lo + 32 <= nkb ? 0xffffffffu : (lo < nkb ? (1u << (nkb - lo)) - 1u : 0u);
+}
+// Blocks of word w that some query block of tile t skips / keeps.
+SA_DEVI uint32_t skip_word(const Ctl& c, int t, int w, int nkb) {
+  if (!((c.tvalid >> t) & 1)) return 0u;
+  return ~(c.kept[t][0][w] & c.kept[t][1][w]) & valid_bits(w, nkb);
+}
+SA_DEVI uint32_t kept_word(const Ctl& c, int t, int w, int nkb) {
+  if (!((c.tvalid >> t) & 1)) return 0u;
+  return (c.kept[t][0][w] | c.kept[t][1][w]) & valid_bits(w, nkb);
+}
+SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct, int nkb) {
+  return (uint64_t)skip_word(c, t, 2 * ct, nkb) | ((uint64_t)skip_word(c, t, 2 * ct + 1, nkb) << 32);
+}
+
+// The walk over work items; identical in every role. Union masks of the current
+// centroid tile (phase 0) or 32-block word (phase 1) are held in registers.
 struct Walk {
-  int phase = 0, tile = 0, word = 0;
-  uint64_t tmask = 0;  // phase 0: skipped blocks of `tile` not yet walked
-  uint32_t kmask = 0;  // phase 1: kept blocks of `word` not yet walked
+  int phase = 0, tile = 0, word = -1;
   bool in_tile = false;
+  uint64_t tmask = 0, sk0 = 0, sk1 = 0;  // phase 0: union / per-tile skipped blocks
+  uint32_t kmask = 0, kw0 = 0, kw1 = 0;  // phase 1: union / per-tile kept blocks
   template <int ORDER>
   SA_DEVI Item next(const Ctl& c, int nkb) {
     const int ntiles = (nkb + KC - 1) / KC;
@@ -116,139 +138,123 @@ struct Walk {
         if (!in_tile) {
           if (tile >= ntiles) {
             phase = 1;
-            word = 0;
-            kmask = c.keptU[0];
             continue;
           }
-          tmask = (uint64_t)c.skipU[2 * tile] | ((uint64_t)c.skipU[2 * tile + 1] << 32);
+          sk0 = skip64(c, 0, tile, nkb);
+          sk1 = skip64(c, 1, tile, nkb);
+          tmask = sk0 | sk1;
           if (tmask) {
             in_tile = true;
-            return Item{kTile, tile};
+            return Item{kTile, tile, (sk0 != 0) | ((sk1 != 0) << 1)};
           }
           ++tile;
           continue;
         }
-        if (ORDER == 1 && tmask) {
-          // skipped blocks of this tile, two at a time
-          const int j1 = tile * KC + __ffsll((long long)tmask) - 1;
+        if (ORDER == 1 && tmask) {  // skipped blocks of this centroid tile, one at a time
+          const int c1 = __ffsll((long long)tmask) - 1;
           tmask &= tmask - 1;
-          int j2 = -1;
-          if (tmask) {
-            j2 = tile * KC + __ffsll((long long)tmask) - 1;
-            tmask &= tmask - 1;
-          }
-          return Item{kMat, j1, j2};
+          return Item{kMat, tile * KC + c1, (int)((sk0 >> c1) & 1u) | (int)(((sk1 >> c1) & 1u) << 1)};
         }
         in_tile = false;
         ++tile;
         continue;
       }
       while (!kmask) {
-        if (++word >= (nkb + 31) / 32) return Item{kNone, 0};
-        kmask = c.keptU[word];
-      }
-      const int j = word * 32 + __ffs(kmask) - 1;
-      kmask &= kmask - 1;
-      return Item{kExact, j};
-    }
-  }
-};
-
-// MMA-side event stream. The logits of the next TILE/EXACT item are issued before
-// the value product of the current one (look-ahead), except after an order-1 TILE:
-// there they follow the tile's order-1 products, which use the other S/P buffer.
-enum : int { eS = 0, ePV = 1, eMat = 2, eNone = 3 };
-struct Event {
-  int kind;   // eS, ePV, eMat, eNone
-  Item item;
-  int buf, use;   // S / PV: S-buffer and its use count; MAT: A slot and its use count
-  int tbuf;       // MAT: S-buffer of the tile the block belongs to
-};
-struct EventGen {
-  Walk cur, ahead;
-  int ns_ahead = 0, ns_cur = 0, nmat = 0, tile_buf = 0;
-  bool started = false;
-  Event q0, q1;  // queued events (at most two)
-  int nq = 0;
-
-  template <int ORDER>
-  SA_DEVI Item next_s(const Ctl& c, int nkb) {
-    while (true) {
-      Item it = ahead.template next<ORDER>(c, nkb);
-      if (it.kind != kMat) return it;
-    }
-  }
-  template <int ORDER>
-  SA_DEVI Event next(const Ctl& c, int nkb) {
-    if (nq) {
-      const Event e = q0;
-      q0 = q1;
-      --nq;
-      return e;
-    }
-    if (!started) {
-      started = true;
-      Item s = next_s<ORDER>(c, nkb);
-      if (s.kind == kNone) return Event{eNone, s, 0, 0, 0};
-      const int n = ns_ahead++;
-      return Event{eS, s, n & 1, n >> 1, 0};
-    }
-    Item it = cur.template next<ORDER>(c, nkb);
-    if (it.kind == kNone) return Event{eNone, it, 0, 0, 0};
-    if (it.kind == kMat) {
-      const int n = nmat++;
-      return Event{eMat, it, n % NA, n / NA, tile_buf};
-    }
-    const int n = ns_cur++;
-    if (it.kind == kTile) tile_buf = n & 1;
-    const Event pv{ePV, it, n & 1, n >> 1, 0};
-    Event first = pv;
-    bool have_first = false;
-    if (ns_ahead <= n) {  // this item's logits were deferred
-      const Item s = next_s<ORDER>(c, nkb);
-      const int m = ns_ahead++;
-      first = Event{eS, s, m & 1, m >> 1, 0};
-      have_first = true;
-    }
-    if (!(ORDER == 1 && it.kind == kTile)) {
-      const Item s = next_s<ORDER>(c, nkb);
-      if (s.kind != kNone) {
-        const int m = ns_ahead++;
-        const Event la{eS, s, m & 1, m >> 1, 0};
-        if (have_first) {
-          q0 = la;
-          nq = 1;
-        } else {
-          first = la;
-          have_first = true;
+        if (++word >= (nkb + 31) / 32) {
+          word = (nkb + 31) / 32;  // stays at the end: later calls return kNone again
+          return Item{kNone, 0, 0};
         }
+        kw0 = kept_word(c, 0, word, nkb);
+        kw1 = kept_word(c, 1, word, nkb);
+        kmask = kw0 | kw1;
       }
+      const int b = __ffs(kmask) - 1;
+      kmask &= kmask - 1;
+      return Item{kExact, word * 32 + b, (int)((kw0 >> b) & 1u) | (int)(((kw1 >> b) & 1u) << 1)};
     }
-    if (have_first) {
-      if (nq == 0) q0 = pv; else q1 = pv;
-      ++nq;
-    }
-    return first;
   }
 };
 
-// TMEM column of A slot `slot` (128 columns: the operands of two skipped blocks) for a
-// tile whose S/P buffer is `tbuf`. Slot 1 reuses that buffer once its P has been read;
-// slot 2 is the other S/P buffer, left free during a tile's order-1 products (the
-// logits of the next item are issued after them).
-SA_DEVI uint32_t a_col(int slot, int tbuf) {
-  return slot == 0 ? COL_A0 : COL_R0 + 128 * (slot == 1 ? tbuf : 1 - tbuf);
+// Steps: what the producer loads into one or two ring units and the MMA threads then
+// issue. An SX step carries the value products of the previous TILE/EXACT item
+// ("pending", one per tile that took part) and the logits of the next one; its units
+// are [V or Vsum of the pending item] + [K or Kbar of the new item].
+enum : int { stSX = 0, stFlush = 1, stMat = 2, stEnd = 3 };
+struct Step {
+  int type, nunits;
+  int cur_kind, cur_mask, cur_j;     // SX: new TILE/EXACT item; MAT: the block
+  int pend_kind, pend_mask, pend_j;  // SX / FLUSH: item whose value products are due
+};
+struct StepGen {
+  Walk wk;
+  int pend_kind = 0, pend_mask = 0, pend_j = 0;
+  bool flush_next = false;
+  template <int ORDER>
+  SA_DEVI Step next(const Ctl& c, int nkb) {
+    if (flush_next) {  // order 1: a TILE's value products come before its MAT items
+      flush_next = false;
+      const Step s{stFlush, 1, 0, 0, 0, pend_kind, pend_mask, pend_j};
+      pend_mask = 0;
+      return s;
+    }
+    const Item it = wk.template next<ORDER>(c, nkb);
+    if (it.kind == kNone) {
+      if (pend_mask) {
+        const Step s{stFlush, 1, 0, 0, 0, pend_kind, pend_mask, pend_j};
+        pend_mask = 0;
+        return s;
+      }
+      return Step{stEnd, 1, 0, 0, 0, 0, 0, 0};
+    }
+    if (it.kind == kMat) return Step{stMat, 1, kMat, it.mask, it.j, 0, 0, 0};
+    const Step s{stSX, pend_mask ? 2 : 1, it.kind, it.mask, it.j, pend_kind, pend_mask, pend_j};
+    pend_kind = it.kind;
+    pend_mask = it.mask;
+    pend_j = it.j;
+    if (ORDER == 1 && it.kind == kTile) flush_next = true;
+    return s;
+  }
+};
+SA_DEVI int encode(const Step& s) {
+  return s.type | (s.cur_kind << 4) | (s.pend_kind << 8) | (s.cur_mask << 12) | (s.pend_mask << 14) |
+         (s.nunits << 16);
 }
 
 template <int D, int BLK>
 struct Bytes {
   static constexpr int SUB = D / 64;                    // 64-column sub-tiles per row
-  static constexpr uint32_t KB = SUB * KC * 128;        // centroid tile
+  static constexpr uint32_t KB = SUB * KC * 128;        // one plane of a centroid tile
   static constexpr uint32_t VS = SUB * KC * 128;        // value-sum tile
   static constexpr uint32_t M = SUB * D * 128;          // one M_j
   static constexpr uint32_t KV = SUB * BLK * 128;       // one K or V block
-  static constexpr uint32_t Q = SUB * TQ * 128;         // query tile
+  static constexpr uint32_t Q = SUB * TQ * 128;         // one query tile
 };
+
+// Element c (0..63) of a row's 64 fp16 probabilities held as 32 packed registers;
+// c is the same for every thread of the warp. A tree of selects on the bits of c
+// (inline PTX, so that the compiler does not turn it into an indexed load from local
+// memory).
+SA_DEVI uint32_t sel(bool p, uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("{\n .reg .pred q;\n setp.ne.u32 q, %3, 0;\n selp.b32 %0, %1, %2, q;\n}\n"
+      : "=r"(r) : "r"(a), "r"(b), "r"((uint32_t)p));
+  return r;
+}
+SA_DEVI float stash_get(const uint32_t* st, int c) {
+  const int i = c >> 1;
+  uint32_t l1[16], l2[8], l3[4], l4[2];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) l1[k] = sel(i & 1, st[2 * k + 1], st[2 * k]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) l2[k] = sel(i & 2, l1[2 * k + 1], l1[2 * k]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) l3[k] = sel(i & 4, l2[2 * k + 1], l2[2 * k]);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) l4[k] = sel(i & 8, l3[2 * k + 1], l3[2 * k]);
+  const uint32_t v = sel(i & 16, l4[1], l4[0]);
+  const uint16_t hv = (c & 1) ? (uint16_t)(v >> 16) : (uint16_t)(v & 0xffffu);
+  return __half2float(__ushort_as_half(hv));
+}
 
 // TMEM store of W consecutive 32-bit columns (W = 16 or 32).
 template <int W>
@@ -261,26 +267,25 @@ SA_DEVI void tmem_st_w(uint32_t taddr, const uint32_t* r) {
   }
 }
 
-// Softmax warps. Thread (warp w, lane l) owns query row r = 32*(w%4) + l and the
-// column half w/4 of every logit tile; the two threads of a row meet through an
-// mbarrier of their warp pair (bounded waits, so an abort never strands a partner).
+// Softmax warpgroup of tile t = warp / 4. Thread (warp w, lane l) owns query row
+// r = 32*(w%4) + l of the tile: all its logits, its running max and sum, its O row.
 template <int D, int BLK, int ORDER>
 SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem, tc::Waiter& wt,
                           int warp, int lane) {
-  constexpr int SUB = D / 64;
-  constexpr int DH = D / 2;  // O columns per thread
-  constexpr int AW = D / 4;  // A-operand columns (fp16 pairs) per thread
-  const int qw = warp & 3, ch = warp >> 2;
+  using By = Bytes<D, BLK>;
+  constexpr int QW = D / 2;  // fp16 pairs per query row
+  const int t = warp >> 2, qw = warp & 3;
   const int r = 32 * qw + lane;
   const uint32_t lane_off = (uint32_t)(32 * qw) << 16;
-  const int h = BLK == 64 ? (r >> 6) : 0;  // which query block of the tile
+  const uint32_t rt = tmem + lane_off + COL_R + 128 * t;  // logits / P / order-1 operand
+  const uint32_t ot = tmem + lane_off + COL_O + 128 * t;  // O rows
+  const int h = BLK == 64 ? (r >> 6) : 0;                  // query block of the row
   const float sl2 = p.scale * kLog2e;
   const int nkb = p.nkb;
-  const int bh = blockIdx.y, q0 = blockIdx.x * TQ;
+  const int bh = blockIdx.y, row0 = blockIdx.x * (NT * TQ) + t * TQ;
+  const uint32_t* kept_h = c.kept[t][h];
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
   auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
-  float* red = reinterpret_cast<float*>(gbase + OFF_RED);       // max [2][2][TQ], sum [2][TQ]
-  __half* stash = reinterpret_cast<__half*>(gbase + OFF_STASH);  // [KC][TQ]
   // One arrival per warp: every lane's tensor-memory stores are ordered before the
   // warp barrier, and lane 0 arrives after it.
   auto warp_arrive = [&](uint32_t b) {
@@ -288,236 +293,226 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(b);
   };
-  const uint32_t pbar = bar(c.pair[qw]);
-  int pair_phase = 0;
-  auto pair_sync = [&]() {
-    warp_arrive(pbar);
-    const bool r2 = uni(wt.fast(pbar, pair_phase & 1, 14));
-    ++pair_phase;
-    return r2;
-  };
 
   bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
-  // fp16 copy of this thread's half of its Q row, in registers (order-1 operands)
-  uint32_t q16[AW];
+  // fp16 copy of this thread's Q row, in registers (order-1 operands)
+  uint32_t q16[ORDER == 1 ? QW : 1];
+  if constexpr (ORDER == 1) {
 #pragma unroll
-  for (int i = 0; i < 4 * SUB; ++i) {
-    const int cc = ch * 4 * SUB + i;
-    const int s = cc / 8, cw = cc % 8;
-    const uint32_t off = s * TQ * 128 + r * 128 + ((cw ^ (r & 7)) << 4);
-    const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
-    const uint4 y = make_uint4(bf16x2_to_f16x2(x.x), bf16x2_to_f16x2(x.y), bf16x2_to_f16x2(x.z),
-                               bf16x2_to_f16x2(x.w));
-    q16[4 * i + 0] = y.x;
-    q16[4 * i + 1] = y.y;
-    q16[4 * i + 2] = y.z;
-    q16[4 * i + 3] = y.w;
+    for (int i = 0; i < QW / 4; ++i) {
+      const int s = i / 8, cw = i % 8;
+      const uint32_t off = t * By::Q + s * TQ * 128 + r * 128 + ((cw ^ (r & 7)) << 4);
+      const uint4 x = *reinterpret_cast<const uint4*>(gbase + OFF_Q + off);
+      q16[4 * i + 0] = bf16x2_to_f16x2(x.x);
+      q16[4 * i + 1] = bf16x2_to_f16x2(x.y);
+      q16[4 * i + 2] = bf16x2_to_f16x2(x.z);
+      q16[4 * i + 3] = bf16x2_to_f16x2(x.w);
+    }
   }
-  tc::fence_proxy_async();
   {
     uint32_t z[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) z[i] = 0u;
 #pragma unroll
-    for (int k = 0; k < DH / 32; ++k) tc::tmem_st32(tmem + lane_off + COL_O + ch * DH + 32 * k, z);
+    for (int k = 0; k < D / 32; ++k) tc::tmem_st32(ot + 32 * k, z);
     tc::tmem_wait_st();
   }
   warp_arrive(bar(c.init_done));
 
   float m_ref = -INFINITY, l = 0.f;
-  // The last O-writing MMA issued before our next value product: kind 0 = value
-  // product of S-buffer lw_buf, kind 1 = order-1 product of A slot lw_buf.
-  int lw_kind = -1, lw_buf = 0, lw_use = 0;
-  auto wait_last_writer = [&](int where) {
-    if (lw_kind < 0) return true;
-    const uint32_t b = lw_kind == 0 ? bar(c.pv_done[lw_buf]) : bar(c.a_done[lw_buf]);
-    const bool r2 = uni(wt.wait(b, lw_use & 1, where));
-    tc::fence_after_sync();
-    return r2;
-  };
+  int ns = 0;                // S items of this tile so far (s_full phases)
+  uint32_t stash[ORDER == 1 ? KC / 2 : 1];  // P of the current centroid tile, fp16 pairs
+  const uint64_t sl2x2 = tc::f2(sl2, sl2);
 
-  Walk wk;
-  int ns = 0, nmat = 0, cur_buf = 0, cur_use = 0, cur_tile = 0, prev_buf = -1;
-  bool r_slots_free = false;  // this tile's value product has read its P
-
-  // One TILE (IS_TILE, NH = 32) or EXACT (NH = BLK / 2) item: this thread's NH logits.
-  auto s_item = [&](const Item& it, int sb, int n, auto nh_tag, auto tile_tag) -> bool {
-    constexpr int NH = decltype(nh_tag)::value;
+  // One TILE (N = KC) or EXACT (N = BLK) item: this thread's N logits in R_t.
+  auto s_item = [&](const Item& it, auto n_tag, auto tile_tag) __attribute__((always_inline)) -> bool {
+    constexpr int N = decltype(n_tag)::value;
     constexpr bool TILE = decltype(tile_tag)::value;
-    constexpr int NK = NH / 32;
-    const uint32_t sa = tmem + lane_off + COL_R0 + 128 * sb;
-    const int col0 = ch * NH;
-    uint32_t sv[NH];
-#pragma unroll
-    for (int k = 0; k < NK; ++k)
-      tc::tmem_ld32(sa + col0 + 32 * k, sv + 32 * k);
-    tc::tmem_wait_ld();
+    constexpr int NK = N / 32;
+    if (!uni(wt.fast(smem_u32(&c.s_full[t]), ns & 1, 11))) return false;
+    ++ns;
+    tc::fence_after_sync();
     uint32_t mbits[NK];
+    bool masked = TILE;  // the same for the whole warp
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
       if (TILE) {
-        const int j0 = it.j * KC + col0 + 32 * k;
-        mbits[k] = c.skipU[j0 >> 5] & ~c.kept[h][j0 >> 5];
+        // a centroid column counts for the rows whose query block skips its block
+        const int w = (it.j * KC + 32 * k) >> 5;
+        mbits[k] = ~kept_h[w] & valid_bits(w, nkb);
       } else {
-        const int t0 = it.j * BLK + col0 + 32 * k;
+        const int t0 = it.j * BLK + 32 * k;
         mbits[k] = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
-        if (BLK == 64 && !((c.kept[h][it.j >> 5] >> (it.j & 31)) & 1u)) mbits[k] = 0u;
+        if (BLK == 64 && !((kept_h[it.j >> 5] >> (it.j & 31)) & 1u)) mbits[k] = 0u;
+        masked = masked || mbits[k] != 0xffffffffu;
       }
     }
-    // Logits in base-2 units; masked columns become -inf, which the exponential maps
-    // to an exact zero, so the second pass needs no per-column tests.
-    float xv[NH];
+    // Raw logits; masked columns become -inf, which the exponential maps to an exact
+    // zero. A TILE's 64 logits are read twice from TMEM (max, then exponentials) so
+    // that only 32 are held at once; an EXACT item's are read once.
+    constexpr int NR = TILE ? 32 : N;
+    float xv[NR];
+    auto fetch = [&, masked](int k0) __attribute__((always_inline)) {
+      uint32_t sv[NR];
 #pragma unroll
-    for (int k = 0; k < NK; ++k)
+      for (int k = 0; k < NR / 32; ++k) tc::tmem_ld32(rt + 32 * (k0 + k), sv + 32 * k);
+      tc::tmem_wait_ld();
+      if (masked) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        xv[32 * k + i] = ((mbits[k] >> i) & 1u) ? __uint_as_float(sv[32 * k + i]) * sl2 : -INFINITY;
-    float mx;
-    {
+        for (int k = 0; k < NR / 32; ++k)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            xv[32 * k + i] = ((mbits[k0 + k] >> i) & 1u) ? __uint_as_float(sv[32 * k + i]) : -INFINITY;
+      } else {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) xv[i] = __uint_as_float(sv[i]);
+      }
+    };
+    // row max of the raw logits (the scale is positive), in base-2 units after scaling
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k0 = 0; k0 < NK; k0 += NR / 32) {
+      fetch(k0);
       float m8[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) m8[a] = xv[a];
 #pragma unroll
-      for (int i = 8; i < NH; ++i) m8[i % 8] = fmaxf(m8[i % 8], xv[i]);
-      mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int i = 8; i < NR; i += 16) {
+#pragma unroll
+        for (int a = 0; a < 8; ++a) m8[a] = i + 8 + a < NR ? tc::max3(m8[a], xv[i + a], xv[i + 8 + a])
+                                                           : fmaxf(m8[a], xv[i + a]);
+      }
+      mx = tc::max3(mx, tc::max3(m8[0], m8[1], m8[2]),
+                    tc::max3(tc::max3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
     }
-    float* rmax = red + (n & 1) * 2 * TQ;
-    rmax[ch * TQ + r] = mx;
-    if (!pair_sync()) return false;
-    mx = fmaxf(mx, rmax[(1 - ch) * TQ + r]);
+    mx *= sl2;
     // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
     // reference; rows that had no reference yet just take one (O is still zero).
     const bool grow = mx > m_ref + kThresh;
     const bool need_o = grow && m_ref != -INFINITY;
     const float f = need_o ? tc::ex2(m_ref - mx) : 1.f;
     if (grow) m_ref = mx;
-    l *= f;
-    if (__any_sync(0xffffffffu, need_o)) {
-      if (!wait_last_writer(12)) return false;
-#pragma unroll
-      for (int k = 0; k < DH / 32; ++k) {
-        uint32_t v[32];
-        const uint32_t oa = tmem + lane_off + COL_O + ch * DH + 32 * k;
-        tc::tmem_ld32(oa, v);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-        tc::tmem_st32(oa, v);
-      }
-      tc::tmem_wait_st();
-    }
-    // P = 2^(x - m_ref) as fp16 pairs over the logits of both halves (all of them were
-    // read before the pair met, so the writes cannot overtake a partner's read).
-    float l4[4] = {0.f, 0.f, 0.f, 0.f};
-    // TILE: column of the possibly partial last block within this half, and its P
-    const int jl = TILE ? nkb - 1 - (it.j * KC + col0) : -1;
+    // A row with no unmasked logit so far keeps m_ref = -inf; its P must be 0, not NaN.
+    const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+    const uint64_t nmr2 = tc::f2(-mr, -mr);
+    // P = 2^(x * scale * log2(e) - m_ref) as fp16 pairs, written over the logits
+    // already read; row sums in two packed accumulators.
+    uint64_t acc0 = tc::f2(0.f, 0.f), acc1 = acc0;
+    // TILE: column of the possibly partial last block, and its P
+    const int jl = TILE ? nkb - 1 - it.j * KC : -1;
     float plast = 0.f;
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
+      if (TILE) fetch(k);
+      const float* xk = TILE ? xv : xv + 32 * k;
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        const float x0 = tc::ex2(xv[32 * k + i] - m_ref);
-        const float x1 = tc::ex2(xv[32 * k + i + 1] - m_ref);
-        l4[(i / 2) & 3] += x0 + x1;
+        const uint64_t y = tc::fma2(tc::f2(xk[i], xk[i + 1]), sl2x2, nmr2);
+        float y0, y1;
+        tc::f2_split(y, y0, y1);
+        const float x0 = tc::ex2(y0), x1 = tc::ex2(y1);
+        const uint64_t e = tc::f2(x0, x1);
+        if ((i / 2) & 1) acc1 = tc::add2(acc1, e); else acc0 = tc::add2(acc0, e);
         pk[i / 2] = pack_f16(x0, x1);
-        if (TILE) {
-          stash[(col0 + 32 * k + i) * TQ + r] = __float2half_rn(x0);
-          stash[(col0 + 32 * k + i + 1) * TQ + r] = __float2half_rn(x1);
-          plast = (32 * k + i == jl) ? x0 : ((32 * k + i + 1 == jl) ? x1 : plast);
-        }
+        if (TILE) plast = (32 * k + i == jl) ? x0 : ((32 * k + i + 1 == jl) ? x1 : plast);
       }
-      tc::tmem_st16(sa + col0 / 2 + 16 * k, pk);
+      if constexpr (TILE && ORDER == 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) stash[16 * k + i] = pk[i];
+      }
+      tc::tmem_st16(rt + 16 * k, pk);
     }
-    if (TILE) {
-      // order-0 denominator weight n_j: b for every block but a partial last one
-      float lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      lt *= (float)BLK;
-      lt += plast * (float)(p.Nk - nkb * BLK);
-      l += lt;
-    } else {
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+    // O_t rescale. Every product into O_t issued so far is complete: the logits of
+    // this item were issued after them and have landed; the value product of this
+    // item waits for p_full.
+    if (__any_sync(0xffffffffu, need_o)) {
+#pragma unroll
+      for (int k = 0; k < D / 32; ++k) {
+        uint32_t v[32];
+        tc::tmem_ld32(ot + 32 * k, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+        tc::tmem_st32(ot + 32 * k, v);
+      }
     }
+    float a0, a1, a2, a3;
+    tc::f2_split(acc0, a0, a1);
+    tc::f2_split(acc1, a2, a3);
+    float ls = (a0 + a1) + (a2 + a3);
+    // order-0 denominator weight n_j: b for every block but a partial last one
+    if (TILE) ls = ls * (float)BLK + plast * (float)(p.Nk - nkb * BLK);
+    l = l * f + ls;
     tc::tmem_wait_st();
-    warp_arrive(bar(c.p_full[sb]));
-    if (TILE && !pair_sync()) return false;  // the partner's half of the stash is visible
+    warp_arrive(smem_u32(&c.p_full[t]));
     return true;
   };
 
+  Walk wk;
+  Item it{kNone, 0, 0};
+  int ntile = 0, na = 0, cur_tile = 0;  // order-1 TILEs, MAT items of this tile so far
+  int since_tile = 0;                   // MAT items since the tile's TILE item
+  // ---- phase 0: centroid tiles and their order-1 products ----
   while (ok) {
-    const Item it = wk.next<ORDER>(c, nkb);
-    if (it.kind == kNone) break;
-    if (it.kind == kMat) {
-      if constexpr (ORDER == 1) {
-        const int n = nmat++;
-        const int slot = n % NA, use = n / NA;
-        if (use >= 1) ok = uni(wt.fast(bar(c.a_done[slot]), (use - 1) & 1, 10));
-        if (ok && slot == 1 && !r_slots_free) {
-          ok = uni(wt.wait(bar(c.pv_done[cur_buf]), cur_use & 1, 15));
-          r_slots_free = true;
-        }
-        if (!ok) break;
-        tc::fence_after_sync();
-        const uint32_t ab = tmem + lane_off + a_col(slot, cur_buf) + ch * AW;
-        const int jb[2] = {it.j, it.j2};
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          if (jb[b] < 0) break;
-          const float pj = __half2float(stash[(jb[b] - cur_tile * KC) * TQ + r]);
-          const __half2 al = __float2half2_rn(pj * p.scale);
-          uint32_t a[AW];
-#pragma unroll
-          for (int i = 0; i < AW; ++i) {
-            const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
-            a[i] = *reinterpret_cast<const uint32_t*>(&y);
-          }
-          tmem_st_w<AW>(ab + b * (D / 2), a);
-        }
-        tc::tmem_wait_st();
-        warp_arrive(bar(c.a_full[slot]));
-        lw_kind = 1;
-        lw_buf = slot;
-        lw_use = use;
-      }
+    it = wk.next<ORDER>(c, nkb);
+    if (it.kind == kExact || it.kind == kNone) break;
+    if (!((it.mask >> t) & 1)) continue;
+    if (it.kind == kTile) {
+      ok = s_item(it, std::integral_constant<int, KC>{}, std::true_type{});
+      since_tile = 0;
+      cur_tile = it.j;
       continue;
     }
-    // ---- TILE or EXACT: logits in an S buffer ----
-    if (prev_buf >= 0) warp_arrive(bar(c.s_free[prev_buf]));
-    const int n = ns++;
-    const int sb = n & 1, use = n >> 1;
-    prev_buf = sb;
-    ok = uni(wt.fast(bar(c.s_full[sb]), use & 1, 11));
-    if (!ok) break;
-    tc::fence_after_sync();
-    if (it.kind == kTile) {
-      cur_buf = sb;
-      cur_use = use;
-      cur_tile = it.j;
-      r_slots_free = false;
-      ok = s_item(it, sb, n, std::integral_constant<int, KC / 2>{}, std::true_type{});
-    } else {
-      ok = s_item(it, sb, n, std::integral_constant<int, BLK / 2>{}, std::false_type{});
+    if constexpr (ORDER == 1) {
+      // Slot s of R_t (columns [s d/2, (s+1) d/2)) is free once the products that
+      // last read it are complete: the tile's value product (P sits in slot 0) for
+      // the first item after a TILE, which also covers the second (everything issued
+      // before the TILE's logits is complete); then the item two before.
+      const int s = na & 1, use = na >> 1;
+      if (since_tile == 0) {
+        ok = uni(wt.fast(bar(c.pv_done[t]), ntile & 1, 15));
+        ++ntile;
+      } else if (since_tile >= 2) {
+        ok = uni(wt.fast(bar(c.a_done[t][s]), (use - 1) & 1, 10));
+      }
+      ++since_tile;
+      ++na;
+      if (!ok) break;
+      tc::fence_after_sync();
+      const float pj = stash_get(stash, it.j - cur_tile * KC);
+      const __half2 al = __float2half2_rn(pj * p.scale);
+#pragma unroll
+      for (int k = 0; k < QW / 32; ++k) {
+        uint32_t a[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[32 * k + i]), al);
+          a[i] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+        tc::tmem_st32(rt + s * (D / 2) + 32 * k, a);
+      }
+      tc::tmem_wait_st();
+      warp_arrive(bar(c.a_full[t][s]));
     }
-    lw_kind = 0;
-    lw_buf = sb;
-    lw_use = use;
+  }
+  // ---- phase 1: kept blocks ----
+  while (ok && it.kind == kExact) {
+    if ((it.mask >> t) & 1) ok = s_item(it, std::integral_constant<int, BLK>{}, std::false_type{});
+    it = wk.next<ORDER>(c, nkb);
   }
 
-  // ---- epilogue: O / l over both column halves ----
-  if (ok) ok = wait_last_writer(13);
-  float* rsum = red + 4 * TQ;
-  rsum[ch * TQ + r] = l;
-  if (ok) ok = pair_sync();
+  // ---- epilogue: O / l ----
+  if (ok) ok = uni(wt.wait(bar(c.o_final[t]), 0, 13));
+  tc::fence_after_sync();
   if (!ok) return;
-  const float lt = l + rsum[(1 - ch) * TQ + r];
-  const bool store = q0 + r < p.Nq;
-  const float inv = lt > 0.f ? 1.f / lt : 0.f;
-  const size_t rowoff = ((size_t)bh * p.Nq + q0 + (store ? r : 0)) * D + ch * DH;
+  const bool store = row0 + r < p.Nq;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const size_t rowoff = ((size_t)bh * p.Nq + row0 + (store ? r : 0)) * D;
 #pragma unroll
-  for (int k = 0; k < DH / 32; ++k) {
+  for (int k = 0; k < D / 32; ++k) {
     uint32_t v[32];
-    tc::tmem_ld32(tmem + lane_off + COL_O + ch * DH + 32 * k, v);
+    tc::tmem_ld32(ot + 32 * k, v);
     tc::tmem_wait_ld();
     if (!store) continue;
     if (p.out_dtype == 0) {
@@ -551,7 +546,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * TQ;
+  const int q0 = blockIdx.x * (NT * TQ);
   const int nkb = p.nkb;
 
   // A failure reported by an earlier CTA (or call) makes the rest of the grid skip
@@ -564,22 +559,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   if (warp == 8 && lane == 0) {
     for (int u = 0; u < NU; ++u) {
       tc::mbar_init(bar(c.full[u]), 1);
-      tc::mbar_init(bar(c.empty[u]), 1);
+      tc::mbar_init(bar(c.empty[u]), NT);  // one release per MMA thread
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(bar(c.s_full[b]), 1);
-      tc::mbar_init(bar(c.pv_done[b]), 1);
-      tc::mbar_init(bar(c.p_full[b]), NSOFT / 32);
-      tc::mbar_init(bar(c.s_free[b]), NSOFT / 32);
-    }
-    for (int a = 0; a < NA; ++a) {
-      tc::mbar_init(bar(c.a_done[a]), 1);
-      tc::mbar_init(bar(c.a_full[a]), NSOFT / 32);
+    for (int t = 0; t < NT; ++t) {
+      tc::mbar_init(bar(c.s_full[t]), 1);
+      tc::mbar_init(bar(c.pv_done[t]), 1);
+      tc::mbar_init(bar(c.o_final[t]), 1);
+      tc::mbar_init(bar(c.p_full[t]), 4);
+      for (int s = 0; s < 2; ++s) {
+        tc::mbar_init(bar(c.a_done[t][s]), 1);
+        tc::mbar_init(bar(c.a_full[t][s]), 4);
+      }
     }
     tc::mbar_init(bar(c.q_full), 1);
     tc::mbar_init(bar(c.init_done), NSOFT / 32);
-    tc::mbar_init(bar(c.drain), 1);
-    for (int w = 0; w < 4; ++w) tc::mbar_init(bar(c.pair[w]), 2);
     tc::fence_mbar_init();
     tc::fence_proxy_async();
   }
@@ -588,32 +581,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
     tc::tmem_relinquish();
   }
   if (warp < 8) {
-    // Kept bitmaps of the one (block 128) or two (block 64) query blocks of the tile.
-    const int nh = BLK == 128 ? 1 : 2;
-    for (int w = tid; w < 2 * MAXW; w += NSOFT) (&c.kept[0][0])[w] = 0u;
+    // Kept bitmaps of the query blocks of both tiles: one per tile (block 128) or
+    // two (block 64, one per 64-row half).
+    for (int w = tid; w < NT * 2 * MAXW; w += NSOFT) (&c.kept[0][0][0])[w] = 0u;
     asm volatile("bar.sync 1, %0;\n" ::"n"(NSOFT) : "memory");
-    for (int h = 0; h < nh; ++h) {
-      const int qb = q0 / BLK + h;
-      if (qb >= p.nqb) continue;
-      const size_t row = (size_t)bh * p.nqb + qb;
-      const int n = min(max(p.kv_cnt[row], 0), p.cap);
-      const int32_t* src = p.kv_idx + row * p.cap;
-      for (int x = tid; x < n; x += NSOFT) {
-        const int j = src[x];
-        if (j >= 0 && j < nkb) atomicOr(&c.kept[h][j >> 5], 1u << (j & 31));
+    for (int t = 0; t < NT; ++t)
+      for (int hh = 0; hh < (BLK == 64 ? 2 : 1); ++hh) {
+        const int r0 = q0 + t * TQ + hh * 64;
+        if (r0 >= p.Nq) continue;
+        const size_t row = (size_t)bh * p.nqb + r0 / BLK;
+        const int n = min(max(p.kv_cnt[row], 0), p.cap);
+        const int32_t* src = p.kv_idx + row * p.cap;
+        for (int x = tid; x < n; x += NSOFT) {
+          const int j = src[x];
+          if (j >= 0 && j < nkb) atomicOr(&c.kept[t][hh][j >> 5], 1u << (j & 31));
+        }
       }
-    }
     asm volatile("bar.sync 1, %0;\n" ::"n"(NSOFT) : "memory");
-    const bool has1 = BLK == 64 && (q0 / BLK + 1) < p.nqb;
-    for (int w = tid; w < MAXW; w += NSOFT) {
-      const int lo = w * 32;
-      const uint32_t valid = lo + 32 <= nkb ? 0xffffffffu : (lo < nkb ? (1u << (nkb - lo)) - 1u : 0u);
-      const uint32_t k0 = c.kept[0][w];
-      const uint32_t k1 = BLK == 128 ? k0 : (has1 ? c.kept[1][w] : k0);
-      if (BLK == 128 || !has1) c.kept[1][w] = k0;
-      c.keptU[w] = (k0 | k1) & valid;
-      c.skipU[w] = (~k0 | ~k1) & valid;
+    // a half without a query block of its own (block 128, or past Nq) repeats half 0
+    for (int w = tid; w < NT * MAXW; w += NSOFT) {
+      const int t = w / MAXW, ww = w % MAXW;
+      if (BLK == 128 || q0 + t * TQ + 64 >= p.Nq) c.kept[t][1][ww] = c.kept[t][0][ww];
     }
+    if (tid == 0) c.tvalid = (q0 < p.Nq ? 1 : 0) | (q0 + TQ < p.Nq ? 2 : 0);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -630,149 +620,157 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
     // =========================== TMA producer ===========================
     if (lane == 0) {
       tc::prefetch_tmap(&p.tmQ);
-      tc::mbar_arrive_expect_tx(bar(c.q_full), By::Q);
-      for (int s = 0; s < SUB; ++s)
-        tc::tma_load_3d(base + OFF_Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s, q0, bh);
-      EventGen gen;
+      const int ntq = q0 + TQ < p.Nq ? 2 : 1;
+      tc::mbar_arrive_expect_tx(bar(c.q_full), ntq * By::Q);
+      for (int t = 0; t < ntq; ++t)
+        for (int s = 0; s < SUB; ++s)
+          tc::tma_load_3d(base + OFF_Q + t * By::Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s,
+                          q0 + t * TQ, bh);
+      StepGen gen;
       int u = 0;
       bool ok = true;
       while (ok) {
-        const Event e = gen.next<ORDER>(c, nkb);
-        const int slot = u % NU;
-        if (u >= NU) ok = wt.fast(bar(c.empty[slot]), ((u / NU) - 1) & 1, 1);
+        const Step s = gen.next<ORDER>(c, nkb);
+        for (int i = 0; i < s.nunits && ok; ++i) {
+          const int v = u + i;
+          if (v >= NU) ok = wt.fast(bar(c.empty[v % NU]), ((v / NU) - 1) & 1, 1);
+        }
         if (!ok) break;
-        const uint32_t dst = base + OFF_U + slot * UNIT;
+        const int slot = u % NU;
         const uint32_t fb = bar(c.full[slot]);
-        const Item& it = e.item;
-        // The MMA thread reads the event of a unit after the unit's full barrier.
-        c.evq[slot] = make_int4(e.kind | (it.kind << 4) | ((it.j2 >= 0) << 8), it.j,
-                                e.buf | (e.tbuf << 4), e.use);
-        if (e.kind == eNone) {
+        // The MMA thread reads the record after the unit's full barrier.
+        c.evq[slot] = make_int4(encode(s), s.cur_j, s.pend_j, 0);
+        if (s.type == stEnd) {
           tc::mbar_arrive(fb);  // terminal record, no data
           ++u;
           break;
         }
-        if (e.kind == eS && it.kind == kTile) {
-          tc::mbar_arrive_expect_tx(fb, 2 * By::KB);
-          for (int pl = 0; pl < 2; ++pl)
-            for (int s = 0; s < SUB; ++s)
-              tc::tma_load_3d(dst + pl * By::KB + s * KC * 128, &p.tmKb, fb, 64 * s, it.j * KC,
-                              2 * bh + pl);
-        } else if (e.kind == ePV && it.kind == kTile) {
-          tc::mbar_arrive_expect_tx(fb, By::VS);
-          for (int s = 0; s < SUB; ++s)
-            tc::tma_load_3d(dst + s * KC * 128, &p.tmVs, fb, 64 * s, it.j * KC, bh);
-        } else if (e.kind == eMat) {
-          tc::mbar_arrive_expect_tx(fb, By::M);
-          for (int s = 0; s < SUB; ++s)
-            tc::tma_load_3d(dst + s * D * 128, &p.tmM, fb, 64 * s, 0, bh * nkb + it.j);
-          if (it.j2 >= 0) {  // the pair's second block goes to the next unit
-            ++u;
-            const int s2 = u % NU;
-            if (u >= NU) ok = wt.fast(bar(c.empty[s2]), ((u / NU) - 1) & 1, 1);
-            if (!ok) break;
-            const uint32_t fb2 = bar(c.full[s2]);
-            tc::mbar_arrive_expect_tx(fb2, By::M);
-            for (int s = 0; s < SUB; ++s)
-              tc::tma_load_3d(base + OFF_U + s2 * UNIT + s * D * 128, &p.tmM, fb2, 64 * s, 0,
-                              bh * nkb + it.j2);
+        auto dst = [&](int i) { return base + OFF_U + ((u + i) % NU) * UNIT; };
+        uint32_t bytes = 0;
+        if (s.type != stMat && s.pend_mask) bytes += s.pend_kind == kTile ? By::VS : By::KV;
+        if (s.type == stSX) bytes += s.cur_kind == kTile ? 2 * By::KB : By::KV;
+        if (s.type == stMat) bytes += By::M;
+        // every load of the step completes on the first unit's barrier
+        tc::mbar_arrive_expect_tx(fb, bytes);
+        int ui = 0;
+        if (s.type != stMat && s.pend_mask) {  // values of the pending item
+          if (s.pend_kind == kTile) {
+            for (int k = 0; k < SUB; ++k)
+              tc::tma_load_3d(dst(0) + k * KC * 128, &p.tmVs, fb, 64 * k, s.pend_j * KC, bh);
+          } else {
+            for (int k = 0; k < SUB; ++k)
+              tc::tma_load_3d(dst(0) + k * BLK * 128, &p.tmV, fb, 64 * k, s.pend_j * BLK, bh);
           }
-        } else {
-          const CUtensorMap* m = e.kind == eS ? &p.tmK : &p.tmV;
-          tc::mbar_arrive_expect_tx(fb, By::KV);
-          for (int s = 0; s < SUB; ++s)
-            tc::tma_load_3d(dst + s * BLK * 128, m, fb, 64 * s, it.j * BLK, bh);
+          ui = 1;
         }
-        ++u;
+        if (s.type == stSX) {  // keys of the new item
+          if (s.cur_kind == kTile) {
+            for (int pl = 0; pl < 2; ++pl)
+              for (int k = 0; k < SUB; ++k)
+                tc::tma_load_3d(dst(ui) + pl * By::KB + k * KC * 128, &p.tmKb, fb, 64 * k,
+                                s.cur_j * KC, 2 * bh + pl);
+          } else {
+            for (int k = 0; k < SUB; ++k)
+              tc::tma_load_3d(dst(ui) + k * BLK * 128, &p.tmK, fb, 64 * k, s.cur_j * BLK, bh);
+          }
+        }
+        if (s.type == stMat)
+          for (int k = 0; k < SUB; ++k)
+            tc::tma_load_3d(dst(0) + k * D * 128, &p.tmM, fb, 64 * k, 0, bh * nkb + s.cur_j);
+        // the second unit's barrier only keeps its phase count in step
+        if (s.nunits == 2) tc::mbar_arrive(bar(c.full[(u + 1) % NU]));
+        u += s.nunits;
       }
       // Drain: every load issued must land before the CTA exits.
       tc::wait_drain(bar(c.q_full), 0, kWaitLimit);
       for (int v = max(0, u - NU); v < u; ++v)
         tc::wait_drain(bar(c.full[v % NU]), (v / NU) & 1, kWaitLimit);
     }
-  } else if (warp == 9) {
-    // =========================== MMA issuer ===========================
+  } else if (warp == 9 || warp == 10) {
+    // ===================== MMA issuers: warp 9 + t for tile t =====================
     if (lane == 0) {
+      const int t = warp - 9;
       constexpr uint32_t I_S_TILE = tc::idesc_f16(1, 1, 0, KC);
-      constexpr uint32_t I_PV_TILE = tc::idesc_f16(0, 0, 1, D);
       constexpr uint32_t I_S_EX = tc::idesc_f16(1, 1, 0, BLK);
-      constexpr uint32_t I_PV_EX = tc::idesc_f16(0, 0, 1, D);
-      constexpr uint32_t I_MAT = tc::idesc_f16(0, 0, 1, D);
+      constexpr uint32_t I_PV = tc::idesc_f16(0, 0, 1, D);
       bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
       tc::fence_after_sync();
-      // Descriptor bases; per k-step only the start-address field (low bits) moves.
-      const uint64_t dQ = tc::sdesc(base + OFF_Q, 16, 1024);
-      for (int u = 0; ok; ++u) {
+      const uint32_t o_t = tmem + COL_O + 128 * t, r_t = tmem + COL_R + 128 * t;
+      // Descriptor base of Q_t; per k-step only the start-address field (low bits) moves.
+      const uint64_t dq = tc::sdesc(base + OFF_Q + t * By::Q, 16, 1024);
+      int np = 0, na = 0;  // p_full phases; order-1 items of this tile
+      for (int u = 0; ok;) {
         const int slot = u % NU;
         ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
         if (!ok) break;
-        const int4 rec = c.evq[slot];  // ordered by the full-barrier wait (asm with memory clobber)
-        const int kind = rec.x & 15, ikind = (rec.x >> 4) & 15, buf = rec.z & 15, tbuf = rec.z >> 4;
-        const bool pair = (rec.x >> 8) & 1;
-        const int use = rec.w;
-        if (kind == eNone) break;
-        const uint32_t src = base + OFF_U + slot * UNIT;
-        if (kind == eS) {
-          if (use >= 1) ok = wt.fast(bar(c.s_free[buf]), (use - 1) & 1, 5);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t dt = tmem + COL_R0 + 128 * buf;
-          const bool tile = ikind == kTile;
-          const int rows = tile ? KC : BLK;
-          const uint64_t bd0 = tc::sdesc(src, 16, 1024);
-          const uint32_t idesc = tile ? I_S_TILE : I_S_EX;
-          // tile: the hi plane, then the lo plane of the centroids, into the same logits
-          const int planes = tile ? 2 : 1;
-          for (int pl = 0; pl < planes; ++pl)
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
-              const uint32_t boff = (pl * By::KB + (kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
-              tc::mma_ss(dt, dQ + aoff, bd0 + boff, idesc, (pl | kk) > 0);
-            }
-          tc::mma_commit(bar(c.s_full[buf]));
-        } else if (kind == ePV) {
-          ok = wt.fast(bar(c.p_full[buf]), use & 1, 6);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t pa = tmem + COL_R0 + 128 * buf;
-          const bool tile = ikind == kTile;
-          const int rows = tile ? KC : BLK;
-          const uint64_t bd0 = tc::sdesc(src, rows * 128, 1024);
-          const uint32_t idesc = tile ? I_PV_TILE : I_PV_EX;
-          for (int kk = 0; kk < rows / 16; ++kk)
-            tc::mma_ts(tmem + COL_O, pa + kk * 8, bd0 + ((kk * 2048) >> 4), idesc, 1);
-          tc::mma_commit(bar(c.pv_done[buf]));
-        } else {
-          const int slot2 = (u + 1) % NU;
-          if (pair) ok = wt.fast(bar(c.full[slot2]), ((u + 1) / NU) & 1, 4);
-          if (ok) ok = wt.fast(bar(c.a_full[buf]), use & 1, 7);
-          if (!ok) break;
-          tc::fence_after_sync();
-          const uint32_t aa = tmem + a_col(buf, tbuf);
-          const uint64_t bd0 = tc::sdesc(src, D * 128, 1024);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_ts(tmem + COL_O, aa + kk * 8, bd0 + ((kk * 2048) >> 4), I_MAT, 1);
-          if (pair) {
-            const uint64_t bd1 = tc::sdesc(base + OFF_U + slot2 * UNIT, D * 128, 1024);
+        const int rec = c.evq[slot].x;  // ordered by the full-barrier wait (asm with memory clobber)
+        const int type = rec & 15, ck = (rec >> 4) & 15, pk = (rec >> 8) & 15;
+        const int cm = (rec >> 12) & 3, pm = (rec >> 14) & 3, nun = (rec >> 16) & 3;
+        if (type == stEnd) break;
+        const int slot2 = (u + 1) % NU;
+        const uint32_t src0 = base + OFF_U + slot * UNIT, src1 = base + OFF_U + slot2 * UNIT;
+        bool issued = false;
+        if (type == stMat) {
+          if ((cm >> t) & 1) {
+            const int s = na & 1, use = na >> 1;
+            ++na;
+            ok = wt.fast(bar(c.a_full[t][s]), use & 1, 7);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint64_t b0 = tc::sdesc(src0, D * 128, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              tc::mma_ts(tmem + COL_O, aa + D / 2 + kk * 8, bd1 + ((kk * 2048) >> 4), I_MAT, 1);
+              tc::mma_ts(o_t, r_t + s * (D / 2) + kk * 8, b0 + ((kk * 2048) >> 4), I_PV, 1);
+            tc::mma_commit(bar(c.a_done[t][s]));
+            issued = true;
           }
-          tc::mma_commit(bar(c.a_done[buf]));
-          if (pair) {
-            tc::mma_commit(bar(c.empty[slot]));
-            ++u;
-            tc::mma_commit(bar(c.empty[slot2]));
-            continue;
+        } else {
+          // SX / FLUSH: value product of the pending item, then logits of the new one
+          if ((pm >> t) & 1) {
+            ok = wt.fast(bar(c.p_full[t]), np & 1, 6);
+            ++np;
+            if (!ok) break;
+            tc::fence_after_sync();
+            const int rows = pk == kTile ? KC : BLK;
+            const uint64_t bd = tc::sdesc(src0, rows * 128, 1024);
+            for (int kk = 0; kk < rows / 16; ++kk)
+              tc::mma_ts(o_t, r_t + kk * 8, bd + ((kk * 2048) >> 4), I_PV, 1);
+            if (ORDER == 1 && pk == kTile) tc::mma_commit(bar(c.pv_done[t]));
+            issued = true;
+          }
+          if (type == stSX && ((cm >> t) & 1)) {
+            const bool tile = ck == kTile;
+            const int rows = tile ? KC : BLK;
+            const uint64_t bd0 = tc::sdesc(pm ? src1 : src0, 16, 1024);
+            const uint32_t idesc = tile ? I_S_TILE : I_S_EX;
+            // tile: the hi plane, then the lo plane of the centroids, into the same logits
+            const int planes = tile ? 2 : 1;
+            for (int pl = 0; pl < planes; ++pl)
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
+                const uint32_t boff = (pl * By::KB + (kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
+                tc::mma_ss(r_t, dq + aoff, bd0 + boff, idesc, (pl | kk) > 0);
+              }
+            tc::mma_commit(bar(c.s_full[t]));
+            issued = true;
           }
         }
-        tc::mma_commit(bar(c.empty[slot]));
+        // Release the step's units: after this thread's products have read them, or at
+        // once if it issued none.
+        if (issued) {
+          tc::mma_commit(bar(c.empty[slot]));
+          if (nun == 2) tc::mma_commit(bar(c.empty[slot2]));
+        } else {
+          tc::mbar_arrive(bar(c.empty[slot]));
+          if (nun == 2) tc::mbar_arrive(bar(c.empty[slot2]));
+        }
+        u += nun;
       }
-      // Drain: wait for every MMA issued so far before TMEM is released.
-      tc::mma_commit(bar(c.drain));
-      tc::wait_drain(bar(c.drain), 0, kWaitLimit);
+      // Every MMA this thread issued is complete once o_final[t] fires: the softmax
+      // warps of tile t read O_t after it, and TMEM is released after it.
+      tc::mma_commit(bar(c.o_final[t]));
+      tc::wait_drain(bar(c.o_final[t]), 0, kWaitLimit);
     }
   }
   }
@@ -841,7 +839,7 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   auto kern = forward_tc_kernel<D, BLK, ORDER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + TQ - 1) / TQ, a.B * a.H);
+  dim3 grid((a.Nq + NT * TQ - 1) / (NT * TQ), a.B * a.H);
   kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(p);
   return cudaGetLastError();
 }
