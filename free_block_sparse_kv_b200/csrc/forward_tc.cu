@@ -469,6 +469,15 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       // last read it are complete: the tile's value product (P sits in slot 0) for
       // the first item after a TILE, which also covers the second (everything issued
       // before the TILE's logits is complete); then the item two before.
+      // The operand does not depend on the slot: compute it first, then wait.
+      const float pj = stash_get(stash, it.j - cur_tile * KC);
+      const __half2 al = __float2half2_rn(pj * p.scale);
+      uint32_t a[QW];
+#pragma unroll
+      for (int i = 0; i < QW; ++i) {
+        const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
+        a[i] = *reinterpret_cast<const uint32_t*>(&y);
+      }
       const int s = na & 1, use = na >> 1;
       if (since_tile == 0) {
         ok = uni(wt.fast(bar(c.pv_done[t]), ntile & 1, 15));
@@ -480,18 +489,8 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       ++na;
       if (!ok) break;
       tc::fence_after_sync();
-      const float pj = stash_get(stash, it.j - cur_tile * KC);
-      const __half2 al = __float2half2_rn(pj * p.scale);
 #pragma unroll
-      for (int k = 0; k < QW / 32; ++k) {
-        uint32_t a[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[32 * k + i]), al);
-          a[i] = *reinterpret_cast<const uint32_t*>(&y);
-        }
-        tc::tmem_st32(rt + s * (D / 2) + 32 * k, a);
-      }
+      for (int k = 0; k < QW / 32; ++k) tc::tmem_st32(rt + s * (D / 2) + 32 * k, a + 32 * k);
       tc::tmem_wait_st();
       warp_arrive(bar(c.a_full[t][s]));
     }
