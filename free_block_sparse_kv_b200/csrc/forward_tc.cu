@@ -10,9 +10,9 @@
 // the first-order correction), all merged into one online softmax.
 //
 // Two query tiles per CTA. Neighbouring query blocks skip mostly the same key blocks,
-// so every operand tile that TMA brings in (centroids, value sums, M_j, K_j, V_j)
-// serves both tiles: half the L2 traffic per tensor-core flop of one tile per CTA.
-// Each tile takes part only in the work items its own rows need.
+// so every operand that TMA brings in (centroids, value sums, M_j, K, V) serves both
+// tiles: half the L2 traffic per tensor-core flop of one tile per CTA. Each tile takes
+// part only in the work items its own rows need.
 //
 // Roles (384 threads):
 //   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: one thread per query
@@ -20,27 +20,29 @@
 //              running max (rescaling O lazily, only when a row's max grows by more
 //              than 2^11), write P back to TMEM as the A operand of the value product,
 //              and build the order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
-//   warp 8     TMA producer: both Q tiles once, then every operand tile through a
-//              5 x 32 KB ring.
+//   warp 8     TMA producer: both Q tiles once, then every operand through a ring of
+//              5 x 32 KB units (each unit holds two 16 KB pieces or one M_j).
 //   warps 9-10 one MMA-issuing thread per tile (warp 9 also allocates TMEM). Issuing
 //              a 128x128x16 tcgen05.mma takes about as long as the tensor core takes to
 //              run it, so one thread cannot also wait and commit without leaving the
 //              pipe idle; two issuers keep it fed.
 //   warp 11    idle (it completes the control warpgroup for the register split).
-// TMEM columns: O_0 [0, 128), O_1 [128, 256); R_t = [256 + 128 t, 384 + 128 t) holds
-// tile t's logits, then its P (fp16), or two order-1 operands (two slots of d/2
-// columns, so that one is built while the other is in use).
+// TMEM columns: O_0 [0, 128), O_1 [128, 256); tile t owns two 64-column buffers at
+// 256 + 128 t + 64 b (b = 0, 1). Every work item of a tile takes the tile's next
+// buffer in turn: 64 logits (then their P as fp16), or one order-1 operand. The
+// logits of a tile's next item are therefore computed while its softmax works on
+// the current one, and one order-1 operand is built while the other is in use.
 //
 // Work items, in order (the same walk runs in every role):
 //   TILE c   64 centroids (bf16 hi + lo) and value sums (fp16):
 //            S_t = Q_t Kbar_hi^T + Q_t Kbar_lo^T, P_t, O_t += P_t Vsum
 //   MAT j    each skipped block of the current centroid tile (order 1):
 //            O_t += A_t,j M_j (fp16)
-//   EXACT j  each kept block: S_t = Q_t K_j^T (bf16), P_t, O_t += P_t V_j (fp16)
-// For each tile, the value product of its last item and the logits of its next item
-// are issued back to back, so a tile's softmax runs while the other tile's products
-// run. Order-1 TILE items are an exception: their value product follows at once,
-// because R_t then holds A operands.
+//   EXACT    each 64-key half (block 128) or block (block 64) of each kept block:
+//            S_t = Q_t K^T (bf16), P_t, O_t += P_t V (fp16)
+// For each tile, the logits of its next item are issued before the value product of
+// its current one. Order-1 TILE items are an exception: their value product follows
+// at once, because the order-1 operands of the centroid tile come next.
 // Every mbarrier wait is bounded: on timeout the CTA sets err_flag, abandons its work,
 // drains its own TMA loads and MMAs, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -56,15 +58,16 @@ namespace tcf {
 
 constexpr int TQ = 128;        // query rows per tile
 constexpr int NT = 2;          // tiles per CTA
-constexpr int KC = 64;         // centroids per TILE item
+constexpr int KC = 64;         // centroids per TILE item; keys per EXACT item
 constexpr int NU = 5;          // ring units
 constexpr int UNIT = 32768;    // bytes per ring unit
+constexpr int HALF = UNIT / 2; // bytes per piece slot
 constexpr int MAXW = 64;       // bitmap words (2048 blocks)
 constexpr int NSOFT = 256;     // softmax threads (2 warpgroups, one per tile)
-constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, MMA, 2 idle)
+constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, 2 MMA, 1 idle)
 // Register split after launch (168 per thread at launch = 64,512 per CTA): the
 // control warpgroup gives registers back, the softmax warpgroups take them.
-constexpr int kRegCtl = 120, kRegSoft = 192;
+constexpr int kRegCtl = 104, kRegSoft = 200;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
 constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
@@ -89,9 +92,10 @@ struct Params {
 
 struct Ctl {  // control block in shared memory
   uint64_t full[NU], empty[NU];
-  uint64_t s_full[NT], p_full[NT], pv_done[NT], o_final[NT];
-  uint64_t a_full[NT][2], a_done[NT][2];  // order-1 operand slots of each tile
-  uint64_t q_full, init_done;
+  // per tile and TMEM buffer: logits landed, P written, order-1 operand written,
+  // buffer released (the last product reading it is complete)
+  uint64_t s_full[NT][2], p_full[NT][2], a_full[NT][2], rel[NT][2];
+  uint64_t o_final[NT], q_full, init_done;
   int4 evq[NU];             // step record of the first ring unit of each step
   uint32_t tmem_base;
   int abort;
@@ -104,6 +108,7 @@ enum : int { kTile = 0, kMat = 1, kExact = 2, kNone = 3 };
 struct Item {
   int kind, j;  // TILE: j = centroid-tile index; MAT / EXACT: j = block index
   int mask;     // bit t: tile t takes part
+  int half;     // EXACT, block 128: which 64 keys of the block
 };
 
 SA_DEVI uint32_t valid_bits(int w, int nkb) {
@@ -125,8 +130,9 @@ SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct, int nkb) {
 
 // The walk over work items; identical in every role. Union masks of the current
 // centroid tile (phase 0) or 32-block word (phase 1) are held in registers.
+template <int BLK>
 struct Walk {
-  int phase = 0, tile = 0, word = -1;
+  int phase = 0, tile = 0, word = -1, half = 0, jcur = 0, mcur = 0;
   bool in_tile = false;
   uint64_t tmask = 0, sk0 = 0, sk1 = 0;  // phase 0: union / per-tile skipped blocks
   uint32_t kmask = 0, kw0 = 0, kw1 = 0;  // phase 1: union / per-tile kept blocks
@@ -145,7 +151,7 @@ struct Walk {
           tmask = sk0 | sk1;
           if (tmask) {
             in_tile = true;
-            return Item{kTile, tile, (sk0 != 0) | ((sk1 != 0) << 1)};
+            return Item{kTile, tile, (sk0 != 0) | ((sk1 != 0) << 1), 0};
           }
           ++tile;
           continue;
@@ -153,16 +159,20 @@ struct Walk {
         if (ORDER == 1 && tmask) {  // skipped blocks of this centroid tile, one at a time
           const int c1 = __ffsll((long long)tmask) - 1;
           tmask &= tmask - 1;
-          return Item{kMat, tile * KC + c1, (int)((sk0 >> c1) & 1u) | (int)(((sk1 >> c1) & 1u) << 1)};
+          return Item{kMat, tile * KC + c1, (int)((sk0 >> c1) & 1u) | (int)(((sk1 >> c1) & 1u) << 1), 0};
         }
         in_tile = false;
         ++tile;
         continue;
       }
+      if (BLK == 128 && half == 1) {  // second 64 keys of the current kept block
+        half = 0;
+        return Item{kExact, jcur, mcur, 1};
+      }
       while (!kmask) {
         if (++word >= (nkb + 31) / 32) {
           word = (nkb + 31) / 32;  // stays at the end: later calls return kNone again
-          return Item{kNone, 0, 0};
+          return Item{kNone, 0, 0, 0};
         }
         kw0 = kept_word(c, 0, word, nkb);
         kw1 = kept_word(c, 1, word, nkb);
@@ -170,47 +180,55 @@ struct Walk {
       }
       const int b = __ffs(kmask) - 1;
       kmask &= kmask - 1;
-      return Item{kExact, word * 32 + b, (int)((kw0 >> b) & 1u) | (int)(((kw1 >> b) & 1u) << 1)};
+      jcur = word * 32 + b;
+      mcur = (int)((kw0 >> b) & 1u) | (int)(((kw1 >> b) & 1u) << 1);
+      if (BLK == 128) half = 1;
+      return Item{kExact, jcur, mcur, 0};
     }
   }
 };
 
 // Steps: what the producer loads into one or two ring units and the MMA threads then
-// issue. An SX step carries the value products of the previous TILE/EXACT item
-// ("pending", one per tile that took part) and the logits of the next one; its units
-// are [V or Vsum of the pending item] + [K or Kbar of the new item].
+// issue. A unit holds two 16 KB pieces (a 64-row K, V, centroid plane or value-sum
+// tile) or one M_j. An SX step carries the logits of the next TILE/EXACT item and
+// the value products of the previous one ("pending", one per tile that took part);
+// its pieces are [V or Vsum of the pending item] + [K, or Kbar hi + lo, of the new].
 enum : int { stSX = 0, stFlush = 1, stMat = 2, stEnd = 3 };
 struct Step {
   int type, nunits;
-  int cur_kind, cur_mask, cur_j;     // SX: new TILE/EXACT item; MAT: the block
-  int pend_kind, pend_mask, pend_j;  // SX / FLUSH: item whose value products are due
+  int cur_kind, cur_mask, cur_j, cur_half;      // SX: new TILE/EXACT item; MAT: the block
+  int pend_kind, pend_mask, pend_j, pend_half;  // SX / FLUSH: item whose value products are due
 };
+template <int BLK>
 struct StepGen {
-  Walk wk;
-  int pend_kind = 0, pend_mask = 0, pend_j = 0;
+  Walk<BLK> wk;
+  int pend_kind = 0, pend_mask = 0, pend_j = 0, pend_half = 0;
   bool flush_next = false;
   template <int ORDER>
   SA_DEVI Step next(const Ctl& c, int nkb) {
     if (flush_next) {  // order 1: a TILE's value products come before its MAT items
       flush_next = false;
-      const Step s{stFlush, 1, 0, 0, 0, pend_kind, pend_mask, pend_j};
+      const Step s{stFlush, 1, 0, 0, 0, 0, pend_kind, pend_mask, pend_j, pend_half};
       pend_mask = 0;
       return s;
     }
     const Item it = wk.template next<ORDER>(c, nkb);
     if (it.kind == kNone) {
       if (pend_mask) {
-        const Step s{stFlush, 1, 0, 0, 0, pend_kind, pend_mask, pend_j};
+        const Step s{stFlush, 1, 0, 0, 0, 0, pend_kind, pend_mask, pend_j, pend_half};
         pend_mask = 0;
         return s;
       }
-      return Step{stEnd, 1, 0, 0, 0, 0, 0, 0};
+      return Step{stEnd, 1, 0, 0, 0, 0, 0, 0, 0, 0};
     }
-    if (it.kind == kMat) return Step{stMat, 1, kMat, it.mask, it.j, 0, 0, 0};
-    const Step s{stSX, pend_mask ? 2 : 1, it.kind, it.mask, it.j, pend_kind, pend_mask, pend_j};
+    if (it.kind == kMat) return Step{stMat, 1, kMat, it.mask, it.j, 0, 0, 0, 0, 0};
+    const int pieces = (pend_mask ? 1 : 0) + (it.kind == kTile ? 2 : 1);
+    const Step s{stSX, (pieces + 1) / 2, it.kind, it.mask, it.j, it.half,
+                 pend_kind, pend_mask, pend_j, pend_half};
     pend_kind = it.kind;
     pend_mask = it.mask;
     pend_j = it.j;
+    pend_half = it.half;
     if (ORDER == 1 && it.kind == kTile) flush_next = true;
     return s;
   }
@@ -223,11 +241,10 @@ SA_DEVI int encode(const Step& s) {
 template <int D, int BLK>
 struct Bytes {
   static constexpr int SUB = D / 64;                    // 64-column sub-tiles per row
-  static constexpr uint32_t KB = SUB * KC * 128;        // one plane of a centroid tile
-  static constexpr uint32_t VS = SUB * KC * 128;        // value-sum tile
+  static constexpr uint32_t PIECE = SUB * 64 * 128;     // 64 rows: K, V, Kbar plane, Vsum
   static constexpr uint32_t M = SUB * D * 128;          // one M_j
-  static constexpr uint32_t KV = SUB * BLK * 128;       // one K or V block
   static constexpr uint32_t Q = SUB * TQ * 128;         // one query tile
+  static_assert(PIECE <= HALF && M <= UNIT, "ring pieces");
 };
 
 // Element c (0..63) of a row's 64 fp16 probabilities held as 32 packed registers;
@@ -256,17 +273,6 @@ SA_DEVI float stash_get(const uint32_t* st, int c) {
   return __half2float(__ushort_as_half(hv));
 }
 
-// TMEM store of W consecutive 32-bit columns (W = 16 or 32).
-template <int W>
-SA_DEVI void tmem_st_w(uint32_t taddr, const uint32_t* r) {
-  if constexpr (W == 32) {
-    tc::tmem_st32(taddr, r);
-  } else {
-    static_assert(W == 16, "width");
-    tc::tmem_st16(taddr, r);
-  }
-}
-
 // Softmax warpgroup of tile t = warp / 4. Thread (warp w, lane l) owns query row
 // r = 32*(w%4) + l of the tile: all its logits, its running max and sum, its O row.
 template <int D, int BLK, int ORDER>
@@ -277,7 +283,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   const int t = warp >> 2, qw = warp & 3;
   const int r = 32 * qw + lane;
   const uint32_t lane_off = (uint32_t)(32 * qw) << 16;
-  const uint32_t rt = tmem + lane_off + COL_R + 128 * t;  // logits / P / order-1 operand
+  const uint32_t rt = tmem + lane_off + COL_R + 128 * t;  // buffer 0 of this tile
   const uint32_t ot = tmem + lane_off + COL_O + 128 * t;  // O rows
   const int h = BLK == 64 ? (r >> 6) : 0;                  // query block of the row
   const float sl2 = p.scale * kLog2e;
@@ -320,42 +326,49 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   warp_arrive(bar(c.init_done));
 
   float m_ref = -INFINITY, l = 0.f;
-  int ns = 0;                // S items of this tile so far (s_full phases)
+  int n = 0;                 // items of this tile so far; item n uses buffer n & 1
+  // Per-buffer phase parities as bit masks (bit b for buffer b): next s_full wait;
+  // number of items so far (rel phases); whether the buffer has been used.
+  uint32_t sph = 0, rcnt = 0, rany = 0;
   uint32_t stash[ORDER == 1 ? KC / 2 : 1];  // P of the current centroid tile, fp16 pairs
   const uint64_t sl2x2 = tc::f2(sl2, sl2);
 
-  // One TILE (N = KC) or EXACT (N = BLK) item: this thread's N logits in R_t.
-  auto s_item = [&](const Item& it, auto n_tag, auto tile_tag) __attribute__((always_inline)) -> bool {
-    constexpr int N = decltype(n_tag)::value;
+  // One TILE or EXACT item: this thread's 64 logits in buffer b.
+  auto s_item = [&](const Item& it, auto tile_tag) __attribute__((always_inline)) -> bool {
     constexpr bool TILE = decltype(tile_tag)::value;
-    constexpr int NK = N / 32;
-    if (!uni(wt.fast(smem_u32(&c.s_full[t]), ns & 1, 11))) return false;
-    ++ns;
+    const int idx = n++;
+    const int b = idx & 1;
+    const uint32_t buf = rt + 64 * b;
+    if (!uni(wt.fast(bar(c.s_full[t][b]), (sph >> b) & 1, 11))) return false;
+    sph ^= 1u << b;
+    rcnt ^= 1u << b;
+    rany |= 1u << b;
     tc::fence_after_sync();
-    uint32_t mbits[NK];
+    uint32_t mbits[2];
     bool masked = TILE;  // the same for the whole warp
 #pragma unroll
-    for (int k = 0; k < NK; ++k) {
+    for (int k = 0; k < 2; ++k) {
       if (TILE) {
         // a centroid column counts for the rows whose query block skips its block
         const int w = (it.j * KC + 32 * k) >> 5;
         mbits[k] = ~kept_h[w] & valid_bits(w, nkb);
       } else {
-        const int t0 = it.j * BLK + 32 * k;
+        const int t0 = it.j * BLK + 64 * it.half + 32 * k;
         mbits[k] = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
         if (BLK == 64 && !((kept_h[it.j >> 5] >> (it.j & 31)) & 1u)) mbits[k] = 0u;
         masked = masked || mbits[k] != 0xffffffffu;
       }
     }
     // Raw logits; masked columns become -inf, which the exponential maps to an exact
-    // zero. A TILE's 64 logits are read twice from TMEM (max, then exponentials) so
-    // that only 32 are held at once; an EXACT item's are read once.
-    constexpr int NR = TILE ? 32 : N;
+    // zero. A TILE's logits are read twice from TMEM (max, then exponentials), 32 at
+    // a time, which keeps registers free for the order-1 state; an EXACT item's 64 are
+    // read once.
+    constexpr int NR = TILE ? 32 : 64;
     float xv[NR];
     auto fetch = [&, masked](int k0) __attribute__((always_inline)) {
       uint32_t sv[NR];
 #pragma unroll
-      for (int k = 0; k < NR / 32; ++k) tc::tmem_ld32(rt + 32 * (k0 + k), sv + 32 * k);
+      for (int k = 0; k < NR / 32; ++k) tc::tmem_ld32(buf + 32 * (k0 + k), sv + 32 * k);
       tc::tmem_wait_ld();
       if (masked) {
 #pragma unroll
@@ -371,19 +384,20 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     // row max of the raw logits (the scale is positive), in base-2 units after scaling
     float mx = -INFINITY;
 #pragma unroll
-    for (int k0 = 0; k0 < NK; k0 += NR / 32) {
+    for (int k0 = 0; k0 < 2; k0 += NR / 32) {
       fetch(k0);
       float m8[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) m8[a] = xv[a];
+      for (int a = 0; a < 8; ++a) m8[a] = tc::max3(xv[a], xv[8 + a], xv[16 + a]);
 #pragma unroll
-      for (int i = 8; i < NR; i += 16) {
+      for (int a = 0; a < 8; ++a) m8[a] = NR == 64 ? tc::max3(m8[a], xv[24 + a], xv[(32 + a) % NR]) : fmaxf(m8[a], xv[24 + a]);
+      if (NR == 64) {
 #pragma unroll
-        for (int a = 0; a < 8; ++a) m8[a] = i + 8 + a < NR ? tc::max3(m8[a], xv[i + a], xv[i + 8 + a])
-                                                           : fmaxf(m8[a], xv[i + a]);
+        for (int a = 0; a < 8; ++a) m8[a] = tc::max3(m8[a], xv[(40 + a) % NR], xv[(48 + a) % NR]);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) m8[a] = fmaxf(m8[a], xv[(56 + a) % NR]);
       }
-      mx = tc::max3(mx, tc::max3(m8[0], m8[1], m8[2]),
-                    tc::max3(tc::max3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+      mx = tc::max3(mx, tc::max3(tc::max3(m8[0], m8[1], m8[2]), tc::max3(m8[3], m8[4], m8[5]), m8[6]), m8[7]);
     }
     mx *= sl2;
     // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
@@ -402,7 +416,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     const int jl = TILE ? nkb - 1 - it.j * KC : -1;
     float plast = 0.f;
 #pragma unroll
-    for (int k = 0; k < NK; ++k) {
+    for (int k = 0; k < 2; ++k) {
       if (TILE) fetch(k);
       const float* xk = TILE ? xv : xv + 32 * k;
       uint32_t pk[16];
@@ -421,14 +435,19 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
 #pragma unroll
         for (int i = 0; i < 16; ++i) stash[16 * k + i] = pk[i];
       }
-      tc::tmem_st16(rt + 16 * k, pk);
+      tc::tmem_st16(buf + 16 * k, pk);
     }
-    // O_t rescale. Every product into O_t issued so far is complete: the logits of
-    // this item were issued after them and have landed; the value product of this
-    // item waits for p_full.
+    // O_t rescale, once the products into O_t issued so far are complete: the last
+    // one is the previous item's (value product or order-1 product), released on the
+    // other buffer; the value product of this item waits for p_full.
+    bool waited = true;
     if (__any_sync(0xffffffffu, need_o)) {
+      if (idx > 0) {
+        waited = uni(wt.fast(bar(c.rel[t][1 - b]), ((rcnt >> (1 - b)) & 1) ^ 1, 12));
+        tc::fence_after_sync();
+      }
 #pragma unroll
-      for (int k = 0; k < D / 32; ++k) {
+      for (int k = 0; k < D / 32 && waited; ++k) {
         uint32_t v[32];
         tc::tmem_ld32(ot + 32 * k, v);
         tc::tmem_wait_ld();
@@ -445,60 +464,60 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     if (TILE) ls = ls * (float)BLK + plast * (float)(p.Nk - nkb * BLK);
     l = l * f + ls;
     tc::tmem_wait_st();
-    warp_arrive(smem_u32(&c.p_full[t]));
+    if (!waited) return false;
+    warp_arrive(bar(c.p_full[t][b]));
     return true;
   };
 
-  Walk wk;
-  Item it{kNone, 0, 0};
-  int ntile = 0, na = 0, cur_tile = 0;  // order-1 TILEs, MAT items of this tile so far
-  int since_tile = 0;                   // MAT items since the tile's TILE item
+  Walk<BLK> wk;
+  Item it{kNone, 0, 0, 0};
+  int cur_tile = 0;
   // ---- phase 0: centroid tiles and their order-1 products ----
   while (ok) {
-    it = wk.next<ORDER>(c, nkb);
+    it = wk.template next<ORDER>(c, nkb);
     if (it.kind == kExact || it.kind == kNone) break;
     if (!((it.mask >> t) & 1)) continue;
     if (it.kind == kTile) {
-      ok = s_item(it, std::integral_constant<int, KC>{}, std::true_type{});
-      since_tile = 0;
+      ok = s_item(it, std::true_type{});
       cur_tile = it.j;
       continue;
     }
     if constexpr (ORDER == 1) {
-      // Slot s of R_t (columns [s d/2, (s+1) d/2)) is free once the products that
-      // last read it are complete: the tile's value product (P sits in slot 0) for
-      // the first item after a TILE, which also covers the second (everything issued
-      // before the TILE's logits is complete); then the item two before.
-      // The operand does not depend on the slot: compute it first, then wait.
+      // The operand does not depend on the buffer: compute (the first 32 columns of) it
+      // first, then wait until the products that last read the buffer (two items
+      // back) are complete.
       const float pj = stash_get(stash, it.j - cur_tile * KC);
       const __half2 al = __float2half2_rn(pj * p.scale);
-      uint32_t a[QW];
+      auto part = [&](int k, uint32_t* a) __attribute__((always_inline)) {
 #pragma unroll
-      for (int i = 0; i < QW; ++i) {
-        const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[i]), al);
-        a[i] = *reinterpret_cast<const uint32_t*>(&y);
-      }
-      const int s = na & 1, use = na >> 1;
-      if (since_tile == 0) {
-        ok = uni(wt.fast(bar(c.pv_done[t]), ntile & 1, 15));
-        ++ntile;
-      } else if (since_tile >= 2) {
-        ok = uni(wt.fast(bar(c.a_done[t][s]), (use - 1) & 1, 10));
-      }
-      ++since_tile;
-      ++na;
+        for (int i = 0; i < 32; ++i) {
+          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&q16[32 * k + i]), al);
+          a[i] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+      };
+      uint32_t a[32];
+      part(0, a);
+      const int b = n & 1;
+      ++n;
+      if ((rany >> b) & 1) ok = uni(wt.fast(bar(c.rel[t][b]), ((rcnt >> b) & 1) ^ 1, 10));
+      rcnt ^= 1u << b;
+      rany |= 1u << b;
       if (!ok) break;
       tc::fence_after_sync();
+      tc::tmem_st32(rt + 64 * b, a);
 #pragma unroll
-      for (int k = 0; k < QW / 32; ++k) tc::tmem_st32(rt + s * (D / 2) + 32 * k, a + 32 * k);
+      for (int k = 1; k < QW / 32; ++k) {
+        part(k, a);
+        tc::tmem_st32(rt + 64 * b + 32 * k, a);
+      }
       tc::tmem_wait_st();
-      warp_arrive(bar(c.a_full[t][s]));
+      warp_arrive(bar(c.a_full[t][b]));
     }
   }
   // ---- phase 1: kept blocks ----
   while (ok && it.kind == kExact) {
-    if ((it.mask >> t) & 1) ok = s_item(it, std::integral_constant<int, BLK>{}, std::false_type{});
-    it = wk.next<ORDER>(c, nkb);
+    if ((it.mask >> t) & 1) ok = s_item(it, std::false_type{});
+    it = wk.template next<ORDER>(c, nkb);
   }
 
   // ---- epilogue: O / l ----
@@ -561,13 +580,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       tc::mbar_init(bar(c.empty[u]), NT);  // one release per MMA thread
     }
     for (int t = 0; t < NT; ++t) {
-      tc::mbar_init(bar(c.s_full[t]), 1);
-      tc::mbar_init(bar(c.pv_done[t]), 1);
       tc::mbar_init(bar(c.o_final[t]), 1);
-      tc::mbar_init(bar(c.p_full[t]), 4);
-      for (int s = 0; s < 2; ++s) {
-        tc::mbar_init(bar(c.a_done[t][s]), 1);
-        tc::mbar_init(bar(c.a_full[t][s]), 4);
+      for (int b = 0; b < 2; ++b) {
+        tc::mbar_init(bar(c.s_full[t][b]), 1);
+        tc::mbar_init(bar(c.rel[t][b]), 1);
+        tc::mbar_init(bar(c.p_full[t][b]), 4);
+        tc::mbar_init(bar(c.a_full[t][b]), 4);
       }
     }
     tc::mbar_init(bar(c.q_full), 1);
@@ -625,7 +643,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         for (int s = 0; s < SUB; ++s)
           tc::tma_load_3d(base + OFF_Q + t * By::Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s,
                           q0 + t * TQ, bh);
-      StepGen gen;
+      StepGen<BLK> gen;
       int u = 0;
       bool ok = true;
       while (ok) {
@@ -637,45 +655,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         if (!ok) break;
         const int slot = u % NU;
         const uint32_t fb = bar(c.full[slot]);
-        // The MMA thread reads the record after the unit's full barrier.
+        // The MMA threads read the record after the unit's full barrier.
         c.evq[slot] = make_int4(encode(s), s.cur_j, s.pend_j, 0);
         if (s.type == stEnd) {
           tc::mbar_arrive(fb);  // terminal record, no data
           ++u;
           break;
         }
-        auto dst = [&](int i) { return base + OFF_U + ((u + i) % NU) * UNIT; };
+        // piece slot k of the step: unit k / 2, half k % 2
+        auto piece = [&](int k) { return base + OFF_U + ((u + k / 2) % NU) * UNIT + (k % 2) * HALF; };
         uint32_t bytes = 0;
-        if (s.type != stMat && s.pend_mask) bytes += s.pend_kind == kTile ? By::VS : By::KV;
-        if (s.type == stSX) bytes += s.cur_kind == kTile ? 2 * By::KB : By::KV;
-        if (s.type == stMat) bytes += By::M;
+        if (s.type == stMat) bytes = By::M;
+        else bytes = By::PIECE * ((s.pend_mask ? 1 : 0) + (s.type == stSX ? (s.cur_kind == kTile ? 2 : 1) : 0));
         // every load of the step completes on the first unit's barrier
         tc::mbar_arrive_expect_tx(fb, bytes);
-        int ui = 0;
-        if (s.type != stMat && s.pend_mask) {  // values of the pending item
-          if (s.pend_kind == kTile) {
-            for (int k = 0; k < SUB; ++k)
-              tc::tma_load_3d(dst(0) + k * KC * 128, &p.tmVs, fb, 64 * k, s.pend_j * KC, bh);
-          } else {
-            for (int k = 0; k < SUB; ++k)
-              tc::tma_load_3d(dst(0) + k * BLK * 128, &p.tmV, fb, 64 * k, s.pend_j * BLK, bh);
+        int k = 0;
+        if (s.type == stMat) {
+          for (int x = 0; x < SUB; ++x)
+            tc::tma_load_3d(piece(0) + x * D * 128, &p.tmM, fb, 64 * x, 0, bh * nkb + s.cur_j);
+        } else {
+          if (s.pend_mask) {  // values of the pending item
+            if (s.pend_kind == kTile) {
+              for (int x = 0; x < SUB; ++x)
+                tc::tma_load_3d(piece(0) + x * 64 * 128, &p.tmVs, fb, 64 * x, s.pend_j * KC, bh);
+            } else {
+              for (int x = 0; x < SUB; ++x)
+                tc::tma_load_3d(piece(0) + x * 64 * 128, &p.tmV, fb, 64 * x,
+                                s.pend_j * BLK + 64 * s.pend_half, bh);
+            }
+            k = 1;
           }
-          ui = 1;
-        }
-        if (s.type == stSX) {  // keys of the new item
-          if (s.cur_kind == kTile) {
-            for (int pl = 0; pl < 2; ++pl)
-              for (int k = 0; k < SUB; ++k)
-                tc::tma_load_3d(dst(ui) + pl * By::KB + k * KC * 128, &p.tmKb, fb, 64 * k,
-                                s.cur_j * KC, 2 * bh + pl);
-          } else {
-            for (int k = 0; k < SUB; ++k)
-              tc::tma_load_3d(dst(ui) + k * BLK * 128, &p.tmK, fb, 64 * k, s.cur_j * BLK, bh);
+          if (s.type == stSX) {  // keys of the new item
+            if (s.cur_kind == kTile) {
+              for (int pl = 0; pl < 2; ++pl)
+                for (int x = 0; x < SUB; ++x)
+                  tc::tma_load_3d(piece(k + pl) + x * 64 * 128, &p.tmKb, fb, 64 * x, s.cur_j * KC,
+                                  2 * bh + pl);
+            } else {
+              for (int x = 0; x < SUB; ++x)
+                tc::tma_load_3d(piece(k) + x * 64 * 128, &p.tmK, fb, 64 * x,
+                                s.cur_j * BLK + 64 * s.cur_half, bh);
+            }
           }
         }
-        if (s.type == stMat)
-          for (int k = 0; k < SUB; ++k)
-            tc::tma_load_3d(dst(0) + k * D * 128, &p.tmM, fb, 64 * k, 0, bh * nkb + s.cur_j);
         // the second unit's barrier only keeps its phase count in step
         if (s.nunits == 2) tc::mbar_arrive(bar(c.full[(u + 1) % NU]));
         u += s.nunits;
@@ -689,15 +711,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
     // ===================== MMA issuers: warp 9 + t for tile t =====================
     if (lane == 0) {
       const int t = warp - 9;
-      constexpr uint32_t I_S_TILE = tc::idesc_f16(1, 1, 0, KC);
-      constexpr uint32_t I_S_EX = tc::idesc_f16(1, 1, 0, BLK);
+      constexpr uint32_t I_S = tc::idesc_f16(1, 1, 0, 64);
       constexpr uint32_t I_PV = tc::idesc_f16(0, 0, 1, D);
       bool ok = wt.wait(bar(c.init_done), 0, 2) && wt.wait(bar(c.q_full), 0, 3);
       tc::fence_after_sync();
       const uint32_t o_t = tmem + COL_O + 128 * t, r_t = tmem + COL_R + 128 * t;
       // Descriptor base of Q_t; per k-step only the start-address field (low bits) moves.
       const uint64_t dq = tc::sdesc(base + OFF_Q + t * By::Q, 16, 1024);
-      int np = 0, na = 0;  // p_full phases; order-1 items of this tile
+      int n = 0;                // items of this tile; item n uses buffer n & 1
+      uint32_t pph = 0, aph = 0;  // p_full / a_full phase parities, bit b for buffer b
+      int pbuf = 0;             // buffer of this tile's pending item
       for (int u = 0; ok;) {
         const int slot = u % NU;
         ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
@@ -707,53 +730,61 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         const int cm = (rec >> 12) & 3, pm = (rec >> 14) & 3, nun = (rec >> 16) & 3;
         if (type == stEnd) break;
         const int slot2 = (u + 1) % NU;
-        const uint32_t src0 = base + OFF_U + slot * UNIT, src1 = base + OFF_U + slot2 * UNIT;
+        auto piece = [&](int k) {
+          return base + OFF_U + (k / 2 ? slot2 : slot) * UNIT + (k % 2) * HALF;
+        };
         bool issued = false;
         if (type == stMat) {
           if ((cm >> t) & 1) {
-            const int s = na & 1, use = na >> 1;
-            ++na;
-            ok = wt.fast(bar(c.a_full[t][s]), use & 1, 7);
+            const int b = n & 1;
+            ++n;
+            ok = wt.fast(bar(c.a_full[t][b]), (aph >> b) & 1, 7);
+            aph ^= 1u << b;
             if (!ok) break;
             tc::fence_after_sync();
-            const uint64_t b0 = tc::sdesc(src0, D * 128, 1024);
+            const uint64_t b0 = tc::sdesc(piece(0), D * 128, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              tc::mma_ts(o_t, r_t + s * (D / 2) + kk * 8, b0 + ((kk * 2048) >> 4), I_PV, 1);
-            tc::mma_commit(bar(c.a_done[t][s]));
+              tc::mma_ts(o_t, r_t + 64 * b + kk * 8, b0 + ((kk * 2048) >> 4), I_PV, 1);
+            tc::mma_commit(bar(c.rel[t][b]));
             issued = true;
           }
         } else {
-          // SX / FLUSH: value product of the pending item, then logits of the new one
-          if ((pm >> t) & 1) {
-            ok = wt.fast(bar(c.p_full[t]), np & 1, 6);
-            ++np;
-            if (!ok) break;
-            tc::fence_after_sync();
-            const int rows = pk == kTile ? KC : BLK;
-            const uint64_t bd = tc::sdesc(src0, rows * 128, 1024);
-            for (int kk = 0; kk < rows / 16; ++kk)
-              tc::mma_ts(o_t, r_t + kk * 8, bd + ((kk * 2048) >> 4), I_PV, 1);
-            if (ORDER == 1 && pk == kTile) tc::mma_commit(bar(c.pv_done[t]));
-            issued = true;
-          }
+          const int kp = pm ? 1 : 0;  // piece of the new item's keys
+          int nbuf = pbuf;
+          // logits of the new item first, into this tile's next buffer
           if (type == stSX && ((cm >> t) & 1)) {
-            const bool tile = ck == kTile;
-            const int rows = tile ? KC : BLK;
-            const uint64_t bd0 = tc::sdesc(pm ? src1 : src0, 16, 1024);
-            const uint32_t idesc = tile ? I_S_TILE : I_S_EX;
-            // tile: the hi plane, then the lo plane of the centroids, into the same logits
-            const int planes = tile ? 2 : 1;
-            for (int pl = 0; pl < planes; ++pl)
+            const int b = n & 1;
+            ++n;
+            const uint32_t dt = r_t + 64 * b;
+            const int planes = ck == kTile ? 2 : 1;  // centroids: hi plane, then lo plane
+            for (int pl = 0; pl < planes; ++pl) {
+              const uint64_t bd = tc::sdesc(piece(kp + pl), 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t aoff = ((kk / 4) * TQ * 128 + (kk % 4) * 32) >> 4;
-                const uint32_t boff = (pl * By::KB + (kk / 4) * rows * 128 + (kk % 4) * 32) >> 4;
-                tc::mma_ss(r_t, dq + aoff, bd0 + boff, idesc, (pl | kk) > 0);
+                const uint32_t boff = ((kk / 4) * 64 * 128 + (kk % 4) * 32) >> 4;
+                tc::mma_ss(dt, dq + aoff, bd + boff, I_S, (pl | kk) > 0);
               }
-            tc::mma_commit(bar(c.s_full[t]));
+            }
+            tc::mma_commit(bar(c.s_full[t][b]));
+            nbuf = b;
             issued = true;
           }
+          // then the value product of the pending item, once its P is written
+          if ((pm >> t) & 1) {
+            ok = wt.fast(bar(c.p_full[t][pbuf]), (pph >> pbuf) & 1, 6);
+            pph ^= 1u << pbuf;
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint64_t bd = tc::sdesc(piece(0), 64 * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc::mma_ts(o_t, r_t + 64 * pbuf + kk * 8, bd + ((kk * 2048) >> 4), I_PV, 1);
+            tc::mma_commit(bar(c.rel[t][pbuf]));
+            issued = true;
+          }
+          pbuf = nbuf;
         }
         // Release the step's units: after this thread's products have read them, or at
         // once if it issued none.
@@ -817,8 +848,8 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   Params p;
   const uint64_t bh = (uint64_t)a.B * a.H;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  bool ok = map3d(&p.tmQ, BF, a.q, D, a.Nq, bh, TQ) && map3d(&p.tmK, BF, a.k, D, a.Nk, bh, BLK) &&
-            map3d(&p.tmV, HF, a.v, D, a.Nk, bh, BLK) &&
+  bool ok = map3d(&p.tmQ, BF, a.q, D, a.Nq, bh, TQ) && map3d(&p.tmK, BF, a.k, D, a.Nk, bh, 64) &&
+            map3d(&p.tmV, HF, a.v, D, a.Nk, bh, 64) &&
             map3d(&p.tmKb, BF, a.kbar16, D, a.nkb, 2 * bh, KC) &&
             map3d(&p.tmVs, HF, a.vsum16, D, a.nkb, bh, KC);
   if (ORDER == 1) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh * a.nkb, D);
