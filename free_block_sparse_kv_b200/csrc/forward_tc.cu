@@ -21,7 +21,7 @@
 //              than 2^11), write P back to TMEM as the A operand of the value product,
 //              and build the order-1 operand A_j = (scale * alpha_tj) q_t in TMEM.
 //   warp 8     TMA producer: both Q tiles once, then every operand through a ring of
-//              5 x 32 KB units (each unit holds two 16 KB pieces or one M_j).
+//              4 x 32 KB units (each unit holds two 16 KB pieces or one M_j).
 //   warps 9-10 one MMA-issuing thread per tile (warp 9 also allocates TMEM). Issuing
 //              a 128x128x16 tcgen05.mma takes about as long as the tensor core takes to
 //              run it, so one thread cannot also wait and commit without leaving the
@@ -59,7 +59,7 @@ namespace tcf {
 constexpr int TQ = 128;        // query rows per tile
 constexpr int NT = 2;          // tiles per CTA
 constexpr int KC = 64;         // centroids per TILE item; keys per EXACT item
-constexpr int NU = 5;          // ring units
+constexpr int NU = 4;          // ring units
 constexpr int UNIT = 32768;    // bytes per ring unit
 constexpr int HALF = UNIT / 2; // bytes per piece slot
 constexpr int MAXW = 64;       // bitmap words (2048 blocks)
@@ -67,7 +67,7 @@ constexpr int NSOFT = 256;     // softmax threads (2 warpgroups, one per tile)
 constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, 2 MMA, 1 idle)
 // Register split after launch (168 per thread at launch = 64,512 per CTA): the
 // control warpgroup gives registers back, the softmax warpgroups take them.
-constexpr int kRegCtl = 104, kRegSoft = 200;
+constexpr int kRegCtl = 72, kRegSoft = 216;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
 constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
@@ -77,7 +77,9 @@ constexpr uint32_t COL_O = 0, COL_R = 256;
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr int OFF_Q = 0;                        // Q tiles, bf16, swizzled (2 x 32 KB)
 constexpr int OFF_U = 65536;                    // ring
-constexpr int OFF_CTL = OFF_U + NU * UNIT;      // control block (2 KB)
+constexpr int OFF_STASH = OFF_U + NU * UNIT;    // P of each tile's current centroid tile,
+                                                // fp16 [tile][column][row] (32 KB)
+constexpr int OFF_CTL = OFF_STASH + NT * 64 * TQ * 2;  // control block (2 KB)
 constexpr int SMEM_BYTES = OFF_CTL + 2048 + 1024;
 
 struct Params {
@@ -247,32 +249,6 @@ struct Bytes {
   static_assert(PIECE <= HALF && M <= UNIT, "ring pieces");
 };
 
-// Element c (0..63) of a row's 64 fp16 probabilities held as 32 packed registers;
-// c is the same for every thread of the warp. A tree of selects on the bits of c
-// (inline PTX, so that the compiler does not turn it into an indexed load from local
-// memory).
-SA_DEVI uint32_t sel(bool p, uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("{\n .reg .pred q;\n setp.ne.u32 q, %3, 0;\n selp.b32 %0, %1, %2, q;\n}\n"
-      : "=r"(r) : "r"(a), "r"(b), "r"((uint32_t)p));
-  return r;
-}
-SA_DEVI float stash_get(const uint32_t* st, int c) {
-  const int i = c >> 1;
-  uint32_t l1[16], l2[8], l3[4], l4[2];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) l1[k] = sel(i & 1, st[2 * k + 1], st[2 * k]);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) l2[k] = sel(i & 2, l1[2 * k + 1], l1[2 * k]);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) l3[k] = sel(i & 4, l2[2 * k + 1], l2[2 * k]);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) l4[k] = sel(i & 8, l3[2 * k + 1], l3[2 * k]);
-  const uint32_t v = sel(i & 16, l4[1], l4[0]);
-  const uint16_t hv = (c & 1) ? (uint16_t)(v >> 16) : (uint16_t)(v & 0xffffu);
-  return __half2float(__ushort_as_half(hv));
-}
-
 // Softmax warpgroup of tile t = warp / 4. Thread (warp w, lane l) owns query row
 // r = 32*(w%4) + l of the tile: all its logits, its running max and sum, its O row.
 template <int D, int BLK, int ORDER>
@@ -330,7 +306,8 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   // Per-buffer phase parities as bit masks (bit b for buffer b): next s_full wait;
   // number of items so far (rel phases); whether the buffer has been used.
   uint32_t sph = 0, rcnt = 0, rany = 0;
-  uint32_t stash[ORDER == 1 ? KC / 2 : 1];  // P of the current centroid tile, fp16 pairs
+  // P of the current centroid tile, this thread's row: stash[c * TQ] is column c
+  uint16_t* stash = reinterpret_cast<uint16_t*>(gbase + OFF_STASH) + t * 64 * TQ + r;
   const uint64_t sl2x2 = tc::f2(sl2, sl2);
 
   // One TILE or EXACT item: this thread's 64 logits in buffer b.
@@ -426,14 +403,17 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
         float y0, y1;
         tc::f2_split(y, y0, y1);
         const float x0 = tc::ex2(y0), x1 = tc::ex2(y1);
-        const uint64_t e = tc::f2(x0, x1);
-        if ((i / 2) & 1) acc1 = tc::add2(acc1, e); else acc0 = tc::add2(acc0, e);
+        const uint64_t ev = tc::f2(x0, x1);
+        if ((i / 2) & 1) acc1 = tc::add2(acc1, ev); else acc0 = tc::add2(acc0, ev);
         pk[i / 2] = pack_f16(x0, x1);
         if (TILE) plast = (32 * k + i == jl) ? x0 : ((32 * k + i + 1 == jl) ? x1 : plast);
       }
       if constexpr (TILE && ORDER == 1) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) stash[16 * k + i] = pk[i];
+        for (int i = 0; i < 16; ++i) {
+          stash[(32 * k + 2 * i) * TQ] = (uint16_t)(pk[i] & 0xffffu);
+          stash[(32 * k + 2 * i + 1) * TQ] = (uint16_t)(pk[i] >> 16);
+        }
       }
       tc::tmem_st16(buf + 16 * k, pk);
     }
@@ -483,10 +463,10 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       continue;
     }
     if constexpr (ORDER == 1) {
-      // The operand does not depend on the buffer: compute (the first 32 columns of) it
+      // The operand does not depend on the buffer: compute (its first 32 columns)
       // first, then wait until the products that last read the buffer (two items
       // back) are complete.
-      const float pj = stash_get(stash, it.j - cur_tile * KC);
+      const float pj = __half2float(__ushort_as_half(stash[(it.j - cur_tile * KC) * TQ]));
       const __half2 al = __float2half2_rn(pj * p.scale);
       auto part = [&](int k, uint32_t* a) __attribute__((always_inline)) {
 #pragma unroll
