@@ -14,6 +14,7 @@ bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -83,6 +84,38 @@ def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dic
                 if w.order == 1:
                     order1 += 2.0 * nq[i] * w.d * w.d * skipped
     return dict(exact=exact, order0=order0, order1=order1, total=exact + order0 + order1)
+
+
+FORWARD_SOURCES = ("forward_tc.cu", "tc.cuh", "common.cuh")
+
+
+def forward_sources_sha256() -> str:
+    """Hash of the forward kernel's sources, to tell whether a DRAM capture still applies."""
+    h = hashlib.sha256()
+    for name in FORWARD_SOURCES:
+        with open(os.path.join(ROOT, "free_block_sparse_kv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def forward_traffic(w: W.Workload):
+    """DRAM bytes (read + write) of one forward launch on this workload, from the ncu capture
+    summarised under profiles/, or None when there is none or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", f"forward_dram_{w.name}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                key, _, val = line.strip().partition(":")
+                vals[key.strip("- `")] = val.strip().strip("`")
+    try:
+        if vals.get("sources_sha256") != forward_sources_sha256():
+            return None
+        return float(vals["dram_bytes_read_per_launch"]) + float(vals["dram_bytes_write_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def pool_bytes(w: W.Workload, with_q: bool) -> float:
@@ -351,7 +384,8 @@ def main():
                           stage_ms[1], "forward": stage_ms[2]},
             "roofline": {"kernel": "sparse_attn_forward", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": forward_traffic(w),
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                          "peak_kind": f"bf16 sustained ({pk['source']})",
                          "flops_per_launch": fl},
             "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")

@@ -179,6 +179,13 @@ SA_DEVI uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
 
 // Instruction descriptor for kind::f16 with fp32 accumulation; M = 128.
 // fmt: 0 = f16, 1 = bf16. b_mn: 0 = B K-major, 1 = B MN-major. A is K-major.
+// Same with the major-ness of A selectable (a_mn = 1: A is M-major, e.g. the transpose of a
+// row-major tile) and the M dimension.
+__host__ __device__ constexpr uint32_t idesc_f16_mn(int a_fmt, int b_fmt, int a_mn, int b_mn, int N,
+                                                    int M) {
+  return (1u << 4) | ((uint32_t)a_fmt << 7) | ((uint32_t)b_fmt << 10) | ((uint32_t)a_mn << 15) |
+         ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_f16(int a_fmt, int b_fmt, int b_mn, int N) {
   return (1u << 4) | ((uint32_t)a_fmt << 7) | ((uint32_t)b_fmt << 10) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
