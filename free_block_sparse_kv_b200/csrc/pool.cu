@@ -205,15 +205,17 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
     tc::fence_after_sync();
     const int a = 32 * (warp & 3) + lane;
     constexpr int HC = D / 2;  // columns per thread
-    uint16_t* mg = M + (((size_t)bh * nkb + j) * D + (a < D ? a : 0)) * D;
+    constexpr int ROWB = D * 2;
+    static_assert(D * ROWB <= 2 * G::TILE, "M stage");
     const float ka = a < D ? ks[a] : 0.f;
+    // fp16 rows into the (consumed) K and V tiles, then coalesced 16-byte stores
 #pragma unroll
     for (int cb = 0; cb < HC; cb += 32) {
       const int c0 = (warp >> 2) * HC + cb;
       uint32_t x[32];
       tc::tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, x);
       tc::tmem_wait_ld();
-      if (done && a < D) {
+      if (a < D) {
         uint32_t h[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
@@ -221,9 +223,16 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                           __uint_as_float(x[2 * e + 1]) - ka * vs[c0 + 2 * e + 1]);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(mg + c0 + 8 * e) =
+          *reinterpret_cast<uint4*>(sk + swz(a, c0 / 8 + e, ROWB)) =
               make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]);
       }
+    }
+    __syncthreads();
+    if (done) {
+      uint16_t* mg = M + ((size_t)bh * nkb + j) * D * D;
+      for (int r = r0; r < D; r += RPP)
+        *reinterpret_cast<uint4*>(mg + (size_t)r * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(sk + swz(r, ch, ROWB));
     }
     tc::fence_before_sync();
     __syncthreads();
