@@ -89,8 +89,23 @@ struct Params {
   void* out;
   int32_t* err_flag;
   int cap, Nq, Nk, nqb, nkb, out_dtype;
+  int nx, nbh;  // CTAs (pairs of query tiles) per (batch, head); batch x heads
   float scale;
 };
+
+// The CTA's pair of query tiles and its (batch, head). The grid is one-dimensional and
+// puts every (batch, head)'s last pair, which may hold fewer rows, after all full pairs,
+// so that the shorter CTAs fill the last wave.
+SA_DEVI void cta_coords(const Params& p, int& x, int& bh) {
+  const int L = blockIdx.x, nfull = p.nx - 1;
+  if (L < nfull * p.nbh) {
+    x = L % nfull;
+    bh = L / nfull;
+  } else {
+    x = p.nx - 1;
+    bh = L - nfull * p.nbh;
+  }
+}
 
 struct Ctl {  // control block in shared memory
   uint64_t full[NU], empty[NU];
@@ -253,7 +268,7 @@ struct Bytes {
 // r = 32*(w%4) + l of the tile: all its logits, its running max and sum, its O row.
 template <int D, int BLK, int ORDER>
 SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem, tc::Waiter& wt,
-                          int warp, int lane) {
+                          int warp, int lane, int cx, int bh) {
   using By = Bytes<D, BLK>;
   constexpr int QW = D / 2;  // fp16 pairs per query row
   const int t = warp >> 2, qw = warp & 3;
@@ -264,7 +279,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   const int h = BLK == 64 ? (r >> 6) : 0;                  // query block of the row
   const float sl2 = p.scale * kLog2e;
   const int nkb = p.nkb;
-  const int bh = blockIdx.y, row0 = blockIdx.x * (NT * TQ) + t * TQ;
+  const int row0 = cx * (NT * TQ) + t * TQ;
   const uint32_t* kept_h = c.kept[t][h];
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
   auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
@@ -543,8 +558,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * (NT * TQ);
+  int cx, bh;
+  cta_coords(p, cx, bh);
+  const int q0 = cx * (NT * TQ);
   const int nkb = p.nkb;
 
   // A failure reported by an earlier CTA (or call) makes the rest of the grid skip
@@ -610,7 +626,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegSoft));
-    softmax_role<D, BLK, ORDER>(p, c, gbase, tmem, wt, warp, lane);
+    softmax_role<D, BLK, ORDER>(p, c, gbase, tmem, wt, warp, lane, cx, bh);
   } else {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegCtl));
   if (warp == 8) {
@@ -846,10 +862,13 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   p.nkb = a.nkb;
   p.out_dtype = a.out_dtype;
   p.scale = a.scale;
+  p.nx = (a.Nq + NT * TQ - 1) / (NT * TQ);
+  p.nbh = (int)bh;
+  if ((uint64_t)p.nx * bh > 0x7fffffffull) return cudaErrorInvalidValue;
   auto kern = forward_tc_kernel<D, BLK, ORDER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Nq + NT * TQ - 1) / (NT * TQ), a.B * a.H);
+  dim3 grid(p.nx * p.nbh);
   kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(p);
   return cudaGetLastError();
 }
