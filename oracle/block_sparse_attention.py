@@ -36,7 +36,16 @@ design notes):
     (cumulative >= tau);
   * structured mode: anchors G_s = {(s mod T_per) + T_per * m}, window
     [t - W, t + W] clipped to the video; a KV block is kept for a query block
-    when any (query token, key token) pair of the two blocks is allowed.
+    when any (query token, key token) pair of the two blocks is allowed;
+  * hybrid order (order 2, PISA "Algorithme Central", global first-order
+    correction): Hbar is the plain mean of the per-block matrices M_j over all
+    blocks of the head, and the numerator gains scale * q_t Hbar * sum_j alpha_tj
+    over the skipped blocks (no denominator term, as for order 1);
+  * covariance-aware top-k (PISA "Routage Sensible a la Covariance"): the
+    norm ||H_j - Hbar||_2 is read as the 2-norm of the matrix entries
+    (Frobenius), and the selection score is s_ij + ln ||H_j - Hbar||, the log of
+    the first-order error bound alpha_ij * scale * |qbar_i| * ||H_j - Hbar||
+    up to a term that is the same for every block of the row.
 """
 from __future__ import annotations
 
@@ -84,6 +93,19 @@ def pool_keys_values(k: np.ndarray, v: np.ndarray, block: int, order: int):
             mats.append((kj - kb).T @ vj)
     m = np.stack(mats) if order == 1 else None
     return np.stack(kbar), np.stack(vsum), np.asarray(counts, dtype=np.int64), m
+
+
+def global_first_order(mats: np.ndarray) -> np.ndarray:
+    """Hbar = mean over all blocks of the per-block first-order matrices M_j
+    [PISA §2 "Algorithme Central": global first-order statistic]."""
+    return np.asarray(mats, np.float64).mean(axis=0)
+
+
+def covariance_norms(mats: np.ndarray, hbar: np.ndarray) -> np.ndarray:
+    """||M_j - Hbar|| per block, as the 2-norm of the matrix entries
+    [PISA §2 "Routage Sensible a la Covariance"]."""
+    diff = np.asarray(mats, np.float64) - np.asarray(hbar, np.float64)[None]
+    return np.sqrt((diff * diff).sum(axis=(1, 2)))
 
 
 # ---------------------------------------------------------------------------
@@ -187,7 +209,7 @@ def structured_kept(Nq: int, Nk: int, block: int, frame_tokens: int, n_frames: i
 
 def forward_rows(q_rows: np.ndarray, row_qblock, k: np.ndarray, v: np.ndarray,
                  kbar: np.ndarray, vsum: np.ndarray, counts: np.ndarray, mats,
-                 kept, block: int, order: int, scale: float) -> np.ndarray:
+                 kept, block: int, order: int, scale: float, hbar=None) -> np.ndarray:
     """Output rows o_t = N_t / D_t for the query rows q_rows.
 
     row_qblock[t] is the query block of row t; kept[i] lists the kept KV blocks
@@ -196,8 +218,10 @@ def forward_rows(q_rows: np.ndarray, row_qblock, k: np.ndarray, v: np.ndarray,
       centroid logits c_j  = scale * q_t . kbar_j     for skipped blocks j
       m = max of all of them
       N_t = sum_r e^(l_r - m) v_r
-            + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j)
+            + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j
+                                     + [order 2] scale * q_t Hbar)
       D_t = sum_r e^(l_r - m) + sum_j e^(c_j - m) n_j
+    Order 2 (hybrid) needs ``hbar``, the mean of the per-block M_j.
     """
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -222,22 +246,40 @@ def forward_rows(q_rows: np.ndarray, row_qblock, k: np.ndarray, v: np.ndarray,
                 term += scale * (qt @ mats[j])
             num += w * term
             den += w * counts[j]
+        if order == 2 and skipped:
+            num += scale * wc.sum() * (qt @ hbar)
         out[t] = num / den
     return out
 
 
 def forward_head(q, k, v, kept, block: int, order: int, scale: float, rows=None):
     """Pool K/V and run :func:`forward_rows` on all rows of a head, or on ``rows``."""
-    kbar, vsum, counts, mats = pool_keys_values(k, v, block, order)
+    kbar, vsum, counts, mats = pool_keys_values(k, v, block, 1 if order == 2 else order)
+    hbar = global_first_order(mats) if order == 2 else None
     q = np.asarray(q, np.float64)
     rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
     return forward_rows(q[rows], rows // block, k, v, kbar, vsum, counts, mats,
-                        kept, block, order, scale)
+                        kept, block, order, scale, hbar=hbar)
 
 
-def route_head(q, k, block: int, mode: str, scale: float, keep=None, tau=None):
-    """Pooled routing for one head. Returns (kept lists, scores, prefix lengths)."""
+def covariance_scores(scores: np.ndarray, cnorms: np.ndarray) -> np.ndarray:
+    """Covariance-aware selection scores s_ij + ln ||M_j - Hbar||
+    [PISA §2 "Routage Sensible a la Covariance"]."""
+    with np.errstate(divide="ignore"):
+        return np.asarray(scores, np.float64) + np.log(np.asarray(cnorms, np.float64))[None, :]
+
+
+def route_head(q, k, block: int, mode: str, scale: float, keep=None, tau=None, v=None):
+    """Pooled routing for one head. Returns (kept lists, scores, prefix lengths).
+
+    mode "topk_cov" needs ``v`` (for the per-block M_j) and returns the
+    covariance-aware scores."""
     qbar = pool_queries(q, block)
+    if mode == "topk_cov":
+        kbar, _, _, mats = pool_keys_values(k, v, block, 1)
+        s = covariance_scores(routing_scores(qbar, kbar, scale),
+                              covariance_norms(mats, global_first_order(mats)))
+        return route_topk(s, keep), s, [keep] * s.shape[0]
     kbar = pool_keys_values(k, np.zeros((k.shape[0], 1)), block, 0)[0]
     s = routing_scores(qbar, kbar, scale)
     if mode == "topk":

@@ -261,3 +261,68 @@ def test_mass_boundary_is_inclusive(golden_dir):
     g = _load(golden_dir, "routing_d4.json")
     kept, cnt = O.route_mass(np.array(g["equal_scores"]), g["equal_scores_tau"])
     assert kept[0].tolist() == g["equal_scores_kept"] and cnt[0] == 2
+
+
+# ---------------------------------------------------------------------------
+# Hybrid order (global first-order matrix) and covariance-aware routing
+# ---------------------------------------------------------------------------
+
+def _shared_deviation_head(n_blocks, block, d, seed, sign=None):
+    """Keys c_j + e_r and values s_j * w_r: every block has the same deviations e_r
+    (summing to zero over the block) and the same values up to a sign s_j, so
+    M_j = s_j * sum_r e_r w_r^T is one matrix for all blocks (or its negative)."""
+    rng = np.random.default_rng(seed)
+    e = rng.standard_normal((block, d))
+    e -= e.mean(axis=0)
+    w = rng.standard_normal((block, d))
+    sign = np.ones(n_blocks) if sign is None else np.asarray(sign, float)
+    centers = rng.standard_normal((n_blocks, d))
+    k = np.concatenate([centers[j] + e for j in range(n_blocks)])
+    v = np.concatenate([sign[j] * w for j in range(n_blocks)])
+    q = rng.standard_normal((n_blocks * block, d))
+    return q, k, v
+
+
+def test_hybrid_equals_per_block_order1_when_blocks_share_their_first_order_matrix():
+    q, k, v = _shared_deviation_head(4, 16, 8, seed=11)
+    kbar, vsum, counts, mats = O.pool_keys_values(k, v, 16, 1)
+    np.testing.assert_allclose(mats, np.broadcast_to(mats[0], mats.shape), atol=1e-12)
+    np.testing.assert_allclose(O.global_first_order(mats), mats[0], atol=1e-12)
+    kept = [np.array([i]) for i in range(4)]
+    o1 = O.forward_head(q, k, v, kept, 16, 1, 0.3)
+    o2 = O.forward_head(q, k, v, kept, 16, 2, 0.3)
+    o0 = O.forward_head(q, k, v, kept, 16, 0, 0.3)
+    np.testing.assert_allclose(o2, o1, atol=1e-12)
+    assert np.abs(o2 - o0).max() > 1e-3  # the first-order term is present
+
+
+def test_hybrid_equals_order0_when_the_mean_first_order_matrix_vanishes():
+    q, k, v = _shared_deviation_head(4, 16, 8, seed=12, sign=[1, -1, 1, -1])
+    _, _, _, mats = O.pool_keys_values(k, v, 16, 1)
+    np.testing.assert_allclose(O.global_first_order(mats), 0.0, atol=1e-12)
+    kept = [np.array([i]) for i in range(4)]
+    np.testing.assert_allclose(O.forward_head(q, k, v, kept, 16, 2, 0.3),
+                               O.forward_head(q, k, v, kept, 16, 0, 0.3), atol=1e-12)
+
+
+def test_covariance_norms_hand_example():
+    # block 1: keys (+-1, 0), values (+-1/2, 0) -> M_1 = [[1, 0], [0, 0]]
+    # block 2: keys (0, +-1), values (0, +-1/2) -> M_2 = [[0, 0], [0, 1]]
+    k = np.array([[1.0, 0.0], [-1.0, 0.0], [0.0, 1.0], [0.0, -1.0]])
+    v = np.array([[0.5, 0.0], [-0.5, 0.0], [0.0, 0.5], [0.0, -0.5]])
+    _, _, _, mats = O.pool_keys_values(k, v, 2, 1)
+    np.testing.assert_allclose(mats[0], [[1, 0], [0, 0]], atol=1e-15)
+    np.testing.assert_allclose(mats[1], [[0, 0], [0, 1]], atol=1e-15)
+    hbar = O.global_first_order(mats)
+    np.testing.assert_allclose(hbar, [[0.5, 0], [0, 0.5]], atol=1e-15)
+    np.testing.assert_allclose(O.covariance_norms(mats, hbar), [math.sqrt(0.5)] * 2, atol=1e-15)
+
+
+def test_covariance_score_can_overtake_the_attention_score():
+    # scores 1.0 and 0.9; norms 1 and e: the second block gains ln e = 1 and wins top-1
+    s = np.array([[1.0, 0.9]])
+    c = np.array([1.0, math.e])
+    cs = O.covariance_scores(s, c)
+    np.testing.assert_allclose(cs, [[1.0, 1.9]], atol=1e-15)
+    assert [list(x) for x in O.route_topk(cs, 1)] == [[1]]
+    assert [list(x) for x in O.route_topk(s, 1)] == [[0]]
