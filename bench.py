@@ -68,6 +68,7 @@ def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dic
     exact kept block j, query block i:     4 * nq_i * n_j * d
     skipped block, order 0 (logit + value): 4 * nq_i * d
     skipped block, order 1 (q M_j):         2 * nq_i * d * d
+    order 2 (q Hbar, once per query block with a skipped block): 2 * nq_i * d * d
     """
     nq = np.array([min(w.block, w.Nq - i * w.block) for i in range(w.nqb)], np.float64)
     nk = np.array([min(w.block, w.Nk - j * w.block) for j in range(w.nkb)], np.float64)
@@ -83,6 +84,8 @@ def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dic
                 order0 += 4.0 * nq[i] * w.d * skipped
                 if w.order == 1:
                     order1 += 2.0 * nq[i] * w.d * w.d * skipped
+                elif w.order == 2 and skipped:
+                    order1 += 2.0 * nq[i] * w.d * w.d
     return dict(exact=exact, order0=order0, order1=order1, total=exact + order0 + order1)
 
 
@@ -119,14 +122,18 @@ def forward_traffic(w: W.Workload):
 
 
 def pool_bytes(w: W.Workload, with_q: bool) -> float:
-    """Algorithmic HBM bytes of one pool launch: read K, V (and Q), write the tables
-    and the fp16 copy of V."""
+    """Algorithmic HBM bytes of one pool stage: read K, V (and Q), write the tables
+    and the fp16 copy of V; for order 2 also the two passes over M (global matrix,
+    covariance norms)."""
     bh = w.B * w.H
     rd = bh * w.Nk * w.d * 2 * 2 + (bh * w.Nq * w.d * 2 if with_q else 0)
     wr = bh * w.nkb * w.d * (4 + 4 + 4 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
     wr += bh * w.Nk * w.d * 2   # fp16 copy of V
-    if w.order == 1:
+    if w.order >= 1:
         wr += bh * w.nkb * w.d * w.d * 2
+    if w.order == 2:  # the global matrix and the covariance norms read the M table twice
+        rd += 2 * bh * w.nkb * w.d * w.d * 2
+        wr += bh * w.d * w.d * 6 + bh * w.nkb * 4
     return float(rd + wr)
 
 
@@ -206,8 +213,9 @@ def time_oracle(w: W.Workload, seconds: float) -> dict:
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
                                  w.n_anchors, w.period, 0, w.q_frame0)
     else:
-        kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau)[0]
-    kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, w.order)
+        kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau, v=v)[0]
+    kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, min(w.order, 1))
+    hbar = O.global_first_order(mats) if w.order == 2 else None
     t_setup = time.perf_counter() - t0
     rng = np.random.default_rng(0)
     order = rng.permutation(w.Nq)
@@ -217,7 +225,7 @@ def time_oracle(w: W.Workload, seconds: float) -> dict:
     while done < w.Nq and time.perf_counter() - t1 < seconds:
         rows = order[done:done + 16]
         O.forward_rows(q64[rows], rows // w.block, k, v, kbar, vsum, counts, mats, kept, w.block,
-                       w.order, w.scale)
+                       w.order, w.scale, hbar=hbar)
         done += len(rows)
     t_rows = time.perf_counter() - t1
     # one head's setup is amortised over its Nq rows
@@ -374,6 +382,8 @@ def main():
             "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                        "block": w.block, "order": w.order, "mode": w.mode,
                        "keep": (f"top {w.rho[0]}/{w.rho[1]}" if w.mode == "topk" else
+                                f"top {w.rho[0]}/{w.rho[1]}, covariance-aware"
+                                if w.mode == "topk_cov" else
                                 f"mass {w.tau}" if w.mode == "mass" else "window+anchors"),
                        "output": "fp32",
                        "l2": "inputs exceed L2 (Q+K+V %.2f GB per GPU)" % (
@@ -391,7 +401,7 @@ def main():
             "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")
                               / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
             "clocks": clocks.summary(),
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (5 if w.order == 2 else 3) * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

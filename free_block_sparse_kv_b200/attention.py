@@ -23,8 +23,11 @@ class Tables:
     vsum: torch.Tensor      # [B,H,nkb,d] fp32
     kbar16: torch.Tensor    # [B,H,2,nkb,d] bf16: centroid hi and lo parts
     vsum16: torch.Tensor    # [B,H,nkb,d] fp16
-    M: Optional[torch.Tensor]  # [B,H,nkb,d,d] fp16 (order 1)
+    M: Optional[torch.Tensor]  # [B,H,nkb,d,d] fp16 (order 1 or 2)
     v16: torch.Tensor       # [B,H,Nk,d] fp16 copy of V
+    hbar: Optional[torch.Tensor] = None    # [B,H,d,d] fp32 global first-order matrix (order 2)
+    hbar16: Optional[torch.Tensor] = None  # [B,H,d,d] fp16
+    cov: Optional[torch.Tensor] = None     # [B,H,nkb] fp32 ||M_j - Hbar|| (order 2)
 
 
 @dataclasses.dataclass
@@ -35,7 +38,7 @@ class Problem:
     Nk: int
     d: int
     block: int
-    order: int
+    order: int  # 0, 1 (first-order term per block) or 2 (global first-order term)
 
     @property
     def nqb(self) -> int:
@@ -55,8 +58,11 @@ def allocate_tables(p: Problem, device) -> Tables:
         vsum=torch.empty(p.B, p.H, p.nkb, p.d, **f32),
         kbar16=torch.empty(p.B, p.H, 2, p.nkb, p.d, dtype=torch.bfloat16, device=device),
         vsum16=torch.empty(p.B, p.H, p.nkb, p.d, **h16),
-        M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **h16) if p.order == 1 else None,
+        M=torch.empty(p.B, p.H, p.nkb, p.d, p.d, **h16) if p.order >= 1 else None,
         v16=torch.empty(p.B, p.H, p.Nk, p.d, **h16),
+        hbar=torch.empty(p.B, p.H, p.d, p.d, **f32) if p.order == 2 else None,
+        hbar16=torch.empty(p.B, p.H, p.d, p.d, **h16) if p.order == 2 else None,
+        cov=torch.empty(p.B, p.H, p.nkb, **f32) if p.order == 2 else None,
     )
 
 
@@ -72,13 +78,21 @@ def _check_inputs(q, k, v):
 
 
 def pool(q, k, v, p: Problem, t: Tables, stream=None):
+    """Pooled tables; with order 2 also the global first-order matrix and the
+    per-block covariance norms."""
     C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar, t.kbar_t,
                        t.vsum, t.kbar16, t.vsum16, t.M, t.v16, stream)
+    if p.order == 2:
+        C.sparse_attn_hbar(t.M, p.B, p.H, p.nkb, p.d, t.hbar, t.hbar16, t.cov, stream)
 
 
 def route(p: Problem, t: Tables, kv_idx, kv_cnt, mode: str, rho=(1, 4), tau=0.9, scale=None,
           stream=None):
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
+    if mode == "topk_cov":
+        C.sparse_attn_route_cov(t.qbar, t.kbar_t, t.cov, p.B, p.H, p.nqb, p.nkb, p.d, rho[0],
+                                rho[1], scale, kv_idx, kv_cnt, kv_idx.shape[-1], stream)
+        return
     m = C.SA_ROUTE_TOPK if mode == "topk" else C.SA_ROUTE_MASS
     C.sparse_attn_route(t.qbar, t.kbar_t, p.B, p.H, p.nqb, p.nkb, p.d, m, rho[0], rho[1], tau,
                         scale, kv_idx, kv_cnt, kv_idx.shape[-1], stream)
@@ -95,7 +109,8 @@ def forward(q, k, v, p: Problem, t: Tables, kv_idx, kv_cnt, out, scale=None, err
             stream=None):
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
     dt = C.SA_OUT_F32 if out.dtype == torch.float32 else C.SA_OUT_BF16
-    C.sparse_attn_forward(q, k, t.v16, t.kbar16, t.vsum16, t.M, kv_idx, kv_cnt, kv_idx.shape[-1],
+    m = t.hbar16 if p.order == 2 else t.M
+    C.sparse_attn_forward(q, k, t.v16, t.kbar16, t.vsum16, m, kv_idx, kv_cnt, kv_idx.shape[-1],
                           p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, scale, out, dt, err_flag,
                           stream)
 
@@ -103,7 +118,8 @@ def forward(q, k, v, p: Problem, t: Tables, kv_idx, kv_cnt, out, scale=None, err
 class BlockSparseAttention:
     """Reusable buffers plus the three-stage call for one problem shape.
 
-    mode "topk" keeps ceil(rho * nkb) blocks per query block, "mass" the shortest
+    mode "topk" keeps ceil(rho * nkb) blocks per query block, "topk_cov" the same
+    number by the covariance-aware score (order 2), "mass" the shortest
     prefix covering tau of the pooled softmax, "structured" the window + rotating
     anchor geometry given in ``geometry`` (frame_tokens, n_frames, window,
     n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
@@ -112,7 +128,9 @@ class BlockSparseAttention:
     def __init__(self, p: Problem, mode: str, rho=(1, 4), tau=0.9, geometry=None,
                  out_dtype=torch.float32, device="cuda"):
         self.p, self.mode, self.rho, self.tau, self.geometry = p, mode, rho, tau, geometry
-        if mode == "topk":
+        if mode == "topk_cov" and p.order != 2:
+            raise ValueError("covariance-aware routing needs order 2 (the covariance norms)")
+        if mode in ("topk", "topk_cov"):
             cap = -(-rho[0] * p.nkb // rho[1])
         else:
             cap = p.nkb

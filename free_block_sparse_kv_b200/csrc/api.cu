@@ -78,7 +78,7 @@ const char* sparse_attn_last_error(void) { return g_last_error.c_str(); }
 int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
                             size_t sizes[7]) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
-  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
   SA_REQUIRE(sizes != nullptr, "sizes must not be NULL");
   const size_t bh = (size_t)B * H, nqb = cdiv(Nq, block), nkb = cdiv(Nk, block);
   sizes[0] = bh * nqb * d * sizeof(float);
@@ -86,7 +86,7 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
   sizes[2] = bh * nkb * d * sizeof(float);
   sizes[3] = bh * 2 * nkb * d * 2;
   sizes[4] = bh * nkb * d * 2;
-  sizes[5] = order == 1 ? bh * nkb * d * d * 2 : 0;
+  sizes[5] = order >= 1 ? bh * nkb * d * d * 2 : 0;
   sizes[6] = bh * (size_t)Nk * d * 2;
   return ok();
 }
@@ -96,7 +96,7 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
                      uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
                      void* stream) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
-  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
   const bool do_q = q != nullptr && Nq > 0;
   if ((long long)B * H == 0 || (Nk == 0 && !do_q)) return ok();
   if (Nk > 0) {
@@ -107,7 +107,7 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
     SA_REQUIRE_PTR(kbar16);
     SA_REQUIRE_PTR(vsum16);
     SA_REQUIRE_PTR(v16);
-    if (order == 1) SA_REQUIRE_PTR(M);
+    if (order >= 1) SA_REQUIRE_PTR(M);
   }
   if (do_q) {
     SA_REQUIRE_PTR(q);
@@ -149,6 +149,47 @@ int sparse_attn_route(const float* qbar, const float* kbar_t, int B, int H, int 
   return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
 }
 
+int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* cov, int B, int H,
+                          int nqb, int nkb, int d, int rho_num, int rho_den, float scale,
+                          int32_t* kv_idx, int32_t* kv_cnt, int cap, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && nqb >= 0 && nkb >= 0, "B, H, nqb, nkb must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(std::isfinite(scale), "scale must be finite");
+  if ((long long)B * H * nqb == 0) return ok();
+  SA_REQUIRE(nkb >= 1 && nkb <= SA_MAX_KV_BLOCKS, "nkb must be in [1, %d] (got %d)",
+             SA_MAX_KV_BLOCKS, nkb);
+  SA_REQUIRE(rho_num > 0 && rho_den > 0 && rho_num <= rho_den,
+             "top-k needs 0 < rho_num <= rho_den (got %d/%d)", rho_num, rho_den);
+  const int keep = (int)(((long long)rho_num * nkb + rho_den - 1) / rho_den);
+  SA_REQUIRE(cap >= keep, "cap %d is below the keep count %d", cap, keep);
+  SA_REQUIRE_PTR(qbar);
+  SA_REQUIRE_PTR(kbar_t);
+  SA_REQUIRE_PTR(cov);
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  if (int rc = check_device()) return rc;
+  sa::RouteArgs p{qbar, kbar_t, B, H, nqb, nkb, d, SA_ROUTE_TOPK, keep, 1.f, scale, kv_idx, kv_cnt,
+                  cap, cov};
+  return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
+}
+
+int sparse_attn_hbar(const uint16_t* M, int B, int H, int nkb, int d, float* hbar,
+                     uint16_t* hbar16, float* cov, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && nkb >= 0, "B, H, nkb must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  if ((long long)B * H == 0) return ok();
+  SA_REQUIRE(nkb >= 1 && nkb <= 65535, "nkb must be in [1, 65535] (got %d)", nkb);
+  SA_REQUIRE_PTR(M);
+  SA_REQUIRE_PTR(hbar);
+  SA_REQUIRE_PTR(hbar16);
+  if (cov) SA_REQUIRE_PTR(cov);
+  if (int rc = check_device()) return rc;
+  sa::HbarArgs p{M, B, H, nkb, d, hbar, hbar16, cov};
+  return launched(sa::launch_hbar(p, static_cast<cudaStream_t>(stream)), "hbar launch");
+}
+
 int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block, int frame_tokens,
                                 int n_frames, int window, int n_anchors, int period, int step,
                                 int q_frame0, int32_t* kv_idx, int32_t* kv_cnt, int cap,
@@ -181,7 +222,7 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v1
                         int Nk, int d, int block, int order, float scale, void* out, int out_dtype,
                         int32_t* err_flag, void* stream) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
-  SA_REQUIRE(order == 0 || order == 1, "order must be 0 or 1");
+  SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
   SA_REQUIRE(out_dtype == SA_OUT_F32 || out_dtype == SA_OUT_BF16, "out_dtype must be F32 or BF16");
   SA_REQUIRE(std::isfinite(scale), "scale must be finite");
   if ((long long)B * H * Nq == 0) return ok();
@@ -194,13 +235,13 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v1
   SA_REQUIRE_PTR(v16);
   SA_REQUIRE_PTR(kbar16);
   SA_REQUIRE_PTR(vsum16);
-  if (order == 1) SA_REQUIRE_PTR(M);
+  if (order >= 1) SA_REQUIRE_PTR(M);
   SA_REQUIRE_PTR(kv_idx);
   SA_REQUIRE_PTR(kv_cnt);
   SA_REQUIRE_PTR(out);
   if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
   if (int rc = check_device()) return rc;
-  sa::ForwardArgs p{q, k, v16, kbar16, vsum16, order == 1 ? M : nullptr, kv_idx, kv_cnt, cap,
+  sa::ForwardArgs p{q, k, v16, kbar16, vsum16, order >= 1 ? M : nullptr, kv_idx, kv_cnt, cap,
                     B, H, Nq, Nk, d, block, order, cdiv(Nq, block), nkb, scale, out, out_dtype,
                     err_flag};
   return launched(sa::launch_forward(p, static_cast<cudaStream_t>(stream)), "forward launch");

@@ -150,7 +150,8 @@ SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct, int nkb) {
 template <int BLK>
 struct Walk {
   int phase = 0, tile = 0, word = -1, half = 0, jcur = 0, mcur = 0;
-  bool in_tile = false;
+  int gmask = 0;       // order 2: tiles with a skipped block so far
+  bool in_tile = false, gdone = false;
   uint64_t tmask = 0, sk0 = 0, sk1 = 0;  // phase 0: union / per-tile skipped blocks
   uint32_t kmask = 0, kw0 = 0, kw1 = 0;  // phase 1: union / per-tile kept blocks
   template <int ORDER>
@@ -160,6 +161,10 @@ struct Walk {
       if (phase == 0) {
         if (!in_tile) {
           if (tile >= ntiles) {
+            if (ORDER == 2 && !gdone && gmask) {  // the global first-order item
+              gdone = true;
+              return Item{kMat, -1, gmask, 0};
+            }
             phase = 1;
             continue;
           }
@@ -168,7 +173,9 @@ struct Walk {
           tmask = sk0 | sk1;
           if (tmask) {
             in_tile = true;
-            return Item{kTile, tile, (sk0 != 0) | ((sk1 != 0) << 1), 0};
+            const int m = (sk0 != 0) | ((sk1 != 0) << 1);
+            gmask |= m;
+            return Item{kTile, tile, m, 0};
           }
           ++tile;
           continue;
@@ -246,7 +253,7 @@ struct StepGen {
     pend_mask = it.mask;
     pend_j = it.j;
     pend_half = it.half;
-    if (ORDER == 1 && it.kind == kTile) flush_next = true;
+    if (ORDER >= 1 && it.kind == kTile) flush_next = true;
     return s;
   }
 };
@@ -293,8 +300,9 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
 
   bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
   // fp16 copy of this thread's Q row, in registers (order-1 operands)
-  uint32_t q16[ORDER == 1 ? QW : 1];
-  if constexpr (ORDER == 1) {
+  uint32_t q16[ORDER >= 1 ? QW : 1];
+  float qmax = 0.f;  // largest |q| of the row (order 2: keeps the global operand in fp16 range)
+  if constexpr (ORDER >= 1) {
 #pragma unroll
     for (int i = 0; i < QW / 4; ++i) {
       const int s = i / 8, cw = i % 8;
@@ -314,9 +322,17 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     for (int k = 0; k < D / 32; ++k) tc::tmem_st32(ot + 32 * k, z);
     tc::tmem_wait_st();
   }
+  if constexpr (ORDER == 2) {
+#pragma unroll
+    for (int i = 0; i < QW; ++i) {
+      const __half2 h = *reinterpret_cast<const __half2*>(&q16[i]);
+      qmax = fmaxf(qmax, fmaxf(fabsf(__low2float(h)), fabsf(__high2float(h))));
+    }
+  }
   warp_arrive(bar(c.init_done));
 
   float m_ref = -INFINITY, l = 0.f;
+  float asum = 0.f;          // order 2: sum of the skipped blocks' alpha, relative to m_ref
   int n = 0;                 // items of this tile so far; item n uses buffer n & 1
   // Per-buffer phase parities as bit masks (bit b for buffer b): next s_full wait;
   // number of items so far (rel phases); whether the buffer has been used.
@@ -455,6 +471,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     tc::f2_split(acc0, a0, a1);
     tc::f2_split(acc1, a2, a3);
     float ls = (a0 + a1) + (a2 + a3);
+    if (ORDER == 2 && TILE) asum = asum * f + ls;  // alpha of the skipped blocks (P is 0 elsewhere)
     // order-0 denominator weight n_j: b for every block but a partial last one
     if (TILE) ls = ls * (float)BLK + plast * (float)(p.Nk - nkb * BLK);
     l = l * f + ls;
@@ -477,12 +494,45 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       cur_tile = it.j;
       continue;
     }
-    if constexpr (ORDER == 1) {
+    if constexpr (ORDER >= 1) {
       // The operand does not depend on the buffer: compute (its first 32 columns)
       // first, then wait until the products that last read the buffer (two items
       // back) are complete.
-      const float pj = __half2float(__ushort_as_half(stash[(it.j - cur_tile * KC) * TQ]));
-      const __half2 al = __float2half2_rn(pj * p.scale);
+      float as;  // scale * alpha of the item's row
+      if constexpr (ORDER == 1) {
+        as = __half2float(__ushort_as_half(stash[(it.j - cur_tile * KC) * TQ])) * p.scale;
+      } else {
+        // The global item: A = (scale * sum_j alpha_tj) q_t must stay in fp16 range. A row
+        // whose operand would exceed 2^14 moves its reference up by E (a rescale by 2^-E
+        // of O, l and the alpha sum, as when its max grows), after the last product into
+        // O_t (the previous item's) is complete.
+        const float g = asum * p.scale * qmax;
+        const int E = g > 16384.f ? (int)ceilf(log2f(g * (1.f / 16384.f))) : 0;
+        if (__any_sync(0xffffffffu, E > 0)) {
+          const float f = exp2f((float)-E);
+          if (n > 0) {
+            const int pb = (n - 1) & 1;
+            ok = uni(wt.fast(bar(c.rel[t][pb]), ((rcnt >> pb) & 1) ^ 1, 12));
+            tc::fence_after_sync();
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k) {
+            uint32_t v[32];
+            tc::tmem_ld32(ot + 32 * k, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            tc::tmem_st32(ot + 32 * k, v);
+          }
+          tc::tmem_wait_st();
+          m_ref += (float)E;
+          l *= f;
+          asum *= f;
+        }
+        as = asum * p.scale;
+      }
+      const __half2 al = __float2half2_rn(as);
       auto part = [&](int k, uint32_t* a) __attribute__((always_inline)) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -667,8 +717,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         tc::mbar_arrive_expect_tx(fb, bytes);
         int k = 0;
         if (s.type == stMat) {
+          // order 1: M_j of the head; order 2: the head's global matrix
+          const int mz = ORDER == 2 ? bh : bh * nkb + s.cur_j;
           for (int x = 0; x < SUB; ++x)
-            tc::tma_load_3d(piece(0) + x * D * 128, &p.tmM, fb, 64 * x, 0, bh * nkb + s.cur_j);
+            tc::tma_load_3d(piece(0) + x * D * 128, &p.tmM, fb, 64 * x, 0, mz);
         } else {
           if (s.pend_mask) {  // values of the pending item
             if (s.pend_kind == kTile) {
@@ -849,6 +901,7 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
             map3d(&p.tmKb, BF, a.kbar16, D, a.nkb, 2 * bh, KC) &&
             map3d(&p.tmVs, HF, a.vsum16, D, a.nkb, bh, KC);
   if (ORDER == 1) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh * a.nkb, D);
+  else if (ORDER == 2) ok = ok && map3d(&p.tmM, HF, a.M, D, D, bh, D);
   else p.tmM = p.tmVs;
   if (!ok) return cudaErrorInvalidValue;
   p.kv_idx = a.kv_idx;
@@ -878,8 +931,10 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
 cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st) {
 #define SA_TC_CASE(D_, B_, O_) \
   if (p.d == D_ && p.block == B_ && p.order == O_) return tcf::launch_t<D_, B_, O_>(p, st);
-  SA_TC_CASE(64, 64, 0) SA_TC_CASE(64, 64, 1) SA_TC_CASE(64, 128, 0) SA_TC_CASE(64, 128, 1)
-  SA_TC_CASE(128, 64, 0) SA_TC_CASE(128, 64, 1) SA_TC_CASE(128, 128, 0) SA_TC_CASE(128, 128, 1)
+  SA_TC_CASE(64, 64, 0) SA_TC_CASE(64, 64, 1) SA_TC_CASE(64, 64, 2)
+  SA_TC_CASE(64, 128, 0) SA_TC_CASE(64, 128, 1) SA_TC_CASE(64, 128, 2)
+  SA_TC_CASE(128, 64, 0) SA_TC_CASE(128, 64, 1) SA_TC_CASE(128, 64, 2)
+  SA_TC_CASE(128, 128, 0) SA_TC_CASE(128, 128, 1) SA_TC_CASE(128, 128, 2)
 #undef SA_TC_CASE
   return cudaErrorInvalidValue;
 }

@@ -19,6 +19,15 @@ struct RouteArgs {
   float tau, scale;
   int32_t *kv_idx, *kv_cnt;
   int cap;
+  const float* cov = nullptr;  // per-block covariance norms: score += ln cov_j (top-k)
+};
+
+struct HbarArgs {
+  const uint16_t* M;
+  int B, H, nkb, d;
+  float* hbar;
+  uint16_t* hbar16;
+  float* cov;
 };
 
 struct MaskArgs {
@@ -42,5 +51,6 @@ cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);
 cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st);
+cudaError_t launch_hbar(const HbarArgs& p, cudaStream_t st);
 
 }  // namespace sa

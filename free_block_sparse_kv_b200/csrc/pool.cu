@@ -254,8 +254,10 @@ static cudaError_t launch_pool_t(const PoolArgs& p, cudaStream_t st) {
 }
 
 cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st) {
+  // order 2 (global first-order term) needs the per-block matrices like order 1
+  const int order = p.order == 2 ? 1 : p.order;
 #define SA_POOL_CASE(D_, B_, O_) \
-  if (p.d == D_ && p.block == B_ && p.order == O_) return launch_pool_t<D_, B_, O_>(p, st);
+  if (p.d == D_ && p.block == B_ && order == O_) return launch_pool_t<D_, B_, O_>(p, st);
   SA_POOL_CASE(64, 64, 0) SA_POOL_CASE(64, 64, 1) SA_POOL_CASE(64, 128, 0) SA_POOL_CASE(64, 128, 1)
   SA_POOL_CASE(128, 64, 0) SA_POOL_CASE(128, 64, 1) SA_POOL_CASE(128, 128, 0) SA_POOL_CASE(128, 128, 1)
 #undef SA_POOL_CASE

@@ -131,7 +131,7 @@ template <int D, int SLOTS>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, int nqb, int nkb,
              int mode, int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
-             int32_t* __restrict__ kv_cnt, int cap) {
+             int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov) {
   extern __shared__ __align__(16) float rsm[];
   float* qs = rsm;                         // [D][kRouteRows]
   float* sc = rsm + D * kRouteRows;        // [kRouteRows][nkb] scores
@@ -165,8 +165,10 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
       acc[6] = fmaf(qb.z, kv, acc[6]);
       acc[7] = fmaf(qb.w, kv, acc[7]);
     }
+    // covariance-aware top-k: the log of block j's covariance norm joins every row's score
+    const float bias = cov ? logf(cov[(size_t)bh * nkb + j]) : 0.f;
 #pragma unroll
-    for (int r = 0; r < kRouteRows; ++r) sc[r * nkb + j] = scale * acc[r];
+    for (int r = 0; r < kRouteRows; ++r) sc[r * nkb + j] = scale * acc[r] + bias;
   }
   __syncthreads();
 
@@ -185,7 +187,7 @@ static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   dim3 grid((p.nqb + kRouteRows - 1) / kRouteRows, p.B * p.H);
   kern<<<grid, kRouteThreads, smem, st>>>(p.qbar, p.kbar_t, p.nqb, p.nkb, p.mode, p.keep, p.tau,
-                                          p.scale, p.kv_idx, p.kv_cnt, p.cap);
+                                          p.scale, p.kv_idx, p.kv_cnt, p.cap, p.cov);
   return cudaGetLastError();
 }
 

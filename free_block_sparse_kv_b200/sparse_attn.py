@@ -19,7 +19,8 @@ SA_OUT_F32, SA_OUT_BF16 = 0, 1
 
 # Entry points declared in include/sparse_attn.h.
 EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
-           "sparse_attn_structured_mask", "sparse_attn_forward", "sparse_attn_last_error")
+           "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
+           "sparse_attn_forward", "sparse_attn_last_error")
 
 
 class SparseAttnError(RuntimeError):
@@ -47,6 +48,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_table_sizes.argtypes = [_I] * 7 + [ctypes.POINTER(ctypes.c_size_t)]
     lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 7 + [_P]
     lib.sparse_attn_route.argtypes = [_P, _P] + [_I] * 8 + [_F, _F, _P, _P, _I, _P]
+    lib.sparse_attn_route_cov.argtypes = [_P, _P, _P] + [_I] * 7 + [_F, _P, _P, _I, _P]
+    lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
     for name in EXPORTS[:-1]:
@@ -96,6 +99,18 @@ def sparse_attn_route(qbar, kbar_t, B, H, nqb, nkb, d, mode, rho_num, rho_den, t
     _check(load_library().sparse_attn_route(
         _ptr(qbar), _ptr(kbar_t), B, H, nqb, nkb, d, mode, rho_num, rho_den, tau, scale,
         _ptr(kv_idx), _ptr(kv_cnt), cap, _stream(stream)))
+
+
+def sparse_attn_route_cov(qbar, kbar_t, cov, B, H, nqb, nkb, d, rho_num, rho_den, scale, kv_idx,
+                          kv_cnt, cap, stream=None):
+    _check(load_library().sparse_attn_route_cov(
+        _ptr(qbar), _ptr(kbar_t), _ptr(cov), B, H, nqb, nkb, d, rho_num, rho_den, scale,
+        _ptr(kv_idx), _ptr(kv_cnt), cap, _stream(stream)))
+
+
+def sparse_attn_hbar(M, B, H, nkb, d, hbar, hbar16, cov, stream=None):
+    _check(load_library().sparse_attn_hbar(
+        _ptr(M), B, H, nkb, d, _ptr(hbar), _ptr(hbar16), _ptr(cov), _stream(stream)))
 
 
 def sparse_attn_structured_mask(B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors,

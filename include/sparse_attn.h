@@ -61,7 +61,9 @@ enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
 
 /*
  * Byte sizes of the pooled tables for a problem, written to sizes[0..6] in the
- * order qbar, kbar_t, vsum, kbar16, vsum16, M (0 when order == 0), v16.
+ * order qbar, kbar_t, vsum, kbar16, vsum16, M (0 when order == 0), v16. Order 2 needs
+ * the M table like order 1; its global tables (see sparse_attn_hbar) take
+ * B*H*d*d*4 (hbar), B*H*d*d*2 (hbar16) and B*H*nkb*4 (cov) bytes.
  * nqb = ceil(Nq / block), nkb = ceil(Nk / block).
  */
 int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int order,
@@ -73,7 +75,7 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
  * centroids). One pass over Q, K and V.
  *   q       [B,H,Nq,d] bf16, may be NULL (then qbar is not written and may be NULL)
  *   k, v    [B,H,Nk,d] bf16
- *   order   0 or 1; with 1, M is written and must not be NULL
+ *   order   0, 1 or 2; with 1 or 2, M is written and must not be NULL
  *   qbar    [B,H,nqb,d]  fp32   mean of each query block's rows
  *   kbar_t  [B,H,d,nkb]  fp32   block centroids, dim-major (routing reads it)
  *   vsum    [B,H,nkb,d]  fp32   value sums S_j
@@ -118,6 +120,34 @@ int sparse_attn_route(const float* qbar, const float* kbar_t,
                       int32_t* kv_idx, int32_t* kv_cnt, int cap, void* stream);
 
 /*
+ * Global first-order statistic (PISA §2 Algorithme Central: Hbar, the mean of the
+ * per-block first-order matrices over all blocks, used in place of each skipped
+ * block's own matrix) and per-block covariance norms (PISA §2 Routage Sensible à la
+ * Covariance: ||H_j - Hbar||, here the 2-norm of the matrix entries).
+ *   M       [B,H,nkb,d,d] fp16, as written by the pool with order 1 or 2
+ *   hbar    [B,H,d,d] fp32    Hbar = (1/nkb) sum_j M_j (fp32 accumulate)
+ *   hbar16  [B,H,d,d] fp16    Hbar rounded to nearest (the forward's order-2 operand)
+ *   cov     [B,H,nkb] fp32    sqrt(sum over entries of (M_j - Hbar)^2); may be NULL
+ * Two launches on the stream (mean, then norms).
+ */
+int sparse_attn_hbar(const uint16_t* M, int B, int H, int nkb, int d, float* hbar,
+                     uint16_t* hbar16, float* cov, void* stream);
+
+/*
+ * Covariance-aware top-k (PISA §2 Routage Sensible à la Covariance). As
+ * sparse_attn_route with SA_ROUTE_TOPK, on the scores
+ *   s'_ij = scale * qbar_i . kbar_j + ln cov_j
+ * (fp32): the log of the first-order error bound alpha_ij * scale * |qbar_i| *
+ * ||H_j - Hbar|| of the hybrid order, up to a term that is the same for every
+ * block of the row.
+ *   cov     [B,H,nkb] fp32, as written by sparse_attn_hbar (positive)
+ */
+int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* cov,
+                          int B, int H, int nqb, int nkb, int d, int rho_num, int rho_den,
+                          float scale, int32_t* kv_idx, int32_t* kv_cnt, int cap,
+                          void* stream);
+
+/*
  * Structured mask (LVSA §2 Mécanisme Central). Tokens are frame-major with
  * frame_tokens tokens per frame; query token t lies in frame
  * q_frame0 + t / frame_tokens and key token r in frame r / frame_tokens.
@@ -135,14 +165,18 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
 
 /*
  * Forward (PISA §2 Algorithme Central and Implémentation Matérielle, phases 1-3,
- * with the first-order term per block). For each query row t of query block i:
+ * with the first-order term per block, or global with order 2). For each query
+ * row t of query block i:
  *   exact logits    scale * q_t . k_r   for the tokens r of the kept blocks of i
  *   centroid logits scale * q_t . kbar_j for the other blocks j
- *   N_t = sum_r e^(l_r - m) v_r + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j)
+ *   N_t = sum_r e^(l_r - m) v_r + sum_j e^(c_j - m) (S_j + [order 1] scale * q_t M_j
+ *                                                      + [order 2] scale * q_t Hbar)
  *   D_t = sum_r e^(l_r - m)     + sum_j e^(c_j - m) n_j
  *   o_t = N_t / D_t
  *   q, k              [B,H,Nq,d] / [B,H,Nk,d] bf16, as for the pool
- *   v16, kbar16, vsum16, M  as written by the pool (M NULL when order == 0)
+ *   v16, kbar16, vsum16  as written by the pool
+ *   M                 order 1: the pool's M table; order 2: hbar16 [B,H,d,d] from
+ *                     sparse_attn_hbar; order 0: NULL
  *   kv_idx, kv_cnt    as written by routing or the structured mask: indices of
  *                     each row must be distinct and < nkb; entries outside
  *                     [0, nkb) are ignored; kv_cnt is clamped to [0, cap]

@@ -75,7 +75,7 @@ def pool_queries(q: np.ndarray, block: int) -> np.ndarray:
 
 
 def pool_keys_values(k: np.ndarray, v: np.ndarray, block: int, order: int):
-    """Per KV block j: centroid kbar_j, value sum S_j, token count n_j and (order 1) M_j.
+    """Per KV block j: centroid kbar_j, value sum S_j, token count n_j and (order 1 or 2) M_j.
 
     M_j[a, c] = sum over tokens r of block j of (k_r[a] - kbar_j[a]) * v_r[c]:
     the first-order Taylor matrix of the block (key dim a, value dim c).
@@ -89,9 +89,9 @@ def pool_keys_values(k: np.ndarray, v: np.ndarray, block: int, order: int):
         kbar.append(kb)
         vsum.append(vj.sum(axis=0))
         counts.append(e - s)
-        if order == 1:
+        if order >= 1:
             mats.append((kj - kb).T @ vj)
-    m = np.stack(mats) if order == 1 else None
+    m = np.stack(mats) if order >= 1 else None
     return np.stack(kbar), np.stack(vsum), np.asarray(counts, dtype=np.int64), m
 
 

@@ -27,6 +27,8 @@ SMALL = {
                                 period=6, steps=(0, 5)),
     "worldmodel-small": W.shrink(W.WORKLOADS["worldmodel-chunk"], name="worldmodel-small", B=2, H=2,
                                  Nq=500, Nk=6500, grid=(13, 10, 50), q_frame0=12),
+    "hybrid-small": W.shrink(W.WORKLOADS["dit720p-hybrid-21x45x80"], name="hybrid-small", H=2,
+                             Nq=9480, Nk=9480, grid=(6, 20, 79)),
 }
 
 
@@ -35,14 +37,15 @@ def err_stats(got: np.ndarray, want: np.ndarray):
     return float(diff.max()), float(diff.sum() / np.abs(want).sum())
 
 
-def oracle_kept(w: W.Workload, q, k, step: int = 0):
-    """Oracle kept lists of one head and the per-row gate flags (True = pinned)."""
+def oracle_kept(w: W.Workload, q, k, step: int = 0, v=None):
+    """Oracle kept lists of one head and the per-row gate flags (True = pinned).
+    Covariance-aware routing needs the head's values ``v``."""
     if w.mode == "structured":
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
                                  w.n_anchors, w.period, step, w.q_frame0)
         return kept, np.ones(len(kept), bool)
-    if w.mode == "topk":
-        kept, s, counts = O.route_head(q, k, w.block, "topk", w.scale, keep=w.keep())
+    if w.mode in ("topk", "topk_cov"):
+        kept, s, counts = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), v=v)
         gaps, _, _ = O.gate_diagnostics(s, counts)
         return kept, gaps > GATE
     kept, s, counts = O.route_head(q, k, w.block, "mass", w.scale, tau=w.tau)

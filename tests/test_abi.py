@@ -40,6 +40,7 @@ def test_table_sizes():
         40 * 591 * 128 * 4, 40 * 591 * 128 * 4, 40 * 591 * 128 * 4,
         40 * 2 * 591 * 128 * 2, 40 * 591 * 128 * 2, 40 * 591 * 128 * 128 * 2, 40 * 75600 * 128 * 2)
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[5] == 0
+    assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 2)[5] == 4 * 16 * 1000 * 128 * 128 * 2
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[0] == 4 * 16 * 25 * 128 * 4
 
 
@@ -51,7 +52,8 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 96, 64, 0),
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 64, 32, 0),
         lambda: C.sparse_attn_table_sizes(-1, 1, 64, 64, 64, 64, 0),
-        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, p, p, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 3, p, p, p, p, p, p, p, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, None, p, 0),
         lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
         lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
         lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, None, 0),
@@ -59,6 +61,15 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 0, 3, 2, 0.9, 0.1, p, p, 10, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 1, 1, 4, 1.5, 0.1, p, p, 10, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 7, 1, 4, 0.9, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_route_cov(p, p, None, 1, 1, 4, 10, 64, 1, 4, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_route_cov(p, p, p, 1, 1, 4, 10, 64, 1, 4, 0.1, p, p, 2, 0),
+        lambda: C.sparse_attn_route_cov(p, p, p, 1, 1, 4, 10, 96, 1, 4, 0.1, p, p, 10, 0),
+        lambda: C.sparse_attn_hbar(p, 1, 1, 4, 96, p, p, p, 0),
+        lambda: C.sparse_attn_hbar(None, 1, 1, 4, 64, p, p, p, 0),
+        lambda: C.sparse_attn_hbar(p, 1, 1, 4, 64, p, None, p, 0),
+        lambda: C.sparse_attn_hbar(p, 1, 1, 0, 64, p, p, p, 0),
+        lambda: C.sparse_attn_forward(p, p, p, p, p, None, p, p, 1, 1, 1, 64, 64, 64, 64, 2, 0.1, p,
+                                      0, None, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 6400, 64, 10, 10, 1, 1, 1, 0, 0, p, p, 100, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 64, 64, 8, 8, 1, 1, 0, 0, 0, p, p, 1, 0),
         lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 0, 64, 64, 0, 0.1, p, 0,

@@ -95,10 +95,19 @@ def test_pool_matches_oracle(name, small_inputs):
             v16 = t.v16[b, h].float().cpu().numpy()
             # fp16 rounding of V (round to nearest even; exact except for subnormals)
             assert np.array_equal(v16, v.astype(np.float16).astype(np.float32))
-            if w.order == 1:
+            if w.order >= 1:
                 mg = t.M[b, h].float().cpu().numpy()
                 tol = 2 ** -10 * np.abs(mats) + 1e-3
                 assert np.all(np.abs(mg - mats) <= tol), float(np.abs(mg - mats).max())
+            if w.order == 2:
+                # mean of the fp16 M table: each entry within the table's rounding
+                hbar = O.global_first_order(mats)
+                err = np.abs(t.hbar[b, h].cpu().numpy() - hbar)
+                assert err.max() <= 2 ** -11 * np.abs(mats).max() + 1e-5, float(err.max())
+                np.testing.assert_array_equal(t.hbar16[b, h].cpu().numpy(),
+                                              t.hbar[b, h].cpu().numpy().astype(np.float16))
+                cov = O.covariance_norms(mats, hbar)
+                np.testing.assert_allclose(t.cov[b, h].cpu().numpy(), cov, rtol=1e-3)
 
 
 # --- routing and structured masks ----------------------------------------------
@@ -112,11 +121,11 @@ def test_route_masks_bit_exact_above_gate(name, small_inputs):
     for b in range(w.B):
         for h in range(w.H):
             q, k = W.bits_to_f32(qb[b, h]), W.bits_to_f32(kb[b, h])
-            kept, gate = oracle_kept(w, q, k)
+            kept, gate = oracle_kept(w, q, k, v=W.bits_to_f32(vb[b, h]))
             got = lists_to_sets(idx[b, h], cnt[b, h])
             for i in range(w.nqb):
                 total += 1
-                if w.mode == "topk":
+                if w.mode in ("topk", "topk_cov"):
                     assert len(got[i]) == w.keep()
                 if gate[i]:
                     pinned += 1
@@ -162,8 +171,8 @@ def test_forward_matches_oracle_on_oracle_masks(name, out_dtype, small_inputs):
     kept_all = {}
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     for b, h in heads:
-        q, k = W.bits_to_f32(qb[b, h]), W.bits_to_f32(kb[b, h])
-        kept_all[(b, h)] = oracle_kept(w, q, k, step)[0]
+        q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+        kept_all[(b, h)] = oracle_kept(w, q, k, step, v=v)[0]
     cap = max(len(r) for kept in kept_all.values() for r in kept)
     idx, cnt = _oracle_lists_to_device(w, kept_all, cap)
     p = _problem(w)
@@ -202,7 +211,7 @@ def test_pipeline_matches_oracle(name, small_inputs):
         for b in range(w.B):
             for h in range(w.H):
                 q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
-                kept, _ = oracle_kept(w, q, k, step)
+                kept, _ = oracle_kept(w, q, k, step, v=v)
                 want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=rows))
                 got_all.append(out[b, h, rows].cpu().numpy())
         mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
@@ -224,7 +233,7 @@ def test_full_size_sampled(name):
     pinned = total = 0
     for b, h in heads:
         q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
-        kept, gate = oracle_kept(w, q, k, step)
+        kept, gate = oracle_kept(w, q, k, step, v=v)
         got = lists_to_sets(idx[b, h], cnt[b, h])
         for i in range(w.nqb):
             total += 1
