@@ -211,7 +211,7 @@ def time_oracle(w: W.Workload, seconds: float) -> dict:
     t0 = time.perf_counter()
     if w.mode == "structured":
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
-                                 w.n_anchors, w.period, 0, w.q_frame0)
+                                 w.n_anchors, w.period, 0, w.q_frame0, budget=w.budget)
     else:
         kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau, v=v)[0]
     kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, min(w.order, 1))
@@ -288,7 +288,7 @@ def main():
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     p = A.Problem(w.B, w.H, w.Nq, w.Nk, w.d, w.block, w.order)
     geometry = dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
-                    n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0)
+                    n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0, budget=w.budget)
     op = A.BlockSparseAttention(p, w.mode, rho=w.rho, tau=w.tau,
                                 geometry=geometry if w.mode == "structured" else None,
                                 out_dtype=torch.float32, device=dev)

@@ -99,7 +99,13 @@ def route(p: Problem, t: Tables, kv_idx, kv_cnt, mode: str, rho=(1, 4), tau=0.9,
 
 
 def structured_mask(p: Problem, kv_idx, kv_cnt, frame_tokens, n_frames, window, n_anchors, period,
-                    step, q_frame0=0, stream=None):
+                    step, q_frame0=0, budget=0, stream=None):
+    """Window + rotating anchors; budget > 0 uses the adaptive (extended) windows."""
+    if budget:
+        C.sparse_attn_structured_mask_adaptive(p.B, p.H, p.Nq, p.Nk, p.block, frame_tokens,
+                                               n_frames, window, n_anchors, period, step, q_frame0,
+                                               budget, kv_idx, kv_cnt, kv_idx.shape[-1], stream)
+        return
     C.sparse_attn_structured_mask(p.B, p.H, p.Nq, p.Nk, p.block, frame_tokens, n_frames, window,
                                   n_anchors, period, step, q_frame0, kv_idx, kv_cnt,
                                   kv_idx.shape[-1], stream)
@@ -121,7 +127,7 @@ class BlockSparseAttention:
     mode "topk" keeps ceil(rho * nkb) blocks per query block, "topk_cov" the same
     number by the covariance-aware score (order 2), "mass" the shortest
     prefix covering tau of the pooled softmax, "structured" the window + rotating
-    anchor geometry given in ``geometry`` (frame_tokens, n_frames, window,
+    anchor geometry given in ``geometry`` (frame_tokens, n_frames, window, budget,
     n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
     """
 
@@ -147,7 +153,7 @@ class BlockSparseAttention:
             g = self.geometry
             structured_mask(p, self.kv_idx, self.kv_cnt, g["frame_tokens"], g["n_frames"],
                             g["window"], g["n_anchors"], g["period"], step, g.get("q_frame0", 0),
-                            stream)
+                            g.get("budget", 0), stream)
         else:
             route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
                   stream=stream)

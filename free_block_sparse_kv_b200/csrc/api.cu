@@ -194,6 +194,16 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block, int fra
                                 int n_frames, int window, int n_anchors, int period, int step,
                                 int q_frame0, int32_t* kv_idx, int32_t* kv_cnt, int cap,
                                 void* stream) {
+  return sparse_attn_structured_mask_adaptive(B, H, Nq, Nk, block, frame_tokens, n_frames, window,
+                                              n_anchors, period, step, q_frame0, 0, kv_idx, kv_cnt,
+                                              cap, stream);
+}
+
+int sparse_attn_structured_mask_adaptive(int B, int H, int Nq, int Nk, int block, int frame_tokens,
+                                         int n_frames, int window, int n_anchors, int period,
+                                         int step, int q_frame0, int budget, int32_t* kv_idx,
+                                         int32_t* kv_cnt, int cap, void* stream) {
+  SA_REQUIRE(budget >= 0, "budget must be >= 0 (got %d)", budget);
   SA_REQUIRE(B >= 0 && H >= 0 && Nq >= 0 && Nk >= 0, "B, H, Nq, Nk must be >= 0");
   SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
   SA_REQUIRE(block == 64 || block == 128, "block must be 64 or 128 (got %d)", block);
@@ -212,7 +222,7 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block, int fra
   SA_REQUIRE_PTR(kv_cnt);
   if (int rc = check_device()) return rc;
   sa::MaskArgs p{B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors, period, step,
-                 q_frame0, cdiv(Nq, block), nkb, kv_idx, kv_cnt, cap};
+                 q_frame0, cdiv(Nq, block), nkb, kv_idx, kv_cnt, cap, budget};
   return launched(sa::launch_structured_mask(p, static_cast<cudaStream_t>(stream)), "mask launch");
 }
 

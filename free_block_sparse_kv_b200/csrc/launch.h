@@ -35,6 +35,7 @@ struct MaskArgs {
   int nqb, nkb;
   int32_t *kv_idx, *kv_cnt;
   int cap;
+  int budget = 0;  // > 0: adaptive windows reaching |A(t)| = budget frames
 };
 
 struct ForwardArgs {

@@ -213,6 +213,27 @@ cudaError_t launch_route(const RouteArgs& p, cudaStream_t st) {
 // [f_lo - window, f_hi + window]. Key block j (frames [g_lo, g_hi]) is kept when
 // that interval meets [g_lo, g_hi] or when an anchor frame lies in [g_lo, g_hi].
 // ---------------------------------------------------------------------------
+// Adaptive window of query frame f (LVSA §2 Fenêtres Adaptatives Étendues): the local
+// window [f - W, f + W] inside the video grows one frame at a time, alternately after
+// and before it (a side at the edge is skipped), while |G u window| < budget.
+SA_DEVI void adaptive_window(const MaskArgs& p, int f, int base, int n_valid, int& lo, int& hi) {
+  const int T = p.n_frames;
+  auto is_anchor = [&](int x) {
+    return x >= base && x < T && (x - base) % p.period == 0 && (x - base) / p.period < p.n_anchors;
+  };
+  lo = max(0, f - p.window);
+  hi = min(T - 1, f + p.window);
+  int inside = 0;
+  for (int x = lo; x <= hi; ++x) inside += is_anchor(x);
+  int size = (hi - lo + 1) + n_valid - inside;
+  bool after = true;
+  while (size < p.budget && (lo > 0 || hi < T - 1)) {
+    const int x = ((after && hi < T - 1) || lo == 0) ? ++hi : --lo;
+    if (!is_anchor(x)) ++size;
+    after = !after;
+  }
+}
+
 __global__ void structured_mask_kernel(MaskArgs p) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= (long long)p.B * p.H * p.nqb) return;
@@ -220,8 +241,22 @@ __global__ void structured_mask_kernel(MaskArgs p) {
   const int ft = p.frame_tokens;
   const int qs = i * p.block, qe = min(p.Nq, qs + p.block) - 1;
   const int f_lo = p.q_frame0 + qs / ft, f_hi = p.q_frame0 + qe / ft;
-  const int w_lo = f_lo - p.window, w_hi = f_hi + p.window;
   const int base = p.step % p.period;
+  int w_lo = f_lo - p.window, w_hi = f_hi + p.window;
+  if (p.budget > 0) {
+    // every frame's window contains the frame, so the union over the block's frames
+    // is one interval
+    int n_valid = 0;
+    for (int m = 0; m < p.n_anchors && base + m * p.period < p.n_frames; ++m) ++n_valid;
+    w_lo = p.n_frames;
+    w_hi = -1;
+    for (int f = f_lo; f <= f_hi; ++f) {
+      int lo, hi;
+      adaptive_window(p, f, base, n_valid, lo, hi);
+      w_lo = min(w_lo, lo);
+      w_hi = max(w_hi, hi);
+    }
+  }
   int32_t* out = p.kv_idx + tid * p.cap;
   int cnt = 0;
   for (int j = 0; j < p.nkb; ++j) {

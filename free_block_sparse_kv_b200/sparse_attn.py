@@ -20,6 +20,7 @@ SA_OUT_F32, SA_OUT_BF16 = 0, 1
 # Entry points declared in include/sparse_attn.h.
 EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
            "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
+           "sparse_attn_structured_mask_adaptive",
            "sparse_attn_forward", "sparse_attn_last_error")
 
 
@@ -51,6 +52,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_route_cov.argtypes = [_P, _P, _P] + [_I] * 7 + [_F, _P, _P, _I, _P]
     lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
+    lib.sparse_attn_structured_mask_adaptive.argtypes = [_I] * 13 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = _I
@@ -118,6 +120,14 @@ def sparse_attn_structured_mask(B, H, Nq, Nk, block, frame_tokens, n_frames, win
     _check(load_library().sparse_attn_structured_mask(
         B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors, period, step, q_frame0,
         _ptr(kv_idx), _ptr(kv_cnt), cap, _stream(stream)))
+
+
+def sparse_attn_structured_mask_adaptive(B, H, Nq, Nk, block, frame_tokens, n_frames, window,
+                                         n_anchors, period, step, q_frame0, budget, kv_idx, kv_cnt,
+                                         cap, stream=None):
+    _check(load_library().sparse_attn_structured_mask_adaptive(
+        B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors, period, step, q_frame0,
+        budget, _ptr(kv_idx), _ptr(kv_cnt), cap, _stream(stream)))
 
 
 def sparse_attn_forward(q, k, v16, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H, Nq, Nk, d, block,

@@ -59,6 +59,7 @@ class Workload:
     window: int = 3
     n_anchors: int = 4
     period: int = 10
+    budget: int = 0                 # > 0: adaptive windows reaching |A(t)| = budget frames
     steps: tuple = (0,)
     seed: int = 0
 
@@ -119,6 +120,12 @@ WORKLOADS = {
         name="longvideo-41x30x52", B=1, H=12, Nq=63960, Nk=63960, d=128, block=128, order=0,
         mode="structured", recipe="patches", grid=(41, 30, 52), window=3, n_anchors=4,
         period=10, steps=tuple(range(10))),
+    # The same long video with LVSA's extended adaptive windows: every frame attends to
+    # 11 frames (4 anchors + 7 window frames), windows growing past anchors and edges.
+    "longvideo-adaptive-41x30x52": Workload(
+        name="longvideo-adaptive-41x30x52", B=1, H=12, Nq=63960, Nk=63960, d=128, block=128,
+        order=0, mode="structured", recipe="patches", grid=(41, 30, 52), window=3, n_anchors=4,
+        period=10, budget=11, steps=tuple(range(10))),
     # Autoregressive world-model chunk: frame 40 attends to frames 0..40.
     "worldmodel-chunk": Workload(
         name="worldmodel-chunk", B=4, H=16, Nq=1560, Nk=63960, d=128, block=64, order=1,

@@ -164,6 +164,21 @@ int sparse_attn_structured_mask(int B, int H, int Nq, int Nk, int block,
                                 int32_t* kv_idx, int32_t* kv_cnt, int cap, void* stream);
 
 /*
+ * Structured mask with extended adaptive windows (LVSA §2 Fenêtres Adaptatives
+ * Étendues). As sparse_attn_structured_mask, but each query frame's window
+ * { f-window .. f+window } (inside the video) grows one frame at a time, alternately
+ * after and before it (a side at the edge of the video is skipped), while
+ * |G u window| < budget, so that overlaps with the anchors and clipping at the edges
+ * are made up: |A(f)| = max(|G u {f-window .. f+window}|, min(budget, n_frames)).
+ * budget = 0 gives sparse_attn_structured_mask.
+ */
+int sparse_attn_structured_mask_adaptive(int B, int H, int Nq, int Nk, int block,
+                                         int frame_tokens, int n_frames, int window,
+                                         int n_anchors, int period, int step, int q_frame0,
+                                         int budget, int32_t* kv_idx, int32_t* kv_cnt, int cap,
+                                         void* stream);
+
+/*
  * Forward (PISA §2 Algorithme Central and Implémentation Matérielle, phases 1-3,
  * with the first-order term per block, or global with order 2). For each query
  * row t of query block i:

@@ -36,7 +36,9 @@ design notes):
     (cumulative >= tau);
   * structured mode: anchors G_s = {(s mod T_per) + T_per * m}, window
     [t - W, t + W] clipped to the video; a KV block is kept for a query block
-    when any (query token, key token) pair of the two blocks is allowed;
+    when any (query token, key token) pair of the two blocks is allowed; with a
+    budget C (LVSA extended adaptive windows) the window grows one frame at a
+    time, alternately after and before it, until |A(t)| reaches C;
   * hybrid order (order 2, PISA "Algorithme Central", global first-order
     correction): Hbar is the plain mean of the per-block matrices M_j over all
     blocks of the head, and the numerator gains scale * q_t Hbar * sum_j alpha_tj
@@ -179,14 +181,30 @@ def anchor_frames(step: int, period: int, n_anchors: int, n_frames: int):
     return {base + period * m for m in range(n_anchors) if base + period * m < n_frames}
 
 
-def attend_frames(t: int, step: int, window: int, period: int, n_anchors: int, n_frames: int):
-    """A(t) = G_s u W(t), with W(t) = {t - window, ..., t + window} inside the video."""
-    local = {f for f in range(t - window, t + window + 1) if 0 <= f < n_frames}
-    return anchor_frames(step, period, n_anchors, n_frames) | local
+def attend_frames(t: int, step: int, window: int, period: int, n_anchors: int, n_frames: int,
+                  budget: int = 0):
+    """A(t) = G_s u W(t), with W(t) = {t - window, ..., t + window} inside the video.
+
+    budget C > 0 [LVSA §2 "Fenêtres Adaptatives Étendues"]: while |G_s u W(t)| < C and
+    W(t) is not the whole video, the window grows by one frame, alternately after and
+    before it (skipping a side that has reached the edge), so that overlaps with the
+    anchors and clipping at the edges are made up: |A(t)| = max(|G_s u W(t)|, min(C, T)).
+    """
+    anchors = anchor_frames(step, period, n_anchors, n_frames)
+    lo, hi = max(0, t - window), min(n_frames - 1, t + window)
+    after = True
+    while budget > 0 and len(anchors | set(range(lo, hi + 1))) < budget and (lo > 0 or hi < n_frames - 1):
+        if (after and hi < n_frames - 1) or lo == 0:
+            hi += 1
+        else:
+            lo -= 1
+        after = not after
+    return anchors | set(range(lo, hi + 1))
 
 
 def structured_kept(Nq: int, Nk: int, block: int, frame_tokens: int, n_frames: int,
-                    window: int, n_anchors: int, period: int, step: int, q_frame0: int = 0):
+                    window: int, n_anchors: int, period: int, step: int, q_frame0: int = 0,
+                    budget: int = 0):
     """Kept KV blocks per query block: block j is kept for query block i when some
     query token of i and some key token of j lie in frames (tq, tk) with tk in A(tq)."""
     key_frames = [{r // frame_tokens for r in range(ks, ke)} for ks, ke in block_ranges(Nk, block)]
@@ -195,7 +213,7 @@ def structured_kept(Nq: int, Nk: int, block: int, frame_tokens: int, n_frames: i
         q_frames = sorted({(q_frame0 * frame_tokens + t) // frame_tokens for t in range(qs, qe)})
         allowed = set()
         for t in q_frames:
-            allowed |= attend_frames(t, step, window, period, n_anchors, n_frames)
+            allowed |= attend_frames(t, step, window, period, n_anchors, n_frames, budget)
         row = [j for j, kf in enumerate(key_frames) if kf & allowed]
         kept.append(np.asarray(row, dtype=np.int64))
     return kept

@@ -27,6 +27,10 @@ SMALL = {
                                 period=6, steps=(0, 5)),
     "worldmodel-small": W.shrink(W.WORKLOADS["worldmodel-chunk"], name="worldmodel-small", B=2, H=2,
                                  Nq=500, Nk=6500, grid=(13, 10, 50), q_frame0=12),
+    "longvideo-adaptive-small": W.shrink(W.WORKLOADS["longvideo-adaptive-41x30x52"],
+                                         name="longvideo-adaptive-small", H=2, Nq=9500, Nk=9500,
+                                         grid=(19, 10, 50), window=2, n_anchors=3, period=6,
+                                         budget=9, steps=(0, 5)),
     "hybrid-small": W.shrink(W.WORKLOADS["dit720p-hybrid-21x45x80"], name="hybrid-small", H=2,
                              Nq=9480, Nk=9480, grid=(6, 20, 79)),
 }
@@ -42,7 +46,7 @@ def oracle_kept(w: W.Workload, q, k, step: int = 0, v=None):
     Covariance-aware routing needs the head's values ``v``."""
     if w.mode == "structured":
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
-                                 w.n_anchors, w.period, step, w.q_frame0)
+                                 w.n_anchors, w.period, step, w.q_frame0, budget=w.budget)
         return kept, np.ones(len(kept), bool)
     if w.mode in ("topk", "topk_cov"):
         kept, s, counts = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), v=v)

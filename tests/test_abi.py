@@ -72,6 +72,8 @@ def test_host_argument_checks(lib):
                                       0, None, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 6400, 64, 10, 10, 1, 1, 1, 0, 0, p, p, 100, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 64, 64, 8, 8, 1, 1, 0, 0, 0, p, p, 1, 0),
+        lambda: C.sparse_attn_structured_mask_adaptive(1, 1, 64, 64, 64, 8, 8, 1, 1, 2, 0, 0, -1, p,
+                                                       p, 1, 0),
         lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 0, 64, 64, 0, 0.1, p, 0,
                                       None, 0),
         lambda: C.sparse_attn_forward(p, p, p, p, p, None, p, p, 1, 1, 1, 64, 64, 64, 64, 1, 0.1, p,

@@ -27,7 +27,7 @@ def _problem(w):
 
 def _geometry(w):
     return dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
-                n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0)
+                n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0, budget=w.budget)
 
 
 def _run(w, q, k, v, step=0, out_dtype=torch.float32):
@@ -133,18 +133,21 @@ def test_route_masks_bit_exact_above_gate(name, small_inputs):
     assert pinned >= 0.5 * total, (pinned, total)
 
 
-@pytest.mark.parametrize("name", ["longvideo-small", "longvideo-41x30x52", "worldmodel-chunk"])
-def test_structured_mask_bit_exact(name):
+@pytest.mark.parametrize("name", ["longvideo-small", "longvideo-41x30x52", "worldmodel-chunk",
+                                  "longvideo-adaptive-small", "longvideo-adaptive-41x30x52"])
+@pytest.mark.parametrize("budget", [None, 0, 6, 40])
+def test_structured_mask_bit_exact(name, budget):
     w = SMALL.get(name) or W.WORKLOADS[name]
+    budget = w.budget if budget is None else budget
     p = A.Problem(1, 2, w.Nq, w.Nk, w.d, w.block, w.order)
     steps = range(w.period) if w.mode == "structured" else (0, 3)
     for step in steps:
         idx, cnt = A.allocate_lists(p, p.nkb, "cuda")
         A.structured_mask(p, idx, cnt, w.frame_tokens, w.n_frames, w.window, w.n_anchors,
-                          w.period, step, w.q_frame0)
+                          w.period, step, w.q_frame0, budget=budget)
         torch.cuda.synchronize()
         want = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
-                                 w.n_anchors, w.period, step, w.q_frame0)
+                                 w.n_anchors, w.period, step, w.q_frame0, budget=budget)
         for h in range(2):
             got = lists_to_sets(idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy())
             assert got == [x.tolist() for x in want], (name, step)

@@ -69,6 +69,25 @@ def test_golden_structured(golden_dir):
     assert [x.tolist() for x in kept] == g["kept"]
 
 
+def test_golden_structured_adaptive(golden_dir):
+    g = _load(golden_dir, "structured_adaptive.json")
+    kept = O.structured_kept(g["Nq"], g["Nk"], g["block"], g["frame_tokens"], g["n_frames"],
+                             g["window"], g["n_anchors"], g["period"], g["step"], budget=g["budget"])
+    assert [x.tolist() for x in kept] == g["kept"]
+
+
+@pytest.mark.parametrize("n_frames,window,n_anchors,period,budget", [
+    (41, 3, 4, 10, 11), (41, 3, 4, 10, 21), (12, 0, 3, 4, 5), (9, 2, 2, 5, 40), (20, 1, 5, 4, 3)])
+def test_adaptive_window_reaches_the_budget(n_frames, window, n_anchors, period, budget):
+    for step in range(period):
+        for t in range(n_frames):
+            base = O.attend_frames(t, step, window, period, n_anchors, n_frames)
+            ext = O.attend_frames(t, step, window, period, n_anchors, n_frames, budget)
+            assert base <= ext
+            assert len(ext) == max(len(base), min(budget, n_frames)), (step, t)
+            assert t in ext
+
+
 # --- rho = 1 is dense attention ----------------------------------------------
 
 @pytest.mark.parametrize("order", [0, 1])
