@@ -43,6 +43,14 @@ design notes):
     correction): Hbar is the plain mean of the per-block matrices M_j over all
     blocks of the head, and the numerator gains scale * q_t Hbar * sum_j alpha_tj
     over the skipped blocks (no denominator term, as for order 1);
+  * error-aware routing (EAR §2 B): with the query centroid qbar_i as the proxy
+    query, the error of block j is err_ij = || sum_r (exp(s_r) - exp(s_c)) v_r ||^2
+    with s_r = scale qbar_i.k_r and s_c = scale qbar_i.kbar_j: the squared error
+    of the centroid substitution (order 0) on the block's share of the unnormalised
+    attention numerator. The score is ln(err_ij / n_j) (error per unit of cost, the
+    cost being the block's token count; the log only changes the scale), blocks are
+    ranked by it, ties by index, and the top ceil(rho nkb) are kept (the greedy
+    selection under a density budget, with the budget read as a block count);
   * covariance-aware top-k (PISA "Routage Sensible a la Covariance"): the
     norm ||H_j - Hbar||_2 is read as the 2-norm of the matrix entries
     (Frobenius), and the selection score is s_ij + ln ||H_j - Hbar||, the log of
@@ -287,12 +295,39 @@ def covariance_scores(scores: np.ndarray, cnorms: np.ndarray) -> np.ndarray:
         return np.asarray(scores, np.float64) + np.log(np.asarray(cnorms, np.float64))[None, :]
 
 
+def ear_scores(qbar: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, scale: float):
+    """Error-aware routing scores ln(err_ij / n_j)  [EAR §2 B: the squared error of the
+    centroid approximation per block, query centroids as proxies, error per unit of
+    cost]. err_ij = 0 (a block whose keys all give the same logit) scores -inf.
+
+    Every weight of row i and block j is taken relative to m = the largest exact logit
+    of the block: err = exp(2 m) * || sum_r (exp(s_r - m) - exp(s_c - m)) v_r ||^2.
+    """
+    qbar = np.asarray(qbar, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    kbar, _, counts, _ = pool_keys_values(k, v, block, 0)
+    out = np.empty((qbar.shape[0], kbar.shape[0]))
+    for j, (s, e) in enumerate(block_ranges(k.shape[0], block)):
+        logit = scale * (qbar @ k[s:e].T)                 # exact logits s_r, [nqb, n_j]
+        cen = scale * (qbar @ kbar[j])                    # centroid logit s_c
+        m = logit.max(axis=1)
+        x = (np.exp(logit - m[:, None]) - np.exp(cen - m)[:, None]) @ v[s:e]
+        err = (x * x).sum(axis=1)
+        with np.errstate(divide="ignore"):
+            out[:, j] = np.log(err) + 2.0 * m - np.log(counts[j])
+    return out
+
+
 def route_head(q, k, block: int, mode: str, scale: float, keep=None, tau=None, v=None):
     """Pooled routing for one head. Returns (kept lists, scores, prefix lengths).
 
-    mode "topk_cov" needs ``v`` (for the per-block M_j) and returns the
-    covariance-aware scores."""
+    modes "topk_cov" and "ear" need ``v`` (the per-block M_j; the numerator errors)
+    and return their own scores."""
     qbar = pool_queries(q, block)
+    if mode == "ear":
+        s = ear_scores(qbar, k, v, block, scale)
+        return route_topk(s, keep), s, [keep] * s.shape[0]
     if mode == "topk_cov":
         kbar, _, _, mats = pool_keys_values(k, v, block, 1)
         s = covariance_scores(routing_scores(qbar, kbar, scale),

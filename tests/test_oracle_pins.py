@@ -345,3 +345,107 @@ def test_covariance_score_can_overtake_the_attention_score():
     np.testing.assert_allclose(cs, [[1.0, 1.9]], atol=1e-15)
     assert [list(x) for x in O.route_topk(cs, 1)] == [[1]]
     assert [list(x) for x in O.route_topk(s, 1)] == [[0]]
+
+
+# --- error-aware routing (SVG-EAR §2 B) -----------------------------------------
+
+def test_golden_ear(golden_dir):
+    g = _load(golden_dir, "ear_d2.json")
+    q, k, v = (np.array(g[x], float) for x in ("q", "k", "v"))
+    qbar = O.pool_queries(q, g["block"])
+    got = O.ear_scores(qbar, k, v, g["block"], g["scale"])
+    want = np.array([[float(x) for x in row] for row in g["scores"]])
+    assert got.shape == want.shape
+    np.testing.assert_allclose(got[:, 0], want[:, 0], rtol=0, atol=1e-12)
+    assert np.isneginf(got[0, 1])
+
+
+def test_ear_constant_values_reduce_to_the_denominator_gap():
+    # With v_r = u for every token of the block, the numerator error is u times the
+    # scalar gap sum_r exp(s_r) - n exp(s_c), which is >= 0 by Jensen's inequality.
+    rng = np.random.default_rng(11)
+    block, d, scale = 8, 4, 0.5
+    k = _rand(rng, 24, d)
+    u = _rand(rng, d)
+    v = np.tile(u, (24, 1))
+    qbar = _rand(rng, 3, d)
+    got = O.ear_scores(qbar, k, v, block, scale)
+    for j in range(3):
+        kb = k[block * j:block * (j + 1)]
+        for i in range(3):
+            gap = np.exp(scale * kb @ qbar[i]).sum() - block * np.exp(scale * kb.mean(0) @ qbar[i])
+            assert gap > 0
+            want = 2 * np.log(gap) + np.log(u @ u) - np.log(block)
+            assert abs(got[i, j] - want) < 1e-10
+
+
+def test_ear_invariants():
+    rng = np.random.default_rng(12)
+    block, d, scale = 16, 8, 0.35
+    k, v = _rand(rng, 40, d), _rand(rng, 40, d)
+    qbar = _rand(rng, 5, d)
+    base = O.ear_scores(qbar, k, v, block, scale)
+    assert np.all(np.isfinite(base))
+    # values scaled by c: error scaled by c^2
+    np.testing.assert_allclose(O.ear_scores(qbar, k, 3.0 * v, block, scale), base + 2 * np.log(3.0),
+                               atol=1e-10)
+    # one key shift delta for every token of block 1: every logit of the block, the
+    # centroid's included, moves by scale * qbar.delta, so the error moves by twice that
+    delta = _rand(rng, d)
+    k2 = k.copy()
+    k2[16:32] += delta
+    got = O.ear_scores(qbar, k2, v, block, scale)
+    np.testing.assert_allclose(got[:, 1], base[:, 1] + 2 * scale * qbar @ delta, atol=1e-9)
+    np.testing.assert_allclose(got[:, [0, 2]], base[:, [0, 2]], atol=1e-12)
+    # the tokens' order inside a block does not matter
+    perm = np.concatenate([rng.permutation(16), 16 + rng.permutation(16), 32 + rng.permutation(8)])
+    np.testing.assert_allclose(O.ear_scores(qbar, k[perm], v[perm], block, scale), base, atol=1e-10)
+
+
+def test_ear_error_vanishes_for_keys_the_proxy_cannot_tell_apart():
+    # keys that differ only orthogonally to qbar give every token the centroid's logit
+    rng = np.random.default_rng(13)
+    d, block = 4, 8
+    qbar = np.array([[1.0, 0.0, 0.0, 0.0]])
+    k = _rand(rng, 16, d)
+    k[:8, 0] = 0.7
+    v = _rand(rng, 16, d)
+    got = O.ear_scores(qbar, k, v, block, 1.0)
+    assert got[0, 0] < got[0, 1] - 20 or np.isneginf(got[0, 0])
+    k[:8] = k[0]
+    assert np.isneginf(O.ear_scores(qbar, k, v, block, 1.0)[0, 0])
+
+
+def test_ear_prefers_a_heterogeneous_block_over_a_high_score_homogeneous_one():
+    # SVG-EAR §2 B: a block with a high attention score can be well approximated by its
+    # centroid, a low-score block with heterogeneous keys cannot.
+    rng = np.random.default_rng(14)
+    d, block = 8, 16
+    qbar = np.zeros((1, d))
+    qbar[0, 0] = 2.0
+    k = np.zeros((32, d))
+    k[:16] = 1.0 + 0.01 * _rand(rng, 16, d)     # high score, nearly identical keys
+    k[16:] = 0.3 * _rand(rng, 16, d)            # low score, spread-out keys
+    k[16:, 0] += 0.2
+    v = _rand(rng, 32, d)
+    scale = 0.5
+    att = O.routing_scores(qbar, np.stack([k[:16].mean(0), k[16:].mean(0)]), scale)
+    ear = O.ear_scores(qbar, k, v, block, scale)
+    assert att[0, 0] > att[0, 1]
+    assert ear[0, 1] > ear[0, 0]
+    kept_att = O.route_head(np.tile(qbar, (block, 1)), k, block, "topk", scale, keep=1)[0][0]
+    kept_ear = O.route_head(np.tile(qbar, (block, 1)), k, block, "ear", scale, keep=1, v=v)[0][0]
+    assert kept_att.tolist() == [0] and kept_ear.tolist() == [1]
+
+
+def test_ear_divides_the_error_by_the_block_size():
+    # Block 0 holds every token of the partial block 1 twice: the numerator error doubles
+    # in amplitude (x4 squared) while the cost doubles, so the scores differ by ln 2.
+    rng = np.random.default_rng(15)
+    d = 4
+    kb, vb = _rand(rng, 4, d), _rand(rng, 4, d)
+    k = np.concatenate([np.repeat(kb, 2, axis=0), kb])   # block 0: 8 tokens, block 1: 4
+    v = np.concatenate([np.repeat(vb, 2, axis=0), vb])
+    qbar = _rand(rng, 2, d)
+    got = O.ear_scores(qbar, k, v, 8, 0.5)
+    np.testing.assert_allclose(got[:, 0] - got[:, 1], np.log(4.0) - np.log(2.0), atol=1e-10)
