@@ -303,8 +303,11 @@ def main():
         ev[1].record(stream)
         if w.mode == "structured":
             A.structured_mask(p, op.kv_idx, op.kv_cnt, w.frame_tokens, w.n_frames, w.window,
-                              w.n_anchors, w.period, s, w.q_frame0)
+                              w.n_anchors, w.period, s, w.q_frame0, budget=w.budget)
         else:
+            if w.mode == "ear":
+                A.ear_scores(k, p, op.tables, err_flag=op.err_flag)
+                ev[4].record(stream)
             A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
         ev[2].record(stream)
         A.forward(q, k, v, p, op.tables, op.kv_idx, op.kv_cnt, op.out)
@@ -314,7 +317,7 @@ def main():
         op(q, k, v, step=steps_cycle[i % len(steps_cycle)])
     torch.cuda.synchronize(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     dev_id = str(getattr(props, "uuid", local))
@@ -333,6 +336,8 @@ def main():
     ms_step = start.elapsed_time(end) / args.steps
     ms_step_max = max_over_ranks(ms_step)
     stage_ms = [float(np.mean([e[s].elapsed_time(e[s + 1]) for e in evs])) for s in range(3)]
+    # error-aware routing: the probe's share of the route stage (events 1 -> 4)
+    ear_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs])) if w.mode == "ear" else None
 
     # per-launch forward work for the lists of the last step
     kv_idx, kv_cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
@@ -384,6 +389,8 @@ def main():
                        "keep": (f"top {w.rho[0]}/{w.rho[1]}" if w.mode == "topk" else
                                 f"top {w.rho[0]}/{w.rho[1]}, covariance-aware"
                                 if w.mode == "topk_cov" else
+                                f"top {w.rho[0]}/{w.rho[1]}, error-aware"
+                                if w.mode == "ear" else
                                 f"mass {w.tau}" if w.mode == "mass" else "window+anchors"),
                        "output": "fp32",
                        "l2": "inputs exceed L2 (Q+K+V %.2f GB per GPU)" % (
@@ -401,11 +408,23 @@ def main():
             "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")
                               / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
             "clocks": clocks.summary(),
-            "gpu_launches": (5 if w.order == 2 else 3) * args.steps,
+            "gpu_launches": (5 if w.order == 2 else 4 if w.mode == "ear" else 3) * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
         line["pool_roofline"]["frac"] = line["pool_roofline"]["achieved"] / pk["hbm"]
+        if ear_ms is not None:
+            # the probe's algorithmic work: logits and the value product, each
+            # 2 * nqb * Nk * d per head (the 2-piece splits are not counted)
+            ear_fl = 4.0 * w.B * w.H * w.nqb * w.Nk * w.d
+            line["stages_ms"]["ear_probe"] = ear_ms
+            line["ear_roofline"] = {"kernel": "sparse_attn_ear_scores", "bound": "tensor",
+                                    "achieved": ear_fl / (ear_ms / 1e3) / 1e12,
+                                    "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                                    "peak_kind": f"bf16 sustained ({pk['source']})",
+                                    "flops_per_launch": ear_fl}
+            line["ear_roofline"]["frac"] = (line["ear_roofline"]["achieved"]
+                                            / pk["bf16_sustained"])
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as tdist

@@ -28,6 +28,7 @@ class Tables:
     hbar: Optional[torch.Tensor] = None    # [B,H,d,d] fp32 global first-order matrix (order 2)
     hbar16: Optional[torch.Tensor] = None  # [B,H,d,d] fp16
     cov: Optional[torch.Tensor] = None     # [B,H,nkb] fp32 ||M_j - Hbar|| (order 2)
+    scores: Optional[torch.Tensor] = None  # [B,H,nqb,nkb] fp32 error-aware routing scores
 
 
 @dataclasses.dataclass
@@ -49,7 +50,7 @@ class Problem:
         return -(-self.Nk // self.block)
 
 
-def allocate_tables(p: Problem, device) -> Tables:
+def allocate_tables(p: Problem, device, ear: bool = False) -> Tables:
     f32 = dict(dtype=torch.float32, device=device)
     h16 = dict(dtype=torch.float16, device=device)
     return Tables(
@@ -63,6 +64,7 @@ def allocate_tables(p: Problem, device) -> Tables:
         hbar=torch.empty(p.B, p.H, p.d, p.d, **f32) if p.order == 2 else None,
         hbar16=torch.empty(p.B, p.H, p.d, p.d, **h16) if p.order == 2 else None,
         cov=torch.empty(p.B, p.H, p.nkb, **f32) if p.order == 2 else None,
+        scores=torch.empty(p.B, p.H, p.nqb, p.nkb, **f32) if ear else None,
     )
 
 
@@ -86,9 +88,21 @@ def pool(q, k, v, p: Problem, t: Tables, stream=None):
         C.sparse_attn_hbar(t.M, p.B, p.H, p.nkb, p.d, t.hbar, t.hbar16, t.cov, stream)
 
 
+def ear_scores(k, p: Problem, t: Tables, scale=None, err_flag=None, stream=None):
+    """Error-aware routing scores ln(err_ij / n_j) into ``t.scores`` (needs the pooled
+    query centroids and the fp16 values of the pool)."""
+    scale = 1.0 / math.sqrt(p.d) if scale is None else scale
+    C.sparse_attn_ear_scores(t.qbar, k, t.v16, p.B, p.H, p.nqb, p.Nk, p.d, p.block, scale,
+                             t.scores, err_flag, stream)
+
+
 def route(p: Problem, t: Tables, kv_idx, kv_cnt, mode: str, rho=(1, 4), tau=0.9, scale=None,
           stream=None):
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
+    if mode == "ear":
+        C.sparse_attn_route_scores(t.scores, p.B, p.H, p.nqb, p.nkb, rho[0], rho[1], kv_idx,
+                                   kv_cnt, kv_idx.shape[-1], stream)
+        return
     if mode == "topk_cov":
         C.sparse_attn_route_cov(t.qbar, t.kbar_t, t.cov, p.B, p.H, p.nqb, p.nkb, p.d, rho[0],
                                 rho[1], scale, kv_idx, kv_cnt, kv_idx.shape[-1], stream)
@@ -125,7 +139,8 @@ class BlockSparseAttention:
     """Reusable buffers plus the three-stage call for one problem shape.
 
     mode "topk" keeps ceil(rho * nkb) blocks per query block, "topk_cov" the same
-    number by the covariance-aware score (order 2), "mass" the shortest
+    number by the covariance-aware score (order 2), "ear" the same number by the
+    error of the centroid approximation per token (SVG-EAR), "mass" the shortest
     prefix covering tau of the pooled softmax, "structured" the window + rotating
     anchor geometry given in ``geometry`` (frame_tokens, n_frames, window, budget,
     n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
@@ -136,11 +151,11 @@ class BlockSparseAttention:
         self.p, self.mode, self.rho, self.tau, self.geometry = p, mode, rho, tau, geometry
         if mode == "topk_cov" and p.order != 2:
             raise ValueError("covariance-aware routing needs order 2 (the covariance norms)")
-        if mode in ("topk", "topk_cov"):
+        if mode in ("topk", "topk_cov", "ear"):
             cap = -(-rho[0] * p.nkb // rho[1])
         else:
             cap = p.nkb
-        self.tables = allocate_tables(p, device)
+        self.tables = allocate_tables(p, device, ear=mode == "ear")
         self.kv_idx, self.kv_cnt = allocate_lists(p, cap, device)
         self.out = torch.empty(p.B, p.H, p.Nq, p.d, dtype=out_dtype, device=device)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=device)
@@ -155,6 +170,8 @@ class BlockSparseAttention:
                             g["window"], g["n_anchors"], g["period"], step, g.get("q_frame0", 0),
                             g.get("budget", 0), stream)
         else:
+            if self.mode == "ear":
+                ear_scores(k, p, self.tables, err_flag=self.err_flag, stream=stream)
             route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
                   stream=stream)
         forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out,

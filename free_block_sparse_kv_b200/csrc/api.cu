@@ -174,6 +174,51 @@ int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* c
   return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
 }
 
+int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v16, int B, int H,
+                           int nqb, int Nk, int d, int block, float scale, float* scores,
+                           int32_t* err_flag, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && nqb >= 0 && Nk >= 0, "B, H, nqb, Nk must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(block == 64 || block == 128, "block must be 64 or 128 (got %d)", block);
+  SA_REQUIRE(std::isfinite(scale), "scale must be finite");
+  if ((long long)B * H * nqb == 0 || Nk == 0) return ok();
+  const int nkb = cdiv(Nk, block);
+  SA_REQUIRE(nkb <= SA_MAX_KV_BLOCKS, "nkb must be <= %d (got %d)", SA_MAX_KV_BLOCKS, nkb);
+  SA_REQUIRE_PTR(qbar);
+  SA_REQUIRE_PTR(k);
+  SA_REQUIRE_PTR(v16);
+  SA_REQUIRE(scores != nullptr && ((uintptr_t)scores & 3u) == 0,
+             "scores must be a non-null 4-byte aligned pointer");
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
+  if (int rc = check_device()) return rc;
+  sa::EarArgs p{qbar, k, v16, B, H, Nk, d, block, nqb, nkb, scale, scores, err_flag};
+  return launched(sa::launch_ear(p, static_cast<cudaStream_t>(stream)), "ear launch");
+}
+
+int sparse_attn_route_scores(const float* scores, int B, int H, int nqb, int nkb, int rho_num,
+                             int rho_den, int32_t* kv_idx, int32_t* kv_cnt, int cap,
+                             void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && nqb >= 0 && nkb >= 0, "B, H, nqb, nkb must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  if ((long long)B * H * nqb == 0) return ok();
+  SA_REQUIRE(nkb >= 1 && nkb <= SA_MAX_KV_BLOCKS, "nkb must be in [1, %d] (got %d)",
+             SA_MAX_KV_BLOCKS, nkb);
+  SA_REQUIRE(rho_num > 0 && rho_den > 0 && rho_num <= rho_den,
+             "top-k needs 0 < rho_num <= rho_den (got %d/%d)", rho_num, rho_den);
+  const int keep = (int)(((long long)rho_num * nkb + rho_den - 1) / rho_den);
+  SA_REQUIRE(cap >= keep, "cap %d is below the keep count %d", cap, keep);
+  SA_REQUIRE(scores != nullptr && ((uintptr_t)scores & 3u) == 0,
+             "scores must be a non-null 4-byte aligned pointer");
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  if (int rc = check_device()) return rc;
+  // d only picks the kernel instance; the centroid tables are not read
+  sa::RouteArgs p{nullptr, nullptr, B, H, nqb, nkb, 64, SA_ROUTE_TOPK, keep, 1.f, 1.f, kv_idx,
+                  kv_cnt, cap, nullptr, scores};
+  return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
+}
+
 int sparse_attn_hbar(const uint16_t* M, int B, int H, int nkb, int d, float* hbar,
                      uint16_t* hbar16, float* cov, void* stream) {
   SA_REQUIRE(B >= 0 && H >= 0 && nkb >= 0, "B, H, nkb must be >= 0");

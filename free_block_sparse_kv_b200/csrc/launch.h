@@ -19,7 +19,18 @@ struct RouteArgs {
   float tau, scale;
   int32_t *kv_idx, *kv_cnt;
   int cap;
-  const float* cov = nullptr;  // per-block covariance norms: score += ln cov_j (top-k)
+  const float* cov = nullptr;     // per-block covariance norms: score += ln cov_j (top-k)
+  const float* scores = nullptr;  // [B*H][nqb][nkb] precomputed scores (top-k over them)
+};
+
+struct EarArgs {
+  const float* qbar;
+  const uint16_t *k, *v16;
+  int B, H, Nk, d, block, nqb, nkb;
+  float scale;
+  float* scores;
+  int32_t* err_flag;
+  int run = 0;  // key blocks per CTA (0: default)
 };
 
 struct HbarArgs {
@@ -53,5 +64,6 @@ cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);
 cudaError_t launch_forward(const ForwardArgs& p, cudaStream_t st);
 cudaError_t launch_hbar(const HbarArgs& p, cudaStream_t st);
+cudaError_t launch_ear(const EarArgs& p, cudaStream_t st);
 
 }  // namespace sa

@@ -131,7 +131,8 @@ template <int D, int SLOTS>
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, int nqb, int nkb,
              int mode, int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
-             int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov) {
+             int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov,
+             const float* __restrict__ pre) {
   extern __shared__ __align__(16) float rsm[];
   float* qs = rsm;                         // [D][kRouteRows]
   float* sc = rsm + D * kRouteRows;        // [kRouteRows][nkb] scores
@@ -140,14 +141,20 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
   const int i0 = blockIdx.x * kRouteRows;
   const int rows = min(kRouteRows, nqb - i0);
 
-  for (int x = tid; x < D * kRouteRows; x += kRouteThreads) {
+  for (int x = tid; x < D * kRouteRows && !pre; x += kRouteThreads) {
     const int r = x % kRouteRows, c = x / kRouteRows;
     qs[x] = (r < rows) ? qbar[((size_t)bh * nqb + i0 + r) * D + c] : 0.f;
   }
   __syncthreads();
 
+  if (pre) {
+    // precomputed scores (error-aware routing): copy the rows, coalesced
+    for (int r = 0; r < rows; ++r)
+      for (int j = tid; j < nkb; j += kRouteThreads)
+        sc[r * nkb + j] = pre[((size_t)bh * nqb + i0 + r) * nkb + j];
+  }
   const float* kt = kbar_t + (size_t)bh * D * nkb;
-  for (int j = tid; j < nkb; j += kRouteThreads) {
+  for (int j = tid; j < nkb && !pre; j += kRouteThreads) {
     float acc[kRouteRows];
 #pragma unroll
     for (int r = 0; r < kRouteRows; ++r) acc[r] = 0.f;
@@ -187,7 +194,7 @@ static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   dim3 grid((p.nqb + kRouteRows - 1) / kRouteRows, p.B * p.H);
   kern<<<grid, kRouteThreads, smem, st>>>(p.qbar, p.kbar_t, p.nqb, p.nkb, p.mode, p.keep, p.tau,
-                                          p.scale, p.kv_idx, p.kv_cnt, p.cap, p.cov);
+                                          p.scale, p.kv_idx, p.kv_cnt, p.cap, p.cov, p.scores);
   return cudaGetLastError();
 }
 

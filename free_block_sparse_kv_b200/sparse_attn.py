@@ -20,8 +20,8 @@ SA_OUT_F32, SA_OUT_BF16 = 0, 1
 # Entry points declared in include/sparse_attn.h.
 EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
            "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
-           "sparse_attn_structured_mask_adaptive",
-           "sparse_attn_forward", "sparse_attn_last_error")
+           "sparse_attn_structured_mask_adaptive", "sparse_attn_ear_scores",
+           "sparse_attn_route_scores", "sparse_attn_forward", "sparse_attn_last_error")
 
 
 class SparseAttnError(RuntimeError):
@@ -51,6 +51,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_route.argtypes = [_P, _P] + [_I] * 8 + [_F, _F, _P, _P, _I, _P]
     lib.sparse_attn_route_cov.argtypes = [_P, _P, _P] + [_I] * 7 + [_F, _P, _P, _I, _P]
     lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
+    lib.sparse_attn_ear_scores.argtypes = [_P, _P, _P] + [_I] * 6 + [_F, _P, _P, _P]
+    lib.sparse_attn_route_scores.argtypes = [_P] + [_I] * 6 + [_P, _P, _I, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_structured_mask_adaptive.argtypes = [_I] * 13 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
@@ -113,6 +115,20 @@ def sparse_attn_route_cov(qbar, kbar_t, cov, B, H, nqb, nkb, d, rho_num, rho_den
 def sparse_attn_hbar(M, B, H, nkb, d, hbar, hbar16, cov, stream=None):
     _check(load_library().sparse_attn_hbar(
         _ptr(M), B, H, nkb, d, _ptr(hbar), _ptr(hbar16), _ptr(cov), _stream(stream)))
+
+
+def sparse_attn_ear_scores(qbar, k, v16, B, H, nqb, Nk, d, block, scale, scores, err_flag=None,
+                           stream=None):
+    _check(load_library().sparse_attn_ear_scores(
+        _ptr(qbar), _ptr(k), _ptr(v16), B, H, nqb, Nk, d, block, scale, _ptr(scores),
+        _ptr(err_flag), _stream(stream)))
+
+
+def sparse_attn_route_scores(scores, B, H, nqb, nkb, rho_num, rho_den, kv_idx, kv_cnt, cap,
+                             stream=None):
+    _check(load_library().sparse_attn_route_scores(
+        _ptr(scores), B, H, nqb, nkb, rho_num, rho_den, _ptr(kv_idx), _ptr(kv_cnt), cap,
+        _stream(stream)))
 
 
 def sparse_attn_structured_mask(B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors,

@@ -44,7 +44,7 @@ class Workload:
     d: int
     block: int
     order: int                      # 0 or 1: compensation order for skipped blocks
-    mode: str                       # "topk", "topk_cov", "mass" or "structured"
+    mode: str                       # "topk", "topk_cov", "ear", "mass" or "structured"
     rho: tuple = (1, 4)             # keep fraction rho_num / rho_den (topk)
     tau: float = 0.9                # covered mass (mass)
     recipe: str = "blocks"          # "blocks", "patches" or "drift"
@@ -90,7 +90,7 @@ class Workload:
 
     def cap(self) -> int:
         """Row capacity of the kept-index lists."""
-        return self.keep() if self.mode in ("topk", "topk_cov") else self.nkb
+        return self.keep() if self.mode in ("topk", "topk_cov", "ear") else self.nkb
 
     def dense_flops(self) -> float:
         """Dense-equivalent attention flops of one call: 4 * B * H * Nq * Nk * d."""
@@ -115,6 +115,11 @@ WORKLOADS = {
     "dit720p-hybrid-21x45x80": Workload(
         name="dit720p-hybrid-21x45x80", B=1, H=40, Nq=75600, Nk=75600, d=128, block=128, order=2,
         mode="topk_cov", rho=(1, 10), recipe="patches", grid=(21, 45, 80), outlier_p=0.05),
+    # The same 720p call with SVG-EAR's routing: blocks ranked by the error of their
+    # centroid approximation per token, order-0 (centroid) compensation for the rest.
+    "dit720p-ear-21x45x80": Workload(
+        name="dit720p-ear-21x45x80", B=1, H=40, Nq=75600, Nk=75600, d=128, block=128, order=0,
+        mode="ear", rho=(1, 10), recipe="patches", grid=(21, 45, 80), outlier_p=0.05),
     # Long video with a local window and rotating anchor frames (denoising steps 0..9).
     "longvideo-41x30x52": Workload(
         name="longvideo-41x30x52", B=1, H=12, Nq=63960, Nk=63960, d=128, block=128, order=0,

@@ -148,6 +148,39 @@ int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* c
                           void* stream);
 
 /*
+ * Error-aware routing scores (SVG-EAR §2 B, Routage Sensible à l'Erreur: the squared
+ * error of the centroid approximation per key block, query centroids as proxies,
+ * normalised by the block's size; §2 C: computed in one streaming pass, no logit is
+ * written). For query centroid i and key block j with n_j tokens:
+ *   s_r = scale * qbar_i . k_r (r in block j),  s_c = mean_r s_r = scale * qbar_i . kbar_j,
+ *   err_ij = || sum_r (exp(s_r) - exp(s_c)) v_r ||^2,
+ *   scores[i][j] = ln(err_ij / n_j)   (-inf when err_ij = 0).
+ * Computed with qbar as two bf16 pieces and the weight differences as two fp16
+ * pieces on the tensor cores, fp32 accumulation, every weight relative to the
+ * block's largest logit.
+ *   qbar      [B,H,nqb,d] fp32 (as written by the pool)
+ *   k         [B,H,Nk,d]  bf16;  v16 [B,H,Nk,d] fp16 (as written by the pool)
+ *   scores    [B,H,nqb,nkb] fp32, nkb = ceil(Nk / block); every entry is written
+ *   err_flag  optional int32 (4-byte aligned): nonzero after a launch whose waits
+ *             gave up (that launch's scores are then undefined)
+ * k, v16 and qbar must be 16-byte aligned. One launch; nkb <= SA_MAX_KV_BLOCKS.
+ */
+int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v16,
+                           int B, int H, int nqb, int Nk, int d, int block, float scale,
+                           float* scores, int32_t* err_flag, void* stream);
+
+/*
+ * Top-k over precomputed block scores (the greedy error-per-cost choice of SVG-EAR
+ * §2 B under a density budget read as a block count): keeps, per query block, the
+ * first ceil(rho_num * nkb / rho_den) blocks in the order (score descending, j
+ * ascending); -inf scores sort last. Same list format as sparse_attn_route.
+ *   scores  [B,H,nqb,nkb] fp32, e.g. from sparse_attn_ear_scores (no NaN)
+ */
+int sparse_attn_route_scores(const float* scores, int B, int H, int nqb, int nkb,
+                             int rho_num, int rho_den, int32_t* kv_idx, int32_t* kv_cnt,
+                             int cap, void* stream);
+
+/*
  * Structured mask (LVSA §2 Mécanisme Central). Tokens are frame-major with
  * frame_tokens tokens per frame; query token t lies in frame
  * q_frame0 + t / frame_tokens and key token r in frame r / frame_tokens.

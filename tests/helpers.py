@@ -33,7 +33,19 @@ SMALL = {
                                          budget=9, steps=(0, 5)),
     "hybrid-small": W.shrink(W.WORKLOADS["dit720p-hybrid-21x45x80"], name="hybrid-small", H=2,
                              Nq=9480, Nk=9480, grid=(6, 20, 79)),
+    "ear-small": W.shrink(W.WORKLOADS["dit720p-ear-21x45x80"], name="ear-small", H=2, Nq=9480,
+                          Nk=9480, grid=(6, 20, 79)),
 }
+
+# Error-aware scores (ln of the error per token). The GPU takes the logits with a 16-bit
+# split of qbar and the weight differences with a 22-bit split, in fp32 arithmetic, so
+# the error X of a block (relative to the block's largest weight) carries an absolute
+# error of a few 1e-6. Where X >= EAR_X_FLOOR that is below 1e-3 relative, i.e. below
+# EAR_TOL in the score (twice the log of X); a kept-set decision is pinned when the
+# oracle's score gap at the cutoff exceeds two such errors.
+EAR_X_FLOOR = 1e-2
+EAR_TOL = 2e-3
+EAR_GATE = 2 * EAR_TOL
 
 
 def err_stats(got: np.ndarray, want: np.ndarray):
@@ -43,15 +55,15 @@ def err_stats(got: np.ndarray, want: np.ndarray):
 
 def oracle_kept(w: W.Workload, q, k, step: int = 0, v=None):
     """Oracle kept lists of one head and the per-row gate flags (True = pinned).
-    Covariance-aware routing needs the head's values ``v``."""
+    Covariance-aware and error-aware routing need the head's values ``v``."""
     if w.mode == "structured":
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
                                  w.n_anchors, w.period, step, w.q_frame0, budget=w.budget)
         return kept, np.ones(len(kept), bool)
-    if w.mode in ("topk", "topk_cov"):
+    if w.mode in ("topk", "topk_cov", "ear"):
         kept, s, counts = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), v=v)
         gaps, _, _ = O.gate_diagnostics(s, counts)
-        return kept, gaps > GATE
+        return kept, gaps > (EAR_GATE if w.mode == "ear" else GATE)
     kept, s, counts = O.route_head(q, k, w.block, "mass", w.scale, tau=w.tau)
     gaps, lo, hi = O.gate_diagnostics(s, counts, tau=w.tau)
     return kept, (gaps > GATE) & (lo > GATE) & (hi > GATE)

@@ -70,6 +70,17 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_hbar(p, 1, 1, 0, 64, p, p, p, 0),
         lambda: C.sparse_attn_forward(p, p, p, p, p, None, p, p, 1, 1, 1, 64, 64, 64, 64, 2, 0.1, p,
                                       0, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 640, 96, 64, 0.1, p, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 640, 64, 32, 0.1, p, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p + 8, p, 1, 1, 4, 640, 64, 64, 0.1, p, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 640, 64, 64, 0.1, None, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 640, 64, 64, 0.1, p + 2, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 640, 64, 64, float("inf"), p, None, 0),
+        lambda: C.sparse_attn_ear_scores(p, p, p, 1, 1, 4, 64 * 4096, 64, 64, 0.1, p, None, 0),
+        lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 10, 1, 4, p, p, 2, 0),
+        lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 10, 5, 4, p, p, 10, 0),
+        lambda: C.sparse_attn_route_scores(None, 1, 1, 4, 10, 1, 4, p, p, 10, 0),
+        lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 0, 1, 4, p, p, 10, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 6400, 64, 10, 10, 1, 1, 1, 0, 0, p, p, 100, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 64, 64, 8, 8, 1, 1, 0, 0, 0, p, p, 1, 0),
         lambda: C.sparse_attn_structured_mask_adaptive(1, 1, 64, 64, 64, 8, 8, 1, 1, 2, 0, 0, -1, p,

@@ -11,8 +11,8 @@ from free_block_sparse_kv_b200 import attention as A
 from free_block_sparse_kv_b200 import sparse_attn as C
 from free_block_sparse_kv_b200 import workloads as W
 from oracle import block_sparse_attention as O
-from tests.helpers import (GATE, MAX_ABS, MEAN_REL, SMALL, err_stats, lists_to_sets, oracle_kept,
-                           sample_rows)
+from tests.helpers import (EAR_TOL, EAR_X_FLOOR, GATE, MAX_ABS, MEAN_REL, SMALL, err_stats,
+                           lists_to_sets, oracle_kept, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -125,7 +125,7 @@ def test_route_masks_bit_exact_above_gate(name, small_inputs):
             got = lists_to_sets(idx[b, h], cnt[b, h])
             for i in range(w.nqb):
                 total += 1
-                if w.mode in ("topk", "topk_cov"):
+                if w.mode in ("topk", "topk_cov", "ear"):
                     assert len(got[i]) == w.keep()
                 if gate[i]:
                     pinned += 1
@@ -151,6 +151,85 @@ def test_structured_mask_bit_exact(name, budget):
         for h in range(2):
             got = lists_to_sets(idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy())
             assert got == [x.tolist() for x in want], (name, step)
+
+
+# --- error-aware routing scores ---------------------------------------------------
+
+def _ear_check(scores_gpu, q, k, v, block, scale):
+    """GPU scores of one head against the oracle: within EAR_TOL wherever the block's
+    relative error X is above the floor, and small (or -inf) on both sides below it."""
+    qbar = O.pool_queries(q, block)
+    want = O.ear_scores(qbar, k, v, block, scale)
+    got = np.asarray(scores_gpu, np.float64)
+    assert not np.isnan(got).any()
+    # X relative to the block's largest weight: err = X^2 exp(2 m), score = ln(err / n)
+    m = np.stack([(scale * (qbar @ k[s:e].T)).max(axis=1)
+                  for s, e in O.block_ranges(k.shape[0], block)], axis=1)
+    n = np.array([e - s for s, e in O.block_ranges(k.shape[0], block)], np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        x_want = np.exp(0.5 * (want + np.log(n)) - m)
+        x_got = np.exp(0.5 * (got + np.log(n)) - m)
+    big = x_want >= EAR_X_FLOOR
+    assert big.mean() > 0.5, big.mean()
+    err = np.abs(got[big] - want[big])
+    assert err.max() <= EAR_TOL, float(err.max())
+    assert np.all(x_got[~big] <= 2 * EAR_X_FLOOR), float(x_got[~big].max())
+    return err.max()
+
+
+@pytest.mark.parametrize("d,block,Nq,Nk", [(64, 64, 700, 4097), (64, 128, 3000, 6500),
+                                           (128, 64, 300, 6401), (128, 128, 9000, 1000),
+                                           (128, 128, 128, 100)])
+def test_ear_scores_match_oracle(d, block, Nq, Nk):
+    """Random inputs: several centroid tiles (the last partial), several runs of key
+    blocks (the last partial), a ragged last key block (one token where Nk % block == 1,
+    whose score is -inf on both sides) and a single partial block."""
+    B, H = 1, 2
+    qb, kb, vb = (_rand_bits((B, H, N, d), s) for N, s in ((Nq, 21), (Nk, 22), (Nk, 23)))
+    p = A.Problem(B, H, Nq, Nk, d, block, 0)
+    t = A.allocate_tables(p, "cuda", ear=True)
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.pool(q_d, k_d, v_d, p, t)
+    A.ear_scores(k_d, p, t, err_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        got = t.scores[0, h].cpu().numpy()
+        _ear_check(got, q, k, v, block, 1 / np.sqrt(d))
+        if Nk % block == 1:
+            assert np.all(np.isneginf(got[:, -1]))
+
+
+def test_ear_scores_match_oracle_on_the_workload(small_inputs):
+    w, qb, kb, vb = small_inputs("ear-small")
+    op, _ = _run(w, _dev(qb), _dev(kb), _dev(vb))
+    for b in range(w.B):
+        for h in range(w.H):
+            q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+            _ear_check(op.tables.scores[b, h].cpu().numpy(), q, k, v, w.block, w.scale)
+
+
+def test_route_scores_selects_like_the_oracle_on_given_scores():
+    """Top-k over given scores is integer work: exact against the oracle's selection,
+    with many exact ties, -inf entries and a keep count that splits tied groups."""
+    B, H, nqb, nkb = 1, 3, 37, 300
+    rng = np.random.default_rng(31)
+    s = rng.integers(0, 40, size=(B, H, nqb, nkb)).astype(np.float32) * np.float32(0.25)
+    s[rng.random(s.shape) < 0.1] = -np.inf
+    s[0, 2] = -np.inf                            # a head where every score is -inf
+    scores = torch.from_numpy(s).cuda()
+    for rho in ((1, 10), (1, 3), (1, 1)):
+        keep = -(-rho[0] * nkb // rho[1])
+        idx = torch.zeros(B, H, nqb, keep, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(B, H, nqb, dtype=torch.int32, device="cuda")
+        C.sparse_attn_route_scores(scores, B, H, nqb, nkb, rho[0], rho[1], idx, cnt, keep)
+        torch.cuda.synchronize()
+        for h in range(H):
+            want = O.route_topk(s[0, h].astype(np.float64), keep)
+            got = lists_to_sets(idx[0, h].cpu().numpy(), cnt[0, h].cpu().numpy())
+            assert got == [x.tolist() for x in want], (rho, h)
 
 
 # --- forward ------------------------------------------------------------------
