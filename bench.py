@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run on this many heads instead of the workload's (profiler captures)")
     return ap.parse_args()
 
 
@@ -89,7 +91,7 @@ def executed_flops(w: W.Workload, kv_idx: np.ndarray, kv_cnt: np.ndarray) -> dic
     return dict(exact=exact, order0=order0, order1=order1, total=exact + order0 + order1)
 
 
-FORWARD_SOURCES = ("forward_tc.cu", "tc.cuh", "common.cuh")
+FORWARD_SOURCES = ("forward_tc.cu", "tc.cuh", "common.cuh", "tmap.h")
 
 
 def forward_sources_sha256() -> str:
@@ -265,6 +267,8 @@ def run_reference(args, w):
 def main():
     args = parse()
     w = W.WORKLOADS[args.workload]
+    if args.heads:
+        w = W.shrink(w, H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
         return
@@ -306,7 +310,7 @@ def main():
                               w.n_anchors, w.period, s, w.q_frame0, budget=w.budget)
         else:
             if w.mode == "ear":
-                A.ear_scores(k, p, op.tables, err_flag=op.err_flag)
+                A.ear_scores(k, v, p, op.tables, err_flag=op.err_flag)
                 ev[4].record(stream)
             A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
         ev[2].record(stream)

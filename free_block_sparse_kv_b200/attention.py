@@ -88,11 +88,11 @@ def pool(q, k, v, p: Problem, t: Tables, stream=None):
         C.sparse_attn_hbar(t.M, p.B, p.H, p.nkb, p.d, t.hbar, t.hbar16, t.cov, stream)
 
 
-def ear_scores(k, p: Problem, t: Tables, scale=None, err_flag=None, stream=None):
+def ear_scores(k, v, p: Problem, t: Tables, scale=None, err_flag=None, stream=None):
     """Error-aware routing scores ln(err_ij / n_j) into ``t.scores`` (needs the pooled
-    query centroids and the fp16 values of the pool)."""
+    query centroids)."""
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
-    C.sparse_attn_ear_scores(t.qbar, k, t.v16, p.B, p.H, p.nqb, p.Nk, p.d, p.block, scale,
+    C.sparse_attn_ear_scores(t.qbar, k, v, p.B, p.H, p.nqb, p.Nk, p.d, p.block, scale,
                              t.scores, err_flag, stream)
 
 
@@ -171,7 +171,7 @@ class BlockSparseAttention:
                             g.get("budget", 0), stream)
         else:
             if self.mode == "ear":
-                ear_scores(k, p, self.tables, err_flag=self.err_flag, stream=stream)
+                ear_scores(k, v, p, self.tables, err_flag=self.err_flag, stream=stream)
             route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
                   stream=stream)
         forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out,

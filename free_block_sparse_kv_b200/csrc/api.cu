@@ -174,7 +174,7 @@ int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* c
   return launched(sa::launch_route(p, static_cast<cudaStream_t>(stream)), "route launch");
 }
 
-int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v16, int B, int H,
+int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v, int B, int H,
                            int nqb, int Nk, int d, int block, float scale, float* scores,
                            int32_t* err_flag, void* stream) {
   SA_REQUIRE(B >= 0 && H >= 0 && nqb >= 0 && Nk >= 0, "B, H, nqb, Nk must be >= 0");
@@ -187,12 +187,12 @@ int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t*
   SA_REQUIRE(nkb <= SA_MAX_KV_BLOCKS, "nkb must be <= %d (got %d)", SA_MAX_KV_BLOCKS, nkb);
   SA_REQUIRE_PTR(qbar);
   SA_REQUIRE_PTR(k);
-  SA_REQUIRE_PTR(v16);
+  SA_REQUIRE_PTR(v);
   SA_REQUIRE(scores != nullptr && ((uintptr_t)scores & 3u) == 0,
              "scores must be a non-null 4-byte aligned pointer");
   if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
   if (int rc = check_device()) return rc;
-  sa::EarArgs p{qbar, k, v16, B, H, Nk, d, block, nqb, nkb, scale, scores, err_flag};
+  sa::EarArgs p{qbar, k, v, B, H, Nk, d, block, nqb, nkb, scale, scores, err_flag};
   return launched(sa::launch_ear(p, static_cast<cudaStream_t>(stream)), "ear launch");
 }
 

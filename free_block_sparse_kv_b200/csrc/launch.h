@@ -25,7 +25,7 @@ struct RouteArgs {
 
 struct EarArgs {
   const float* qbar;
-  const uint16_t *k, *v16;
+  const uint16_t *k, *v;
   int B, H, Nk, d, block, nqb, nkb;
   float scale;
   float* scores;

@@ -117,10 +117,10 @@ def sparse_attn_hbar(M, B, H, nkb, d, hbar, hbar16, cov, stream=None):
         _ptr(M), B, H, nkb, d, _ptr(hbar), _ptr(hbar16), _ptr(cov), _stream(stream)))
 
 
-def sparse_attn_ear_scores(qbar, k, v16, B, H, nqb, Nk, d, block, scale, scores, err_flag=None,
+def sparse_attn_ear_scores(qbar, k, v, B, H, nqb, Nk, d, block, scale, scores, err_flag=None,
                            stream=None):
     _check(load_library().sparse_attn_ear_scores(
-        _ptr(qbar), _ptr(k), _ptr(v16), B, H, nqb, Nk, d, block, scale, _ptr(scores),
+        _ptr(qbar), _ptr(k), _ptr(v), B, H, nqb, Nk, d, block, scale, _ptr(scores),
         _ptr(err_flag), _stream(stream)))
 
 

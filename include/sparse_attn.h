@@ -155,17 +155,17 @@ int sparse_attn_route_cov(const float* qbar, const float* kbar_t, const float* c
  *   s_r = scale * qbar_i . k_r (r in block j),  s_c = mean_r s_r = scale * qbar_i . kbar_j,
  *   err_ij = || sum_r (exp(s_r) - exp(s_c)) v_r ||^2,
  *   scores[i][j] = ln(err_ij / n_j)   (-inf when err_ij = 0).
- * Computed with qbar as two bf16 pieces and the weight differences as two fp16
- * pieces on the tensor cores, fp32 accumulation, every weight relative to the
- * block's largest logit.
+ * Computed on the tensor cores with fp32 accumulation: qbar as two bf16 pieces
+ * (about 16 significant bits), the weight differences as two bf16 pieces (the top
+ * 16 bits of each), every weight relative to the block's largest logit.
  *   qbar      [B,H,nqb,d] fp32 (as written by the pool)
- *   k         [B,H,Nk,d]  bf16;  v16 [B,H,Nk,d] fp16 (as written by the pool)
+ *   k, v      [B,H,Nk,d]  bf16, as for the pool
  *   scores    [B,H,nqb,nkb] fp32, nkb = ceil(Nk / block); every entry is written
  *   err_flag  optional int32 (4-byte aligned): nonzero after a launch whose waits
  *             gave up (that launch's scores are then undefined)
- * k, v16 and qbar must be 16-byte aligned. One launch; nkb <= SA_MAX_KV_BLOCKS.
+ * k, v and qbar must be 16-byte aligned. One launch; nkb <= SA_MAX_KV_BLOCKS.
  */
-int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v16,
+int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t* v,
                            int B, int H, int nqb, int Nk, int d, int block, float scale,
                            float* scores, int32_t* err_flag, void* stream);
 

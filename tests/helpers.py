@@ -38,13 +38,14 @@ SMALL = {
 }
 
 # Error-aware scores (ln of the error per token). The GPU takes the logits with a 16-bit
-# split of qbar and the weight differences with a 22-bit split, in fp32 arithmetic, so
-# the error X of a block (relative to the block's largest weight) carries an absolute
-# error of a few 1e-6. Where X >= EAR_X_FLOOR that is below 1e-3 relative, i.e. below
-# EAR_TOL in the score (twice the log of X); a kept-set decision is pinned when the
+# split of qbar and the weight differences with a 16-bit split (each within 2^-15 of
+# its value) in fp32 arithmetic. The relative error of X (the block's numerator error,
+# relative to the block's largest weight) is then a few 2^-16 / sqrt(3) per term, summed
+# with random signs over the block, about 1e-5 of X where X >= EAR_X_FLOOR; the score is
+# ln ||X||^2, so its error stays below EAR_TOL. A kept-set decision is pinned when the
 # oracle's score gap at the cutoff exceeds two such errors.
 EAR_X_FLOOR = 1e-2
-EAR_TOL = 2e-3
+EAR_TOL = 2e-4
 EAR_GATE = 2 * EAR_TOL
 
 

@@ -191,7 +191,7 @@ def test_ear_scores_match_oracle(d, block, Nq, Nk):
     q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     A.pool(q_d, k_d, v_d, p, t)
-    A.ear_scores(k_d, p, t, err_flag=flag)
+    A.ear_scores(k_d, v_d, p, t, err_flag=flag)
     torch.cuda.synchronize()
     assert int(flag.item()) == 0
     for h in range(H):
@@ -315,6 +315,8 @@ def test_full_size_sampled(name):
     pinned = total = 0
     for b, h in heads:
         q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+        if w.mode == "ear":
+            _ear_check(op.tables.scores[b, h].cpu().numpy(), q, k, v, w.block, w.scale)
         kept, gate = oracle_kept(w, q, k, step, v=v)
         got = lists_to_sets(idx[b, h], cnt[b, h])
         for i in range(w.nqb):
