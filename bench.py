@@ -211,6 +211,12 @@ def time_oracle(w: W.Workload, seconds: float) -> dict:
     from oracle import block_sparse_attention as O
     q, k, v = W.head_inputs(w, 0, 0)
     t0 = time.perf_counter()
+    if w.clusters:
+        from oracle import cluster_layout as K
+        cq, ck, iters = w.clusters
+        pq = K.group_major_permutation(K.kmeans(q, cq, iters)[0], cq)[0]
+        pk = K.group_major_permutation(K.kmeans(k, ck, iters)[0], ck)[0]
+        q, k, v = q[pq], k[pk], v[pk]
     if w.mode == "structured":
         kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
                                  w.n_anchors, w.period, 0, w.q_frame0, budget=w.budget)
@@ -235,7 +241,8 @@ def time_oracle(w: W.Workload, seconds: float) -> dict:
     tflops = 4.0 * w.Nk * w.d / per_row / 1e12
     cores = len(os.sched_getaffinity(0))
     return dict(value=tflops, unit=UNIT, cores=cores, kind="oracle",
-                sample=f"{w.name}: head (0,0) pooled and routed ({t_setup:.1f} s), then {done} of "
+                sample=f"{w.name}: head (0,0) {'clustered, ' if w.clusters else ''}pooled and "
+                       f"routed ({t_setup:.1f} s), then {done} of "
                        f"{w.Nq} query rows forwarded ({t_rows:.1f} s); scaled per row to the "
                        f"dense-equivalent flops of one call",
                 seconds=t_setup + t_rows, ms_per_call_est=per_row * w.Nq * w.B * w.H * 1e3)
@@ -295,33 +302,43 @@ def main():
                     n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0, budget=w.budget)
     op = A.BlockSparseAttention(p, w.mode, rho=w.rho, tau=w.tau,
                                 geometry=geometry if w.mode == "structured" else None,
-                                out_dtype=torch.float32, device=dev)
+                                out_dtype=torch.float32, device=dev,
+                                clusters=w.clusters or None)
     stream = torch.cuda.current_stream(dev)
     steps_cycle = w.steps if w.mode == "structured" else (0,)
 
     def stage_step(s, ev):
-        """One step with events around each stage (pool, mask/route, forward)."""
+        """One step with events around each stage: (clustering), pool, mask/route,
+        forward, (output back to the query order)."""
         use_q = w.mode != "structured"
         ev[0].record(stream)
-        A.pool(q if use_q else None, k, v, p, op.tables)
+        qq, kk, vv, out = q, k, v, op.out
+        if w.clusters:
+            qq, kk, vv = op.cluster(q, k, v)
+            out = op.out_p
+        ev[5].record(stream)
+        A.pool(qq if use_q else None, kk, vv, p, op.tables)
         ev[1].record(stream)
         if w.mode == "structured":
             A.structured_mask(p, op.kv_idx, op.kv_cnt, w.frame_tokens, w.n_frames, w.window,
                               w.n_anchors, w.period, s, w.q_frame0, budget=w.budget)
         else:
             if w.mode == "ear":
-                A.ear_scores(k, v, p, op.tables, err_flag=op.err_flag)
+                A.ear_scores(kk, vv, p, op.tables, err_flag=op.err_flag)
                 ev[4].record(stream)
             A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
         ev[2].record(stream)
-        A.forward(q, k, v, p, op.tables, op.kv_idx, op.kv_cnt, op.out)
+        A.forward(qq, kk, vv, p, op.tables, op.kv_idx, op.kv_cnt, out)
         ev[3].record(stream)
+        if w.clusters:
+            A.permute_rows(op.out_p, op.cl_q.perm, op.out, gather=False)
+        ev[6].record(stream)
 
     for i in range(args.warmup):
         op(q, k, v, step=steps_cycle[i % len(steps_cycle)])
     torch.cuda.synchronize(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     dev_id = str(getattr(props, "uuid", local))
@@ -339,7 +356,9 @@ def main():
     op.check()
     ms_step = start.elapsed_time(end) / args.steps
     ms_step_max = max_over_ranks(ms_step)
-    stage_ms = [float(np.mean([e[s].elapsed_time(e[s + 1]) for e in evs])) for s in range(3)]
+    mean_ms = lambda a, b: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+    stage_ms = [mean_ms(5, 1), mean_ms(1, 2), mean_ms(2, 3)]  # pool, route / mask, forward
+    cluster_ms = (mean_ms(0, 5), mean_ms(3, 6)) if w.clusters else None
     # error-aware routing: the probe's share of the route stage (events 1 -> 4)
     ear_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs])) if w.mode == "ear" else None
 
@@ -412,11 +431,18 @@ def main():
             "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")
                               / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
             "clocks": clocks.summary(),
-            "gpu_launches": (5 if w.order == 2 else 4 if w.mode == "ear" else 3) * args.steps,
+            "gpu_launches": ((5 if w.order == 2 else 4 if w.mode == "ear" else 3)
+                             + (2 * (7 + 7 * w.clusters[2]) + 4 if w.clusters else 0))
+                            * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
         line["pool_roofline"]["frac"] = line["pool_roofline"]["achieved"] / pk["hbm"]
+        if cluster_ms is not None:
+            line["stages_ms"]["cluster"] = cluster_ms[0]
+            line["stages_ms"]["unpermute"] = cluster_ms[1]
+            line["config"]["clusters"] = {"C_q": w.clusters[0], "C_k": w.clusters[1],
+                                          "iters": w.clusters[2]}
         if ear_ms is not None:
             # the probe's algorithmic work: logits and the value product, each
             # 2 * nqb * Nk * d per head (the 2-piece splits are not counted)

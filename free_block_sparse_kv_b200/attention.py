@@ -13,6 +13,7 @@ from typing import Optional
 import torch
 
 from . import sparse_attn as C
+from . import sparse_attn as _C
 
 
 @dataclasses.dataclass
@@ -66,6 +67,44 @@ def allocate_tables(p: Problem, device, ear: bool = False) -> Tables:
         cov=torch.empty(p.B, p.H, p.nkb, **f32) if p.order == 2 else None,
         scores=torch.empty(p.B, p.H, p.nqb, p.nkb, **f32) if ear else None,
     )
+
+
+@dataclasses.dataclass
+class Clustering:
+    """Buffers of one tensor's k-means and its group-major layout (include/sparse_attn.h)."""
+    C: int
+    iters: int
+    centroids: torch.Tensor  # [B,H,C,d] fp64
+    cwork: torch.Tensor      # scratch bytes
+    iwork: torch.Tensor      # scratch int32
+    labels: torch.Tensor     # [B,H,N] int32
+    perm: torch.Tensor       # [B,H,N] int32: perm[p] = original index at position p
+    offsets: torch.Tensor    # [B,H,C+1] int32
+
+
+def allocate_clustering(B, H, N, d, C, iters, device) -> Clustering:
+    _, s_cw, s_iw = _C.sparse_attn_kmeans_sizes(B, H, N, d, C)
+    i32 = dict(dtype=torch.int32, device=device)
+    return Clustering(
+        C=C, iters=iters,
+        centroids=torch.empty(B, H, C, d, dtype=torch.float64, device=device),
+        cwork=torch.empty(max(s_cw, 16), dtype=torch.uint8, device=device),
+        iwork=torch.empty(max(s_iw // 4, 4), **i32),
+        labels=torch.empty(B, H, N, **i32), perm=torch.empty(B, H, N, **i32),
+        offsets=torch.empty(B, H, C + 1, **i32))
+
+
+def kmeans(x, cl: Clustering, err_flag=None, stream=None):
+    """k-means of x's rows per (b, h) and the stable group-major order of the labels."""
+    B, H, N, d = x.shape
+    _C.sparse_attn_kmeans(x, B, H, N, d, cl.C, cl.iters, cl.centroids, cl.cwork, cl.iwork,
+                          cl.labels, cl.perm, cl.offsets, err_flag, stream)
+
+
+def permute_rows(src, perm, dst, gather=True, stream=None):
+    """gather: dst[p] = src[perm[p]]; otherwise dst[perm[p]] = src[p] (per (b, h))."""
+    B, H, N, d = src.shape
+    _C.sparse_attn_permute_rows(src, perm, B, H, N, d * src.element_size(), gather, dst, stream)
 
 
 def allocate_lists(p: Problem, cap: int, device):
@@ -144,11 +183,15 @@ class BlockSparseAttention:
     prefix covering tau of the pooled softmax, "structured" the window + rotating
     anchor geometry given in ``geometry`` (frame_tokens, n_frames, window, budget,
     n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
+    ``clusters`` = (C_q, C_k, iters) first clusters Q and K by k-means and runs the
+    three stages on their group-major copies (V follows K), returning the output in the
+    original query order.
     """
 
     def __init__(self, p: Problem, mode: str, rho=(1, 4), tau=0.9, geometry=None,
-                 out_dtype=torch.float32, device="cuda"):
+                 out_dtype=torch.float32, device="cuda", clusters=None):
         self.p, self.mode, self.rho, self.tau, self.geometry = p, mode, rho, tau, geometry
+        self.clusters = clusters
         if mode == "topk_cov" and p.order != 2:
             raise ValueError("covariance-aware routing needs order 2 (the covariance norms)")
         if mode in ("topk", "topk_cov", "ear"):
@@ -159,9 +202,40 @@ class BlockSparseAttention:
         self.kv_idx, self.kv_cnt = allocate_lists(p, cap, device)
         self.out = torch.empty(p.B, p.H, p.Nq, p.d, dtype=out_dtype, device=device)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=device)
+        if clusters:
+            # cluster-permuted layout: (C_q, C_k, iters); blocks are cut from the
+            # group-major order of each tensor's k-means labels
+            if mode == "structured":
+                raise ValueError("the structured mask works on frame order, not on clusters")
+            cq, ck, iters = clusters
+            self.cl_q = allocate_clustering(p.B, p.H, p.Nq, p.d, cq, iters, device)
+            self.cl_k = allocate_clustering(p.B, p.H, p.Nk, p.d, ck, iters, device)
+            bf = dict(dtype=torch.bfloat16, device=device)
+            self.q_p = torch.empty(p.B, p.H, p.Nq, p.d, **bf)
+            self.k_p = torch.empty(p.B, p.H, p.Nk, p.d, **bf)
+            self.v_p = torch.empty(p.B, p.H, p.Nk, p.d, **bf)
+            self.out_p = torch.empty_like(self.out)
+
+    def cluster(self, q, k, v, stream=None):
+        """k-means of Q and K and the group-major copies of Q, K and V."""
+        kmeans(q, self.cl_q, self.err_flag, stream)
+        kmeans(k, self.cl_k, self.err_flag, stream)
+        permute_rows(q, self.cl_q.perm, self.q_p, True, stream)
+        permute_rows(k, self.cl_k.perm, self.k_p, True, stream)
+        permute_rows(v, self.cl_k.perm, self.v_p, True, stream)
+        return self.q_p, self.k_p, self.v_p
 
     def __call__(self, q, k, v, step: int = 0, stream=None) -> torch.Tensor:
         _check_inputs(q, k, v)
+        if self.clusters:
+            qp, kp, vp = self.cluster(q, k, v, stream)
+            self._attend(qp, kp, vp, self.out_p, step, stream)
+            permute_rows(self.out_p, self.cl_q.perm, self.out, False, stream)
+            return self.out
+        self._attend(q, k, v, self.out, step, stream)
+        return self.out
+
+    def _attend(self, q, k, v, out, step, stream):
         p = self.p
         pool(q if self.mode != "structured" else None, k, v, p, self.tables, stream)
         if self.mode == "structured":
@@ -174,9 +248,8 @@ class BlockSparseAttention:
                 ear_scores(k, v, p, self.tables, err_flag=self.err_flag, stream=stream)
             route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
                   stream=stream)
-        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, self.out,
+        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, out,
                 err_flag=self.err_flag, stream=stream)
-        return self.out
 
     def check(self):
         """Raise if a bounded device wait of an earlier call gave up (synchronises)."""

@@ -271,6 +271,54 @@ int sparse_attn_structured_mask_adaptive(int B, int H, int Nq, int Nk, int block
   return launched(sa::launch_structured_mask(p, static_cast<cudaStream_t>(stream)), "mask launch");
 }
 
+int sparse_attn_kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
+  SA_REQUIRE(B >= 0 && H >= 0 && N >= 0, "B, H, N must be >= 0");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(C >= 1 && C <= SA_MAX_CLUSTERS, "C must be in [1, %d] (got %d)", SA_MAX_CLUSTERS, C);
+  SA_REQUIRE(sizes != nullptr, "sizes must not be NULL");
+  sa::kmeans_sizes(B, H, N, d, C, sizes);
+  return ok();
+}
+
+int sparse_attn_kmeans(const uint16_t* x, int B, int H, int N, int d, int C, int iters,
+                       double* centroids, void* cwork, int32_t* iwork, int32_t* labels,
+                       int32_t* perm, int32_t* offsets, int32_t* err_flag, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && N >= 0, "B, H, N must be >= 0");
+  SA_REQUIRE((long long)B * H <= 65535, "B*H must be <= 65535");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(C >= 1 && C <= SA_MAX_CLUSTERS, "C must be in [1, %d] (got %d)", SA_MAX_CLUSTERS, C);
+  SA_REQUIRE(iters >= 0 && iters <= 1000, "iters must be in [0, 1000] (got %d)", iters);
+  if ((long long)B * H == 0 || N == 0) return ok();
+  SA_REQUIRE(C <= N, "C must be <= N (C %d, N %d)", C, N);
+  SA_REQUIRE_PTR(x);
+  SA_REQUIRE_PTR(centroids);
+  SA_REQUIRE_PTR(cwork);
+  SA_REQUIRE_PTR(iwork);
+  SA_REQUIRE_PTR(labels);
+  SA_REQUIRE_PTR(perm);
+  SA_REQUIRE_PTR(offsets);
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
+  if (int rc = check_device()) return rc;
+  sa::KmeansArgs p{x, B, H, N, d, C, iters, centroids, cwork, iwork, labels, perm, offsets,
+                   err_flag};
+  return launched(sa::launch_kmeans(p, static_cast<cudaStream_t>(stream)), "kmeans launch");
+}
+
+int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H, int N,
+                             int row_bytes, int gather, void* dst, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && N >= 0, "B, H, N must be >= 0");
+  SA_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "row_bytes must be a positive multiple of 16");
+  SA_REQUIRE(gather == 0 || gather == 1, "gather must be 0 or 1");
+  if ((long long)B * H * N == 0) return ok();
+  SA_REQUIRE_PTR(src);
+  SA_REQUIRE_PTR(perm);
+  SA_REQUIRE_PTR(dst);
+  SA_REQUIRE(src != dst, "src and dst must not be the same buffer");
+  if (int rc = check_device()) return rc;
+  sa::PermuteArgs p{src, perm, B, H, N, row_bytes, gather != 0, dst};
+  return launched(sa::launch_permute_rows(p, static_cast<cudaStream_t>(stream)), "permute launch");
+}
+
 int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
                         const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H, int Nq,

@@ -1,0 +1,646 @@
+// k-means clustering of one tensor's rows per (batch, head) and the group-major token
+// layout built from it.
+//
+// Follows "SVG-EAR: Parameter-Free Linear Compensation for Sparse Video Generation via
+// Error-aware Routing" §2 A (query and key tokens grouped into semantic clusters by
+// k-means before the sparse attention) and "Partition the Support, Reconstruct the
+// Residual: Training-Free Sparse Attention for Video Generation and World Models" §2 C
+// (tokens permuted into contiguous group-major layouts).
+//
+// Lloyd's iteration from the tokens at floor(m N / C): assign every token to its nearest
+// centroid (ties to the lowest index), move every centroid to the mean of its members
+// (one without members stays), and after the last update assign once more. The layout
+// is the stable counting sort of the final labels.
+//
+// Kernels, per iteration:
+//   assign   tcgen05: a tile of 128 tokens against tiles of 128 centroids,
+//            S = X C_hi^T + X C_lo^T (the fp64 centroids as two bf16 pieces), score
+//            ||c||^2 - 2 S in fp32; a token whose two best scores lie closer than the
+//            error bound of that arithmetic goes on a list instead of being decided;
+//   recheck  the listed tokens in fp64 against every centroid (one warp each);
+//   hist / scan / scatter   stable counting sort: one warp per chunk of 1024 tokens;
+//   update   one CTA per cluster sums its members in fp64 (the sums of bf16 values are
+//            exact, so the means are the correctly rounded fp64 means) and writes the
+//            bf16 pieces and the fp32 squared norm the next assignment reads.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace sa {
+namespace km {
+
+constexpr int TT = 128;                      // tokens per assignment tile
+constexpr int TCN = 128;                     // centroids per tile
+constexpr int kChunk = 1024;                 // tokens per sorting warp
+constexpr int kSortWarps = 4;
+constexpr int kMaxC = 4096;
+constexpr uint32_t kWaitLimit = 1u << 18;
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------
+// init and prep
+// ---------------------------------------------------------------------------
+__global__ void init_kernel(const uint16_t* __restrict__ x, int N, int d, int C,
+                            double* __restrict__ cent) {
+  const int m = blockIdx.x, bh = blockIdx.y;
+  const long long r = (long long)m * N / C;
+  const uint16_t* src = x + ((size_t)bh * N + r) * d;
+  double* dst = cent + ((size_t)bh * C + m) * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x)
+    dst[i] = (double)__uint_as_float((uint32_t)src[i] << 16);
+}
+
+// The assignment's operands from the fp64 centroids: bf16 hi = rn(c), lo = rn(c - hi),
+// and ||c||^2 in fp32; padding centroids (m >= C) get zero pieces and +inf. Also clears
+// the head's list of undecided tokens.
+__global__ void prep_kernel(const double* __restrict__ cent, int C, int Cpad, int d,
+                            uint16_t* __restrict__ pieces, float* __restrict__ cnorm,
+                            int32_t* __restrict__ amb_cnt) {
+  const int m = blockIdx.x, bh = blockIdx.y;
+  __shared__ double red[32];
+  uint16_t* hi = pieces + (((size_t)bh * 2 + 0) * Cpad + m) * d;
+  uint16_t* lo = pieces + (((size_t)bh * 2 + 1) * Cpad + m) * d;
+  double s = 0.0;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    if (m < C) {
+      const double c = cent[((size_t)bh * C + m) * d + i];
+      const float cf = (float)c;
+      const __nv_bfloat16 h = __float2bfloat16_rn(cf);
+      const float rest = (float)(c - (double)__bfloat162float(h));
+      const __nv_bfloat16 l = __float2bfloat16_rn(rest);
+      hi[i] = __bfloat16_as_ushort(h);
+      lo[i] = __bfloat16_as_ushort(l);
+      s += c * c;
+    } else {
+      hi[i] = 0;
+      lo[i] = 0;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)blockDim.x / 32; ++w) t += red[w];
+    cnorm[(size_t)bh * Cpad + m] = m < C ? (float)t : INFINITY;
+    if (m == 0) amb_cnt[bh] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// assign (tcgen05)
+// ---------------------------------------------------------------------------
+// One CTA per (head, pair of token tiles), one CTA per SM:
+//   warps 0-3 / 4-7  one thread per token of tile 0 / 1: scores of each centroid tile from
+//                    TMEM, the three best scores and the two best indices;
+//   warp 8           TMA: both token tiles once, then the centroid tiles (hi and lo
+//                    pieces) through a two-stage ring that both tiles read;
+//   warps 9 / 10     MMA issuer of tile 0 / 1: S = X C_hi^T + X C_lo^T into the tile's
+//                    next logit buffer (two per tile, 128 columns each).
+template <int D>
+struct AGeom {
+  static constexpr int SUB = D / 64;
+  static constexpr int XT = TT * D * 2;       // one token tile (bf16)
+  static constexpr int CT = TCN * D * 2;      // one centroid piece tile (bf16)
+  static constexpr int NCS = 2;               // centroid stages
+  static constexpr int OFF_X = 0;             // [2 tiles][SUB][128 rows x 128 B]
+  static constexpr int OFF_C = 2 * XT;        // [NCS][2 pieces][SUB][128 rows x 128 B]
+  static constexpr int OFF_CTL = OFF_C + NCS * 2 * CT;
+  static constexpr int OFF_CN = OFF_CTL + 256;  // [Cpad] ||c||^2, sized at launch
+  static constexpr int TCOLS = 512;           // [2 tiles][2 buffers][128 columns]
+  // one CTA per SM, so that its 512 TMEM columns are always free
+  static constexpr int FLOOR = 232448 / 2 + 1024;
+  static int smem(int Cpad) {
+    const int need = OFF_CN + Cpad * 4 + 1024;  // + alignment slack
+    return need > FLOOR ? need : FLOOR;
+  }
+};
+
+struct ACtl {
+  uint64_t x_full, c_full[2], c_empty[2], s_full[2][2], s_free[2][2], done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct AParams {
+  CUtensorMap tmX, tmC;
+  const float* cnorm;
+  int32_t* labels;
+  int32_t* amb_list;
+  int32_t* amb_pair;
+  int32_t* amb_cnt;
+  int32_t* err_flag;
+  int N, Cpad, npair;
+};
+
+template <int D>
+__global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ AParams p) {
+  using G = AGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t base = smem_u32(smem);
+  ACtl& c = *reinterpret_cast<ACtl*>(smem + G::OFF_CTL);
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int pair = blockIdx.x % p.npair, bh = blockIdx.x / p.npair;
+  const int r0 = pair * 2 * TT;
+  const int ntc = p.Cpad / TCN;
+
+  if (tid == 0) {
+    tc::mbar_init(bar(c.x_full), 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(bar(c.c_full[b]), 1);
+      tc::mbar_init(bar(c.c_empty[b]), 2);
+      for (int g = 0; g < 2; ++g) {
+        tc::mbar_init(bar(c.s_full[g][b]), 1);
+        tc::mbar_init(bar(c.s_free[g][b]), TT);
+      }
+    }
+    tc::mbar_init(bar(c.done), 2);
+    c.abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 9) {
+    tc::tmem_alloc(smem_u32(&c.tmem_base), G::TCOLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = c.tmem_base;
+  tc::Waiter wt{&c.abort, p.err_flag, kWaitLimit};
+
+  if (warp < 8) {
+    // ============ rows: nearest centroids of one token of tile g ============
+    const int g = warp / 4, row = tid & (TT - 1);
+    const int r = r0 + g * TT + row;  // the token
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
+    // the head's ||c||^2 into shared memory once (the eight row warps, then their barrier)
+    float* cn = reinterpret_cast<float*>(smem + G::OFF_CN);
+    for (int m = tid; m < p.Cpad; m += 2 * TT) cn[m] = __ldg(p.cnorm + (size_t)bh * p.Cpad + m);
+    asm volatile("bar.sync 1, %0;\n" ::"r"(2 * TT) : "memory");
+    bool ok = uni(wt.wait(bar(c.x_full), 0, 1));
+    // ||x||^2 from the swizzled token tile (bf16 values, exact products in fp32)
+    float xn = 0.f;
+    if (ok) {
+      const uint8_t* xt = smem + G::OFF_X + g * G::XT;
+      for (int ch = 0; ch < D / 8; ++ch) {
+        const uint32_t off = (ch >> 3) * TT * 128 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        const uint4 w = *reinterpret_cast<const uint4*>(xt + off);
+        const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = bf16_lo(v[e]), b = bf16_hi(v[e]);
+          xn = fmaf(a, a, fmaf(b, b, xn));
+        }
+      }
+    }
+    float best = INFINITY, second = INFINITY, third = INFINITY, cmax2 = 0.f;
+    int bi = 0, si = 0;
+    for (int t = 0; t < ntc && ok; ++t) {
+      const int b = t & 1;
+      ok = uni(wt.wait(bar(c.s_full[g][b]), (t >> 1) & 1, 2));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t scol = tmem + lane_off + 256 * g + TCN * b;
+#pragma unroll 1
+      for (int h = 0; h < TCN / 64; ++h) {
+        uint32_t sr[64];
+        tc::tmem_ld32(scol + 64 * h, sr);
+        tc::tmem_ld32(scol + 64 * h + 32, sr + 32);
+        tc::tmem_wait_ld();
+        if (h == TCN / 64 - 1) {
+          tc::fence_before_sync();
+          tc::mbar_arrive(bar(c.s_free[g][b]));
+        }
+        const int m0 = t * TCN + 64 * h;
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          const float4 n4 = *reinterpret_cast<const float4*>(cn + m0 + e);
+          const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const float s = fmaf(-2.f, __uint_as_float(sr[e + f]), nv[f]);
+            if (nv[f] < INFINITY) cmax2 = fmaxf(cmax2, nv[f]);
+            // three best scores (and the two best indices), without branches
+            const int m = m0 + e + f;
+            const bool lt1 = s < best, lt2 = s < second, lt3 = s < third;
+            third = lt2 ? second : (lt3 ? s : third);
+            si = lt1 ? bi : (lt2 ? m : si);
+            second = lt1 ? best : (lt2 ? s : second);
+            bi = lt1 ? m : bi;
+            best = lt1 ? s : best;
+          }
+        }
+      }
+    }
+    if (ok && r < p.N) {
+      // Error bound of one fp32 score here: the pieces hold c to 2^-17 relative, the
+      // products accumulate in fp32 over 2d terms, ||c||^2 and the final fma round once:
+      // |err| <= 5e-5 |x| |c| + 1.2e-7 |c|^2. A token whose two best scores are closer
+      // than twice that (with 20% to spare) is decided in fp64 instead: only a centroid
+      // scored within that distance of the best can be the true nearest one.
+      const float xa = sqrtf(xn), ca = sqrtf(cmax2);
+      const float thr = 1.2e-4f * xa * ca + 3e-7f * cmax2;
+      p.labels[(size_t)bh * p.N + r] = bi;
+      if (!(second - best > thr)) {
+        // undecided: between the two best if the third is clear of them, else among all
+        const int k = atomicAdd(p.amb_cnt + bh, 1);
+        p.amb_list[(size_t)bh * p.N + k] = r;
+        p.amb_pair[(size_t)bh * p.N + k] = third - best > thr ? (bi | (si << 16)) : -1;
+      }
+    }
+  } else if (warp == 8) {
+    // ======================== TMA producer ========================
+    if (lane == 0) {
+      bool ok = true;
+      tc::mbar_arrive_expect_tx(bar(c.x_full), 2 * G::XT);
+      for (int g = 0; g < 2; ++g)
+        for (int x = 0; x < G::SUB; ++x)
+          tc::tma_load_3d(base + G::OFF_X + g * G::XT + x * TT * 128, &p.tmX, bar(c.x_full),
+                          64 * x, r0 + g * TT, bh);
+      uint32_t used = 0, par = 0;  // per stage: loaded, parity of the last load
+      for (int t = 0; t < ntc && ok; ++t) {
+        const int st = t & 1, ph = (t >> 1) & 1;
+        if (t >= 2) ok = wt.wait(bar(c.c_empty[st]), ph ^ 1, 3);
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(bar(c.c_full[st]), 2 * G::CT);
+        for (int pc = 0; pc < 2; ++pc)
+          for (int x = 0; x < G::SUB; ++x)
+            tc::tma_load_3d(base + G::OFF_C + (st * 2 + pc) * G::CT + x * TCN * 128, &p.tmC,
+                            bar(c.c_full[st]), 64 * x, t * TCN, 2 * bh + pc);
+        used |= 1u << st;
+        par = (par & ~(1u << st)) | ((uint32_t)ph << st);
+      }
+      tc::wait_drain(bar(c.x_full), 0, kWaitLimit);
+      for (int st = 0; st < 2; ++st)
+        if ((used >> st) & 1) tc::wait_drain(bar(c.c_full[st]), (par >> st) & 1, kWaitLimit);
+    }
+  } else if (warp == 9 || warp == 10) {
+    // ================ MMA issuers: warp 9 + g for token tile g ================
+    if (lane == 0) {
+      constexpr uint32_t I_S = tc::idesc_f16(1, 1, 0, TCN);
+      const int g = warp - 9;
+      bool ok = wt.wait(bar(c.x_full), 0, 4);
+      const uint64_t dx = tc::sdesc(base + G::OFF_X + g * G::XT, 16, 1024);
+      for (int t = 0; t < ntc && ok; ++t) {
+        const int b = t & 1, st = t & 1;
+        ok = wt.wait(bar(c.c_full[st]), (t >> 1) & 1, 5) &&
+             (t < 2 || wt.wait(bar(c.s_free[g][b]), ((t >> 1) - 1) & 1, 6));
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint64_t dc = tc::sdesc(base + G::OFF_C + st * 2 * G::CT, 16, 1024);
+        for (int pc = 0; pc < 2; ++pc) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t aoff = ((kk / 4) * TT * 128 + (kk % 4) * 32) >> 4;
+            const uint32_t boff = (pc * G::CT + (kk / 4) * TCN * 128 + (kk % 4) * 32) >> 4;
+            tc::mma_ss(tmem + 256 * g + TCN * b, dx + aoff, dc + boff, I_S, (pc | kk) > 0);
+          }
+        }
+        tc::mma_commit(bar(c.s_full[g][b]));
+        tc::mma_commit(bar(c.c_empty[st]));
+      }
+      tc::mma_commit(bar(c.done));
+      tc::wait_drain(bar(c.done), 0, kWaitLimit);
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 9) {
+    __syncwarp();
+    tc::tmem_dealloc(tmem, G::TCOLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// recheck: the undecided tokens in fp64, one warp per token
+// ---------------------------------------------------------------------------
+// dist_m = sum_i (x_i - c_mi)^2, lane l summing dimensions l, l+32, ... in order and the
+// lanes combined by a fixed butterfly; the smallest distance wins, ties to the lower
+// index. Only the candidates the assignment recorded are compared: its two best
+// centroids, or every centroid when a third one was as close.
+__device__ __forceinline__ double dist64(const double* xv, const double* cm, int d, int lane) {
+  double s = 0.0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (lane + 32 * k < d) {
+      const double t = xv[k] - cm[lane + 32 * k];
+      s = fma(t, t, s);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+__global__ void recheck_kernel(const uint16_t* __restrict__ x, const double* __restrict__ cent,
+                               int N, int d, int C, const int32_t* __restrict__ amb_list,
+                               const int32_t* __restrict__ amb_pair,
+                               const int32_t* __restrict__ amb_cnt, int32_t* __restrict__ labels) {
+  const int bh = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int nw = (int)(blockDim.x / 32);
+  const int cnt = amb_cnt[bh];
+  for (int e = blockIdx.x * nw + threadIdx.x / 32; e < cnt; e += gridDim.x * nw) {
+    const int r = amb_list[(size_t)bh * N + e];
+    const int pair = amb_pair[(size_t)bh * N + e];
+    const uint16_t* xr = x + ((size_t)bh * N + r) * d;
+    double xv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      xv[k] = lane + 32 * k < d ? (double)__uint_as_float((uint32_t)xr[lane + 32 * k] << 16) : 0.0;
+    const double* cb = cent + (size_t)bh * C * d;
+    int bi = 0;
+    if (pair >= 0) {
+      const int a = pair & 0xFFFF, b = pair >> 16;
+      const double da = dist64(xv, cb + (size_t)a * d, d, lane);
+      const double db = dist64(xv, cb + (size_t)b * d, d, lane);
+      bi = (db < da || (db == da && b < a)) ? b : a;
+    } else {
+      double best = INFINITY;
+      for (int m = 0; m < C; ++m) {
+        const double s = dist64(xv, cb + (size_t)m * d, d, lane);
+        if (s < best) {
+          best = s;
+          bi = m;
+        }
+      }
+    }
+    if (lane == 0) labels[(size_t)bh * N + r] = bi;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// stable counting sort of the labels
+// ---------------------------------------------------------------------------
+// counts[bh][chunk][m]: members of cluster m among the chunk's tokens.
+__global__ void hist_kernel(const int32_t* __restrict__ labels, int N, int C, int nchunk,
+                            int32_t* __restrict__ counts) {
+  extern __shared__ int32_t hsm[];  // [kSortWarps][C]
+  const int bh = blockIdx.y, w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kSortWarps + w;
+  int32_t* h = hsm + w * C;
+  for (int m = lane; m < C; m += 32) h[m] = 0;
+  __syncwarp();
+  if (chunk < nchunk) {
+    const int s = chunk * kChunk, e = min(N, s + kChunk);
+    for (int r = s + lane; r < e; r += 32) atomicAdd(h + labels[(size_t)bh * N + r], 1);
+  }
+  __syncwarp();
+  if (chunk < nchunk)
+    for (int m = lane; m < C; m += 32) counts[((size_t)bh * nchunk + chunk) * C + m] = h[m];
+}
+
+// offsets[m] = members of clusters < m; counts becomes the first position of each
+// (chunk, cluster) pair: offsets[m] + members of m in earlier chunks.
+__global__ void scan_kernel(int32_t* __restrict__ counts, int C, int nchunk,
+                            int32_t* __restrict__ offsets) {
+  extern __shared__ int32_t ssm[];  // [C] totals
+  const int bh = blockIdx.x;
+  int32_t* cnt = counts + (size_t)bh * nchunk * C;
+  for (int m = threadIdx.x; m < C; m += blockDim.x) {
+    int run = 0;
+    for (int k = 0; k < nchunk; ++k) {
+      const int v = cnt[(size_t)k * C + m];
+      cnt[(size_t)k * C + m] = run;
+      run += v;
+    }
+    ssm[m] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int m = 0; m < C; ++m) {
+      const int v = ssm[m];
+      ssm[m] = acc;
+      acc += v;
+    }
+    offsets[(size_t)bh * (C + 1) + C] = acc;
+  }
+  __syncthreads();
+  for (int m = threadIdx.x; m < C; m += blockDim.x) {
+    const int o = ssm[m];
+    offsets[(size_t)bh * (C + 1) + m] = o;
+    for (int k = 0; k < nchunk; ++k) cnt[(size_t)k * C + m] += o;
+  }
+}
+
+// Each warp walks its chunk 32 tokens at a time, in token order: lanes holding the same
+// label take consecutive positions in lane order after that label's cursor.
+__global__ void scatter_kernel(const int32_t* __restrict__ labels, int N, int C, int nchunk,
+                               const int32_t* __restrict__ starts, int32_t* __restrict__ perm) {
+  extern __shared__ int32_t csm[];  // [kSortWarps][C] cursors
+  const int bh = blockIdx.y, w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kSortWarps + w;
+  if (chunk >= nchunk) return;
+  int32_t* cur = csm + w * C;
+  for (int m = lane; m < C; m += 32) cur[m] = starts[((size_t)bh * nchunk + chunk) * C + m];
+  __syncwarp();
+  const int s = chunk * kChunk, e = min(N, s + kChunk);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r0 = s; r0 < e; r0 += 32) {
+    const int r = r0 + lane;
+    const bool valid = r < e;
+    const unsigned act = __ballot_sync(0xffffffffu, valid);
+    const int lab = valid ? labels[(size_t)bh * N + r] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, lab) & act;
+    int base = 0;
+    if (valid) base = cur[lab];  // every peer reads the cursor before the leader moves it
+    __syncwarp();
+    if (valid) {
+      perm[(size_t)bh * N + base + __popc(peers & lt)] = r;
+      if ((peers & lt) == 0) cur[lab] = base + __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// update: each centroid to the fp64 mean of its members; one without members stays
+// ---------------------------------------------------------------------------
+// 512 threads: d / 8 threads per row (eight dimensions each, one 16-byte load), so
+// 512 / (d / 8) member rows are read side by side; member k goes to row lane k mod L.
+// Every sum of bf16 values here is exact in fp64, so the split changes nothing; the
+// lanes are still combined in a fixed order.
+constexpr int kUpdThreads = 512;
+
+__global__ void __launch_bounds__(kUpdThreads)
+update_kernel(const uint16_t* __restrict__ x, int N, int d, int C,
+              const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
+              double* __restrict__ cent) {
+  __shared__ double part[kUpdThreads * 8];  // [row lane][d]
+  const int m = blockIdx.x, bh = blockIdx.y;
+  const int cpr = d / 8, lanes = kUpdThreads / cpr;
+  const int rl = threadIdx.x / cpr, ch = threadIdx.x % cpr;
+  const int s = offsets[(size_t)bh * (C + 1) + m], e = offsets[(size_t)bh * (C + 1) + m + 1];
+  if (e == s) return;  // no members: the centroid stays
+  const int32_t* pr = perm + (size_t)bh * N;
+  const uint16_t* xb = x + (size_t)bh * N * d + ch * 8;
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int k = s + rl; k < e; k += lanes) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(xb + (size_t)__ldg(pr + k) * d));
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] += (double)bf16_lo(v[q]);
+      acc[2 * q + 1] += (double)bf16_hi(v[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) part[rl * d + ch * 8 + q] = acc[q];
+  __syncthreads();
+  if (threadIdx.x < d) {
+    double sum = 0.0;
+    for (int l = 0; l < lanes; ++l) sum += part[l * d + threadIdx.x];
+    cent[((size_t)bh * C + m) * d + threadIdx.x] = sum / (double)(e - s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// row permutations
+// ---------------------------------------------------------------------------
+// dst[p] = src[perm[p]] (gather) or dst[perm[p]] = src[p] (scatter), rows of row_bytes
+// (a multiple of 16), 16 bytes per thread step.
+template <bool GATHER>
+__global__ void permute_kernel(const uint8_t* __restrict__ src, const int32_t* __restrict__ perm,
+                               int N, int row_bytes, long long total_vec, uint8_t* __restrict__ dst) {
+  const int vpr = row_bytes / 16;
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < total_vec;
+       v += (long long)gridDim.x * blockDim.x) {
+    const long long row = v / vpr;
+    const int col = (int)(v % vpr);
+    const long long other = (row / N) * N + perm[row];
+    const long long from = GATHER ? other : row, to = GATHER ? row : other;
+    reinterpret_cast<uint4*>(dst + to * row_bytes)[col] =
+        reinterpret_cast<const uint4*>(src + from * row_bytes)[col];
+  }
+}
+
+}  // namespace km
+
+namespace {
+
+size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+template <int D>
+cudaError_t assign_t(const KmeansArgs& a, int Cpad, cudaStream_t st) {
+  using G = km::AGeom<D>;
+  km::AParams p;
+  const uint64_t bh = (uint64_t)a.B * a.H;
+  if (!map3d(&p.tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, D, a.N, bh, km::TT) ||
+      !map3d(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.pieces, D, Cpad, 2 * bh, km::TCN))
+    return cudaErrorInvalidValue;
+  p.cnorm = a.cnorm;
+  p.labels = a.labels;
+  p.amb_list = a.amb_list;
+  p.amb_pair = a.amb_pair;
+  p.amb_cnt = a.amb_cnt;
+  p.err_flag = a.err_flag;
+  p.N = a.N;
+  p.Cpad = Cpad;
+  p.npair = km::cdiv(a.N, 2 * km::TT);
+  auto kern = km::assign_kernel<D>;
+  const int smem = G::smem(Cpad);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(p.npair * bh), 352, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
+  const size_t bh = (size_t)B * H;
+  const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
+  sizes[0] = bh * C * d * sizeof(double);
+  sizes[1] = align256(bh * 2 * Cpad * d * 2) + bh * Cpad * 4;
+  sizes[2] = align256(bh * nchunk * C * 4) + 2 * align256(bh * N * 4) + bh * 4;
+}
+
+cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
+  KmeansArgs a = in;
+  const int bh = a.B * a.H, C = a.C, d = a.d, N = a.N;
+  const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
+  // carve the work buffers
+  a.pieces = reinterpret_cast<uint16_t*>(a.cwork);
+  a.cnorm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.cwork) +
+                                     align256((size_t)bh * 2 * Cpad * d * 2));
+  uint8_t* iw = reinterpret_cast<uint8_t*>(a.iwork);
+  a.counts = reinterpret_cast<int32_t*>(iw);
+  iw += align256((size_t)bh * nchunk * C * 4);
+  a.amb_list = reinterpret_cast<int32_t*>(iw);
+  iw += align256((size_t)bh * N * 4);
+  a.amb_pair = reinterpret_cast<int32_t*>(iw);
+  iw += align256((size_t)bh * N * 4);
+  a.amb_cnt = reinterpret_cast<int32_t*>(iw);
+
+  const int sort_smem = km::kSortWarps * C * 4;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(km::hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                sort_smem)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(km::scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                sort_smem)) != cudaSuccess)
+    return e;
+  const dim3 gsort(km::cdiv(nchunk, km::kSortWarps), bh);
+  auto assign = [&]() -> cudaError_t {
+    cudaError_t r = d == 64 ? assign_t<64>(a, Cpad, st) : assign_t<128>(a, Cpad, st);
+    if (r != cudaSuccess) return r;
+    km::recheck_kernel<<<dim3(32, bh), 256, 0, st>>>(a.x, a.cent, N, d, C, a.amb_list,
+                                                     a.amb_pair, a.amb_cnt, a.labels);
+    return cudaGetLastError();
+  };
+  auto sort = [&]() -> cudaError_t {
+    km::hist_kernel<<<gsort, 32 * km::kSortWarps, sort_smem, st>>>(a.labels, N, C, nchunk,
+                                                                   a.counts);
+    km::scan_kernel<<<bh, 256, C * 4, st>>>(a.counts, C, nchunk, a.offsets);
+    km::scatter_kernel<<<gsort, 32 * km::kSortWarps, sort_smem, st>>>(a.labels, N, C, nchunk,
+                                                                      a.counts, a.perm);
+    return cudaGetLastError();
+  };
+  auto prep = [&]() -> cudaError_t {
+    km::prep_kernel<<<dim3(Cpad, bh), 64, 0, st>>>(a.cent, C, Cpad, d, a.pieces, a.cnorm,
+                                                  a.amb_cnt);
+    return cudaGetLastError();
+  };
+  km::init_kernel<<<dim3(C, bh), 64, 0, st>>>(a.x, N, d, C, a.cent);
+  if ((e = prep()) != cudaSuccess) return e;
+  for (int t = 0; t < a.iters; ++t) {
+    if ((e = assign()) != cudaSuccess) return e;
+    if ((e = sort()) != cudaSuccess) return e;
+    km::update_kernel<<<dim3(C, bh), km::kUpdThreads, 0, st>>>(a.x, N, d, C, a.perm, a.offsets,
+                                                                a.cent);
+    if ((e = prep()) != cudaSuccess) return e;
+  }
+  if ((e = assign()) != cudaSuccess) return e;
+  return sort();
+}
+
+cudaError_t launch_permute_rows(const PermuteArgs& a, cudaStream_t st) {
+  const long long rows = (long long)a.B * a.H * a.N;
+  const long long total = rows * (a.row_bytes / 16);
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const long long want = (total + threads - 1) / threads;
+  const unsigned blocks = (unsigned)(want < 148LL * 64 ? want : 148LL * 64);
+  if (a.gather)
+    km::permute_kernel<true><<<blocks, threads, 0, st>>>(
+        reinterpret_cast<const uint8_t*>(a.src), a.perm, a.N, a.row_bytes, total,
+        reinterpret_cast<uint8_t*>(a.dst));
+  else
+    km::permute_kernel<false><<<blocks, threads, 0, st>>>(
+        reinterpret_cast<const uint8_t*>(a.src), a.perm, a.N, a.row_bytes, total,
+        reinterpret_cast<uint8_t*>(a.dst));
+  return cudaGetLastError();
+}
+
+}  // namespace sa

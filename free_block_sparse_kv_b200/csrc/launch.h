@@ -59,6 +59,31 @@ struct ForwardArgs {
   int32_t* err_flag;
 };
 
+struct KmeansArgs {
+  const uint16_t* x;
+  int B, H, N, d, C, iters;
+  double* cent;
+  void* cwork;
+  int32_t* iwork;
+  int32_t *labels, *perm, *offsets;
+  int32_t* err_flag;
+  // carved from cwork / iwork by the launcher
+  uint16_t* pieces = nullptr;
+  float* cnorm = nullptr;
+  int32_t *counts = nullptr, *amb_list = nullptr, *amb_pair = nullptr, *amb_cnt = nullptr;
+};
+
+struct PermuteArgs {
+  const void* src;
+  const int32_t* perm;
+  int B, H, N, row_bytes;
+  bool gather;
+  void* dst;
+};
+
+void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]);
+cudaError_t launch_kmeans(const KmeansArgs& p, cudaStream_t st);
+cudaError_t launch_permute_rows(const PermuteArgs& p, cudaStream_t st);
 cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);

@@ -21,7 +21,8 @@ SA_OUT_F32, SA_OUT_BF16 = 0, 1
 EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
            "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
            "sparse_attn_structured_mask_adaptive", "sparse_attn_ear_scores",
-           "sparse_attn_route_scores", "sparse_attn_forward", "sparse_attn_last_error")
+           "sparse_attn_route_scores", "sparse_attn_kmeans_sizes", "sparse_attn_kmeans",
+           "sparse_attn_permute_rows", "sparse_attn_forward", "sparse_attn_last_error")
 
 
 class SparseAttnError(RuntimeError):
@@ -53,6 +54,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
     lib.sparse_attn_ear_scores.argtypes = [_P, _P, _P] + [_I] * 6 + [_F, _P, _P, _P]
     lib.sparse_attn_route_scores.argtypes = [_P] + [_I] * 6 + [_P, _P, _I, _P]
+    lib.sparse_attn_kmeans_sizes.argtypes = [_I] * 5 + [ctypes.POINTER(ctypes.c_size_t)]
+    lib.sparse_attn_kmeans.argtypes = [_P] + [_I] * 6 + [_P] * 7 + [_P]
+    lib.sparse_attn_permute_rows.argtypes = [_P, _P] + [_I] * 5 + [_P, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_structured_mask_adaptive.argtypes = [_I] * 13 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
@@ -129,6 +133,25 @@ def sparse_attn_route_scores(scores, B, H, nqb, nkb, rho_num, rho_den, kv_idx, k
     _check(load_library().sparse_attn_route_scores(
         _ptr(scores), B, H, nqb, nkb, rho_num, rho_den, _ptr(kv_idx), _ptr(kv_cnt), cap,
         _stream(stream)))
+
+
+def sparse_attn_kmeans_sizes(B, H, N, d, C):
+    """Byte sizes (centroids, cwork, iwork) of sparse_attn_kmeans's buffers."""
+    out = (ctypes.c_size_t * 3)()
+    _check(load_library().sparse_attn_kmeans_sizes(B, H, N, d, C, out))
+    return tuple(int(x) for x in out)
+
+
+def sparse_attn_kmeans(x, B, H, N, d, C, iters, centroids, cwork, iwork, labels, perm, offsets,
+                       err_flag=None, stream=None):
+    _check(load_library().sparse_attn_kmeans(
+        _ptr(x), B, H, N, d, C, iters, _ptr(centroids), _ptr(cwork), _ptr(iwork), _ptr(labels),
+        _ptr(perm), _ptr(offsets), _ptr(err_flag), _stream(stream)))
+
+
+def sparse_attn_permute_rows(src, perm, B, H, N, row_bytes, gather, dst, stream=None):
+    _check(load_library().sparse_attn_permute_rows(
+        _ptr(src), _ptr(perm), B, H, N, row_bytes, int(gather), _ptr(dst), _stream(stream)))
 
 
 def sparse_attn_structured_mask(B, H, Nq, Nk, block, frame_tokens, n_frames, window, n_anchors,

@@ -60,6 +60,7 @@ class Workload:
     n_anchors: int = 4
     period: int = 10
     budget: int = 0                 # > 0: adaptive windows reaching |A(t)| = budget frames
+    clusters: tuple = ()            # (C_q, C_k, iters): k-means group-major layout first
     steps: tuple = (0,)
     seed: int = 0
 
@@ -120,6 +121,13 @@ WORKLOADS = {
     "dit720p-ear-21x45x80": Workload(
         name="dit720p-ear-21x45x80", B=1, H=40, Nq=75600, Nk=75600, d=128, block=128, order=0,
         mode="ear", rho=(1, 10), recipe="patches", grid=(21, 45, 80), outlier_p=0.05),
+    # The 720p call on the cluster-permuted layout: Q and K grouped by k-means into 296
+    # clusters each (about two blocks per cluster), three Lloyd updates, then blocks cut
+    # from the group-major order.
+    "dit720p-kmeans-21x45x80": Workload(
+        name="dit720p-kmeans-21x45x80", B=1, H=40, Nq=75600, Nk=75600, d=128, block=128,
+        order=1, mode="topk", rho=(1, 10), recipe="patches", grid=(21, 45, 80), outlier_p=0.05,
+        clusters=(296, 296, 3)),
     # Long video with a local window and rotating anchor frames (denoising steps 0..9).
     "longvideo-41x30x52": Workload(
         name="longvideo-41x30x52", B=1, H=12, Nq=63960, Nk=63960, d=128, block=128, order=0,

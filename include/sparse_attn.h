@@ -58,6 +58,7 @@ enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
 
 /* Largest number of KV blocks per head that routing and the forward accept. */
 #define SA_MAX_KV_BLOCKS 2048
+#define SA_MAX_CLUSTERS 4096
 
 /*
  * Byte sizes of the pooled tables for a problem, written to sizes[0..6] in the
@@ -179,6 +180,47 @@ int sparse_attn_ear_scores(const float* qbar, const uint16_t* k, const uint16_t*
 int sparse_attn_route_scores(const float* scores, int B, int H, int nqb, int nkb,
                              int rho_num, int rho_den, int32_t* kv_idx, int32_t* kv_cnt,
                              int cap, void* stream);
+
+/*
+ * Cluster-permuted token layout (SVG-EAR §2 A: query and key tokens grouped into
+ * semantic clusters by k-means; "Partition the Support, Reconstruct the Residual"
+ * (SparsePR) §2 C: tokens permuted into contiguous group-major layouts before the
+ * block-sparse attention).
+ *
+ * sparse_attn_kmeans_sizes: byte sizes of the buffers sparse_attn_kmeans needs:
+ *   sizes[0] centroids (fp64), sizes[1] cwork, sizes[2] iwork.
+ *
+ * sparse_attn_kmeans: Lloyd's k-means on the rows of x per (b, h), then the stable
+ * group-major order of the final labels.
+ *   x          [B,H,N,d] bf16 (Q or K as given), 16-byte aligned
+ *   C          clusters, 1 <= C <= min(N, SA_MAX_CLUSTERS); iters update steps, 0..1000
+ *   centroids  [B,H,C,d] fp64, out: the final centroids
+ *   cwork, iwork  scratch of sizes[1] and sizes[2] bytes (16-byte aligned), contents
+ *              undefined on return
+ *   labels     [B,H,N] int32, out: cluster of every token after the final assignment
+ *   perm       [B,H,N] int32, out: perm[p] = original index of the token at position p
+ *              (tokens by cluster, then by original index)
+ *   offsets    [B,H,C+1] int32, out: positions offsets[m] .. offsets[m+1]-1 hold cluster m
+ *   err_flag   optional int32: nonzero after a launch whose waits gave up
+ * Iteration: every centroid starts at token floor(m N / C); each token goes to its
+ * nearest centroid (squared Euclidean distance, ties to the lowest index), each centroid
+ * with members moves to their mean (fp64; the others stay); after `iters` updates the
+ * tokens are assigned once more. The assignment runs on the tensor cores (fp32 scores
+ * from a two-piece bf16 split of the fp64 centroids); a token whose two best scores lie
+ * within that arithmetic's error bound is decided again in fp64. 7 + 7 * iters
+ * launches on the stream.
+ *
+ * sparse_attn_permute_rows: rows of row_bytes bytes (a multiple of 16) per (b, h);
+ *   gather = 1: dst[p] = src[perm[p]] (into the clustered order);
+ *   gather = 0: dst[perm[p]] = src[p] (back to the original order).
+ * src and dst must not overlap. One launch.
+ */
+int sparse_attn_kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]);
+int sparse_attn_kmeans(const uint16_t* x, int B, int H, int N, int d, int C, int iters,
+                       double* centroids, void* cwork, int32_t* iwork, int32_t* labels,
+                       int32_t* perm, int32_t* offsets, int32_t* err_flag, void* stream);
+int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H, int N,
+                             int row_bytes, int gather, void* dst, void* stream);
 
 /*
  * Structured mask (LVSA §2 Mécanisme Central). Tokens are frame-major with

@@ -35,6 +35,8 @@ SMALL = {
                              Nq=9480, Nk=9480, grid=(6, 20, 79)),
     "ear-small": W.shrink(W.WORKLOADS["dit720p-ear-21x45x80"], name="ear-small", H=2, Nq=9480,
                           Nk=9480, grid=(6, 20, 79)),
+    "kmeans-small": W.shrink(W.WORKLOADS["dit720p-kmeans-21x45x80"], name="kmeans-small", H=2,
+                             Nq=9480, Nk=9480, grid=(6, 20, 79), clusters=(38, 38, 3)),
 }
 
 # Error-aware scores (ln of the error per token). The GPU takes the logits with a 16-bit
@@ -68,6 +70,22 @@ def oracle_kept(w: W.Workload, q, k, step: int = 0, v=None):
     kept, s, counts = O.route_head(q, k, w.block, "mass", w.scale, tau=w.tau)
     gaps, lo, hi = O.gate_diagnostics(s, counts, tau=w.tau)
     return kept, (gaps > GATE) & (lo > GATE) & (hi > GATE)
+
+
+def oracle_layout(w: W.Workload, q, k, v):
+    """The oracle's token layout of one head: (q', k', v', position of every original
+    query row). Without clustering the layout is the given one."""
+    if not w.clusters:
+        return q, k, v, np.arange(q.shape[0])
+    from oracle import cluster_layout as K
+    cq, ck, iters = w.clusters
+    lq, _ = K.kmeans(q, cq, iters)
+    lk, _ = K.kmeans(k, ck, iters)
+    pq, _ = K.group_major_permutation(lq, cq)
+    pk, _ = K.group_major_permutation(lk, ck)
+    pos = np.empty_like(pq)
+    pos[pq] = np.arange(pq.shape[0])
+    return K.permute_rows(q, pq), K.permute_rows(k, pk), K.permute_rows(v, pk), pos
 
 
 def lists_to_sets(kv_idx: np.ndarray, kv_cnt: np.ndarray):

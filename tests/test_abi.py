@@ -42,6 +42,10 @@ def test_table_sizes():
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[5] == 0
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 2)[5] == 4 * 16 * 1000 * 128 * 128 * 2
     assert C.sparse_attn_table_sizes(4, 16, 1560, 63960, 128, 64, 0)[0] == 4 * 16 * 25 * 128 * 4
+    cent, cw, iw = C.sparse_attn_kmeans_sizes(1, 40, 75600, 128, 296)
+    assert cent == 40 * 296 * 128 * 8
+    assert cw >= 40 * 2 * 384 * 128 * 2 + 40 * 384 * 4      # padded bf16 pieces, norms
+    assert iw >= 40 * 74 * 296 * 4 + 2 * 40 * 75600 * 4 + 40 * 4
 
 
 def test_host_argument_checks(lib):
@@ -81,6 +85,16 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 10, 5, 4, p, p, 10, 0),
         lambda: C.sparse_attn_route_scores(None, 1, 1, 4, 10, 1, 4, p, p, 10, 0),
         lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 0, 1, 4, p, p, 10, 0),
+        lambda: C.sparse_attn_kmeans_sizes(1, 1, 64, 96, 4),
+        lambda: C.sparse_attn_kmeans_sizes(1, 1, 64, 64, 0),
+        lambda: C.sparse_attn_kmeans_sizes(1, 1, 64, 64, 5000),
+        lambda: C.sparse_attn_kmeans(p, 1, 1, 64, 64, 65, 2, p, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_kmeans(p, 1, 1, 64, 64, 4, -1, p, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_kmeans(p + 8, 1, 1, 64, 64, 4, 2, p, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_kmeans(p, 1, 1, 64, 64, 4, 2, p, None, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_permute_rows(p, p, 1, 1, 64, 100, 1, p + 16, 0),
+        lambda: C.sparse_attn_permute_rows(p, p, 1, 1, 64, 128, 2, p + 16, 0),
+        lambda: C.sparse_attn_permute_rows(p, p, 1, 1, 64, 128, 1, p, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 6400, 64, 10, 10, 1, 1, 1, 0, 0, p, p, 100, 0),
         lambda: C.sparse_attn_structured_mask(1, 1, 64, 64, 64, 8, 8, 1, 1, 0, 0, 0, p, p, 1, 0),
         lambda: C.sparse_attn_structured_mask_adaptive(1, 1, 64, 64, 64, 8, 8, 1, 1, 2, 0, 0, -1, p,

@@ -12,7 +12,7 @@ from free_block_sparse_kv_b200 import sparse_attn as C
 from free_block_sparse_kv_b200 import workloads as W
 from oracle import block_sparse_attention as O
 from tests.helpers import (EAR_TOL, EAR_X_FLOOR, GATE, MAX_ABS, MEAN_REL, SMALL, err_stats,
-                           lists_to_sets, oracle_kept, sample_rows)
+                           lists_to_sets, oracle_kept, oracle_layout, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,7 @@ def _geometry(w):
 def _run(w, q, k, v, step=0, out_dtype=torch.float32):
     op = A.BlockSparseAttention(_problem(w), w.mode, rho=w.rho, tau=w.tau,
                                 geometry=_geometry(w) if w.mode == "structured" else None,
-                                out_dtype=out_dtype)
+                                out_dtype=out_dtype, clusters=w.clusters or None)
     out = op(q, k, v, step=step)
     torch.cuda.synchronize()
     op.check()
@@ -120,8 +120,8 @@ def test_route_masks_bit_exact_above_gate(name, small_inputs):
     pinned = total = 0
     for b in range(w.B):
         for h in range(w.H):
-            q, k = W.bits_to_f32(qb[b, h]), W.bits_to_f32(kb[b, h])
-            kept, gate = oracle_kept(w, q, k, v=W.bits_to_f32(vb[b, h]))
+            q, k, v, _ = oracle_layout(w, *(W.bits_to_f32(x[b, h]) for x in (qb, kb, vb)))
+            kept, gate = oracle_kept(w, q, k, v=v)
             got = lists_to_sets(idx[b, h], cnt[b, h])
             for i in range(w.nqb):
                 total += 1
@@ -232,6 +232,77 @@ def test_route_scores_selects_like_the_oracle_on_given_scores():
             assert got == [x.tolist() for x in want], (rho, h)
 
 
+# --- k-means and the group-major layout ---------------------------------------------
+
+def _kmeans_check(xb, C, iters, B, H):
+    """GPU k-means of bf16 rows xb [B,H,N,d] against the oracle, bit for bit."""
+    from oracle import cluster_layout as K
+    N, d = xb.shape[2], xb.shape[3]
+    cl = A.allocate_clustering(B, H, N, d, C, iters, "cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = _dev(xb)
+    A.kmeans(x, cl, err_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    for b in range(B):
+        for h in range(H):
+            xf = W.bits_to_f32(xb[b, h])
+            lab, cen = K.kmeans(xf, C, iters)
+            perm, offs = K.group_major_permutation(lab, C)
+            assert np.array_equal(cl.labels[b, h].cpu().numpy(), lab), (b, h)
+            assert np.array_equal(cl.perm[b, h].cpu().numpy(), perm), (b, h)
+            assert np.array_equal(cl.offsets[b, h].cpu().numpy(), offs), (b, h)
+            assert np.array_equal(cl.centroids[b, h].cpu().numpy(), cen), (b, h)
+    return cl, x
+
+
+@pytest.mark.parametrize("d,N,C,iters", [(64, 700, 5, 0), (64, 3000, 130, 2), (128, 4097, 300, 3),
+                                         (128, 1000, 1, 2), (128, 129, 129, 1)])
+def test_kmeans_matches_oracle(d, N, C, iters):
+    """Several token tiles (the last partial), several centroid tiles (the last partial),
+    one cluster, as many clusters as tokens."""
+    _kmeans_check(_rand_bits((1, 2, N, d), 40 + d + N), C, iters, 1, 2)
+
+
+def test_kmeans_ties_and_empty_clusters():
+    """Duplicated tokens: the initial centroids coincide, ties go to the lower index and
+    the higher one is left empty and keeps its position."""
+    rng = np.random.default_rng(41)
+    base = rng.standard_normal((25, 64)).astype(np.float32)
+    xb = W.bf16_round(np.repeat(base, 8, axis=0))[1][None, None]
+    cl, _ = _kmeans_check(xb, 50, 2, 1, 1)
+    offs = cl.offsets[0, 0].cpu().numpy()
+    assert (np.diff(offs) == 0).any()
+
+
+def test_kmeans_on_the_workload(small_inputs):
+    w, qb, kb, _ = small_inputs("kmeans-small")
+    cq, ck, iters = w.clusters
+    _kmeans_check(qb, cq, iters, w.B, w.H)
+    _kmeans_check(kb, ck, iters, w.B, w.H)
+
+
+def test_permute_rows_round_trip():
+    B, H, N, d = 1, 3, 777, 128
+    xb = _rand_bits((B, H, N, d), 42)
+    x = _dev(xb)
+    rng = np.random.default_rng(43)
+    perm = torch.from_numpy(np.stack([rng.permutation(N) for _ in range(B * H)]).reshape(B, H, N)
+                            .astype(np.int32)).cuda()
+    y = torch.empty_like(x)
+    z = torch.empty_like(x)
+    A.permute_rows(x, perm, y, gather=True)
+    A.permute_rows(y, perm, z, gather=False)
+    f = torch.randn(B, H, N, d, device="cuda")
+    g, f2 = torch.empty_like(f), torch.empty_like(f)
+    A.permute_rows(f, perm, g, gather=True)
+    A.permute_rows(g, perm, f2, gather=False)
+    torch.cuda.synchronize()
+    pn = perm.cpu().numpy()
+    assert torch.equal(z, x) and torch.equal(f2, f)
+    assert np.array_equal(y.view(torch.int16).cpu().numpy()[0, 1], xb.view(np.int16)[0, 1][pn[0, 1]])
+
+
 # --- forward ------------------------------------------------------------------
 
 def _oracle_lists_to_device(w, kept_per_head, cap):
@@ -292,9 +363,10 @@ def test_pipeline_matches_oracle(name, small_inputs):
         got_all, want_all = [], []
         for b in range(w.B):
             for h in range(w.H):
-                q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+                q, k, v, pos = oracle_layout(w, *(W.bits_to_f32(x[b, h]) for x in (qb, kb, vb)))
                 kept, _ = oracle_kept(w, q, k, step, v=v)
-                want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=rows))
+                want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale,
+                                               rows=pos[rows]))
                 got_all.append(out[b, h, rows].cpu().numpy())
         mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
         assert mx <= MAX_ABS and mr <= MEAN_REL, (name, step, mx, mr)
@@ -314,7 +386,7 @@ def test_full_size_sampled(name):
     got_all, want_all = [], []
     pinned = total = 0
     for b, h in heads:
-        q, k, v = (W.bits_to_f32(x[b, h]) for x in (qb, kb, vb))
+        q, k, v, pos = oracle_layout(w, *(W.bits_to_f32(x[b, h]) for x in (qb, kb, vb)))
         if w.mode == "ear":
             _ear_check(op.tables.scores[b, h].cpu().numpy(), q, k, v, w.block, w.scale)
         kept, gate = oracle_kept(w, q, k, step, v=v)
@@ -324,7 +396,7 @@ def test_full_size_sampled(name):
             if gate[i]:
                 pinned += 1
                 assert got[i] == kept[i].tolist(), (name, b, h, i)
-        want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=rows))
+        want_all.append(O.forward_head(q, k, v, kept, w.block, w.order, w.scale, rows=pos[rows]))
         got_all.append(out[b, h, rows].cpu().numpy())
     assert pinned >= 0.5 * total, (pinned, total)
     mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
