@@ -304,6 +304,31 @@ int sparse_attn_kmeans(const uint16_t* x, int B, int H, int N, int d, int C, int
   return launched(sa::launch_kmeans(p, static_cast<cudaStream_t>(stream)), "kmeans launch");
 }
 
+int sparse_attn_kmeans_noalloc(const uint16_t* x, int B, int H, int N, int d, int C, int iters,
+                               double* centroids, int32_t* labels, int32_t* perm,
+                               int32_t* offsets, int32_t* err_flag, void* stream) {
+  SA_REQUIRE(B >= 0 && H >= 0 && N >= 0, "B, H, N must be >= 0");
+  SA_REQUIRE(d == 64 || d == 128, "d must be 64 or 128 (got %d)", d);
+  SA_REQUIRE(C >= 1 && C <= SA_MAX_CLUSTERS, "C must be in [1, %d] (got %d)", SA_MAX_CLUSTERS, C);
+  size_t sizes[3];
+  sa::kmeans_sizes(B, H, N, d, C, sizes);
+  const size_t cw = (sizes[1] + 255) & ~(size_t)255;
+  SA_REQUIRE(cw + sizes[2] <= sa::kKmeansScratchBytes,
+             "problem needs %zu scratch bytes; the built-in buffer holds %zu (use sparse_attn_kmeans)",
+             cw + sizes[2], sa::kKmeansScratchBytes);
+  if ((long long)B * H == 0 || N == 0) return sparse_attn_kmeans(x, B, H, N, d, C, iters, centroids,
+                                                                 nullptr, nullptr, labels, perm,
+                                                                 offsets, err_flag, stream);
+  if (int rc = check_device()) return rc;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  uint8_t* scratch = static_cast<uint8_t*>(sa::kmeans_scratch(dev));
+  if (!scratch) return fail(SA_ERR_LAUNCH, "no address for the built-in scratch buffer on device %d", dev);
+  return sparse_attn_kmeans(x, B, H, N, d, C, iters, centroids, scratch,
+                            reinterpret_cast<int32_t*>(scratch + cw), labels, perm, offsets,
+                            err_flag, stream);
+}
+
 int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H, int N,
                              int row_bytes, int gather, void* dst, void* stream) {
   SA_REQUIRE(B >= 0 && H >= 0 && N >= 0, "B, H, N must be >= 0");

@@ -558,6 +558,21 @@ cudaError_t assign_t(const KmeansArgs& a, int Cpad, cudaStream_t st) {
 
 }  // namespace
 
+// Scratch for sparse_attn_kmeans_noalloc: one fixed buffer per device, part of the
+// module's global memory (no allocation at call time).
+static __device__ __align__(256) uint8_t g_kmeans_scratch[kKmeansScratchBytes];
+
+void* kmeans_scratch(int device) {
+  static void* addr[64] = {};
+  if (device < 0 || device >= 64) return nullptr;
+  if (!addr[device]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_kmeans_scratch) != cudaSuccess) return nullptr;
+    addr[device] = a;
+  }
+  return addr[device];
+}
+
 void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
   const size_t bh = (size_t)B * H;
   const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);

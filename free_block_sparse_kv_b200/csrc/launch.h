@@ -82,6 +82,8 @@ struct PermuteArgs {
 };
 
 void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]);
+constexpr size_t kKmeansScratchBytes = (size_t)32 << 20;  // per device, for the no-alloc call
+void* kmeans_scratch(int device);  // device address of that buffer on `device`
 cudaError_t launch_kmeans(const KmeansArgs& p, cudaStream_t st);
 cudaError_t launch_permute_rows(const PermuteArgs& p, cudaStream_t st);
 cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);

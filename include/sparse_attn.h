@@ -223,6 +223,20 @@ int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H,
                              int row_bytes, int gather, void* dst, void* stream);
 
 /*
+ * sparse_attn_kmeans_noalloc: sparse_attn_kmeans without caller scratch. The pages have
+ * no counterpart for this call; it is an interface convenience for callers that cannot
+ * allocate device memory. cwork and iwork come from one built-in 32 MiB buffer per
+ * device (module global memory, obtained with cudaGetSymbolAddress); problems whose
+ * sizes[1] (rounded up to 256 bytes) + sizes[2] exceed it return SA_ERR_INVALID before
+ * anything is enqueued. The buffer is shared by every call on the device: calls must be
+ * ordered (one stream, or synchronised), never concurrent. Results equal
+ * sparse_attn_kmeans's bit for bit.
+ */
+int sparse_attn_kmeans_noalloc(const uint16_t* x, int B, int H, int N, int d, int C, int iters,
+                               double* centroids, int32_t* labels, int32_t* perm,
+                               int32_t* offsets, int32_t* err_flag, void* stream);
+
+/*
  * Structured mask (LVSA §2 Mécanisme Central). Tokens are frame-major with
  * frame_tokens tokens per frame; query token t lies in frame
  * q_frame0 + t / frame_tokens and key token r in frame r / frame_tokens.
