@@ -17,12 +17,14 @@
 //            S = X C_hi^T + X C_lo^T (the fp64 centroids as two bf16 pieces), score
 //            ||c||^2 - 2 S in fp32; a token whose two best scores lie closer than the
 //            error bound of that arithmetic goes on a list instead of being decided;
-//   recheck  the listed tokens in fp64 against every centroid (one warp each);
+//   recheck  the listed tokens in fp64 against every centroid (one CTA each);
 //   hist / scan / scatter   stable counting sort: one warp per chunk of 1024 tokens;
 //   update   one CTA per cluster sums its members in fp64 (the sums of bf16 values are
 //            exact, so the means are the correctly rounded fp64 means) and writes the
 //            bf16 pieces and the fp32 squared norm the next assignment reads.
 #include <cudaTypedefs.h>
+
+#include <cmath>
 
 #include "common.cuh"
 #include "launch.h"
@@ -94,13 +96,16 @@ __global__ void prep_kernel(const double* __restrict__ cent, int C, int Cpad, in
 // ---------------------------------------------------------------------------
 // assign (tcgen05)
 // ---------------------------------------------------------------------------
-// One CTA per (head, pair of token tiles), one CTA per SM:
-//   warps 0-3 / 4-7  one thread per token of tile 0 / 1: scores of each centroid tile from
-//                    TMEM, the three best scores and the two best indices;
-//   warp 8           TMA: both token tiles once, then the centroid tiles (hi and lo
-//                    pieces) through a two-stage ring that both tiles read;
+// One CTA per (head, run of pairs of token tiles), one CTA per SM:
+//   warps 0-3 / 4-7  one thread per token of tile 0 / 1 of the current pair: scores of
+//                    each centroid tile from TMEM, the two best scores and the best index;
+//   warp 8           TMA: the pair's two token tiles, then its centroid tiles (hi and lo
+//                    pieces) through a two-stage ring that both tiles read and that runs
+//                    on across the pairs of the run;
 //   warps 9 / 10     MMA issuer of tile 0 / 1: S = X C_hi^T + X C_lo^T into the tile's
 //                    next logit buffer (two per tile, 128 columns each).
+// The token tiles of the next pair load as soon as both issuers are done with the
+// current ones and every row thread has read its token's norm.
 template <int D>
 struct AGeom {
   static constexpr int SUB = D / 64;
@@ -121,7 +126,7 @@ struct AGeom {
 };
 
 struct ACtl {
-  uint64_t x_full, c_full[2], c_empty[2], s_full[2][2], s_free[2][2], done;
+  uint64_t x_full, x_empty, c_full[2], c_empty[2], s_full[2][2], s_free[2][2], done;
   uint32_t tmem_base;
   int abort;
 };
@@ -131,10 +136,9 @@ struct AParams {
   const float* cnorm;
   int32_t* labels;
   int32_t* amb_list;
-  int32_t* amb_pair;
   int32_t* amb_cnt;
   int32_t* err_flag;
-  int N, Cpad, npair;
+  int N, Cpad, npair, run, nrun;
 };
 
 template <int D>
@@ -147,12 +151,14 @@ __global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ 
   ACtl& c = *reinterpret_cast<ACtl*>(smem + G::OFF_CTL);
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int pair = blockIdx.x % p.npair, bh = blockIdx.x / p.npair;
-  const int r0 = pair * 2 * TT;
+  const int run = blockIdx.x % p.nrun, bh = blockIdx.x / p.nrun;
+  const int pr0 = run * p.run;
+  const int np = min(p.run, p.npair - pr0);  // pairs of this CTA
   const int ntc = p.Cpad / TCN;
 
   if (tid == 0) {
     tc::mbar_init(bar(c.x_full), 1);
+    tc::mbar_init(bar(c.x_empty), 2 + 2 * TT);
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(c.c_full[b]), 1);
       tc::mbar_init(bar(c.c_empty[b]), 2);
@@ -178,17 +184,31 @@ __global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ 
   if (warp < 8) {
     // ============ rows: nearest centroids of one token of tile g ============
     const int g = warp / 4, row = tid & (TT - 1);
-    const int r = r0 + g * TT + row;  // the token
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
     // the head's ||c||^2 into shared memory once (the eight row warps, then their barrier)
     float* cn = reinterpret_cast<float*>(smem + G::OFF_CN);
-    for (int m = tid; m < p.Cpad; m += 2 * TT) cn[m] = __ldg(p.cnorm + (size_t)bh * p.Cpad + m);
+    float* red = reinterpret_cast<float*>(smem + G::OFF_CTL + 128);  // [8] warp maxima
+    float cm = 0.f;  // largest ||c||^2 of the head (real centroids only)
+    for (int m = tid; m < p.Cpad; m += 2 * TT) {
+      const float v = __ldg(p.cnorm + (size_t)bh * p.Cpad + m);
+      cn[m] = v;
+      if (v < INFINITY) cm = fmaxf(cm, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    if (lane == 0) red[warp] = cm;
     asm volatile("bar.sync 1, %0;\n" ::"r"(2 * TT) : "memory");
-    bool ok = uni(wt.wait(bar(c.x_full), 0, 1));
-    // ||x||^2 from the swizzled token tile (bf16 values, exact products in fp32)
-    float xn = 0.f;
-    if (ok) {
+    float cmax2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) cmax2 = fmaxf(cmax2, red[w]);
+    bool ok = true;
+    for (int i = 0; i < np && ok; ++i) {
+      const int r = (pr0 + i) * 2 * TT + g * TT + row;  // the token
+      ok = uni(wt.wait(bar(c.x_full), i & 1, 1));
+      if (!ok) break;
+      // ||x||^2 from the swizzled token tile (bf16 values, exact products in fp32)
+      float xn = 0.f;
       const uint8_t* xt = smem + G::OFF_X + g * G::XT;
       for (int ch = 0; ch < D / 8; ++ch) {
         const uint32_t off = (ch >> 3) * TT * 128 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
@@ -200,85 +220,85 @@ __global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ 
           xn = fmaf(a, a, fmaf(b, b, xn));
         }
       }
-    }
-    float best = INFINITY, second = INFINITY, third = INFINITY, cmax2 = 0.f;
-    int bi = 0, si = 0;
-    for (int t = 0; t < ntc && ok; ++t) {
-      const int b = t & 1;
-      ok = uni(wt.wait(bar(c.s_full[g][b]), (t >> 1) & 1, 2));
-      if (!ok) break;
-      tc::fence_after_sync();
-      const uint32_t scol = tmem + lane_off + 256 * g + TCN * b;
+      tc::mbar_arrive(bar(c.x_empty));  // this thread is done with the token tiles
+      float best = INFINITY, second = INFINITY;
+      int bi = 0;
+      for (int t = 0; t < ntc && ok; ++t) {
+        const int T = i * ntc + t, b = T & 1;
+        ok = uni(wt.wait(bar(c.s_full[g][b]), (T >> 1) & 1, 2));
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t scol = tmem + lane_off + 256 * g + TCN * b;
 #pragma unroll 1
-      for (int h = 0; h < TCN / 64; ++h) {
-        uint32_t sr[64];
-        tc::tmem_ld32(scol + 64 * h, sr);
-        tc::tmem_ld32(scol + 64 * h + 32, sr + 32);
-        tc::tmem_wait_ld();
-        if (h == TCN / 64 - 1) {
-          tc::fence_before_sync();
-          tc::mbar_arrive(bar(c.s_free[g][b]));
-        }
-        const int m0 = t * TCN + 64 * h;
+        for (int h = 0; h < TCN / 64; ++h) {
+          uint32_t sr[64];
+          tc::tmem_ld32(scol + 64 * h, sr);
+          tc::tmem_ld32(scol + 64 * h + 32, sr + 32);
+          tc::tmem_wait_ld();
+          if (h == TCN / 64 - 1) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(c.s_free[g][b]));
+          }
+          const int m0 = t * TCN + 64 * h;
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          const float4 n4 = *reinterpret_cast<const float4*>(cn + m0 + e);
-          const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+          for (int e = 0; e < 64; e += 4) {
+            const float4 n4 = *reinterpret_cast<const float4*>(cn + m0 + e);
+            const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-          for (int f = 0; f < 4; ++f) {
-            const float s = fmaf(-2.f, __uint_as_float(sr[e + f]), nv[f]);
-            if (nv[f] < INFINITY) cmax2 = fmaxf(cmax2, nv[f]);
-            // three best scores (and the two best indices), without branches
-            const int m = m0 + e + f;
-            const bool lt1 = s < best, lt2 = s < second, lt3 = s < third;
-            third = lt2 ? second : (lt3 ? s : third);
-            si = lt1 ? bi : (lt2 ? m : si);
-            second = lt1 ? best : (lt2 ? s : second);
-            bi = lt1 ? m : bi;
-            best = lt1 ? s : best;
+            for (int f = 0; f < 4; ++f) {
+              const float s = fmaf(-2.f, __uint_as_float(sr[e + f]), nv[f]);
+              // the two best scores and the best index (the first on ties)
+              bi = s < best ? m0 + e + f : bi;
+              second = fminf(second, fmaxf(best, s));
+              best = fminf(best, s);
+            }
           }
         }
       }
-    }
-    if (ok && r < p.N) {
-      // Error bound of one fp32 score here: the pieces hold c to 2^-17 relative, the
-      // products accumulate in fp32 over 2d terms, ||c||^2 and the final fma round once:
-      // |err| <= 5e-5 |x| |c| + 1.2e-7 |c|^2. A token whose two best scores are closer
-      // than twice that (with 20% to spare) is decided in fp64 instead: only a centroid
-      // scored within that distance of the best can be the true nearest one.
-      const float xa = sqrtf(xn), ca = sqrtf(cmax2);
-      const float thr = 1.2e-4f * xa * ca + 3e-7f * cmax2;
-      p.labels[(size_t)bh * p.N + r] = bi;
-      if (!(second - best > thr)) {
-        // undecided: between the two best if the third is clear of them, else among all
-        const int k = atomicAdd(p.amb_cnt + bh, 1);
-        p.amb_list[(size_t)bh * p.N + k] = r;
-        p.amb_pair[(size_t)bh * p.N + k] = third - best > thr ? (bi | (si << 16)) : -1;
+      if (ok && r < p.N) {
+        // Error bound of one fp32 score here: the pieces hold c to 2^-17 relative, the
+        // products accumulate in fp32 over 2d terms, ||c||^2 and the final fma round
+        // once: |err| <= 5e-5 |x| |c| + 1.2e-7 |c|^2. A token whose two best scores are
+        // closer than twice that (with 20% to spare) is decided in fp64 instead.
+        const float xa = sqrtf(xn), ca = sqrtf(cmax2);
+        const float thr = 1.2e-4f * xa * ca + 3e-7f * cmax2;
+        p.labels[(size_t)bh * p.N + r] = bi;
+        if (!(second - best > thr)) {
+          const int k = atomicAdd(p.amb_cnt + bh, 1);  // undecided: recheck in fp64
+          p.amb_list[(size_t)bh * p.N + k] = r;
+        }
       }
     }
   } else if (warp == 8) {
     // ======================== TMA producer ========================
     if (lane == 0) {
       bool ok = true;
-      tc::mbar_arrive_expect_tx(bar(c.x_full), 2 * G::XT);
-      for (int g = 0; g < 2; ++g)
-        for (int x = 0; x < G::SUB; ++x)
-          tc::tma_load_3d(base + G::OFF_X + g * G::XT + x * TT * 128, &p.tmX, bar(c.x_full),
-                          64 * x, r0 + g * TT, bh);
-      uint32_t used = 0, par = 0;  // per stage: loaded, parity of the last load
-      for (int t = 0; t < ntc && ok; ++t) {
-        const int st = t & 1, ph = (t >> 1) & 1;
-        if (t >= 2) ok = wt.wait(bar(c.c_empty[st]), ph ^ 1, 3);
+      uint32_t used = 0, par = 0;  // per centroid stage: loaded, parity of the last load
+      int xloads = 0;
+      for (int i = 0; i < np && ok; ++i) {
+        if (i >= 1) ok = wt.wait(bar(c.x_empty), (i - 1) & 1, 7);
         if (!ok) break;
-        tc::mbar_arrive_expect_tx(bar(c.c_full[st]), 2 * G::CT);
-        for (int pc = 0; pc < 2; ++pc)
+        tc::mbar_arrive_expect_tx(bar(c.x_full), 2 * G::XT);
+        for (int g = 0; g < 2; ++g)
           for (int x = 0; x < G::SUB; ++x)
-            tc::tma_load_3d(base + G::OFF_C + (st * 2 + pc) * G::CT + x * TCN * 128, &p.tmC,
-                            bar(c.c_full[st]), 64 * x, t * TCN, 2 * bh + pc);
-        used |= 1u << st;
-        par = (par & ~(1u << st)) | ((uint32_t)ph << st);
+            tc::tma_load_3d(base + G::OFF_X + g * G::XT + x * TT * 128, &p.tmX, bar(c.x_full),
+                            64 * x, (pr0 + i) * 2 * TT + g * TT, bh);
+        ++xloads;
+        for (int t = 0; t < ntc && ok; ++t) {
+          const int T = i * ntc + t, st = T & 1, ph = (T >> 1) & 1;
+          if (T >= 2) ok = wt.wait(bar(c.c_empty[st]), ph ^ 1, 3);
+          if (!ok) break;
+          tc::mbar_arrive_expect_tx(bar(c.c_full[st]), 2 * G::CT);
+          for (int pc = 0; pc < 2; ++pc)
+            for (int x = 0; x < G::SUB; ++x)
+              tc::tma_load_3d(base + G::OFF_C + (st * 2 + pc) * G::CT + x * TCN * 128, &p.tmC,
+                              bar(c.c_full[st]), 64 * x, t * TCN, 2 * bh + pc);
+          used |= 1u << st;
+          par = (par & ~(1u << st)) | ((uint32_t)ph << st);
+        }
       }
-      tc::wait_drain(bar(c.x_full), 0, kWaitLimit);
+      // every load issued lands before the CTA exits
+      if (xloads > 0) tc::wait_drain(bar(c.x_full), (xloads - 1) & 1, kWaitLimit);
       for (int st = 0; st < 2; ++st)
         if ((used >> st) & 1) tc::wait_drain(bar(c.c_full[st]), (par >> st) & 1, kWaitLimit);
     }
@@ -287,25 +307,29 @@ __global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t I_S = tc::idesc_f16(1, 1, 0, TCN);
       const int g = warp - 9;
-      bool ok = wt.wait(bar(c.x_full), 0, 4);
       const uint64_t dx = tc::sdesc(base + G::OFF_X + g * G::XT, 16, 1024);
-      for (int t = 0; t < ntc && ok; ++t) {
-        const int b = t & 1, st = t & 1;
-        ok = wt.wait(bar(c.c_full[st]), (t >> 1) & 1, 5) &&
-             (t < 2 || wt.wait(bar(c.s_free[g][b]), ((t >> 1) - 1) & 1, 6));
-        if (!ok) break;
-        tc::fence_after_sync();
-        const uint64_t dc = tc::sdesc(base + G::OFF_C + st * 2 * G::CT, 16, 1024);
-        for (int pc = 0; pc < 2; ++pc) {
+      bool ok = true;
+      for (int i = 0; i < np && ok; ++i) {
+        ok = wt.wait(bar(c.x_full), i & 1, 4);
+        for (int t = 0; t < ntc && ok; ++t) {
+          const int T = i * ntc + t, b = T & 1, st = T & 1;
+          ok = wt.wait(bar(c.c_full[st]), (T >> 1) & 1, 5) &&
+               (T < 2 || wt.wait(bar(c.s_free[g][b]), ((T >> 1) - 1) & 1, 6));
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint64_t dc = tc::sdesc(base + G::OFF_C + st * 2 * G::CT, 16, 1024);
+          for (int pc = 0; pc < 2; ++pc) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t aoff = ((kk / 4) * TT * 128 + (kk % 4) * 32) >> 4;
-            const uint32_t boff = (pc * G::CT + (kk / 4) * TCN * 128 + (kk % 4) * 32) >> 4;
-            tc::mma_ss(tmem + 256 * g + TCN * b, dx + aoff, dc + boff, I_S, (pc | kk) > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t aoff = ((kk / 4) * TT * 128 + (kk % 4) * 32) >> 4;
+              const uint32_t boff = (pc * G::CT + (kk / 4) * TCN * 128 + (kk % 4) * 32) >> 4;
+              tc::mma_ss(tmem + 256 * g + TCN * b, dx + aoff, dc + boff, I_S, (pc | kk) > 0);
+            }
           }
+          tc::mma_commit(bar(c.s_full[g][b]));
+          tc::mma_commit(bar(c.c_empty[st]));
         }
-        tc::mma_commit(bar(c.s_full[g][b]));
-        tc::mma_commit(bar(c.c_empty[st]));
+        if (ok) tc::mma_commit(bar(c.x_empty));  // the token tiles are read
       }
       tc::mma_commit(bar(c.done));
       tc::wait_drain(bar(c.done), 0, kWaitLimit);
@@ -322,12 +346,13 @@ __global__ void __launch_bounds__(352, 1) assign_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-// recheck: the undecided tokens in fp64, one warp per token
+// recheck: the undecided tokens in fp64, one CTA per token
 // ---------------------------------------------------------------------------
 // dist_m = sum_i (x_i - c_mi)^2, lane l summing dimensions l, l+32, ... in order and the
-// lanes combined by a fixed butterfly; the smallest distance wins, ties to the lower
-// index. Only the candidates the assignment recorded are compared: its two best
-// centroids, or every centroid when a third one was as close.
+// lanes combined by a fixed butterfly. Warp w takes the centroids m = w, w + 8, ...; the
+// smallest distance wins, ties to the lowest index.
+constexpr int kRecheckWarps = 8;
+
 __device__ __forceinline__ double dist64(const double* xv, const double* cm, int d, int lane) {
   double s = 0.0;
 #pragma unroll
@@ -342,40 +367,52 @@ __device__ __forceinline__ double dist64(const double* xv, const double* cm, int
   return s;
 }
 
-__global__ void recheck_kernel(const uint16_t* __restrict__ x, const double* __restrict__ cent,
-                               int N, int d, int C, const int32_t* __restrict__ amb_list,
-                               const int32_t* __restrict__ amb_pair,
-                               const int32_t* __restrict__ amb_cnt, int32_t* __restrict__ labels) {
+__global__ void __launch_bounds__(32 * kRecheckWarps)
+recheck_kernel(const uint16_t* __restrict__ x, const double* __restrict__ cent, int N, int d,
+               int C, const int32_t* __restrict__ amb_list, const int32_t* __restrict__ amb_cnt,
+               int32_t* __restrict__ labels) {
+  __shared__ double wbest[kRecheckWarps];
+  __shared__ int wbi[kRecheckWarps];
   const int bh = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  const int nw = (int)(blockDim.x / 32);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int cnt = amb_cnt[bh];
-  for (int e = blockIdx.x * nw + threadIdx.x / 32; e < cnt; e += gridDim.x * nw) {
+  const double* cb = cent + (size_t)bh * C * d;
+  for (int e = blockIdx.x; e < cnt; e += gridDim.x) {
     const int r = amb_list[(size_t)bh * N + e];
-    const int pair = amb_pair[(size_t)bh * N + e];
     const uint16_t* xr = x + ((size_t)bh * N + r) * d;
     double xv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       xv[k] = lane + 32 * k < d ? (double)__uint_as_float((uint32_t)xr[lane + 32 * k] << 16) : 0.0;
-    const double* cb = cent + (size_t)bh * C * d;
+    double best = INFINITY;
     int bi = 0;
-    if (pair >= 0) {
-      const int a = pair & 0xFFFF, b = pair >> 16;
-      const double da = dist64(xv, cb + (size_t)a * d, d, lane);
-      const double db = dist64(xv, cb + (size_t)b * d, d, lane);
-      bi = (db < da || (db == da && b < a)) ? b : a;
-    } else {
-      double best = INFINITY;
-      for (int m = 0; m < C; ++m) {
-        const double s = dist64(xv, cb + (size_t)m * d, d, lane);
-        if (s < best) {
-          best = s;
-          bi = m;
-        }
-      }
+    int m = warp;
+    for (; m + kRecheckWarps < C; m += 2 * kRecheckWarps) {  // two centroids in flight
+      const double s0 = dist64(xv, cb + (size_t)m * d, d, lane);
+      const double s1 = dist64(xv, cb + (size_t)(m + kRecheckWarps) * d, d, lane);
+      if (s0 < best) { best = s0; bi = m; }
+      if (s1 < best) { best = s1; bi = m + kRecheckWarps; }
     }
-    if (lane == 0) labels[(size_t)bh * N + r] = bi;
+    if (m < C) {
+      const double s0 = dist64(xv, cb + (size_t)m * d, d, lane);
+      if (s0 < best) { best = s0; bi = m; }
+    }
+    if (lane == 0) {
+      wbest[warp] = best;
+      wbi[warp] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double b = wbest[0];
+      int ib = wbi[0];
+      for (int w = 1; w < kRecheckWarps; ++w)
+        if (wbest[w] < b || (wbest[w] == b && wbi[w] < ib)) {
+          b = wbest[w];
+          ib = wbi[w];
+        }
+      labels[(size_t)bh * N + r] = ib;
+    }
+    __syncthreads();
   }
 }
 
@@ -486,15 +523,27 @@ update_kernel(const uint16_t* __restrict__ x, int N, int d, int C,
   const int32_t* pr = perm + (size_t)bh * N;
   const uint16_t* xb = x + (size_t)bh * N * d + ch * 8;
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int k = s + rl; k < e; k += lanes) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(xb + (size_t)__ldg(pr + k) * d));
+  auto add = [&](const uint4& w) {
     const uint32_t v[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       acc[2 * q] += (double)bf16_lo(v[q]);
       acc[2 * q + 1] += (double)bf16_hi(v[q]);
     }
+  };
+  int k = s + rl;
+  for (; k + 3 * lanes < e; k += 4 * lanes) {  // four member rows in flight
+    int r4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r4[u] = __ldg(pr + k + u * lanes);
+    uint4 w4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      w4[u] = __ldg(reinterpret_cast<const uint4*>(xb + (size_t)r4[u] * d));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) add(w4[u]);
   }
+  for (; k < e; k += lanes) add(__ldg(reinterpret_cast<const uint4*>(xb + (size_t)__ldg(pr + k) * d)));
 #pragma unroll
   for (int q = 0; q < 8; ++q) part[rl * d + ch * 8 + q] = acc[q];
   __syncthreads();
@@ -542,17 +591,34 @@ cudaError_t assign_t(const KmeansArgs& a, int Cpad, cudaStream_t st) {
   p.cnorm = a.cnorm;
   p.labels = a.labels;
   p.amb_list = a.amb_list;
-  p.amb_pair = a.amb_pair;
   p.amb_cnt = a.amb_cnt;
   p.err_flag = a.err_flag;
   p.N = a.N;
   p.Cpad = Cpad;
   p.npair = km::cdiv(a.N, 2 * km::TT);
+  // pairs per CTA: the run length that minimises waves x (run + 1/2), one CTA per SM and
+  // the CTA's setup costed as half a pair
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms < 1) sms = 1;
+  double best_cost = 1e300;
+  p.run = 1;
+  for (int run = 1; run <= 32; ++run) {
+    const double ctas = (double)bh * km::cdiv(p.npair, run);
+    const double cost = std::ceil(ctas / sms) * (run + 0.5);
+    if (cost < best_cost) {
+      best_cost = cost;
+      p.run = run;
+    }
+    if (run >= p.npair) break;
+  }
+  p.nrun = km::cdiv(p.npair, p.run);
   auto kern = km::assign_kernel<D>;
   const int smem = G::smem(Cpad);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(p.npair * bh), 352, smem, st>>>(p);
+  kern<<<(unsigned)(p.nrun * bh), 352, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -578,7 +644,7 @@ void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
   const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
   sizes[0] = bh * C * d * sizeof(double);
   sizes[1] = align256(bh * 2 * Cpad * d * 2) + bh * Cpad * 4;
-  sizes[2] = align256(bh * nchunk * C * 4) + 2 * align256(bh * N * 4) + bh * 4;
+  sizes[2] = align256(bh * nchunk * C * 4) + align256(bh * N * 4) + bh * 4;
 }
 
 cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
@@ -594,8 +660,6 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   iw += align256((size_t)bh * nchunk * C * 4);
   a.amb_list = reinterpret_cast<int32_t*>(iw);
   iw += align256((size_t)bh * N * 4);
-  a.amb_pair = reinterpret_cast<int32_t*>(iw);
-  iw += align256((size_t)bh * N * 4);
   a.amb_cnt = reinterpret_cast<int32_t*>(iw);
 
   const int sort_smem = km::kSortWarps * C * 4;
@@ -610,8 +674,8 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   auto assign = [&]() -> cudaError_t {
     cudaError_t r = d == 64 ? assign_t<64>(a, Cpad, st) : assign_t<128>(a, Cpad, st);
     if (r != cudaSuccess) return r;
-    km::recheck_kernel<<<dim3(32, bh), 256, 0, st>>>(a.x, a.cent, N, d, C, a.amb_list,
-                                                     a.amb_pair, a.amb_cnt, a.labels);
+    km::recheck_kernel<<<dim3(256, bh), 32 * km::kRecheckWarps, 0, st>>>(
+        a.x, a.cent, N, d, C, a.amb_list, a.amb_cnt, a.labels);
     return cudaGetLastError();
   };
   auto sort = [&]() -> cudaError_t {

@@ -70,7 +70,7 @@ struct KmeansArgs {
   // carved from cwork / iwork by the launcher
   uint16_t* pieces = nullptr;
   float* cnorm = nullptr;
-  int32_t *counts = nullptr, *amb_list = nullptr, *amb_pair = nullptr, *amb_cnt = nullptr;
+  int32_t *counts = nullptr, *amb_list = nullptr, *amb_cnt = nullptr;
 };
 
 struct PermuteArgs {
