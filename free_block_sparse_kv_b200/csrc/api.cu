@@ -344,6 +344,18 @@ int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H,
   return launched(sa::launch_permute_rows(p, static_cast<cudaStream_t>(stream)), "permute launch");
 }
 
+int sparse_attn_wait_selftest(int32_t* err_flag, int rounds, int32_t* waited, void* stream) {
+  SA_REQUIRE(rounds >= 1 && rounds <= (1 << 20), "rounds must be in [1, 2^20] (got %d)", rounds);
+  SA_REQUIRE(err_flag != nullptr && ((uintptr_t)err_flag & 3u) == 0,
+             "err_flag must be a non-null 4-byte aligned pointer");
+  SA_REQUIRE(waited != nullptr && ((uintptr_t)waited & 3u) == 0,
+             "waited must be a non-null 4-byte aligned pointer");
+  if (int rc = check_device()) return rc;
+  return launched(sa::launch_wait_selftest(err_flag, (uint32_t)rounds, waited,
+                                           static_cast<cudaStream_t>(stream)),
+                  "selftest launch");
+}
+
 int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
                         const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H, int Nq,

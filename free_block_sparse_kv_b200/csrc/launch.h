@@ -86,6 +86,8 @@ constexpr size_t kKmeansScratchBytes = (size_t)32 << 20;  // per device, for the
 void* kmeans_scratch(int device);  // device address of that buffer on `device`
 cudaError_t launch_kmeans(const KmeansArgs& p, cudaStream_t st);
 cudaError_t launch_permute_rows(const PermuteArgs& p, cudaStream_t st);
+cudaError_t launch_wait_selftest(int32_t* err_flag, uint32_t rounds, int32_t* waited,
+                                 cudaStream_t st);
 cudaError_t launch_pool(const PoolArgs& p, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& p, cudaStream_t st);
 cudaError_t launch_structured_mask(const MaskArgs& p, cudaStream_t st);

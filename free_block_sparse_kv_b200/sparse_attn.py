@@ -22,8 +22,8 @@ EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
            "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
            "sparse_attn_structured_mask_adaptive", "sparse_attn_ear_scores",
            "sparse_attn_route_scores", "sparse_attn_kmeans_sizes", "sparse_attn_kmeans",
-           "sparse_attn_permute_rows", "sparse_attn_kmeans_noalloc", "sparse_attn_forward",
-           "sparse_attn_last_error")
+           "sparse_attn_permute_rows", "sparse_attn_kmeans_noalloc", "sparse_attn_wait_selftest",
+           "sparse_attn_forward", "sparse_attn_last_error")
 
 
 class SparseAttnError(RuntimeError):
@@ -59,6 +59,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_kmeans.argtypes = [_P] + [_I] * 6 + [_P] * 7 + [_P]
     lib.sparse_attn_permute_rows.argtypes = [_P, _P] + [_I] * 5 + [_P, _P]
     lib.sparse_attn_kmeans_noalloc.argtypes = [_P] + [_I] * 6 + [_P] * 5 + [_P]
+    lib.sparse_attn_wait_selftest.argtypes = [_P, _I, _P, _P]
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_structured_mask_adaptive.argtypes = [_I] * 13 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
@@ -156,6 +157,11 @@ def sparse_attn_kmeans_noalloc(x, B, H, N, d, C, iters, centroids, labels, perm,
     _check(load_library().sparse_attn_kmeans_noalloc(
         _ptr(x), B, H, N, d, C, iters, _ptr(centroids), _ptr(labels), _ptr(perm), _ptr(offsets),
         _ptr(err_flag), _stream(stream)))
+
+
+def sparse_attn_wait_selftest(err_flag, rounds, waited, stream=None):
+    _check(load_library().sparse_attn_wait_selftest(_ptr(err_flag), rounds, _ptr(waited),
+                                                    _stream(stream)))
 
 
 def sparse_attn_permute_rows(src, perm, B, H, N, row_bytes, gather, dst, stream=None):

@@ -268,6 +268,15 @@ int sparse_attn_structured_mask_adaptive(int B, int H, int Nq, int Nk, int block
                                          void* stream);
 
 /*
+ * Self-test of the device-side failure path: one CTA waits on an mbarrier that nothing
+ * arrives on, with the library's bounded wait (`rounds` try_wait rounds of about 1 us
+ * each, 1 <= rounds <= 2^20). The wait gives up, sets bit 0 of *err_flag (device int32)
+ * and writes 0 to *waited (device int32; 1 would mean the wait had completed). The
+ * context stays usable. One launch.
+ */
+int sparse_attn_wait_selftest(int32_t* err_flag, int rounds, int32_t* waited, void* stream);
+
+/*
  * Forward (PISA §2 Algorithme Central and Implémentation Matérielle, phases 1-3,
  * with the first-order term per block, or global with order 2). For each query
  * row t of query block i:

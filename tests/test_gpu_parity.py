@@ -501,6 +501,23 @@ def test_invalid_arguments_raise():
         C.sparse_attn_pool(x, x, x, 1, 1, 64, 64, 64, 64, 1, f, f, f, x, x, None, x)
 
 
+def test_bounded_wait_gives_up_and_reports(small_inputs):
+    """A wait on an mbarrier that nothing completes ends after its bounded rounds, sets
+    the error word and returns; the context stays usable for a real call afterwards."""
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    waited = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    C.sparse_attn_wait_selftest(flag, 256, waited)
+    torch.cuda.synchronize()
+    assert int(waited.item()) == 0 and int(flag.item()) & 1
+    w, qb, kb, vb = small_inputs("uniform-4k")
+    op, out = _run(w, _dev(qb), _dev(kb), _dev(vb))
+    assert int(op.err_flag.item()) == 0 and torch.isfinite(out).all()
+    with pytest.raises(C.SparseAttnError) as e:   # the host helper turns a set flag into an error
+        op.err_flag.fill_(1)
+        op.check()
+    assert e.value.code == C.SA_ERR_TIMEOUT
+
+
 def test_repeat_calls_are_bitwise_deterministic(small_inputs):
     w, qb, kb, vb = small_inputs("dit-small")
     q, k, v = _dev(qb), _dev(kb), _dev(vb)
