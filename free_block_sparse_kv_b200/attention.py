@@ -217,7 +217,7 @@ class BlockSparseAttention:
             self.out_p = torch.empty_like(self.out)
 
     def cluster(self, q, k, v, stream=None):
-        """k-means of Q and K and the group-major copies of Q, K and V."""
+        """k-means of Q and K and the group-major copies of Q, K and V (every head)."""
         kmeans(q, self.cl_q, self.err_flag, stream)
         kmeans(k, self.cl_k, self.err_flag, stream)
         permute_rows(q, self.cl_q.perm, self.q_p, True, stream)
@@ -227,29 +227,104 @@ class BlockSparseAttention:
 
     def __call__(self, q, k, v, step: int = 0, stream=None) -> torch.Tensor:
         _check_inputs(q, k, v)
-        if self.clusters:
-            qp, kp, vp = self.cluster(q, k, v, stream)
-            self._attend(qp, kp, vp, self.out_p, step, stream)
-            permute_rows(self.out_p, self.cl_q.perm, self.out, False, stream)
-            return self.out
-        self._attend(q, k, v, self.out, step, stream)
+        self._run(q, k, v, self.out, None, step, stream)
         return self.out
 
-    def _attend(self, q, k, v, out, step, stream):
-        p = self.p
-        pool(q if self.mode != "structured" else None, k, v, p, self.tables, stream)
+    def _run(self, q, k, v, out, heads, step, stream):
+        """All stages for the heads ``heads`` = (b, h0, h1) (None: every head). A head
+        range runs as a problem of its own on views of every buffer; heads never
+        interact, so any split of them gives the same output."""
+        if heads is None:
+            p, t, idx, cnt = self.p, self.tables, self.kv_idx, self.kv_cnt
+            sub = lambda x: x
+        else:
+            b, h0, h1 = heads
+            p = dataclasses.replace(self.p, B=1, H=h1 - h0)
+            sub = lambda x: None if x is None else x[b:b + 1, h0:h1]
+            t = Tables(**{f.name: sub(getattr(self.tables, f.name))
+                          for f in dataclasses.fields(Tables)})
+            idx, cnt = sub(self.kv_idx), sub(self.kv_cnt)
+            q, k, v, out = sub(q), sub(k), sub(v), sub(out)
+        if self.clusters:
+            clq = dataclasses.replace(self.cl_q, centroids=sub(self.cl_q.centroids),
+                                      labels=sub(self.cl_q.labels), perm=sub(self.cl_q.perm),
+                                      offsets=sub(self.cl_q.offsets))
+            clk = dataclasses.replace(self.cl_k, centroids=sub(self.cl_k.centroids),
+                                      labels=sub(self.cl_k.labels), perm=sub(self.cl_k.perm),
+                                      offsets=sub(self.cl_k.offsets))
+            qp, kp, vp, op_ = sub(self.q_p), sub(self.k_p), sub(self.v_p), sub(self.out_p)
+            kmeans(q, clq, self.err_flag, stream)
+            kmeans(k, clk, self.err_flag, stream)
+            permute_rows(q, clq.perm, qp, True, stream)
+            permute_rows(k, clk.perm, kp, True, stream)
+            permute_rows(v, clk.perm, vp, True, stream)
+            self._attend(p, t, idx, cnt, qp, kp, vp, op_, step, stream)
+            permute_rows(op_, clq.perm, out, False, stream)
+        else:
+            self._attend(p, t, idx, cnt, q, k, v, out, step, stream)
+
+    def _attend(self, p, t, kv_idx, kv_cnt, q, k, v, out, step, stream):
+        pool(q if self.mode != "structured" else None, k, v, p, t, stream)
         if self.mode == "structured":
             g = self.geometry
-            structured_mask(p, self.kv_idx, self.kv_cnt, g["frame_tokens"], g["n_frames"],
+            structured_mask(p, kv_idx, kv_cnt, g["frame_tokens"], g["n_frames"],
                             g["window"], g["n_anchors"], g["period"], step, g.get("q_frame0", 0),
                             g.get("budget", 0), stream)
         else:
             if self.mode == "ear":
-                ear_scores(k, v, p, self.tables, err_flag=self.err_flag, stream=stream)
-            route(p, self.tables, self.kv_idx, self.kv_cnt, self.mode, self.rho, self.tau,
-                  stream=stream)
-        forward(q, k, v, p, self.tables, self.kv_idx, self.kv_cnt, out,
-                err_flag=self.err_flag, stream=stream)
+                ear_scores(k, v, p, t, err_flag=self.err_flag, stream=stream)
+            route(p, t, kv_idx, kv_cnt, self.mode, self.rho, self.tau, stream=stream)
+        forward(q, k, v, p, t, kv_idx, kv_cnt, out, err_flag=self.err_flag, stream=stream)
+
+    def run_from_host(self, q_h, k_h, v_h, out_h, step: int = 0, chunks: int = 10):
+        """One call with Q, K, V in (pinned) host memory and the output written to the
+        (pinned) host tensor ``out_h``. The heads are split into ``chunks`` ranges: the
+        host-to-device copies run ahead on one stream, each range is computed on the
+        current stream as soon as its inputs are in, and its output goes back on a
+        third stream while the next range computes. Returns after enqueueing; the
+        current stream waits for the last copy back."""
+        p = self.p
+        dev = self.out.device
+        if getattr(self, "_dev_in", None) is None:
+            self._dev_in = tuple(torch.empty(x.shape, dtype=x.dtype, device=dev)
+                                 for x in (q_h, k_h, v_h))
+            self._h2d, self._d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        q, k, v = self._dev_in
+        cs = torch.cuda.current_stream(dev)
+        # Head ranges start at multiples of 4 heads of the flattened (batch, head) index,
+        # so that every per-head table slice starts on a 16-byte boundary (the C ABI's
+        # alignment rule); otherwise the call runs as one range.
+        per_b = max(1, -(-chunks // p.B))              # ranges per batch entry
+        step_h = -(-(-(-p.H // per_b)) // 4) * 4
+        ranges = [(b, h0, min(p.H, h0 + step_h)) for b in range(p.B)
+                  for h0 in range(0, p.H, step_h)]
+        if any((b * p.H + h0) % 4 for b, h0, _ in ranges):
+            ranges = [(b, 0, p.H) for b in range(p.B)] if (p.H % 4 == 0) else None
+        if ranges is None:
+            for dst, src in ((q, q_h), (k, k_h), (v, v_h)):
+                dst.copy_(src, non_blocking=True)
+            self._run(q, k, v, self.out, None, step, None)
+            out_h.copy_(self.out, non_blocking=True)
+            return out_h
+        self._h2d.wait_stream(cs)                      # inputs may still be read by an earlier call
+        ready = []
+        with torch.cuda.stream(self._h2d):
+            for b, h0, h1 in ranges:
+                for dst, src in ((q, q_h), (k, k_h), (v, v_h)):
+                    dst[b, h0:h1].copy_(src[b, h0:h1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self._h2d)
+                ready.append(ev)
+        for (b, h0, h1), ev in zip(ranges, ready):
+            cs.wait_event(ev)
+            self._run(q, k, v, self.out, (b, h0, h1), step, None)
+            done = torch.cuda.Event()
+            done.record(cs)
+            self._d2h.wait_event(done)
+            with torch.cuda.stream(self._d2h):
+                out_h[b, h0:h1].copy_(self.out[b, h0:h1], non_blocking=True)
+        cs.wait_stream(self._d2h)
+        return out_h
 
     def check(self):
         """Raise if a bounded device wait of an earlier call gave up (synchronises)."""

@@ -518,6 +518,28 @@ def test_bounded_wait_gives_up_and_reports(small_inputs):
     assert e.value.code == C.SA_ERR_TIMEOUT
 
 
+@pytest.mark.parametrize("name", ["dit-small", "kmeans-small", "longvideo-small", "worldmodel-small",
+                                  "ear-small", "hybrid-small"])
+def test_host_call_equals_device_call(name, small_inputs):
+    """run_from_host (head ranges, copies overlapped with the compute) gives the device
+    call's output bit for bit."""
+    w, qb, kb, vb = small_inputs(name)
+    if name in ("dit-small", "kmeans-small"):   # enough heads for several ranges of four
+        w = W.shrink(w, H=12, Nq=3000, Nk=3000, grid=(3, 20, 50))
+        qb, kb, vb = W.full_inputs_bits(w)
+    step = w.steps[-1] if w.mode == "structured" else 0
+    op, out = _run(w, _dev(qb), _dev(kb), _dev(vb), step=step)
+    want = out.clone()
+    pin = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_h = torch.empty(want.shape, dtype=want.dtype, pin_memory=True)
+    for chunks in (1, 3, 8):
+        out_h.zero_()
+        op.run_from_host(pin(qb), pin(kb), pin(vb), out_h, step=step, chunks=chunks)
+        torch.cuda.synchronize()
+        op.check()
+        assert torch.equal(out_h, want.cpu()), chunks
+
+
 def test_repeat_calls_are_bitwise_deterministic(small_inputs):
     w, qb, kb, vb = small_inputs("dit-small")
     q, k, v = _dev(qb), _dev(kb), _dev(vb)
