@@ -118,11 +118,17 @@ def _check_inputs(q, k, v):
             raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor [B,H,N,d]")
 
 
-def pool(q, k, v, p: Problem, t: Tables, stream=None):
+def pool(q, k, v, p: Problem, t: Tables, stream=None, kv_block_start: int = 0):
     """Pooled tables; with order 2 also the global first-order matrix and the
-    per-block covariance norms."""
-    C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar, t.kbar_t,
-                       t.vsum, t.kbar16, t.vsum16, t.M, t.v16, stream)
+    per-block covariance norms. kv_block_start > 0 pools only the KV blocks from there
+    on (a growing KV cache whose earlier blocks were pooled by an earlier call)."""
+    if kv_block_start:
+        C.sparse_attn_pool_incremental(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order,
+                                       kv_block_start, t.qbar, t.kbar_t, t.vsum, t.kbar16,
+                                       t.vsum16, t.M, t.v16, stream)
+    else:
+        C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar,
+                           t.kbar_t, t.vsum, t.kbar16, t.vsum16, t.M, t.v16, stream)
     if p.order == 2:
         C.sparse_attn_hbar(t.M, p.B, p.H, p.nkb, p.d, t.hbar, t.hbar16, t.cov, stream)
 

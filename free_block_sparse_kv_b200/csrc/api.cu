@@ -119,6 +119,39 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
   return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
 }
 
+int sparse_attn_pool_incremental(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                                 int H, int Nq, int Nk, int d, int block, int order,
+                                 int kv_block_start, float* qbar, float* kbar_t, float* vsum,
+                                 uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
+                                 void* stream) {
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
+  const int nkb = cdiv(Nk, block);
+  SA_REQUIRE(kv_block_start >= 0 && kv_block_start <= nkb,
+             "kv_block_start must be in [0, nkb] (got %d, nkb %d)", kv_block_start, nkb);
+  const bool do_q = q != nullptr && Nq > 0;
+  if ((long long)B * H == 0 || (kv_block_start == nkb && !do_q)) return ok();
+  if (kv_block_start < nkb) {
+    SA_REQUIRE_PTR(k);
+    SA_REQUIRE_PTR(v);
+    SA_REQUIRE_PTR(kbar_t);
+    SA_REQUIRE_PTR(vsum);
+    SA_REQUIRE_PTR(kbar16);
+    SA_REQUIRE_PTR(vsum16);
+    SA_REQUIRE_PTR(v16);
+    if (order >= 1) SA_REQUIRE_PTR(M);
+  }
+  if (do_q) {
+    SA_REQUIRE_PTR(q);
+    SA_REQUIRE_PTR(qbar);
+  }
+  if (int rc = check_device()) return rc;
+  sa::PoolArgs p{do_q ? q : nullptr, k, v, B, H, Nq, kv_block_start < nkb ? Nk : 0, d, block,
+                 order, cdiv(Nq, block), nkb, qbar, kbar_t, vsum, kbar16, vsum16, M, v16,
+                 kv_block_start};
+  return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
+}
+
 int sparse_attn_route(const float* qbar, const float* kbar_t, int B, int H, int nqb, int nkb, int d,
                       int mode, int rho_num, int rho_den, float tau, float scale, int32_t* kv_idx,
                       int32_t* kv_cnt, int cap, void* stream) {

@@ -11,6 +11,7 @@ struct PoolArgs {
   int B, H, Nq, Nk, d, block, order, nqb, nkb;
   float *qbar, *kbar_t, *vsum;
   uint16_t *kbar16, *vsum16, *M, *v16;
+  int j0 = 0;  // first KV block pooled (the tables of blocks < j0 are left as they are)
 };
 
 struct RouteArgs {

@@ -49,7 +49,7 @@ SA_DEVI uint32_t swz128(int r, int c, int rows) {
 template <int D, int BLK, int ORDER>
 __global__ void __launch_bounds__(kPoolThreads, 3)
 pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-            const uint16_t* __restrict__ v, int Nq, int Nk, int nqb, int nkb,
+            const uint16_t* __restrict__ v, int Nq, int Nk, int nqb, int nkb, int j0,
             float* __restrict__ qbar, float* __restrict__ kbar_t, float* __restrict__ vsum,
             uint16_t* __restrict__ kbar16, uint16_t* __restrict__ vsum16,
             uint16_t* __restrict__ M, uint16_t* __restrict__ v16) {
@@ -94,9 +94,10 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
       for (int e = 0; e < 8; ++e) out_rows[warp * D + ch * 8 + e] = acc[e];
   };
 
-  if (blk >= nkb) {
+  const int nkv = nkb - j0;  // KV blocks pooled by this launch: j0 .. nkb-1
+  if (blk >= nkv) {
     // ---- query block: qbar_i = mean of its rows ----
-    const int i = blk - nkb;
+    const int i = blk - nkv;
     const int start = i * BLK;
     const int n = min(BLK, Nq - start);
     const uint16_t* src = q + ((size_t)bh * Nq + start) * D;
@@ -116,7 +117,7 @@ pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
   }
 
   // ---- KV block j ----
-  const int j = blk;
+  const int j = j0 + blk;
   const int start = j * BLK;
   const int n = min(BLK, Nk - start);
   const uint16_t* kg = k + ((size_t)bh * Nk + start) * D;
@@ -247,8 +248,10 @@ static cudaError_t launch_pool_t(const PoolArgs& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   const int nq_blocks = p.q ? p.nqb : 0;
-  dim3 grid(p.nkb + nq_blocks, p.B * p.H);
-  kern<<<grid, kPoolThreads, G::SMEM, st>>>(p.q, p.k, p.v, p.Nq, p.Nk, p.nqb, p.nkb, p.qbar,
+  const int nkv = p.Nk > 0 ? p.nkb - p.j0 : 0;
+  if (nkv + nq_blocks == 0) return cudaSuccess;
+  dim3 grid(nkv + nq_blocks, p.B * p.H);
+  kern<<<grid, kPoolThreads, G::SMEM, st>>>(p.q, p.k, p.v, p.Nq, p.Nk, p.nqb, p.nkb, p.j0, p.qbar,
                                             p.kbar_t, p.vsum, p.kbar16, p.vsum16, p.M, p.v16);
   return cudaGetLastError();
 }

@@ -18,7 +18,8 @@ SA_ROUTE_TOPK, SA_ROUTE_MASS = 0, 1
 SA_OUT_F32, SA_OUT_BF16 = 0, 1
 
 # Entry points declared in include/sparse_attn.h.
-EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_route",
+EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_pool_incremental",
+           "sparse_attn_route",
            "sparse_attn_route_cov", "sparse_attn_hbar", "sparse_attn_structured_mask",
            "sparse_attn_structured_mask_adaptive", "sparse_attn_ear_scores",
            "sparse_attn_route_scores", "sparse_attn_kmeans_sizes", "sparse_attn_kmeans",
@@ -50,6 +51,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_last_error.argtypes = []
     lib.sparse_attn_table_sizes.argtypes = [_I] * 7 + [ctypes.POINTER(ctypes.c_size_t)]
     lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 7 + [_P]
+    lib.sparse_attn_pool_incremental.argtypes = [_P, _P, _P] + [_I] * 8 + [_P] * 7 + [_P]
     lib.sparse_attn_route.argtypes = [_P, _P] + [_I] * 8 + [_F, _F, _P, _P, _I, _P]
     lib.sparse_attn_route_cov.argtypes = [_P, _P, _P] + [_I] * 7 + [_F, _P, _P, _I, _P]
     lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
@@ -103,6 +105,13 @@ def sparse_attn_pool(q, k, v, B, H, Nq, Nk, d, block, order, qbar, kbar_t, vsum,
     _check(load_library().sparse_attn_pool(
         _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, block, order, _ptr(qbar), _ptr(kbar_t),
         _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _stream(stream)))
+
+
+def sparse_attn_pool_incremental(q, k, v, B, H, Nq, Nk, d, block, order, kv_block_start, qbar,
+                                 kbar_t, vsum, kbar16, vsum16, M, v16, stream=None):
+    _check(load_library().sparse_attn_pool_incremental(
+        _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, block, order, kv_block_start, _ptr(qbar),
+        _ptr(kbar_t), _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _stream(stream)))
 
 
 def sparse_attn_route(qbar, kbar_t, B, H, nqb, nkb, d, mode, rho_num, rho_den, tau, scale, kv_idx,

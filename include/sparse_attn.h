@@ -101,6 +101,22 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      void* stream);
 
 /*
+ * Incremental pooling for a growing KV cache (an autoregressive world model attends a new
+ * chunk of frames to every earlier frame): as sparse_attn_pool, but only the KV blocks
+ * kv_block_start .. nkb-1 are pooled and written (kbar_t, vsum, kbar16, vsum16, M rows and
+ * the v16 tokens of those blocks); the tables of the earlier blocks are left as an earlier
+ * call wrote them. Query blocks are pooled as usual when q is given. Pooling blocks
+ * [0, s) in one call and [s, nkb) in another gives the tables of one full call, bit for
+ * bit. 0 <= kv_block_start <= nkb. For order 2, sparse_attn_hbar is run again afterwards
+ * (it reads every M_j).
+ */
+int sparse_attn_pool_incremental(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 int B, int H, int Nq, int Nk, int d, int block, int order,
+                                 int kv_block_start, float* qbar, float* kbar_t, float* vsum,
+                                 uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
+                                 void* stream);
+
+/*
  * Routing (PISA §2 top-k choice of the critical blocks; SVG-EAR §2 B pooled
  * proxies). Scores s_ij = scale * qbar_i . kbar_j in fp32; blocks are ordered by
  * (s descending, j ascending).

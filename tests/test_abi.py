@@ -85,6 +85,10 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 10, 5, 4, p, p, 10, 0),
         lambda: C.sparse_attn_route_scores(None, 1, 1, 4, 10, 1, 4, p, p, 10, 0),
         lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 0, 1, 4, p, p, 10, 0),
+        lambda: C.sparse_attn_pool_incremental(p, p, p, 1, 1, 64, 640, 64, 64, 0, 11, p, p, p, p,
+                                               p, None, p, 0),
+        lambda: C.sparse_attn_pool_incremental(p, p, p, 1, 1, 64, 640, 64, 64, 1, 2, p, p, p, p,
+                                               p, None, p, 0),
         lambda: C.sparse_attn_wait_selftest(p, 0, p, 0),
         lambda: C.sparse_attn_wait_selftest(None, 10, p, 0),
         lambda: C.sparse_attn_kmeans_sizes(1, 1, 64, 96, 4),

@@ -468,6 +468,30 @@ def test_nothing_kept_and_bad_list_entries(order):
     assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
 
 
+@pytest.mark.parametrize("order", [0, 1])
+def test_incremental_pool_equals_full_pool(order):
+    """A KV cache whose last blocks change: pooling only those blocks over the tables of
+    the old cache gives the tables of a full pool of the new cache, bit for bit."""
+    B, H, d, block, Nk, Nq = 1, 2, 128, 64, 64 * 40 + 24, 300
+    j0 = 33
+    qb = _rand_bits((B, H, Nq, d), 50)
+    kb1, vb1 = _rand_bits((B, H, Nk, d), 51), _rand_bits((B, H, Nk, d), 52)
+    kb2, vb2 = kb1.copy(), vb1.copy()
+    kb2[:, :, j0 * block:] = _rand_bits((B, H, Nk - j0 * block, d), 53)
+    vb2[:, :, j0 * block:] = _rand_bits((B, H, Nk - j0 * block, d), 54)
+    p = A.Problem(B, H, Nq, Nk, d, block, order)
+    t_inc, t_full = A.allocate_tables(p, "cuda"), A.allocate_tables(p, "cuda")
+    q = _dev(qb)
+    A.pool(q, _dev(kb1), _dev(vb1), p, t_inc)
+    A.pool(q, _dev(kb2), _dev(vb2), p, t_inc, kv_block_start=j0)
+    A.pool(q, _dev(kb2), _dev(vb2), p, t_full)
+    torch.cuda.synchronize()
+    for name in ("qbar", "kbar_t", "vsum", "kbar16", "vsum16", "M", "v16"):
+        a, b = getattr(t_inc, name), getattr(t_full, name)
+        if a is not None:
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), name
+
+
 def test_empty_problems_are_no_ops():
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     f = torch.zeros(16, dtype=torch.float32, device="cuda")
