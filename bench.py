@@ -490,7 +490,7 @@ def main():
                               / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
             "clocks": clocks.summary(),
             "gpu_launches": ((5 if w.order == 2 else 4 if w.mode == "ear" else 3)
-                             + (2 * (7 + 7 * w.clusters[2]) + 4 if w.clusters else 0))
+                             + (2 * (7 + 8 * w.clusters[2]) + 4 if w.clusters else 0))
                             * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,

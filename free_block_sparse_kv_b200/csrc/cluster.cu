@@ -19,9 +19,10 @@
 //            error bound of that arithmetic goes on a list instead of being decided;
 //   recheck  the listed tokens in fp64 against every centroid (one CTA each);
 //   hist / scan / scatter   stable counting sort: one warp per chunk of 1024 tokens;
-//   update   one CTA per cluster sums its members in fp64 (the sums of bf16 values are
-//            exact, so the means are the correctly rounded fp64 means) and writes the
-//            bf16 pieces and the fp32 squared norm the next assignment reads.
+//   update   segments of at most 512 sorted members summed in fp64 by one CTA each, then
+//            one CTA per cluster adds its segments (the sums of bf16 values are exact,
+//            so the means are the correctly rounded fp64 means); the bf16 pieces and
+//            fp32 squared norms the next assignment reads follow.
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -39,6 +40,7 @@ constexpr int TCN = 128;                     // centroids per tile
 constexpr int kChunk = 1024;                 // tokens per sorting warp
 constexpr int kSortWarps = 4;
 constexpr int kMaxC = 4096;
+constexpr int kSeg = 512;                    // members per centroid-update segment
 constexpr uint32_t kWaitLimit = 1u << 18;
 
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -440,7 +442,7 @@ __global__ void hist_kernel(const int32_t* __restrict__ labels, int N, int C, in
 // offsets[m] = members of clusters < m; counts becomes the first position of each
 // (chunk, cluster) pair: offsets[m] + members of m in earlier chunks.
 __global__ void scan_kernel(int32_t* __restrict__ counts, int C, int nchunk,
-                            int32_t* __restrict__ offsets) {
+                            int32_t* __restrict__ offsets, int32_t* __restrict__ seg_off) {
   extern __shared__ int32_t ssm[];  // [C] totals
   const int bh = blockIdx.x;
   int32_t* cnt = counts + (size_t)bh * nchunk * C;
@@ -455,13 +457,16 @@ __global__ void scan_kernel(int32_t* __restrict__ counts, int C, int nchunk,
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int acc = 0;
+    int acc = 0, sacc = 0;  // members, and segments of kSeg members, of clusters < m
     for (int m = 0; m < C; ++m) {
       const int v = ssm[m];
       ssm[m] = acc;
+      seg_off[(size_t)bh * (C + 1) + m] = sacc;
       acc += v;
+      sacc += (v + kSeg - 1) / kSeg;
     }
     offsets[(size_t)bh * (C + 1) + C] = acc;
+    seg_off[(size_t)bh * (C + 1) + C] = sacc;
   }
   __syncthreads();
   for (int m = threadIdx.x; m < C; m += blockDim.x) {
@@ -504,54 +509,66 @@ __global__ void scatter_kernel(const int32_t* __restrict__ labels, int N, int C,
 // ---------------------------------------------------------------------------
 // update: each centroid to the fp64 mean of its members; one without members stays
 // ---------------------------------------------------------------------------
-// 512 threads: d / 8 threads per row (eight dimensions each, one 16-byte load), so
-// 512 / (d / 8) member rows are read side by side; member k goes to row lane k mod L.
-// Every sum of bf16 values here is exact in fp64, so the split changes nothing; the
-// lanes are still combined in a fixed order.
+// The sorted members are cut into segments of at most kSeg per cluster (the scan gives
+// each cluster's first segment), so that a very large cluster does not run on one CTA:
+// one CTA sums each segment, then one CTA per cluster adds its segments in order. Every
+// sum of bf16 values here is exact in fp64, so the split changes no bit of the means.
+// Segment CTA: 512 threads, d / 8 per member row (eight dimensions each, one 16-byte
+// load), 512 / (d / 8) member rows side by side, combined in a fixed order.
 constexpr int kUpdThreads = 512;
 
 __global__ void __launch_bounds__(kUpdThreads)
-update_kernel(const uint16_t* __restrict__ x, int N, int d, int C,
-              const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
-              double* __restrict__ cent) {
-  __shared__ double part[kUpdThreads * 8];  // [row lane][d]
-  const int m = blockIdx.x, bh = blockIdx.y;
+segment_sum_kernel(const uint16_t* __restrict__ x, int N, int d, int C, int maxseg,
+                   const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ seg_off, double* __restrict__ part) {
+  __shared__ double lanes_sum[kUpdThreads * 8];  // [row lane][d]
+  const int sg = blockIdx.x, bh = blockIdx.y;
+  const int32_t* so = seg_off + (size_t)bh * (C + 1);
+  if (sg >= so[C]) return;
+  // the segment's cluster: the last m with so[m] <= sg
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    if (so[mid] <= sg) lo = mid; else hi = mid - 1;
+  }
+  const int m = lo;
+  const int32_t* of = offsets + (size_t)bh * (C + 1);
+  const int s = of[m] + (sg - so[m]) * kSeg, e = min(s + kSeg, of[m + 1]);
   const int cpr = d / 8, lanes = kUpdThreads / cpr;
   const int rl = threadIdx.x / cpr, ch = threadIdx.x % cpr;
-  const int s = offsets[(size_t)bh * (C + 1) + m], e = offsets[(size_t)bh * (C + 1) + m + 1];
-  if (e == s) return;  // no members: the centroid stays
   const int32_t* pr = perm + (size_t)bh * N;
   const uint16_t* xb = x + (size_t)bh * N * d + ch * 8;
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  auto add = [&](const uint4& w) {
+  for (int k = s + rl; k < e; k += lanes) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(xb + (size_t)__ldg(pr + k) * d));
     const uint32_t v[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       acc[2 * q] += (double)bf16_lo(v[q]);
       acc[2 * q + 1] += (double)bf16_hi(v[q]);
     }
-  };
-  int k = s + rl;
-  for (; k + 3 * lanes < e; k += 4 * lanes) {  // four member rows in flight
-    int r4[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) r4[u] = __ldg(pr + k + u * lanes);
-    uint4 w4[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      w4[u] = __ldg(reinterpret_cast<const uint4*>(xb + (size_t)r4[u] * d));
-#pragma unroll
-    for (int u = 0; u < 4; ++u) add(w4[u]);
   }
-  for (; k < e; k += lanes) add(__ldg(reinterpret_cast<const uint4*>(xb + (size_t)__ldg(pr + k) * d)));
 #pragma unroll
-  for (int q = 0; q < 8; ++q) part[rl * d + ch * 8 + q] = acc[q];
+  for (int q = 0; q < 8; ++q) lanes_sum[rl * d + ch * 8 + q] = acc[q];
   __syncthreads();
   if (threadIdx.x < d) {
     double sum = 0.0;
-    for (int l = 0; l < lanes; ++l) sum += part[l * d + threadIdx.x];
-    cent[((size_t)bh * C + m) * d + threadIdx.x] = sum / (double)(e - s);
+    for (int l = 0; l < lanes; ++l) sum += lanes_sum[l * d + threadIdx.x];
+    part[((size_t)bh * maxseg + sg) * d + threadIdx.x] = sum;
   }
+}
+
+__global__ void combine_kernel(int d, int C, int maxseg, const int32_t* __restrict__ offsets,
+                               const int32_t* __restrict__ seg_off,
+                               const double* __restrict__ part, double* __restrict__ cent) {
+  const int m = blockIdx.x, bh = blockIdx.y, i = threadIdx.x;
+  const int32_t* of = offsets + (size_t)bh * (C + 1);
+  const int32_t* so = seg_off + (size_t)bh * (C + 1);
+  const int cnt = of[m + 1] - of[m];
+  if (cnt == 0 || i >= d) return;  // no members: the centroid stays
+  double sum = 0.0;
+  for (int sg = so[m]; sg < so[m + 1]; ++sg) sum += part[((size_t)bh * maxseg + sg) * d + i];
+  cent[((size_t)bh * C + m) * d + i] = sum / (double)cnt;
 }
 
 // ---------------------------------------------------------------------------
@@ -643,8 +660,10 @@ void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
   const size_t bh = (size_t)B * H;
   const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
   sizes[0] = bh * C * d * sizeof(double);
-  sizes[1] = align256(bh * 2 * Cpad * d * 2) + bh * Cpad * 4;
-  sizes[2] = align256(bh * nchunk * C * 4) + align256(bh * N * 4) + bh * 4;
+  const size_t maxseg = (size_t)km::cdiv(N, km::kSeg) + C;
+  sizes[1] = align256(bh * 2 * Cpad * d * 2) + align256(bh * Cpad * 4) + bh * maxseg * d * 8;
+  sizes[2] = align256(bh * nchunk * C * 4) + align256(bh * N * 4) + align256(bh * 4) +
+             bh * (C + 1) * 4;
 }
 
 cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
@@ -652,15 +671,21 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   const int bh = a.B * a.H, C = a.C, d = a.d, N = a.N;
   const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
   // carve the work buffers
-  a.pieces = reinterpret_cast<uint16_t*>(a.cwork);
-  a.cnorm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.cwork) +
-                                     align256((size_t)bh * 2 * Cpad * d * 2));
+  const int maxseg = km::cdiv(N, km::kSeg) + C;
+  uint8_t* cw = reinterpret_cast<uint8_t*>(a.cwork);
+  a.pieces = reinterpret_cast<uint16_t*>(cw);
+  cw += align256((size_t)bh * 2 * Cpad * d * 2);
+  a.cnorm = reinterpret_cast<float*>(cw);
+  cw += align256((size_t)bh * Cpad * 4);
+  double* part = reinterpret_cast<double*>(cw);
   uint8_t* iw = reinterpret_cast<uint8_t*>(a.iwork);
   a.counts = reinterpret_cast<int32_t*>(iw);
   iw += align256((size_t)bh * nchunk * C * 4);
   a.amb_list = reinterpret_cast<int32_t*>(iw);
   iw += align256((size_t)bh * N * 4);
   a.amb_cnt = reinterpret_cast<int32_t*>(iw);
+  iw += align256((size_t)bh * 4);
+  int32_t* seg_off = reinterpret_cast<int32_t*>(iw);
 
   const int sort_smem = km::kSortWarps * C * 4;
   cudaError_t e;
@@ -681,7 +706,7 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   auto sort = [&]() -> cudaError_t {
     km::hist_kernel<<<gsort, 32 * km::kSortWarps, sort_smem, st>>>(a.labels, N, C, nchunk,
                                                                    a.counts);
-    km::scan_kernel<<<bh, 256, C * 4, st>>>(a.counts, C, nchunk, a.offsets);
+    km::scan_kernel<<<bh, 256, C * 4, st>>>(a.counts, C, nchunk, a.offsets, seg_off);
     km::scatter_kernel<<<gsort, 32 * km::kSortWarps, sort_smem, st>>>(a.labels, N, C, nchunk,
                                                                       a.counts, a.perm);
     return cudaGetLastError();
@@ -696,8 +721,9 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   for (int t = 0; t < a.iters; ++t) {
     if ((e = assign()) != cudaSuccess) return e;
     if ((e = sort()) != cudaSuccess) return e;
-    km::update_kernel<<<dim3(C, bh), km::kUpdThreads, 0, st>>>(a.x, N, d, C, a.perm, a.offsets,
-                                                                a.cent);
+    km::segment_sum_kernel<<<dim3(maxseg, bh), km::kUpdThreads, 0, st>>>(
+        a.x, N, d, C, maxseg, a.perm, a.offsets, seg_off, part);
+    km::combine_kernel<<<dim3(C, bh), d, 0, st>>>(d, C, maxseg, a.offsets, seg_off, part, a.cent);
     if ((e = prep()) != cudaSuccess) return e;
   }
   if ((e = assign()) != cudaSuccess) return e;

@@ -223,7 +223,7 @@ int sparse_attn_route_scores(const float* scores, int B, int H, int nqb, int nkb
  * with members moves to their mean (fp64; the others stay); after `iters` updates the
  * tokens are assigned once more. The assignment runs on the tensor cores (fp32 scores
  * from a two-piece bf16 split of the fp64 centroids); a token whose two best scores lie
- * within that arithmetic's error bound is decided again in fp64. 7 + 7 * iters
+ * within that arithmetic's error bound is decided again in fp64. 7 + 8 * iters
  * launches on the stream.
  *
  * sparse_attn_permute_rows: rows of row_bytes bytes (a multiple of 16) per (b, h);
