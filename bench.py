@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--graphs", action="store_true",
+                    help="also time the step replayed from CUDA graphs (reported as 'graph')")
     ap.add_argument("--heads", type=int, default=0,
                     help="run on this many heads instead of the workload's (profiler captures)")
     return ap.parse_args()
@@ -393,6 +395,27 @@ def main():
     # error-aware routing: the probe's share of the route stage (events 1 -> 4)
     ear_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs])) if w.mode == "ear" else None
 
+    # The same steps replayed from CUDA graphs (one per denoising step of the cycle): no
+    # host work per launch. Reported beside the eager figure.
+    graph = None
+    if args.graphs:
+        graphs = {st: op.capture(q, k, v, step=st) for st in sorted(set(steps_cycle))}
+        for st in steps_cycle:
+            graphs[st].replay()
+        torch.cuda.synchronize(dev)
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.steps):
+            graphs[steps_cycle[i % len(steps_cycle)]].replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        gms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+        graph = {"ms_per_step": gms, "value": D.weak_scaling_value(w.dense_flops(), world, gms),
+                 "unit": UNIT, "graphs": len(graphs)}
+        del graphs
+
     # World model: the frames before the chunk form a KV cache whose pooled tables carry
     # over between chunks; only the chunk's own blocks are pooled (labelled secondary row).
     secondary = None
@@ -511,6 +534,8 @@ def main():
                                   / FP32_PEAK_TFLOPS, "fp32_peak_tflops": FP32_PEAK_TFLOPS}
         if secondary is not None:
             line["secondary"] = secondary
+        if graph is not None:
+            line["graph"] = graph
         if cluster_ms is not None:
             line["stages_ms"]["cluster"] = cluster_ms[0]
             line["stages_ms"]["unpermute"] = cluster_ms[1]

@@ -282,6 +282,21 @@ class BlockSparseAttention:
             route(p, t, kv_idx, kv_cnt, self.mode, self.rho, self.tau, stream=stream)
         forward(q, k, v, p, t, kv_idx, kv_cnt, out, err_flag=self.err_flag, stream=stream)
 
+    def capture(self, q, k, v, step: int = 0) -> "torch.cuda.CUDAGraph":
+        """Record one call on these buffers as a CUDA graph: replaying it repeats every
+        launch of the call (for the step given) on whatever the buffers hold then, with no
+        host work per launch."""
+        dev = self.out.device
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):   # one eager call first: attributes, tensor maps
+            self(q, k, v, step=step)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(q, k, v, step=step)
+        return g
+
     def run_from_host(self, q_h, k_h, v_h, out_h, step: int = 0, chunks: int = 10):
         """One call with Q, K, V in (pinned) host memory and the output written to the
         (pinned) host tensor ``out_h``. The heads are split into ``chunks`` ranges: the

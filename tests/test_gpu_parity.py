@@ -564,13 +564,49 @@ def test_host_call_equals_device_call(name, small_inputs):
         assert torch.equal(out_h, want.cpu()), chunks
 
 
-def test_repeat_calls_are_bitwise_deterministic(small_inputs):
-    w, qb, kb, vb = small_inputs("dit-small")
+@pytest.mark.parametrize("name", ["dit-small", "ear-small", "kmeans-small", "hybrid-small",
+                                  "longvideo-small"])
+def test_graph_replay_equals_eager_call(name, small_inputs):
+    """A captured call replays the same launches: equal output, also after the inputs
+    change in place."""
+    w, qb, kb, vb = small_inputs(name)
+    step = w.steps[-1] if w.mode == "structured" else 0
     q, k, v = _dev(qb), _dev(kb), _dev(vb)
-    _, a = _run(w, q, k, v)
+    op, out = _run(w, q, k, v, step=step)
+    want = out.clone()
+    g = op.capture(q, k, v, step=step)
+    op.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(op.out, want)
+    k.copy_(torch.roll(k, 7, dims=2))               # new keys, same buffers
+    _, want2 = _run(w, q, k, v, step=step)
+    want2 = want2.clone()
+    op.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    op.check()
+    assert torch.equal(op.out, want2)
+    del g
+
+
+@pytest.mark.parametrize("name", ["dit-small", "ear-small", "kmeans-small", "hybrid-small",
+                                  "worldmodel-small"])
+def test_repeat_calls_are_bitwise_deterministic(name, small_inputs):
+    w, qb, kb, vb = small_inputs(name)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    op, a = _run(w, q, k, v)
     a = a.clone()
+    extra = [op.tables.scores.clone()] if w.mode == "ear" else []
+    if w.clusters:
+        extra += [op.cl_q.perm.clone(), op.cl_k.centroids.clone()]
     _, b = _run(w, q, k, v)
     assert torch.equal(a, b)
+    op2, _ = _run(w, q, k, v)
+    if w.mode == "ear":
+        assert torch.equal(op2.tables.scores, extra[0])
+    if w.clusters:
+        assert torch.equal(op2.cl_q.perm, extra[-2]) and torch.equal(op2.cl_k.centroids, extra[-1])
 
 
 @pytest.mark.parametrize("mode", ["topk", "mass"])
