@@ -299,18 +299,27 @@ class BlockSparseAttention:
 
     def run_from_host(self, q_h, k_h, v_h, out_h, step: int = 0, chunks: int = 10):
         """One call with Q, K, V in (pinned) host memory and the output written to the
-        (pinned) host tensor ``out_h``. The heads are split into ``chunks`` ranges: the
+        (pinned) host tensor ``out_h``.
+
+        The heads are split into ranges of four (``chunks`` ranges or fewer): the
         host-to-device copies run ahead on one stream, each range is computed on the
-        current stream as soon as its inputs are in, and its output goes back on a
-        third stream while the next range computes. Returns after enqueueing; the
-        current stream waits for the last copy back."""
+        current stream as soon as its inputs are in, and its output goes back on a third
+        stream while the next range computes. Successive calls alternate between two
+        sets of device input and output buffers, so the next call's inputs load while
+        this call computes and its outputs drain while the next one computes. Returns
+        after enqueueing; call :meth:`wait_host_copies` (or synchronise) before reading
+        ``out_h``."""
         p = self.p
         dev = self.out.device
-        if getattr(self, "_dev_in", None) is None:
-            self._dev_in = tuple(torch.empty(x.shape, dtype=x.dtype, device=dev)
-                                 for x in (q_h, k_h, v_h))
+        if getattr(self, "_sets", None) is None:
+            mk = lambda x: torch.empty(x.shape, dtype=x.dtype, device=dev)
+            self._sets = [dict(q=mk(q_h), k=mk(k_h), v=mk(v_h), out=torch.empty_like(self.out),
+                               free_in=None, free_out=None) for _ in range(2)]
             self._h2d, self._d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        q, k, v = self._dev_in
+            self._call = 0
+        st = self._sets[self._call % 2]
+        self._call += 1
+        q, k, v, out = st["q"], st["k"], st["v"], st["out"]
         cs = torch.cuda.current_stream(dev)
         # Head ranges start at multiples of 4 heads of the flattened (batch, head) index,
         # so that every per-head table slice starts on a 16-byte boundary (the C ABI's
@@ -320,32 +329,41 @@ class BlockSparseAttention:
         ranges = [(b, h0, min(p.H, h0 + step_h)) for b in range(p.B)
                   for h0 in range(0, p.H, step_h)]
         if any((b * p.H + h0) % 4 for b, h0, _ in ranges):
-            ranges = [(b, 0, p.H) for b in range(p.B)] if (p.H % 4 == 0) else None
-        if ranges is None:
-            for dst, src in ((q, q_h), (k, k_h), (v, v_h)):
-                dst.copy_(src, non_blocking=True)
-            self._run(q, k, v, self.out, None, step, None)
-            out_h.copy_(self.out, non_blocking=True)
-            return out_h
-        self._h2d.wait_stream(cs)                      # inputs may still be read by an earlier call
+            ranges = [(b, 0, p.H) for b in range(p.B)] if (p.H % 4 == 0) else [None]
+        # this set's inputs may still be read by the compute of the call before last, and
+        # its output may still be draining to the host
+        if st["free_in"] is not None:
+            self._h2d.wait_event(st["free_in"])
+        if st["free_out"] is not None:
+            cs.wait_event(st["free_out"])
         ready = []
         with torch.cuda.stream(self._h2d):
-            for b, h0, h1 in ranges:
+            for r in ranges:
+                sl = (slice(None),) if r is None else (r[0], slice(r[1], r[2]))
                 for dst, src in ((q, q_h), (k, k_h), (v, v_h)):
-                    dst[b, h0:h1].copy_(src[b, h0:h1], non_blocking=True)
+                    dst[sl].copy_(src[sl], non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(self._h2d)
                 ready.append(ev)
-        for (b, h0, h1), ev in zip(ranges, ready):
+        for r, ev in zip(ranges, ready):
             cs.wait_event(ev)
-            self._run(q, k, v, self.out, (b, h0, h1), step, None)
+            self._run(q, k, v, out, r, step, None)
             done = torch.cuda.Event()
             done.record(cs)
             self._d2h.wait_event(done)
             with torch.cuda.stream(self._d2h):
-                out_h[b, h0:h1].copy_(self.out[b, h0:h1], non_blocking=True)
-        cs.wait_stream(self._d2h)
+                sl = (slice(None),) if r is None else (r[0], slice(r[1], r[2]))
+                out_h[sl].copy_(out[sl], non_blocking=True)
+        st["free_in"] = torch.cuda.Event()
+        st["free_in"].record(cs)
+        st["free_out"] = torch.cuda.Event()
+        st["free_out"].record(self._d2h)
         return out_h
+
+    def wait_host_copies(self):
+        """Make the current stream wait for every output copy to the host issued so far."""
+        if getattr(self, "_d2h", None) is not None:
+            torch.cuda.current_stream(self.out.device).wait_stream(self._d2h)
 
     def check(self):
         """Raise if a bounded device wait of an earlier call gave up (synchronises)."""
