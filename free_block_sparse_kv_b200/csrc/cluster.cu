@@ -39,7 +39,6 @@ constexpr int TT = 128;                      // tokens per assignment tile
 constexpr int TCN = 128;                     // centroids per tile
 constexpr int kChunk = 1024;                 // tokens per sorting warp
 constexpr int kSortWarps = 4;
-constexpr int kMaxC = 4096;
 constexpr int kSeg = 512;                    // members per centroid-update segment
 constexpr uint32_t kWaitLimit = 1u << 18;
 

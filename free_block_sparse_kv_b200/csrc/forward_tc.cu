@@ -694,7 +694,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       int u = 0;
       bool ok = true;
       while (ok) {
-        const Step s = gen.next<ORDER>(c, nkb);
+        const Step s = gen.template next<ORDER>(c, nkb);
         for (int i = 0; i < s.nunits && ok; ++i) {
           const int v = u + i;
           if (v >= NU) ok = wt.fast(bar(c.empty[v % NU]), ((v / NU) - 1) & 1, 1);
@@ -775,7 +775,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         ok = wt.fast(bar(c.full[slot]), (u / NU) & 1, 4);
         if (!ok) break;
         const int rec = c.evq[slot].x;  // ordered by the full-barrier wait (asm with memory clobber)
-        const int type = rec & 15, ck = (rec >> 4) & 15, pk = (rec >> 8) & 15;
+        const int type = rec & 15, ck = (rec >> 4) & 15;
         const int cm = (rec >> 12) & 3, pm = (rec >> 14) & 3, nun = (rec >> 16) & 3;
         if (type == stEnd) break;
         const int slot2 = (u + 1) % NU;
