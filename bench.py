@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--graphs", action="store_true",
                     help="also time the step replayed from CUDA graphs (reported as 'graph')")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="key-range splits of the forward (0: the library's choice)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run on this many heads instead of the workload's (profiler captures)")
     return ap.parse_args()
@@ -335,7 +337,7 @@ def main():
     op = A.BlockSparseAttention(p, w.mode, rho=w.rho, tau=w.tau,
                                 geometry=geometry if w.mode == "structured" else None,
                                 out_dtype=torch.float32, device=dev,
-                                clusters=w.clusters or None)
+                                clusters=w.clusters or None, splits=args.splits or None)
     stream = torch.cuda.current_stream(dev)
     steps_cycle = w.steps if w.mode == "structured" else (0,)
 
@@ -360,7 +362,7 @@ def main():
                 ev[4].record(stream)
             A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
         ev[2].record(stream)
-        A.forward(qq, kk, vv, p, op.tables, op.kv_idx, op.kv_cnt, out)
+        op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, qq, kk, vv, out)
         ev[3].record(stream)
         if w.clusters:
             A.permute_rows(op.out_p, op.cl_q.perm, op.out, gather=False)
@@ -433,7 +435,7 @@ def main():
             e[1].record(stream)
             A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
             e[2].record(stream)
-            A.forward(q, k, v, p, op.tables, op.kv_idx, op.kv_cnt, op.out)
+            op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, q, k, v, op.out)
             e[3].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -514,8 +516,10 @@ def main():
                               / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
             "clocks": clocks.summary(),
             "gpu_launches": ((5 if w.order == 2 else 4 if w.mode == "ear" else 3)
+                             + (1 if op.last_splits > 1 else 0)  # the merge of the splits
                              + (2 * (7 + 8 * w.clusters[2]) + 4 if w.clusters else 0))
                             * args.steps,
+            "forward_splits": op.last_splits,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

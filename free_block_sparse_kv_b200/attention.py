@@ -7,6 +7,7 @@ Torch only provides device memory and the stream; each stage is one call into
 from __future__ import annotations
 
 import dataclasses
+import functools
 import math
 from typing import Optional
 
@@ -171,13 +172,32 @@ def structured_mask(p: Problem, kv_idx, kv_cnt, frame_tokens, n_frames, window, 
 
 
 def forward(q, k, v, p: Problem, t: Tables, kv_idx, kv_cnt, out, scale=None, err_flag=None,
-            stream=None):
+            stream=None, splits: int = 1, work=None):
+    """The forward; ``splits`` > 1 shares every query tile's key blocks among that many
+    CTAs and merges their partial results (``work``: fp32 scratch of at least
+    ``sparse_attn_forward_work_bytes`` bytes)."""
     scale = 1.0 / math.sqrt(p.d) if scale is None else scale
     dt = C.SA_OUT_F32 if out.dtype == torch.float32 else C.SA_OUT_BF16
     m = t.hbar16 if p.order == 2 else t.M
-    C.sparse_attn_forward(q, k, t.v16, t.kbar16, t.vsum16, m, kv_idx, kv_cnt, kv_idx.shape[-1],
-                          p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, scale, out, dt, err_flag,
-                          stream)
+    if splits > 1:
+        C.sparse_attn_forward_split(q, k, t.v16, t.kbar16, t.vsum16, m, kv_idx, kv_cnt,
+                                    kv_idx.shape[-1], p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order,
+                                    scale, splits, work, out, dt, err_flag, stream)
+    else:
+        C.sparse_attn_forward(q, k, t.v16, t.kbar16, t.vsum16, m, kv_idx, kv_cnt, kv_idx.shape[-1],
+                              p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, scale, out, dt, err_flag,
+                              stream)
+
+
+@functools.lru_cache(maxsize=256)
+def _plan(B, H, Nq, Nk, d, block, sms):
+    return C.sparse_attn_forward_split_plan(B, H, Nq, Nk, d, block, sms)
+
+
+def split_plan(p: Problem, device) -> tuple:
+    """(splits, work bytes) the library picks for this shape on ``device``'s SMs."""
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    return _plan(p.B, p.H, p.Nq, p.Nk, p.d, p.block, sms)
 
 
 class BlockSparseAttention:
@@ -191,13 +211,15 @@ class BlockSparseAttention:
     n_anchors, period, q_frame0) at the step passed to :meth:`__call__`.
     ``clusters`` = (C_q, C_k, iters) first clusters Q and K by k-means and runs the
     three stages on their group-major copies (V follows K), returning the output in the
-    original query order.
+    original query order. ``splits`` = key-range splits of the forward: None lets the
+    library choose per call shape (:func:`split_plan`), an int fixes it.
     """
 
     def __init__(self, p: Problem, mode: str, rho=(1, 4), tau=0.9, geometry=None,
-                 out_dtype=torch.float32, device="cuda", clusters=None):
+                 out_dtype=torch.float32, device="cuda", clusters=None, splits=None):
         self.p, self.mode, self.rho, self.tau, self.geometry = p, mode, rho, tau, geometry
         self.clusters = clusters
+        self.splits, self._work, self.last_splits = splits, None, 1
         if mode == "topk_cov" and p.order != 2:
             raise ValueError("covariance-aware routing needs order 2 (the covariance norms)")
         if mode in ("topk", "topk_cov", "ear"):
@@ -280,7 +302,25 @@ class BlockSparseAttention:
             if self.mode == "ear":
                 ear_scores(k, v, p, t, err_flag=self.err_flag, stream=stream)
             route(p, t, kv_idx, kv_cnt, self.mode, self.rho, self.tau, stream=stream)
-        forward(q, k, v, p, t, kv_idx, kv_cnt, out, err_flag=self.err_flag, stream=stream)
+        self.forward_stage(p, t, kv_idx, kv_cnt, q, k, v, out, stream)
+
+    def forward_stage(self, p, t, kv_idx, kv_cnt, q, k, v, out, stream=None):
+        """The forward of one (sub-)problem, split as :attr:`splits` says. The automatic
+        choice is made for the whole problem, also when a head range runs on its own, so
+        that every form of the call computes each row the same way (bit for bit). The
+        scratch for the partial results is kept and only grows."""
+        S = self.splits if self.splits is not None else split_plan(self.p, self.out.device)[0]
+        work = None
+        if S > 1:
+            need = C.sparse_attn_forward_work_bytes(p.B, p.H, p.Nq, p.d, S) // 4
+            if self._work is None or self._work.numel() < need:
+                self._work = torch.empty(need, dtype=torch.float32, device=self.out.device)
+            work = self._work
+            if isinstance(stream, torch.cuda.Stream):
+                work.record_stream(stream)
+        self.last_splits = S
+        forward(q, k, v, p, t, kv_idx, kv_cnt, out, err_flag=self.err_flag, stream=stream,
+                splits=S, work=work)
 
     def capture(self, q, k, v, step: int = 0) -> "torch.cuda.CUDAGraph":
         """Record one call on these buffers as a CUDA graph: replaying it repeats every

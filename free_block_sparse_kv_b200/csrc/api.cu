@@ -1,9 +1,13 @@
 // C ABI of the library: argument checks on the host, then one kernel launch per
 // entry point on the caller's stream. No allocation, no synchronisation.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <functional>
+#include <queue>
 #include <string>
+#include <vector>
 
 #include "../../include/sparse_attn.h"
 #include "launch.h"
@@ -416,7 +420,108 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v1
   if (int rc = check_device()) return rc;
   sa::ForwardArgs p{q, k, v16, kbar16, vsum16, order >= 1 ? M : nullptr, kv_idx, kv_cnt, cap,
                     B, H, Nq, Nk, d, block, order, cdiv(Nq, block), nkb, scale, out, out_dtype,
-                    err_flag};
+                    err_flag, 1, nullptr};
+  return launched(sa::launch_forward(p, static_cast<cudaStream_t>(stream)), "forward launch");
+}
+
+int sparse_attn_forward_work_bytes(int B, int H, int Nq, int d, int splits, size_t* bytes) {
+  if (int rc = check_shape(B, H, Nq, 1, d, 64)) return rc;
+  SA_REQUIRE(splits >= 1 && splits <= SA_MAX_SPLITS, "splits must be in [1, %d] (got %d)",
+             SA_MAX_SPLITS, splits);
+  SA_REQUIRE(bytes != nullptr, "bytes must be non-null");
+  *bytes = sa::forward_work_floats(B, H, Nq, d, splits) * sizeof(float);
+  return ok();
+}
+
+int sparse_attn_forward_split_plan(int B, int H, int Nq, int Nk, int d, int block, int sms,
+                                   int* splits, size_t* work_bytes) {
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(splits != nullptr && work_bytes != nullptr, "splits and work_bytes must be non-null");
+  SA_REQUIRE(sms >= 0, "sms must be >= 0");
+  if (sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(SA_ERR_LAUNCH, "SM count: %s", cudaGetErrorString(e));
+  }
+  *splits = 1;
+  *work_bytes = 0;
+  const long long bh = (long long)B * H;
+  if (bh == 0 || Nq == 0 || Nk == 0) return ok();
+  // CTAs of the unsplit grid: per (batch, head), the full pairs of 128-row tiles and a
+  // last pair with one or two tiles (cost 1/2 or 1 of a full one).
+  const int nx = cdiv(Nq, 256), ntl = cdiv(cdiv(Nk, block), 64);
+  const int last_tiles = cdiv(Nq - (nx - 1) * 256, 128);
+  if (bh * nx >= 8LL * sms) return ok();  // many waves: the last one costs little
+  // Model: every split CTA costs 1/S of its unsplit cost plus a fixed setup and drain
+  // (about eight work items against ~nkb items per unsplit CTA); CTAs start in grid order
+  // on the first SM that is free. The time of a split count is the makespan, plus a
+  // small charge per split for the merge.
+  const double setup = 8.0 / std::max(1, cdiv(Nk, block));
+  auto makespan = [&](int S) {
+    std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+    for (int i = 0; i < sms; ++i) free_at.push(0.0);
+    double end = 0.0;
+    auto run = [&](double cost, long long n) {
+      for (long long i = 0; i < n; ++i) {
+        const double t = free_at.top() + cost;
+        free_at.pop();
+        free_at.push(t);
+        end = std::max(end, t);
+      }
+    };
+    run(1.0 / S + setup, bh * (nx - 1) * S);
+    run(0.5 * last_tiles / S + setup, bh * S);
+    return end + 0.003 * (S - 1);
+  };
+  double best = makespan(1);
+  for (int S = 2; S <= std::min(ntl, SA_MAX_SPLITS); ++S) {
+    if (bh * nx * S > 400000) break;
+    const double t = makespan(S);
+    if (t < 0.97 * best) {
+      best = t;
+      *splits = S;
+    }
+  }
+  *work_bytes = sa::forward_work_floats(B, H, Nq, d, *splits) * sizeof(float);
+  return ok();
+}
+
+int sparse_attn_forward_split(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
+                              const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H,
+                              int Nq, int Nk, int d, int block, int order, float scale, int splits,
+                              float* work, void* out, int out_dtype, int32_t* err_flag,
+                              void* stream) {
+  SA_REQUIRE(splits >= 1 && splits <= SA_MAX_SPLITS, "splits must be in [1, %d] (got %d)",
+             SA_MAX_SPLITS, splits);
+  if (splits == 1)
+    return sparse_attn_forward(q, k, v16, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H, Nq, Nk, d,
+                               block, order, scale, out, out_dtype, err_flag, stream);
+  if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
+  SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
+  SA_REQUIRE(out_dtype == SA_OUT_F32 || out_dtype == SA_OUT_BF16, "out_dtype must be F32 or BF16");
+  SA_REQUIRE(std::isfinite(scale), "scale must be finite");
+  if ((long long)B * H * Nq == 0) return ok();
+  SA_REQUIRE(Nk >= 1, "Nk must be >= 1 when there are queries");
+  const int nkb = cdiv(Nk, block);
+  SA_REQUIRE(nkb <= SA_MAX_KV_BLOCKS, "nkb must be <= %d (got %d)", SA_MAX_KV_BLOCKS, nkb);
+  SA_REQUIRE(cap >= 0, "cap must be >= 0");
+  SA_REQUIRE_PTR(q);
+  SA_REQUIRE_PTR(k);
+  SA_REQUIRE_PTR(v16);
+  SA_REQUIRE_PTR(kbar16);
+  SA_REQUIRE_PTR(vsum16);
+  if (order >= 1) SA_REQUIRE_PTR(M);
+  SA_REQUIRE_PTR(kv_idx);
+  SA_REQUIRE_PTR(kv_cnt);
+  SA_REQUIRE_PTR(work);
+  SA_REQUIRE_PTR(out);
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
+  if (int rc = check_device()) return rc;
+  sa::ForwardArgs p{q, k, v16, kbar16, vsum16, order >= 1 ? M : nullptr, kv_idx, kv_cnt, cap,
+                    B, H, Nq, Nk, d, block, order, cdiv(Nq, block), nkb, scale, out, out_dtype,
+                    err_flag, splits, work};
   return launched(sa::launch_forward(p, static_cast<cudaStream_t>(stream)), "forward launch");
 }
 

@@ -91,21 +91,27 @@ struct Params {
   int32_t* err_flag;
   int cap, Nq, Nk, nqb, nkb, out_dtype;
   int nx, nbh;  // CTAs (pairs of query tiles) per (batch, head); batch x heads
+  int nsplit;   // key-range splits per pair of query tiles (1: no split)
+  float* part;  // nsplit > 1: partial results [nsplit][nbh][Nq][D] fp32, then (m, l) pairs
   float scale;
 };
 
-// The CTA's pair of query tiles and its (batch, head). The grid is one-dimensional and
-// puts every (batch, head)'s last pair, which may hold fewer rows, after all full pairs,
-// so that the shorter CTAs fill the last wave.
-SA_DEVI void cta_coords(const Params& p, int& x, int& bh) {
+// The CTA's pair of query tiles, its (batch, head) and its key-range split. The grid is
+// one-dimensional and puts every (batch, head)'s last pair, which may hold fewer rows,
+// after all full pairs, so that the shorter CTAs fill the last wave. Neighbouring CTAs
+// share (batch, head) and split, hence their keys and values in L2.
+SA_DEVI void cta_coords(const Params& p, int& x, int& bh, int& split) {
   const int L = blockIdx.x, nfull = p.nx - 1;
-  if (L < nfull * p.nbh) {
+  int r;
+  if (L < nfull * p.nbh * p.nsplit) {
     x = L % nfull;
-    bh = L / nfull;
+    r = L / nfull;
   } else {
     x = p.nx - 1;
-    bh = L - nfull * p.nbh;
+    r = L - nfull * p.nbh * p.nsplit;
   }
+  split = r % p.nsplit;
+  bh = r / p.nsplit;
 }
 
 struct Ctl {  // control block in shared memory
@@ -118,6 +124,7 @@ struct Ctl {  // control block in shared memory
   uint32_t tmem_base;
   int abort;
   int tvalid;               // bit t: tile t has rows below Nq
+  int jlo, jhi, split;      // key blocks of this CTA's split: [jlo, jhi)
   uint32_t kept[NT][2][MAXW];  // kept blocks of each query block (half) of each tile
 };
 static_assert(sizeof(Ctl) <= 2048, "control block");
@@ -129,35 +136,49 @@ struct Item {
   int half;     // EXACT, block 128: which 64 keys of the block
 };
 
-SA_DEVI uint32_t valid_bits(int w, int nkb) {
-  const int lo = w * 32;
-  return lo + 32 <= nkb ? 0xffffffffu : (lo < nkb ? (1u << (nkb - lo)) - 1u : 0u);
+// Key blocks [jlo, jhi) of a split: whole centroid tiles of KC blocks, shared out evenly.
+SA_DEVI void split_range(int split, int nsplit, int nkb, int& jlo, int& jhi) {
+  const int ntl = (nkb + KC - 1) / KC;
+  jlo = min(nkb, (int)((long long)split * ntl / nsplit) * KC);
+  jhi = min(nkb, (int)((long long)(split + 1) * ntl / nsplit) * KC);
+}
+
+// Blocks j of word w (j = 32 w + bit) inside the CTA's key range [jlo, jhi).
+SA_DEVI uint32_t range_bits(int w, int jlo, int jhi) {
+  const int a = max(jlo - 32 * w, 0), b = min(jhi - 32 * w, 32);
+  if (b <= a) return 0u;
+  return (b - a == 32 ? 0xffffffffu : (1u << (b - a)) - 1u) << a;
 }
 // Blocks of word w that some query block of tile t skips / keeps.
-SA_DEVI uint32_t skip_word(const Ctl& c, int t, int w, int nkb) {
+SA_DEVI uint32_t skip_word(const Ctl& c, int t, int w) {
   if (!((c.tvalid >> t) & 1)) return 0u;
-  return ~(c.kept[t][0][w] & c.kept[t][1][w]) & valid_bits(w, nkb);
+  return ~(c.kept[t][0][w] & c.kept[t][1][w]) & range_bits(w, c.jlo, c.jhi);
 }
-SA_DEVI uint32_t kept_word(const Ctl& c, int t, int w, int nkb) {
+SA_DEVI uint32_t kept_word(const Ctl& c, int t, int w) {
   if (!((c.tvalid >> t) & 1)) return 0u;
-  return (c.kept[t][0][w] | c.kept[t][1][w]) & valid_bits(w, nkb);
+  return (c.kept[t][0][w] | c.kept[t][1][w]) & range_bits(w, c.jlo, c.jhi);
 }
-SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct, int nkb) {
-  return (uint64_t)skip_word(c, t, 2 * ct, nkb) | ((uint64_t)skip_word(c, t, 2 * ct + 1, nkb) << 32);
+SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct) {
+  return (uint64_t)skip_word(c, t, 2 * ct) | ((uint64_t)skip_word(c, t, 2 * ct + 1) << 32);
 }
 
 // The walk over work items; identical in every role. Union masks of the current
-// centroid tile (phase 0) or 32-block word (phase 1) are held in registers.
+// centroid tile (phase 0) or 32-block word (phase 1) are held in registers. It covers
+// the key blocks [jlo, jhi) of the CTA's split (every block when there is one split).
 template <int BLK>
 struct Walk {
   int phase = 0, tile = 0, word = -1, half = 0, jcur = 0, mcur = 0;
+  SA_DEVI void start(const Ctl& c) {
+    tile = c.jlo / KC;
+    word = c.jlo / 32 - 1;
+  }
   int gmask = 0;       // order 2: tiles with a skipped block so far
   bool in_tile = false, gdone = false;
   uint64_t tmask = 0, sk0 = 0, sk1 = 0;  // phase 0: union / per-tile skipped blocks
   uint32_t kmask = 0, kw0 = 0, kw1 = 0;  // phase 1: union / per-tile kept blocks
   template <int ORDER>
   SA_DEVI Item next(const Ctl& c, int nkb) {
-    const int ntiles = (nkb + KC - 1) / KC;
+    const int ntiles = (c.jhi + KC - 1) / KC;
     while (true) {
       if (phase == 0) {
         if (!in_tile) {
@@ -169,8 +190,8 @@ struct Walk {
             phase = 1;
             continue;
           }
-          sk0 = skip64(c, 0, tile, nkb);
-          sk1 = skip64(c, 1, tile, nkb);
+          sk0 = skip64(c, 0, tile);
+          sk1 = skip64(c, 1, tile);
           tmask = sk0 | sk1;
           if (tmask) {
             in_tile = true;
@@ -195,12 +216,12 @@ struct Walk {
         return Item{kExact, jcur, mcur, 1};
       }
       while (!kmask) {
-        if (++word >= (nkb + 31) / 32) {
-          word = (nkb + 31) / 32;  // stays at the end: later calls return kNone again
+        if (++word >= (c.jhi + 31) / 32) {
+          word = (c.jhi + 31) / 32;  // stays at the end: later calls return kNone again
           return Item{kNone, 0, 0, 0};
         }
-        kw0 = kept_word(c, 0, word, nkb);
-        kw1 = kept_word(c, 1, word, nkb);
+        kw0 = kept_word(c, 0, word);
+        kw1 = kept_word(c, 1, word);
         kmask = kw0 | kw1;
       }
       const int b = __ffs(kmask) - 1;
@@ -360,7 +381,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       if (TILE) {
         // a centroid column counts for the rows whose query block skips its block
         const int w = (it.j * KC + 32 * k) >> 5;
-        mbits[k] = ~kept_h[w] & valid_bits(w, nkb);
+        mbits[k] = ~kept_h[w] & range_bits(w, c.jlo, c.jhi);
       } else {
         const int t0 = it.j * BLK + 64 * it.half + 32 * k;
         mbits[k] = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
@@ -483,6 +504,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   };
 
   Walk<BLK> wk;
+  wk.start(c);
   Item it{kNone, 0, 0, 0};
   int cur_tile = 0;
   // ---- phase 0: centroid tiles and their order-1 products ----
@@ -573,6 +595,26 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   const bool store = row0 + r < p.Nq;
   const float inv = l > 0.f ? 1.f / l : 0.f;
   const size_t rowoff = ((size_t)bh * p.Nq + row0 + (store ? r : 0)) * D;
+  if (p.nsplit > 1) {
+    // A split's partial result: O relative to 2^m_ref, not yet divided, with (m_ref, l).
+    const size_t prow = ((size_t)c.split * p.nbh + bh) * p.Nq + row0 + (store ? r : 0);
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      uint32_t v[32];
+      tc::tmem_ld32(ot + 32 * k, v);
+      tc::tmem_wait_ld();
+      if (!store) continue;
+      float4* o = reinterpret_cast<float4*>(p.part + prow * D + 32 * k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    }
+    if (store)
+      reinterpret_cast<float2*>(p.part + (size_t)p.nsplit * p.nbh * p.Nq * D)[prow] =
+          make_float2(m_ref, l);
+    return;
+  }
 #pragma unroll
   for (int k = 0; k < D / 32; ++k) {
     uint32_t v[32];
@@ -609,8 +651,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  int cx, bh;
-  cta_coords(p, cx, bh);
+  int cx, bh, split;
+  cta_coords(p, cx, bh, split);
   const int q0 = cx * (NT * TQ);
   const int nkb = p.nkb;
 
@@ -667,7 +709,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
       const int t = w / MAXW, ww = w % MAXW;
       if (BLK == 128 || q0 + t * TQ + 64 >= p.Nq) c.kept[t][1][ww] = c.kept[t][0][ww];
     }
-    if (tid == 0) c.tvalid = (q0 < p.Nq ? 1 : 0) | (q0 + TQ < p.Nq ? 2 : 0);
+    if (tid == 0) {
+      c.tvalid = (q0 < p.Nq ? 1 : 0) | (q0 + TQ < p.Nq ? 2 : 0);
+      split_range(split, p.nsplit, nkb, c.jlo, c.jhi);
+      c.split = split;
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -691,6 +737,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
           tc::tma_load_3d(base + OFF_Q + t * By::Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s,
                           q0 + t * TQ, bh);
       StepGen<BLK> gen;
+      gen.wk.start(c);
       int u = 0;
       bool ok = true;
       while (ok) {
@@ -861,6 +908,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 }
 
 
+// Merge of the key-range splits of every query row: with M = max_s m_s and
+// w_s = 2^(m_s - M), O = sum_s w_s O_s / sum_s w_s l_s (0 for a row with no weight).
+// One warp per row; lane l holds D / 32 consecutive columns.
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int nsplit,
+                                                      long long rows, void* out, int out_dtype) {
+  constexpr int V = D / 32;
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const float2* ml = reinterpret_cast<const float2*>(part + (size_t)nsplit * rows * D);
+  float M = -INFINITY;
+  for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, ml[(size_t)sp * rows + row].x);
+  float acc[V], L = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  if (M != -INFINITY) {
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const float2 x = ml[(size_t)sp * rows + row];
+      if (x.x == -INFINITY) continue;
+      const float w = exp2f(x.x - M);
+      L += w * x.y;
+      const float* o = part + ((size_t)sp * rows + row) * D + V * lane;
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] += w * o[i];
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (out_dtype == 0) {
+    float* o = static_cast<float*>(out) + (size_t)row * D + V * lane;
+#pragma unroll
+    for (int i = 0; i < V; ++i) o[i] = acc[i] * inv;
+  } else {
+    uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(out) + (size_t)row * D + V * lane);
+#pragma unroll
+    for (int i = 0; i < V / 2; ++i) o[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+  }
+}
+
 template <int D, int BLK, int ORDER>
 static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   Params p;
@@ -887,12 +973,20 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   p.scale = a.scale;
   p.nx = (a.Nq + NT * TQ - 1) / (NT * TQ);
   p.nbh = (int)bh;
-  if ((uint64_t)p.nx * bh > 0x7fffffffull) return cudaErrorInvalidValue;
+  p.nsplit = a.splits > 1 ? a.splits : 1;
+  p.part = p.nsplit > 1 ? a.work : nullptr;
+  if (p.nsplit > 1 && !p.part) return cudaErrorInvalidValue;
+  if ((uint64_t)p.nx * bh * p.nsplit > 0x7fffffffull) return cudaErrorInvalidValue;
   auto kern = forward_tc_kernel<D, BLK, ORDER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nx * p.nbh);
+  dim3 grid(p.nx * p.nbh * p.nsplit);
   kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.nsplit == 1) return e;
+  const long long rows = (long long)bh * a.Nq;
+  combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p.part, p.nsplit, rows, a.out,
+                                                                a.out_dtype);
   return cudaGetLastError();
 }
 

@@ -58,7 +58,15 @@ struct ForwardArgs {
   void* out;
   int out_dtype;
   int32_t* err_flag;
+  int splits;   // key-range splits (1: none)
+  float* work;  // splits > 1: partial results, forward_work_floats(...) floats
 };
+
+// Floats of partial results a forward with `splits` key-range splits needs: per split and
+// query row, the row's D accumulators and its (max, sum) pair.
+inline size_t forward_work_floats(int B, int H, int Nq, int d, int splits) {
+  return splits > 1 ? (size_t)splits * B * H * Nq * (size_t)(d + 2) : 0;
+}
 
 struct KmeansArgs {
   const uint16_t* x;

@@ -24,7 +24,8 @@ EXPORTS = ("sparse_attn_table_sizes", "sparse_attn_pool", "sparse_attn_pool_incr
            "sparse_attn_structured_mask_adaptive", "sparse_attn_ear_scores",
            "sparse_attn_route_scores", "sparse_attn_kmeans_sizes", "sparse_attn_kmeans",
            "sparse_attn_permute_rows", "sparse_attn_kmeans_noalloc", "sparse_attn_wait_selftest",
-           "sparse_attn_forward", "sparse_attn_last_error")
+           "sparse_attn_forward", "sparse_attn_forward_split", "sparse_attn_forward_work_bytes",
+           "sparse_attn_forward_split_plan", "sparse_attn_last_error")
 
 
 class SparseAttnError(RuntimeError):
@@ -65,6 +66,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_structured_mask.argtypes = [_I] * 12 + [_P, _P, _I, _P]
     lib.sparse_attn_structured_mask_adaptive.argtypes = [_I] * 13 + [_P, _P, _I, _P]
     lib.sparse_attn_forward.argtypes = [_P] * 8 + [_I] * 8 + [_F, _P, _I, _P, _P]
+    lib.sparse_attn_forward_split.argtypes = [_P] * 8 + [_I] * 8 + [_F, _I, _P, _P, _I, _P, _P]
+    lib.sparse_attn_forward_work_bytes.argtypes = [_I] * 5 + [ctypes.POINTER(ctypes.c_size_t)]
+    lib.sparse_attn_forward_split_plan.argtypes = [_I] * 7 + [ctypes.POINTER(_I),
+                                                              ctypes.POINTER(ctypes.c_size_t)]
     for name in EXPORTS[:-1]:
         getattr(lib, name).restype = _I
     _lib = lib
@@ -199,6 +204,31 @@ def sparse_attn_forward(q, k, v16, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H,
         _ptr(q), _ptr(k), _ptr(v16), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(kv_idx),
         _ptr(kv_cnt), cap, B, H, Nq, Nk, d, block, order, scale, _ptr(out), out_dtype,
         _ptr(err_flag), _stream(stream)))
+
+
+def sparse_attn_forward_split(q, k, v16, kbar16, vsum16, M, kv_idx, kv_cnt, cap, B, H, Nq, Nk, d,
+                              block, order, scale, splits, work, out, out_dtype, err_flag=None,
+                              stream=None):
+    _check(load_library().sparse_attn_forward_split(
+        _ptr(q), _ptr(k), _ptr(v16), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(kv_idx),
+        _ptr(kv_cnt), cap, B, H, Nq, Nk, d, block, order, scale, splits, _ptr(work), _ptr(out),
+        out_dtype, _ptr(err_flag), _stream(stream)))
+
+
+def sparse_attn_forward_work_bytes(B, H, Nq, d, splits) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().sparse_attn_forward_work_bytes(B, H, Nq, d, splits, ctypes.byref(out)))
+    return int(out.value)
+
+
+def sparse_attn_forward_split_plan(B, H, Nq, Nk, d, block, sms=0):
+    """(splits, work bytes) the library picks for this shape on ``sms`` SMs (0: the
+    current device's count)."""
+    n = _I(0)
+    b = ctypes.c_size_t(0)
+    _check(load_library().sparse_attn_forward_split_plan(B, H, Nq, Nk, d, block, sms,
+                                                         ctypes.byref(n), ctypes.byref(b)))
+    return int(n.value), int(b.value)
 
 
 def sparse_attn_last_error() -> str:

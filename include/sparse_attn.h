@@ -59,6 +59,7 @@ enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
 /* Largest number of KV blocks per head that routing and the forward accept. */
 #define SA_MAX_KV_BLOCKS 2048
 #define SA_MAX_CLUSTERS 4096
+#define SA_MAX_SPLITS 16
 
 /*
  * Byte sizes of the pooled tables for a problem, written to sizes[0..6] in the
@@ -326,6 +327,43 @@ int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v1
                         int B, int H, int Nq, int Nk, int d, int block, int order,
                         float scale, void* out, int out_dtype, int32_t* err_flag,
                         void* stream);
+
+/*
+ * The forward with the key blocks of every query tile shared out among `splits` CTAs
+ * (whole runs of 64 blocks each), for grids too small to fill the GPU evenly: each CTA
+ * runs the same online softmax over its own blocks (kept ones exactly, the others by
+ * their compensation terms) and writes its unnormalised numerator with its running
+ * maximum m_s (base 2) and denominator l_s; a second kernel merges the splits of every
+ * row, o_t = sum_s 2^(m_s - M) N_s / sum_s 2^(m_s - M) l_s with M = max_s m_s. The
+ * result equals sparse_attn_forward's up to fp32 rounding (the terms are summed in
+ * another order). The pages describe one pass per query tile; the split is a scheduling
+ * choice of this library.
+ *   splits     1 <= splits <= SA_MAX_SPLITS; 1 is sparse_attn_forward (work may be NULL)
+ *   work       device scratch owned by the caller, 16-byte aligned, at least
+ *              sparse_attn_forward_work_bytes(B, H, Nq, d, splits) bytes:
+ *              [splits][B*H][Nq][d] fp32 numerators, then [splits][B*H][Nq] (m, l) pairs
+ *   others     as for sparse_attn_forward (same checks and the same err_flag contract)
+ * Two launches when splits > 1 (forward, merge), one otherwise.
+ */
+int sparse_attn_forward_split(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
+                              const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, int cap, int B, int H,
+                              int Nq, int Nk, int d, int block, int order, float scale, int splits,
+                              float* work, void* out, int out_dtype, int32_t* err_flag,
+                              void* stream);
+
+/* Bytes of `work` sparse_attn_forward_split needs: splits * B * H * Nq * (d + 2) * 4 when
+ * splits > 1, else 0. Host only. */
+int sparse_attn_forward_work_bytes(int B, int H, int Nq, int d, int splits, size_t* bytes);
+
+/*
+ * Host-side choice of the split count for a problem shape: *splits = 1 unless splitting
+ * shortens a model of the grid's schedule (CTAs of 1/S the work plus a fixed setup,
+ * started in grid order on the first free SM of `sms`) by at least 3%; *work_bytes = the
+ * scratch it needs. sms = 0 asks the current device for its SM count. No launch.
+ */
+int sparse_attn_forward_split_plan(int B, int H, int Nq, int Nk, int d, int block, int sms,
+                                   int* splits, size_t* work_bytes);
 
 /* Message for the last error returned on the calling thread ("" if none). */
 const char* sparse_attn_last_error(void);

@@ -113,12 +113,41 @@ def test_host_argument_checks(lib):
                                       None, 0),
         lambda: C.sparse_attn_forward(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64 * 4096, 64, 64, 0, 0.1,
                                       p, 0, None, 0),
+        lambda: C.sparse_attn_forward_split(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 64, 64, 0, 0.1,
+                                            0, p, p, 0, None, 0),
+        lambda: C.sparse_attn_forward_split(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 64, 64, 0, 0.1,
+                                            17, p, p, 0, None, 0),
+        lambda: C.sparse_attn_forward_split(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 64, 64, 0, 0.1,
+                                            2, None, p, 0, None, 0),
+        lambda: C.sparse_attn_forward_split(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 64, 64, 0, 0.1,
+                                            2, p + 4, p, 0, None, 0),
+        lambda: C.sparse_attn_forward_work_bytes(1, 1, 64, 64, 0),
+        lambda: C.sparse_attn_forward_split_plan(1, 1, 64, 64, 64, 64, -1),
     ]
     for i, call in enumerate(cases):
         with pytest.raises(C.SparseAttnError) as e:
             call()
         assert e.value.code == C.SA_ERR_INVALID, (i, str(e.value))
         assert C.sparse_attn_last_error(), i
+
+
+def test_split_plan_on_the_host(lib):
+    """The split choice for a given SM count (no device needed): no split where the grid
+    spans many waves or the keys form one run of 64 blocks; a split of the world-model
+    chunk whose modelled schedule beats the unsplit one; scratch as documented."""
+    assert C.sparse_attn_forward_split_plan(1, 40, 75600, 75600, 128, 128, 148) == (1, 0)
+    assert C.sparse_attn_forward_split_plan(1, 2, 4096, 4096, 128, 64, 148) == (1, 0)
+    assert C.sparse_attn_forward_split_plan(1, 2, 0, 4096, 128, 64, 148) == (1, 0)
+    n, b = C.sparse_attn_forward_split_plan(4, 16, 1560, 63960, 128, 64, 148)
+    assert 2 <= n <= 16 and b == n * 4 * 16 * 1560 * (128 + 2) * 4
+    # a single (batch, head) with 16 runs of 64 blocks: 7 CTAs on 148 SMs split far
+    n1, _ = C.sparse_attn_forward_split_plan(1, 1, 1560, 63960, 128, 64, 148)
+    assert 8 <= n1 <= 16
+    # never more splits than runs of 64 blocks
+    n2, _ = C.sparse_attn_forward_split_plan(1, 1, 1560, 3 * 64 * 64, 128, 64, 148)
+    assert n2 <= 3
+    assert C.sparse_attn_forward_work_bytes(2, 3, 100, 64, 1) == 0
+    assert C.sparse_attn_forward_work_bytes(2, 3, 100, 64, 4) == 4 * 2 * 3 * 100 * 66 * 4
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -87,6 +87,38 @@ def test_pool_route_forward_stay_in_bounds(N, d, block, order):
         assert np.abs(got - want).max() <= 1e-2
 
 
+@pytest.mark.parametrize("Nq,d,splits,out_dtype", [(77, 64, 2, torch.float32),
+                                                    (300, 128, 3, torch.bfloat16),
+                                                    (129, 128, 5, torch.float32)])
+def test_split_forward_stays_in_bounds(Nq, d, splits, out_dtype):
+    """Partial results and the merge write inside their buffers (scratch sized exactly as
+    the library states); 9,000 keys at block 64 give three runs of 64 blocks."""
+    B, H, Nk, block, order = 1, 2, 9000, 64, 1
+    qb, kb, vb = _bits((B, H, Nq, d), 90), _bits((B, H, Nk, d), 91), _bits((B, H, Nk, d), 92)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    p = A.Problem(B, H, Nq, Nk, d, block, order)
+    t = A.allocate_tables(p, "cuda")
+    A.pool(q, k, v, p, t)
+    keep = -(-p.nkb // 6)
+    idx = torch.empty(B, H, p.nqb, keep, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, H, p.nqb, dtype=torch.int32, device="cuda")
+    A.route(p, t, idx, cnt, "topk", rho=(1, 6))
+    work = Guarded((C.sparse_attn_forward_work_bytes(B, H, Nq, d, splits) // 4,), torch.float32)
+    out = Guarded((B, H, Nq, d), out_dtype)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.forward(q, k, v, p, t, idx, cnt, out.t, err_flag=flag, splits=splits, work=work.t)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    assert work.intact() and out.intact()
+    scale = 1 / np.sqrt(d)
+    for h in range(H):
+        qh, kh, vh = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        kept = O.route_head(qh, kh, block, "topk", scale, keep=keep)[0]
+        want = O.forward_head(qh, kh, vh, kept, block, order, scale)
+        got = out.t[0, h].float().cpu().numpy()
+        assert np.abs(got - want).max() <= 1e-2
+
+
 def test_ear_kmeans_permute_stay_in_bounds():
     B, H, N, d, block = 1, 2, 333, 128, 64
     qb, kb, vb = (_bits((B, H, N, d), 80 + s) for s in range(3))

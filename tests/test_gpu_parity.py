@@ -468,6 +468,89 @@ def test_nothing_kept_and_bad_list_entries(order):
     assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
 
 
+# --- key-range splits of the forward ---------------------------------------------
+
+@pytest.mark.parametrize("Nq,Nk,d,block,order,splits,out_dtype", [
+    (300, 20000, 128, 64, 1, 2, torch.float32),    # 313 blocks: 5 runs of 64
+    (300, 20000, 128, 64, 1, 3, torch.float32),
+    (300, 20000, 128, 64, 0, 5, torch.float32),
+    (300, 20000, 128, 64, 1, 9, torch.float32),    # more splits than runs: 4 empty
+    (700, 17000, 64, 128, 2, 3, torch.float32),    # 133 blocks, ragged last run
+    (260, 30000, 128, 128, 0, 4, torch.bfloat16),  # 235 blocks
+    (77, 9000, 64, 64, 1, 16, torch.float32),      # one query tile, ragged everything
+])
+def test_split_forward_matches_oracle(Nq, Nk, d, block, order, splits, out_dtype):
+    """The forward with key-range splits and the merge, on the oracle's top-k lists,
+    against the oracle; and against the unsplit forward on the same lists."""
+    B, H = 1, 2
+    qb = _rand_bits((B, H, Nq, d), 31)
+    kb = _rand_bits((B, H, Nk, d), 32, 0.5)
+    vb = _rand_bits((B, H, Nk, d), 33)
+    p = A.Problem(B, H, Nq, Nk, d, block, order)
+    scale = 1 / np.sqrt(d)
+    keep = -(-p.nkb // 8)
+    kept = {}
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        kept[(0, h)] = O.route_head(q, k, block, "topk", scale, keep=keep)[0]
+    idx, cnt = _oracle_lists_to_device(W.shrink(W.WORKLOADS["uniform-4k"], B=B, H=H, Nq=Nq,
+                                                Nk=Nk, d=d, block=block), kept, keep)
+    t = A.allocate_tables(p, "cuda")
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    A.pool(q_d, k_d, v_d, p, t)
+    work = torch.empty(C.sparse_attn_forward_work_bytes(B, H, Nq, d, splits) // 4, device="cuda")
+    out = torch.empty(B, H, Nq, d, dtype=out_dtype, device="cuda")
+    ref = torch.empty(B, H, Nq, d, dtype=out_dtype, device="cuda")
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    A.forward(q_d, k_d, v_d, p, t, idx, cnt, out, err_flag=flag, splits=splits, work=work)
+    A.forward(q_d, k_d, v_d, p, t, idx, cnt, ref, err_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    got_all, want_all = [], []
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        want_all.append(O.forward_head(q, k, v, kept[(0, h)], block, order, scale))
+        got_all.append(out[0, h].float().cpu().numpy())
+    got, want = np.concatenate(got_all), np.concatenate(want_all)
+    mx, mr = err_stats(got, want)
+    floor = 0.0
+    if out_dtype == torch.bfloat16:
+        floor = err_stats(torch.from_numpy(want).to(torch.bfloat16).double().numpy(), want)[1]
+    assert mx <= MAX_ABS and mr <= MEAN_REL + floor, (mx, mr, floor)
+    # the split only reorders fp32 sums and moves the fp16 rounding of P with the
+    # running maxima: far below the oracle tolerance
+    d_ab = (out.float() - ref.float()).abs().max().item()
+    assert d_ab <= (2e-3 if out_dtype == torch.float32 else 2e-2), d_ab
+
+
+def test_split_plan_and_work_bytes():
+    """The library's split choice: none for grids of many waves, some for the world-model
+    chunk, never more than the 64-block runs; scratch size as documented."""
+    for (B, H, Nq, Nk, d, block) in [(1, 40, 75600, 75600, 128, 128), (1, 24, 32760, 32760, 128, 128)]:
+        assert C.sparse_attn_forward_split_plan(B, H, Nq, Nk, d, block) == (1, 0)
+    n, b = C.sparse_attn_forward_split_plan(4, 16, 1560, 63960, 128, 64)
+    assert 2 <= n <= 16 and b == n * 4 * 16 * 1560 * 130 * 4
+    n, _ = C.sparse_attn_forward_split_plan(1, 1, 1560, 4096, 128, 64)
+    assert n == 1  # a single run of 64 blocks cannot be split
+    assert C.sparse_attn_forward_work_bytes(2, 3, 100, 64, 1) == 0
+    assert C.sparse_attn_forward_work_bytes(2, 3, 100, 64, 4) == 4 * 2 * 3 * 100 * 66 * 4
+
+
+def test_split_forward_empty_and_invalid():
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(16, dtype=torch.float32, device="cuda")
+    i = torch.zeros(4, dtype=torch.int32, device="cuda")
+    # no queries: nothing to do, even without scratch
+    C.sparse_attn_forward_split(x, x, x, x, x, x, i, i, 1, 1, 1, 0, 100, 128, 128, 1, 0.1, 4,
+                                None, f, 0)
+    with pytest.raises(C.SparseAttnError):  # scratch missing
+        C.sparse_attn_forward_split(x, x, x, x, x, x, i, i, 1, 1, 1, 64, 64, 64, 64, 0, 0.1, 2,
+                                    None, f, 0)
+    with pytest.raises(C.SparseAttnError):  # too many splits
+        C.sparse_attn_forward_split(x, x, x, x, x, x, i, i, 1, 1, 1, 64, 64, 64, 64, 0, 0.1, 17,
+                                    f, f, 0)
+
+
 @pytest.mark.parametrize("order", [0, 1])
 def test_incremental_pool_equals_full_pool(order):
     """A KV cache whose last blocks change: pooling only those blocks over the tables of
@@ -546,10 +629,13 @@ def test_bounded_wait_gives_up_and_reports(small_inputs):
                                   "ear-small", "hybrid-small"])
 def test_host_call_equals_device_call(name, small_inputs):
     """run_from_host (head ranges, copies overlapped with the compute) gives the device
-    call's output bit for bit."""
+    call's output bit for bit (the forward's split count is the whole problem's)."""
     w, qb, kb, vb = small_inputs(name)
     if name in ("dit-small", "kmeans-small"):   # enough heads for several ranges of four
         w = W.shrink(w, H=12, Nq=3000, Nk=3000, grid=(3, 20, 50))
+        qb, kb, vb = W.full_inputs_bits(w)
+    if name == "worldmodel-small":  # ranges of four heads, forward split in two
+        w = W.shrink(w, H=8)
         qb, kb, vb = W.full_inputs_bits(w)
     step = w.steps[-1] if w.mode == "structured" else 0
     op, out = _run(w, _dev(qb), _dev(kb), _dev(vb), step=step)
