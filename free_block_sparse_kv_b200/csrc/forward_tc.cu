@@ -71,6 +71,7 @@ constexpr int NTHREADS = NSOFT + 128;  // + one control warpgroup (producer, 2 M
 constexpr int kRegCtl = 72, kRegSoft = 216;
 static_assert(2 * 128 * kRegSoft + 128 * kRegCtl <= 168 * NTHREADS, "register split");
 constexpr float kThresh = 11.0f;  // lazy-rescale threshold, base-2 units (P < 2^11)
+constexpr float kF16Safe = 32768.f;  // bound kept on the fp16 order-1 operand (fp16 max 65504)
 constexpr uint32_t kWaitLimit = 1u << 18;  // ~0.3 s: far above any legitimate wait
 
 constexpr uint32_t COL_O = 0, COL_R = 256;
@@ -323,7 +324,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   bool ok = uni(wt.wait(bar(c.q_full), 0, 9));
   // fp16 copy of this thread's Q row, in registers (order-1 operands)
   uint32_t q16[ORDER >= 1 ? QW : 1];
-  float qmax = 0.f;  // largest |q| of the row (order 2: keeps the global operand in fp16 range)
+  float qmax = 0.f;  // largest |q| of the row (keeps the order-1/2 operands in fp16 range)
   if constexpr (ORDER >= 1) {
 #pragma unroll
     for (int i = 0; i < QW / 4; ++i) {
@@ -344,7 +345,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     for (int k = 0; k < D / 32; ++k) tc::tmem_st32(ot + 32 * k, z);
     tc::tmem_wait_st();
   }
-  if constexpr (ORDER == 2) {
+  if constexpr (ORDER >= 1) {
 #pragma unroll
     for (int i = 0; i < QW; ++i) {
       const __half2 h = *reinterpret_cast<const __half2*>(&q16[i]);
@@ -352,6 +353,17 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     }
   }
   warp_arrive(bar(c.init_done));
+  // Order 1 builds (scale * alpha) q_t in fp16 with alpha < 2^thr (the rescale threshold):
+  // a row with large |q| lowers its threshold so that the operand stays below 2^15. For
+  // |q| up to 2^15 / (2^11 scale) (181 at d = 128) the threshold stays 2^11.
+  float thr = kThresh;
+  if constexpr (ORDER == 1) {
+    if (p.scale * qmax * exp2f(kThresh) > kF16Safe) {
+      int e;  // kF16Safe / (scale qmax) = m 2^e with m in [0.5, 1): floor(log2) = e - 1
+      frexpf(kF16Safe / (p.scale * qmax), &e);
+      thr = fmaxf(0.f, (float)(e - 1));
+    }
+  }
 
   float m_ref = -INFINITY, l = 0.f;
   float asum = 0.f;          // order 2: sum of the skipped blocks' alpha, relative to m_ref
@@ -430,9 +442,9 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       mx = tc::max3(mx, tc::max3(tc::max3(m8[0], m8[1], m8[2]), tc::max3(m8[3], m8[4], m8[5]), m8[6]), m8[7]);
     }
     mx *= sl2;
-    // Lazy rescale: only rows whose max grew by more than 2^kThresh move their
+    // Lazy rescale: only rows whose max grew by more than 2^thr move their
     // reference; rows that had no reference yet just take one (O is still zero).
-    const bool grow = mx > m_ref + kThresh;
+    const bool grow = mx > m_ref + thr;
     const bool need_o = grow && m_ref != -INFINITY;
     const float f = need_o ? tc::ex2(m_ref - mx) : 1.f;
     if (grow) m_ref = mx;

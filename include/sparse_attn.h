@@ -320,6 +320,11 @@ int sparse_attn_wait_selftest(int32_t* err_flag, int rounds, int32_t* waited, vo
  *                     a non-zero flag after the stream completes means
  *                     SA_ERR_TIMEOUT and the output is not valid. The flag is
  *                     sticky: clear it before the next call.
+ * Ranges: probabilities enter the value products as fp16 at most 2^11 (relative to the
+ * row's running maximum); with order 1 the operand scale * alpha * q_t is fp16 too, and
+ * a row with |q| above 2^15 / (2^11 scale) (181 at d = 128) rescales its maximum earlier
+ * so that the operand stays below 2^15. The pool's fp16 tables (V, value sums, M_j) must
+ * hold values below 65504; nothing checks them.
  */
 int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,

@@ -468,6 +468,50 @@ def test_nothing_kept_and_bad_list_entries(order):
     assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
 
 
+def test_order1_large_queries_keep_the_operand_in_fp16_range():
+    """Order 1 forms (scale * alpha) q_t in fp16 with alpha up to 2^11 relative to the row's
+    running reference. Queries of magnitude ~600 and keys whose logits rise by ~10.8 (base
+    2) from the first centroid tile to the second would put that operand near 2^17; rows
+    with such queries rescale earlier, and the output stays finite and matches the oracle."""
+    B, H, N, d, block = 1, 2, 8192, 128, 64
+    rng = np.random.default_rng(41)
+    q = np.empty((B, H, N, d), np.float32)
+    k = np.empty((B, H, N, d), np.float32)
+    scale = 1 / np.sqrt(d)
+    for h in range(H):
+        u = rng.choice([-1.0, 1.0], size=d).astype(np.float32)
+        q[0, h] = 600.0 * u * (1 + 0.05 * rng.standard_normal((N, 1)).astype(np.float32))
+        # logit of a key a * u / d against q = 600 u is scale * 600 * a; base 2: 76.5 a
+        a = np.where(np.arange(N) < N // 2, 0.0, 10.8 / (scale * 600 * np.log2(np.e)))
+        k[0, h] = (a[:, None] * u[None, :] / d
+                   + 1e-4 * rng.standard_normal((N, d))).astype(np.float32)
+    qb, kb = W.bf16_round(q)[1], W.bf16_round(k)[1]
+    vb = _rand_bits((B, H, N, d), 42)
+    p = A.Problem(B, H, N, N, d, block, 1)
+    keep = -(-p.nkb // 4)
+    kept = {}
+    for h in range(H):
+        qh, kh = W.bits_to_f32(qb[0, h]), W.bits_to_f32(kb[0, h])
+        kept[(0, h)] = O.route_head(qh, kh, block, "topk", scale, keep=keep)[0]
+    idx, cnt = _oracle_lists_to_device(W.shrink(W.WORKLOADS["uniform-4k"], B=B, H=H, Nq=N, Nk=N,
+                                                d=d, block=block), kept, keep)
+    t = A.allocate_tables(p, "cuda")
+    q_d, k_d, v_d = _dev(qb), _dev(kb), _dev(vb)
+    A.pool(q_d, k_d, v_d, p, t)
+    out = torch.empty(B, H, N, d, device="cuda")
+    A.forward(q_d, k_d, v_d, p, t, idx, cnt, out)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out).all())
+    rows = _sample_rows_small(A.Problem(B, H, N, N, d, block, 1), per_tile=1, seed=4)
+    got_all, want_all = [], []
+    for h in range(H):
+        qh, kh, vh = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        want_all.append(O.forward_head(qh, kh, vh, kept[(0, h)], block, 1, scale, rows=rows))
+        got_all.append(out[0, h, rows].cpu().numpy())
+    mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+
+
 # --- key-range splits of the forward ---------------------------------------------
 
 @pytest.mark.parametrize("Nq,Nk,d,block,order,splits,out_dtype", [
