@@ -512,6 +512,47 @@ def test_order1_large_queries_keep_the_operand_in_fp16_range():
     assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
 
 
+@pytest.mark.parametrize("Nq,Nk,block,order,mode", [
+    (1, 5000, 64, 1, "topk"),      # one query row (decode-like), forward split in two
+    (2, 1, 128, 0, "topk"),        # a single key
+    (63, 63, 64, 2, "topk"),       # one partial block on each side
+    (65, 4100, 128, 1, "mass"),    # a full and a one-row query block; ragged keys
+    (129, 9000, 64, 0, "mass"),
+])
+def test_pipeline_tiny_and_ragged_shapes(Nq, Nk, block, order, mode):
+    """The whole call (pool, route, forward through BlockSparseAttention, which may split
+    the forward) on degenerate shapes, against the oracle's own pipeline."""
+    B, H, d = 1, 2, 128
+    qb = _rand_bits((B, H, Nq, d), 51)
+    kb = _rand_bits((B, H, Nk, d), 52)
+    vb = _rand_bits((B, H, Nk, d), 53)
+    p = A.Problem(B, H, Nq, Nk, d, block, order)
+    op = A.BlockSparseAttention(p, mode, rho=(1, 4), tau=0.9)
+    out = op(_dev(qb), _dev(kb), _dev(vb))
+    torch.cuda.synchronize()
+    op.check()
+    scale = 1 / np.sqrt(d)
+    got_all, want_all = [], []
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        if mode == "topk":
+            kept, sc, counts = O.route_head(q, k, block, "topk", scale, keep=-(-p.nkb // 4))
+            gaps, lo, hi = O.gate_diagnostics(sc, counts)
+            pinned = gaps > GATE
+        else:
+            kept, sc, counts = O.route_head(q, k, block, "mass", scale, tau=0.9)
+            gaps, lo, hi = O.gate_diagnostics(sc, counts, tau=0.9)
+            pinned = (gaps > GATE) & (lo > GATE) & (hi > GATE)
+        got = lists_to_sets(op.kv_idx[0, h].cpu().numpy(), op.kv_cnt[0, h].cpu().numpy())
+        for i in range(p.nqb):
+            if pinned[i]:
+                assert got[i] == kept[i].tolist(), (h, i)
+        want_all.append(O.forward_head(q, k, v, kept, block, order, scale))
+        got_all.append(out[0, h].cpu().numpy())
+    mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr, op.last_splits)
+
+
 # --- key-range splits of the forward ---------------------------------------------
 
 @pytest.mark.parametrize("Nq,Nk,d,block,order,splits,out_dtype", [
