@@ -101,8 +101,20 @@ struct Params {
 // one-dimensional and puts every (batch, head)'s last pair, which may hold fewer rows,
 // after all full pairs, so that the shorter CTAs fill the last wave. Neighbouring CTAs
 // share (batch, head) and split, hence their keys and values in L2.
+template <bool SPLIT>
 SA_DEVI void cta_coords(const Params& p, int& x, int& bh, int& split) {
   const int L = blockIdx.x, nfull = p.nx - 1;
+  if constexpr (!SPLIT) {
+    split = 0;
+    if (L < nfull * p.nbh) {
+      x = L % nfull;
+      bh = L / nfull;
+    } else {
+      x = p.nx - 1;
+      bh = L - nfull * p.nbh;
+    }
+    return;
+  }
   int r;
   if (L < nfull * p.nbh * p.nsplit) {
     x = L % nfull;
@@ -125,8 +137,8 @@ struct Ctl {  // control block in shared memory
   uint32_t tmem_base;
   int abort;
   int tvalid;               // bit t: tile t has rows below Nq
-  int jlo, jhi, split;      // key blocks of this CTA's split: [jlo, jhi)
   uint32_t kept[NT][2][MAXW];  // kept blocks of each query block (half) of each tile
+  int jlo, jhi, split;      // key blocks of this CTA's split: [jlo, jhi)
 };
 static_assert(sizeof(Ctl) <= 2048, "control block");
 
@@ -144,34 +156,47 @@ SA_DEVI void split_range(int split, int nsplit, int nkb, int& jlo, int& jhi) {
   jhi = min(nkb, (int)((long long)(split + 1) * ntl / nsplit) * KC);
 }
 
-// Blocks j of word w (j = 32 w + bit) inside the CTA's key range [jlo, jhi).
+// Blocks j of word w (j = 32 w + bit) inside the CTA's key range [jlo, jhi); without
+// splits the range is [0, nkb) with jhi = nkb.
+template <bool SPLIT>
 SA_DEVI uint32_t range_bits(int w, int jlo, int jhi) {
+  if constexpr (!SPLIT) {
+    const int lo = w * 32;
+    return lo + 32 <= jhi ? 0xffffffffu : (lo < jhi ? (1u << (jhi - lo)) - 1u : 0u);
+  }
   const int a = max(jlo - 32 * w, 0), b = min(jhi - 32 * w, 32);
   if (b <= a) return 0u;
   return (b - a == 32 ? 0xffffffffu : (1u << (b - a)) - 1u) << a;
 }
 // Blocks of word w that some query block of tile t skips / keeps.
-SA_DEVI uint32_t skip_word(const Ctl& c, int t, int w) {
+template <bool SPLIT>
+SA_DEVI uint32_t skip_word(const Ctl& c, int t, int w, int jlo, int jhi) {
   if (!((c.tvalid >> t) & 1)) return 0u;
-  return ~(c.kept[t][0][w] & c.kept[t][1][w]) & range_bits(w, c.jlo, c.jhi);
+  return ~(c.kept[t][0][w] & c.kept[t][1][w]) & range_bits<SPLIT>(w, jlo, jhi);
 }
-SA_DEVI uint32_t kept_word(const Ctl& c, int t, int w) {
+template <bool SPLIT>
+SA_DEVI uint32_t kept_word(const Ctl& c, int t, int w, int jlo, int jhi) {
   if (!((c.tvalid >> t) & 1)) return 0u;
-  return (c.kept[t][0][w] | c.kept[t][1][w]) & range_bits(w, c.jlo, c.jhi);
+  return (c.kept[t][0][w] | c.kept[t][1][w]) & range_bits<SPLIT>(w, jlo, jhi);
 }
-SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct) {
-  return (uint64_t)skip_word(c, t, 2 * ct) | ((uint64_t)skip_word(c, t, 2 * ct + 1) << 32);
+template <bool SPLIT>
+SA_DEVI uint64_t skip64(const Ctl& c, int t, int ct, int jlo, int jhi) {
+  return (uint64_t)skip_word<SPLIT>(c, t, 2 * ct, jlo, jhi) |
+         ((uint64_t)skip_word<SPLIT>(c, t, 2 * ct + 1, jlo, jhi) << 32);
 }
 
 // The walk over work items; identical in every role. Union masks of the current
 // centroid tile (phase 0) or 32-block word (phase 1) are held in registers. It covers
 // the key blocks [jlo, jhi) of the CTA's split (every block when there is one split).
-template <int BLK>
+template <int BLK, bool SPLIT>
 struct Walk {
   int phase = 0, tile = 0, word = -1, half = 0, jcur = 0, mcur = 0;
+  int jlo = 0, jhi = 0;  // the split's key blocks, kept in registers
   SA_DEVI void start(const Ctl& c) {
-    tile = c.jlo / KC;
-    word = c.jlo / 32 - 1;
+    jlo = SPLIT ? c.jlo : 0;
+    jhi = c.jhi;
+    tile = jlo / KC;
+    word = jlo / 32 - 1;
   }
   int gmask = 0;       // order 2: tiles with a skipped block so far
   bool in_tile = false, gdone = false;
@@ -179,7 +204,7 @@ struct Walk {
   uint32_t kmask = 0, kw0 = 0, kw1 = 0;  // phase 1: union / per-tile kept blocks
   template <int ORDER>
   SA_DEVI Item next(const Ctl& c, int nkb) {
-    const int ntiles = (c.jhi + KC - 1) / KC;
+    const int ntiles = (jhi + KC - 1) / KC;
     while (true) {
       if (phase == 0) {
         if (!in_tile) {
@@ -191,8 +216,8 @@ struct Walk {
             phase = 1;
             continue;
           }
-          sk0 = skip64(c, 0, tile);
-          sk1 = skip64(c, 1, tile);
+          sk0 = skip64<SPLIT>(c, 0, tile, jlo, jhi);
+          sk1 = skip64<SPLIT>(c, 1, tile, jlo, jhi);
           tmask = sk0 | sk1;
           if (tmask) {
             in_tile = true;
@@ -217,12 +242,12 @@ struct Walk {
         return Item{kExact, jcur, mcur, 1};
       }
       while (!kmask) {
-        if (++word >= (c.jhi + 31) / 32) {
-          word = (c.jhi + 31) / 32;  // stays at the end: later calls return kNone again
+        if (++word >= (jhi + 31) / 32) {
+          word = (jhi + 31) / 32;  // stays at the end: later calls return kNone again
           return Item{kNone, 0, 0, 0};
         }
-        kw0 = kept_word(c, 0, word);
-        kw1 = kept_word(c, 1, word);
+        kw0 = kept_word<SPLIT>(c, 0, word, jlo, jhi);
+        kw1 = kept_word<SPLIT>(c, 1, word, jlo, jhi);
         kmask = kw0 | kw1;
       }
       const int b = __ffs(kmask) - 1;
@@ -246,9 +271,9 @@ struct Step {
   int cur_kind, cur_mask, cur_j, cur_half;      // SX: new TILE/EXACT item; MAT: the block
   int pend_kind, pend_mask, pend_j, pend_half;  // SX / FLUSH: item whose value products are due
 };
-template <int BLK>
+template <int BLK, bool SPLIT>
 struct StepGen {
-  Walk<BLK> wk;
+  Walk<BLK, SPLIT> wk;
   int pend_kind = 0, pend_mask = 0, pend_j = 0, pend_half = 0;
   bool flush_next = false;
   template <int ORDER>
@@ -296,7 +321,7 @@ struct Bytes {
 
 // Softmax warpgroup of tile t = warp / 4. Thread (warp w, lane l) owns query row
 // r = 32*(w%4) + l of the tile: all its logits, its running max and sum, its O row.
-template <int D, int BLK, int ORDER>
+template <int D, int BLK, int ORDER, bool SPLIT>
 SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem, tc::Waiter& wt,
                           int warp, int lane, int cx, int bh) {
   using By = Bytes<D, BLK>;
@@ -311,6 +336,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   const int nkb = p.nkb;
   const int row0 = cx * (NT * TQ) + t * TQ;
   const uint32_t* kept_h = c.kept[t][h];
+  const int jlo = c.jlo, jhi = c.jhi;  // the CTA's key blocks (split)
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
   auto uni = [](bool x) { return __all_sync(0xffffffffu, x); };
   // One arrival per warp: every lane's tensor-memory stores are ordered before the
@@ -393,7 +419,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
       if (TILE) {
         // a centroid column counts for the rows whose query block skips its block
         const int w = (it.j * KC + 32 * k) >> 5;
-        mbits[k] = ~kept_h[w] & range_bits(w, c.jlo, c.jhi);
+        mbits[k] = ~kept_h[w] & range_bits<SPLIT>(w, jlo, jhi);
       } else {
         const int t0 = it.j * BLK + 64 * it.half + 32 * k;
         mbits[k] = t0 + 32 <= p.Nk ? 0xffffffffu : (t0 < p.Nk ? (1u << (p.Nk - t0)) - 1u : 0u);
@@ -515,7 +541,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     return true;
   };
 
-  Walk<BLK> wk;
+  Walk<BLK, SPLIT> wk;
   wk.start(c);
   Item it{kNone, 0, 0, 0};
   int cur_tile = 0;
@@ -607,7 +633,7 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
   const bool store = row0 + r < p.Nq;
   const float inv = l > 0.f ? 1.f / l : 0.f;
   const size_t rowoff = ((size_t)bh * p.Nq + row0 + (store ? r : 0)) * D;
-  if (p.nsplit > 1) {
+  if constexpr (SPLIT) {
     // A split's partial result: O relative to 2^m_ref, not yet divided, with (m_ref, l).
     const size_t prow = ((size_t)c.split * p.nbh + bh) * p.Nq + row0 + (store ? r : 0);
 #pragma unroll
@@ -625,33 +651,33 @@ SA_DEVI void softmax_role(const Params& p, Ctl& c, uint8_t* gbase, uint32_t tmem
     if (store)
       reinterpret_cast<float2*>(p.part + (size_t)p.nsplit * p.nbh * p.Nq * D)[prow] =
           make_float2(m_ref, l);
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int k = 0; k < D / 32; ++k) {
-    uint32_t v[32];
-    tc::tmem_ld32(ot + 32 * k, v);
-    tc::tmem_wait_ld();
-    if (!store) continue;
-    if (p.out_dtype == 0) {
-      float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff + 32 * k);
+    for (int k = 0; k < D / 32; ++k) {
+      uint32_t v[32];
+      tc::tmem_ld32(ot + 32 * k, v);
+      tc::tmem_wait_ld();
+      if (!store) continue;
+      if (p.out_dtype == 0) {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + rowoff + 32 * k);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        o[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
-                           __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
-    } else {
-      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff + 32 * k);
+        for (int i = 0; i < 8; ++i)
+          o[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                             __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
+      } else {
+        uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + rowoff + 32 * k);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        o[i] = make_uint4(pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv),
-                          pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv),
-                          pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv),
-                          pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv));
+        for (int i = 0; i < 4; ++i)
+          o[i] = make_uint4(pack_bf16(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv),
+                            pack_bf16(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv),
+                            pack_bf16(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv),
+                            pack_bf16(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv));
+      }
     }
   }
 }
 
-template <int D, int BLK, int ORDER>
+template <int D, int BLK, int ORDER, bool SPLIT>
 __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_constant__ Params p) {
   using By = Bytes<D, BLK>;
   constexpr int SUB = By::SUB;
@@ -664,7 +690,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   int cx, bh, split;
-  cta_coords(p, cx, bh, split);
+  cta_coords<SPLIT>(p, cx, bh, split);
   const int q0 = cx * (NT * TQ);
   const int nkb = p.nkb;
 
@@ -735,7 +761,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegSoft));
-    softmax_role<D, BLK, ORDER>(p, c, gbase, tmem, wt, warp, lane, cx, bh);
+    softmax_role<D, BLK, ORDER, SPLIT>(p, c, gbase, tmem, wt, warp, lane, cx, bh);
   } else {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegCtl));
   if (warp == 8) {
@@ -748,7 +774,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) forward_tc_kernel(const __grid_co
         for (int s = 0; s < SUB; ++s)
           tc::tma_load_3d(base + OFF_Q + t * By::Q + s * TQ * 128, &p.tmQ, bar(c.q_full), 64 * s,
                           q0 + t * TQ, bh);
-      StepGen<BLK> gen;
+      StepGen<BLK, SPLIT> gen;
       gen.wk.start(c);
       int u = 0;
       bool ok = true;
@@ -989,7 +1015,8 @@ static cudaError_t launch_t(const ForwardArgs& a, cudaStream_t st) {
   p.part = p.nsplit > 1 ? a.work : nullptr;
   if (p.nsplit > 1 && !p.part) return cudaErrorInvalidValue;
   if ((uint64_t)p.nx * bh * p.nsplit > 0x7fffffffull) return cudaErrorInvalidValue;
-  auto kern = forward_tc_kernel<D, BLK, ORDER>;
+  auto kern = p.nsplit > 1 ? forward_tc_kernel<D, BLK, ORDER, true>
+                            : forward_tc_kernel<D, BLK, ORDER, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nx * p.nbh * p.nsplit);
