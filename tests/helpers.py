@@ -37,6 +37,9 @@ SMALL = {
                           Nk=9480, grid=(6, 20, 79)),
     "kmeans-small": W.shrink(W.WORKLOADS["dit720p-kmeans-21x45x80"], name="kmeans-small", H=2,
                              Nq=9480, Nk=9480, grid=(6, 20, 79), clusters=(38, 38, 3)),
+    # error-aware routing on blocks cut from the k-means group-major order
+    "ear-kmeans-small": W.shrink(W.WORKLOADS["dit720p-ear-21x45x80"], name="ear-kmeans-small", H=2,
+                                 Nq=9480, Nk=9480, grid=(6, 20, 79), clusters=(38, 38, 3)),
 }
 
 # Error-aware scores (ln of the error per token). The GPU takes the logits with a 16-bit
