@@ -553,6 +553,38 @@ def test_pipeline_tiny_and_ragged_shapes(Nq, Nk, block, order, mode):
     assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr, op.last_splits)
 
 
+@pytest.mark.parametrize("mode,order,block", [
+    ("topk", 1, 64), ("topk", 0, 128), ("mass", 1, 128), ("topk_cov", 2, 64), ("topk_cov", 2, 128),
+    ("ear", 0, 64),
+])
+def test_pipeline_head_dim_64(mode, order, block):
+    """Every routing mode and order through the d = 64 kernels (pool, route or error-aware
+    probe, forward), against the oracle's own pipeline, with ragged ends."""
+    B, H, N, d = 1, 2, 3000, 64
+    w = W.shrink(W.WORKLOADS["dit-21x30x52"], B=B, H=H, Nq=N, Nk=N, d=d, block=block,
+                 order=order, grid=(3, 20, 50))
+    qb, kb, vb = W.full_inputs_bits(w)
+    p = A.Problem(B, H, N, N, d, block, order)
+    rho = (1, 5)
+    op = A.BlockSparseAttention(p, mode, rho=rho, tau=0.9)
+    out = op(_dev(qb), _dev(kb), _dev(vb))
+    torch.cuda.synchronize()
+    op.check()
+    scale = 1 / np.sqrt(d)
+    keep = -(-p.nkb * rho[0] // rho[1])
+    got_all, want_all = [], []
+    for h in range(H):
+        q, k, v = (W.bits_to_f32(x[0, h]) for x in (qb, kb, vb))
+        if mode == "mass":
+            kept = O.route_head(q, k, block, "mass", scale, tau=0.9)[0]
+        else:
+            kept = O.route_head(q, k, block, mode, scale, keep=keep, v=v)[0]
+        want_all.append(O.forward_head(q, k, v, kept, block, order, scale))
+        got_all.append(out[0, h].cpu().numpy())
+    mx, mr = err_stats(np.concatenate(got_all), np.concatenate(want_all))
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+
+
 # --- key-range splits of the forward ---------------------------------------------
 
 @pytest.mark.parametrize("Nq,Nk,d,block,order,splits,out_dtype", [
