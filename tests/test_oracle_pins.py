@@ -62,6 +62,45 @@ def test_golden_routing(golden_dir):
     assert gaps[0] == 0.0
 
 
+def test_golden_mass_margins(golden_dir):
+    """Cumulative-mass margins at the cutoff of the mass rule, hand-derived (closed
+    forms in the fixture), including k = 1 where the lower margin is undefined."""
+    g = _load(golden_dir, "mass_margins_d4.json")
+    s = np.array([g["scores"]], float)
+    for case in g["cases"]:
+        kept, cnt = O.route_mass(s, case["tau"])
+        assert cnt[0] == case["k"]
+        gaps, lo, hi = O.gate_diagnostics(s, cnt, tau=case["tau"])
+        assert gaps[0] == pytest.approx(case["gap"], abs=1e-15)
+        if case["lo"] == "inf":
+            assert lo[0] == math.inf
+        else:
+            assert lo[0] == pytest.approx(case["lo"], abs=1e-12)
+        assert hi[0] == pytest.approx(case["hi"], abs=1e-12)
+
+
+def test_mass_margins_match_brute_force_sums():
+    """Margins against an independent ranking (Python sort) and exactly rounded sums
+    (math.fsum): tau - C_(k-1) > 0 >= tau - C_k, both reported with the right sign."""
+    rng = np.random.default_rng(11)
+    s = 1.5 * rng.standard_normal((30, 25))
+    for tau in (0.3, 0.75, 0.95):
+        _, counts = O.route_mass(s, tau)
+        _, lo, hi = O.gate_diagnostics(s, counts, tau=tau)
+        for i, row in enumerate(s):
+            z = [math.exp(x - max(row)) for x in row]
+            total = math.fsum(z)
+            ranked = sorted(range(len(row)), key=lambda j: (-row[j], j))
+            k = counts[i]
+            c_k = math.fsum(z[j] for j in ranked[:k]) / total
+            c_km1 = math.fsum(z[j] for j in ranked[:k - 1]) / total
+            assert hi[i] == pytest.approx(c_k - tau, abs=1e-12) and hi[i] >= -1e-12
+            if k == 1:
+                assert lo[i] == math.inf
+            else:
+                assert lo[i] == pytest.approx(tau - c_km1, abs=1e-12) and lo[i] > 0
+
+
 def test_golden_structured(golden_dir):
     g = _load(golden_dir, "structured_small.json")
     kept = O.structured_kept(g["Nq"], g["Nk"], g["block"], g["frame_tokens"], g["n_frames"],
@@ -257,6 +296,44 @@ def test_structured_mask_against_token_pairs():
                             hit = True
                 want.append(hit)
             assert kept[i].tolist() == [j for j, h in enumerate(want) if h]
+
+
+def test_structured_mask_of_a_query_chunk_against_token_pairs():
+    """A query chunk that starts mid-video (q_frame0 > 0, an autoregressive chunk):
+    query token t lies in frame q_frame0 + t // frame_tokens. Brute force over every
+    (query token, key token) pair, with blocks that straddle frames on both sides."""
+    ft, T, b, win, na, per = 7, 9, 5, 1, 2, 4
+    nk = ft * T
+    for q_frame0, nq in ((4, 17), (6, 21), (8, 7)):
+        for step in (0, 3):
+            kept = O.structured_kept(nq, nk, b, ft, T, win, na, per, step, q_frame0=q_frame0)
+            anchors = {(step % per) + per * m for m in range(na)}
+            assert len(kept) == -(-nq // b)
+            for i in range(-(-nq // b)):
+                want = []
+                for j in range(-(-nk // b)):
+                    hit = False
+                    for tq in range(i * b, min(nq, (i + 1) * b)):
+                        for tk in range(j * b, min(nk, (j + 1) * b)):
+                            fq, fk = q_frame0 + tq // ft, tk // ft
+                            if abs(fq - fk) <= win or fk in anchors:
+                                hit = True
+                    want.append(hit)
+                assert kept[i].tolist() == [j for j, h in enumerate(want) if h]
+
+
+@pytest.mark.parametrize("budget", [0, 6])
+def test_structured_mask_of_a_chunk_equals_the_rows_of_the_whole_video(budget):
+    """When a chunk starts on a block boundary, its query blocks are blocks of the whole
+    video: the chunk's mask (q_frame0 > 0) equals those rows of the full mask, with and
+    without adaptive windows."""
+    ft, T, b, win, na, per = 6, 10, 3, 1, 2, 5
+    full = O.structured_kept(ft * T, ft * T, b, ft, T, win, na, per, 2, budget=budget)
+    for f0, nframes in ((2, 2), (5, 3), (9, 1)):
+        chunk = O.structured_kept(ft * nframes, ft * T, b, ft, T, win, na, per, 2, q_frame0=f0,
+                                  budget=budget)
+        first = f0 * ft // b
+        assert [x.tolist() for x in chunk] == [x.tolist() for x in full[first:first + len(chunk)]]
 
 
 def test_structured_kept_fraction_at_long_video_size():
