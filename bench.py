@@ -230,72 +230,134 @@ class ClockSampler:
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
 
-def time_oracle(w: W.Workload, seconds: float) -> dict:
-    """Time the fp64 oracle on a bounded sample: one head's pooling and routing, then
-    query rows (spread over the head) until `seconds` have passed. Scaled to
-    dense-equivalent TFLOPS: rows * Nk * d * 4 per second of the oracle's time."""
-    from oracle import block_sparse_attention as O
-    q, k, v = W.head_inputs(w, 0, 0)
-    t0 = time.perf_counter()
-    if w.clusters:
-        from oracle import cluster_layout as K
-        cq, ck, iters = w.clusters
-        pq = K.group_major_permutation(K.kmeans(q, cq, iters)[0], cq)[0]
-        pk = K.group_major_permutation(K.kmeans(k, ck, iters)[0], ck)[0]
-        q, k, v = q[pq], k[pk], v[pk]
-    if w.mode == "structured":
-        kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames, w.window,
-                                 w.n_anchors, w.period, 0, w.q_frame0, budget=w.budget)
-    else:
-        kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau, v=v)[0]
-    kbar, vsum, counts, mats = O.pool_keys_values(k, v, w.block, min(w.order, 1))
-    hbar = O.global_first_order(mats) if w.order == 2 else None
-    t_setup = time.perf_counter() - t0
-    rng = np.random.default_rng(0)
-    order = rng.permutation(w.Nq)
-    done = 0
-    t1 = time.perf_counter()
-    q64 = q.astype(np.float64)
-    while done < w.Nq and time.perf_counter() - t1 < seconds:
-        rows = order[done:done + 16]
-        O.forward_rows(q64[rows], rows // w.block, k, v, kbar, vsum, counts, mats, kept, w.block,
-                       w.order, w.scale, hbar=hbar)
-        done += len(rows)
-    t_rows = time.perf_counter() - t1
-    # one head's setup is amortised over its Nq rows
-    per_row = t_rows / done + t_setup / w.Nq
-    tflops = 4.0 * w.Nk * w.d / per_row / 1e12
-    cores = len(os.sched_getaffinity(0))
+class OracleSampler:
+    """The fp64 oracle on one head of a workload: pooling and routing once, then query
+    rows (spread over the head in a fixed random order) forwarded in samples."""
+
+    def __init__(self, w: W.Workload):
+        from oracle import block_sparse_attention as O
+        self.O, self.w = O, w
+        q, k, v = W.head_inputs(w, 0, 0)
+        t0 = time.perf_counter()
+        if w.clusters:
+            from oracle import cluster_layout as K
+            cq, ck, iters = w.clusters
+            pq = K.group_major_permutation(K.kmeans(q, cq, iters)[0], cq)[0]
+            pk = K.group_major_permutation(K.kmeans(k, ck, iters)[0], ck)[0]
+            q, k, v = q[pq], k[pk], v[pk]
+        if w.mode == "structured":
+            self.kept = O.structured_kept(w.Nq, w.Nk, w.block, w.frame_tokens, w.n_frames,
+                                          w.window, w.n_anchors, w.period, 0, w.q_frame0,
+                                          budget=w.budget)
+        else:
+            self.kept = O.route_head(q, k, w.block, w.mode, w.scale, keep=w.keep(), tau=w.tau,
+                                     v=v)[0]
+        self.tables = O.pool_keys_values(k, v, w.block, min(w.order, 1))
+        self.hbar = O.global_first_order(self.tables[3]) if w.order == 2 else None
+        self.t_setup = time.perf_counter() - t0
+        self.q64, self.k, self.v = q.astype(np.float64), k, v
+        self.order = np.random.default_rng(0).permutation(w.Nq)
+        self.done = 0
+
+    def rows(self, n: int) -> int:
+        """Forward the next n rows (wrapping around the head); returns n."""
+        w = self.w
+        kbar, vsum, counts, mats = self.tables
+        left = n
+        while left > 0:
+            start = self.done % w.Nq
+            take = min(left, 16, w.Nq - start)
+            rows = self.order[start:start + take]
+            self.O.forward_rows(self.q64[rows], rows // w.block, self.k, self.v, kbar, vsum,
+                                counts, mats, self.kept, w.block, w.order, w.scale,
+                                hbar=self.hbar)
+            self.done += take
+            left -= take
+        return n
+
+    def tflops(self, rows: int, seconds: float) -> float:
+        """Dense-equivalent TFLOPS of `rows` rows forwarded in `seconds`, with the head's
+        pooling and routing amortised over its Nq rows."""
+        per_row = seconds / rows + self.t_setup / self.w.Nq
+        return 4.0 * self.w.Nk * self.w.d / per_row / 1e12
+
+    def ms_per_call(self, rows: int, seconds: float) -> float:
+        """A whole call (every row of every head) extrapolated from the rate measured."""
+        w = self.w
+        return (seconds / rows + self.t_setup / w.Nq) * w.Nq * w.B * w.H * 1e3
+
+
+def host_info() -> dict:
     try:
         blas = ",".join(sorted({c.get("internal_api", "?") for c in
                                 __import__("threadpoolctl").threadpool_info()}))
     except Exception:  # the report is informational
         blas = "unknown"
-    return dict(value=tflops, unit=UNIT, cores=cores, cpu_count=os.cpu_count(), blas=blas,
-                kind="oracle",
+    return dict(cores=len(os.sched_getaffinity(0)), cpu_count=os.cpu_count(), blas=blas)
+
+
+def time_oracle(w: W.Workload, seconds: float) -> dict:
+    """Time the fp64 oracle on a bounded sample: one head's pooling and routing, then query
+    rows until `seconds` have passed. Scaled to dense-equivalent TFLOPS: rows * Nk * d * 4
+    per second of the oracle's time."""
+    smp = OracleSampler(w)
+    t1 = time.perf_counter()
+    done = 0
+    while done < w.Nq and time.perf_counter() - t1 < seconds:
+        done += smp.rows(16)
+    t_rows = time.perf_counter() - t1
+    return dict(value=smp.tflops(done, t_rows), unit=UNIT, **host_info(), kind="oracle",
                 sample=f"{w.name}: head (0,0) {'clustered, ' if w.clusters else ''}pooled and "
-                       f"routed ({t_setup:.1f} s), then {done} of "
+                       f"routed ({smp.t_setup:.1f} s), then {done} of "
                        f"{w.Nq} query rows forwarded ({t_rows:.1f} s); scaled per row to the "
                        f"dense-equivalent flops of one call",
-                seconds=t_setup + t_rows, ms_per_call_est=per_row * w.Nq * w.B * w.H * 1e3)
+                seconds=smp.t_setup + t_rows, ms_per_call_est=smp.ms_per_call(done, t_rows))
+
+
+def reference_rows_per_step(seconds_per_row: float, budget_s: float, steps: int) -> int:
+    """Rows per timed step so that `steps` steps take about `budget_s` seconds (at least 16,
+    a whole number of 16-row chunks)."""
+    rows = int(budget_s / max(steps, 1) / max(seconds_per_row, 1e-9))
+    return max(16, rows - rows % 16)
 
 
 def run_reference(args, w):
+    """The reference arm: the fp64 oracle on the host cores. One step = one bounded sample
+    of the workload (a fixed number of query rows of head (0,0)); W warm-up steps calibrate
+    the sample size so that the K timed steps take about --cpu-seconds."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    res = time_oracle(w, args.cpu_seconds)
+    smp = OracleSampler(w)
+    t0 = time.perf_counter()
+    for _ in range(max(args.warmup, 1)):
+        smp.rows(16)
+    per_row = (time.perf_counter() - t0) / (16 * max(args.warmup, 1))
+    rows_step = reference_rows_per_step(per_row, args.cpu_seconds, args.steps)
+    step_s = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        smp.rows(rows_step)
+        step_s.append(time.perf_counter() - t)
+    total = float(sum(step_s))
+    rows = rows_step * args.steps
+    value = smp.tflops(rows, total)
+    info = host_info()
+    sample = (f"{w.name}: head (0,0) pooled and routed once ({smp.t_setup:.1f} s, amortised "
+              f"over its {w.Nq} rows); each step forwards {rows_step} query rows of that head; "
+              f"{args.steps} timed steps = {rows} rows in {total:.1f} s")
     line = {
-        "impl": "reference", "metric": METRIC, "value": res["value"], "unit": UNIT,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": res["ms_per_call_est"], "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "block": w.block, "order": w.order, "mode": w.mode},
-        "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "cpu_count", "blas", "kind",
-                                             "sample")},
-        "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
+        "step": f"one bounded sample: {rows_step} query rows of head (0,0)",
+        "rows_timed": rows,
+        "ms_per_call_extrapolated": smp.ms_per_call(rows, total),
+        "cpu_baseline": {"value": value, "unit": UNIT, **info, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 

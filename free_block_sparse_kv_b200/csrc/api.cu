@@ -357,10 +357,12 @@ int sparse_attn_kmeans_noalloc(const uint16_t* x, int B, int H, int N, int d, in
                                                                  nullptr, nullptr, labels, perm,
                                                                  offsets, err_flag, stream);
   if (int rc = check_device()) return rc;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  uint8_t* scratch = static_cast<uint8_t*>(sa::kmeans_scratch(dev));
-  if (!scratch) return fail(SA_ERR_LAUNCH, "no address for the built-in scratch buffer on device %d", dev);
+  void* addr = nullptr;
+  const cudaError_t e = sa::kmeans_scratch(&addr);
+  if (e != cudaSuccess)
+    return fail(SA_ERR_LAUNCH, "cudaGetSymbolAddress of the built-in scratch buffer: %s",
+                cudaGetErrorString(e));
+  uint8_t* scratch = static_cast<uint8_t*>(addr);
   return sparse_attn_kmeans(x, B, H, N, d, C, iters, centroids, scratch,
                             reinterpret_cast<int32_t*>(scratch + cw), labels, perm, offsets,
                             err_flag, stream);

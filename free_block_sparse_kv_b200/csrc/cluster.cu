@@ -644,25 +644,46 @@ cudaError_t assign_t(const KmeansArgs& a, int Cpad, cudaStream_t st) {
 // module's global memory (no allocation at call time).
 static __device__ __align__(256) uint8_t g_kmeans_scratch[kKmeansScratchBytes];
 
-void* kmeans_scratch(int device) {
-  static void* addr[64] = {};
-  if (device < 0 || device >= 64) return nullptr;
-  if (!addr[device]) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_kmeans_scratch) != cudaSuccess) return nullptr;
-    addr[device] = a;
+// The buffer's device address on the current device. Looked up on every call: the
+// lookup costs microseconds, and an address kept across calls would go stale if the
+// device's context were reset (the module, and with it the buffer, is then loaded
+// again). On failure the runtime's error state is cleared, so that it does not
+// surface in a later launch check, and the error is returned.
+cudaError_t kmeans_scratch(void** addr) {
+  *addr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(addr, g_kmeans_scratch);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *addr = nullptr;
   }
-  return addr[device];
+  return e;
+}
+
+// Where each work buffer of launch_kmeans sits in cwork and iwork (byte offsets);
+// the sizes the caller allocates are the two ends, so the carving and the sizes
+// cannot disagree.
+KmeansLayout kmeans_layout(int B, int H, int N, int d, int C) {
+  const size_t bh = (size_t)B * H;
+  const size_t Cpad = (size_t)km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
+  const size_t maxseg = (size_t)km::cdiv(N, km::kSeg) + C;
+  KmeansLayout L;
+  L.pieces = 0;                                                // [bh][2][Cpad][d] bf16
+  L.cnorm = L.pieces + align256(bh * 2 * Cpad * d * 2);        // [bh][Cpad] fp32
+  L.part = L.cnorm + align256(bh * Cpad * 4);                  // [bh][maxseg][d] fp64
+  L.cwork_end = L.part + bh * maxseg * d * 8;
+  L.counts = 0;                                                // [bh][nchunk][C] int32
+  L.amb_list = L.counts + align256(bh * nchunk * C * 4);       // [bh][N] int32
+  L.amb_cnt = L.amb_list + align256(bh * N * 4);               // [bh] int32
+  L.seg_off = L.amb_cnt + align256(bh * 4);                    // [bh][C + 1] int32
+  L.iwork_end = L.seg_off + bh * (C + 1) * 4;
+  return L;
 }
 
 void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]) {
-  const size_t bh = (size_t)B * H;
-  const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
-  sizes[0] = bh * C * d * sizeof(double);
-  const size_t maxseg = (size_t)km::cdiv(N, km::kSeg) + C;
-  sizes[1] = align256(bh * 2 * Cpad * d * 2) + align256(bh * Cpad * 4) + bh * maxseg * d * 8;
-  sizes[2] = align256(bh * nchunk * C * 4) + align256(bh * N * 4) + align256(bh * 4) +
-             bh * (C + 1) * 4;
+  const KmeansLayout L = kmeans_layout(B, H, N, d, C);
+  sizes[0] = (size_t)B * H * C * d * sizeof(double);
+  sizes[1] = L.cwork_end;
+  sizes[2] = L.iwork_end;
 }
 
 cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
@@ -671,20 +692,16 @@ cudaError_t launch_kmeans(const KmeansArgs& in, cudaStream_t st) {
   const int Cpad = km::cdiv(C, km::TCN) * km::TCN, nchunk = km::cdiv(N, km::kChunk);
   // carve the work buffers
   const int maxseg = km::cdiv(N, km::kSeg) + C;
+  const KmeansLayout L = kmeans_layout(a.B, a.H, N, d, C);
   uint8_t* cw = reinterpret_cast<uint8_t*>(a.cwork);
-  a.pieces = reinterpret_cast<uint16_t*>(cw);
-  cw += align256((size_t)bh * 2 * Cpad * d * 2);
-  a.cnorm = reinterpret_cast<float*>(cw);
-  cw += align256((size_t)bh * Cpad * 4);
-  double* part = reinterpret_cast<double*>(cw);
   uint8_t* iw = reinterpret_cast<uint8_t*>(a.iwork);
-  a.counts = reinterpret_cast<int32_t*>(iw);
-  iw += align256((size_t)bh * nchunk * C * 4);
-  a.amb_list = reinterpret_cast<int32_t*>(iw);
-  iw += align256((size_t)bh * N * 4);
-  a.amb_cnt = reinterpret_cast<int32_t*>(iw);
-  iw += align256((size_t)bh * 4);
-  int32_t* seg_off = reinterpret_cast<int32_t*>(iw);
+  a.pieces = reinterpret_cast<uint16_t*>(cw + L.pieces);
+  a.cnorm = reinterpret_cast<float*>(cw + L.cnorm);
+  double* part = reinterpret_cast<double*>(cw + L.part);
+  a.counts = reinterpret_cast<int32_t*>(iw + L.counts);
+  a.amb_list = reinterpret_cast<int32_t*>(iw + L.amb_list);
+  a.amb_cnt = reinterpret_cast<int32_t*>(iw + L.amb_cnt);
+  int32_t* seg_off = reinterpret_cast<int32_t*>(iw + L.seg_off);
 
   const int sort_smem = km::kSortWarps * C * 4;
   cudaError_t e;

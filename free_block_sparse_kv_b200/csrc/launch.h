@@ -90,9 +90,15 @@ struct PermuteArgs {
   void* dst;
 };
 
+// Byte offsets of launch_kmeans's work buffers in cwork and iwork, and the two ends.
+struct KmeansLayout {
+  size_t pieces, cnorm, part, cwork_end;
+  size_t counts, amb_list, amb_cnt, seg_off, iwork_end;
+};
+KmeansLayout kmeans_layout(int B, int H, int N, int d, int C);
 void kmeans_sizes(int B, int H, int N, int d, int C, size_t sizes[3]);
 constexpr size_t kKmeansScratchBytes = (size_t)32 << 20;  // per device, for the no-alloc call
-void* kmeans_scratch(int device);  // device address of that buffer on `device`
+cudaError_t kmeans_scratch(void** addr);  // device address of that buffer, current device
 cudaError_t launch_kmeans(const KmeansArgs& p, cudaStream_t st);
 cudaError_t launch_permute_rows(const PermuteArgs& p, cudaStream_t st);
 cudaError_t launch_wait_selftest(int32_t* err_flag, uint32_t rounds, int32_t* waited,

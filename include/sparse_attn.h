@@ -247,7 +247,11 @@ int sparse_attn_permute_rows(const void* src, const int32_t* perm, int B, int H,
  * sizes[1] (rounded up to 256 bytes) + sizes[2] exceed it return SA_ERR_INVALID before
  * anything is enqueued. The buffer is shared by every call on the device: calls must be
  * ordered (one stream, or synchronised), never concurrent. Results equal
- * sparse_attn_kmeans's bit for bit.
+ * sparse_attn_kmeans's bit for bit. Every call looks up the buffer's address on the
+ * current device (cudaGetSymbolAddress; a failed lookup returns SA_ERR_LAUNCH with the
+ * runtime's message and leaves no pending runtime error); the first lookup on a device
+ * may load the library's module there, so make the first call on each device outside
+ * any stream capture.
  */
 int sparse_attn_kmeans_noalloc(const uint16_t* x, int B, int H, int N, int d, int C, int iters,
                                double* centroids, int32_t* labels, int32_t* perm,
