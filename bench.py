@@ -50,6 +50,9 @@ def parse():
                     help="key-range splits of the forward (0: the library's choice)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run on this many heads instead of the workload's (profiler captures)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="measure only --workload (by default the metric workload's line also "
+                         "carries the other configurations under 'workloads')")
     return ap.parse_args()
 
 
@@ -127,19 +130,28 @@ def forward_traffic(w: W.Workload):
 
 
 def pool_bytes(w: W.Workload, with_q: bool) -> float:
-    """Algorithmic HBM bytes of one pool stage: read K, V (and Q), write the tables
-    and the fp16 copy of V; for order 2 also the two passes over M (global matrix,
-    covariance norms)."""
+    """Algorithmic HBM bytes of one pool stage, as the method defines its tables: read K, V
+    (and Q); write the query centroids, the KV centroids and value sums in fp32 with one
+    16-bit copy of each for the tensor cores, and (order 1 or 2) the first-order matrices
+    M_j in 16 bits; for order 2 also the two passes over M (global matrix, covariance
+    norms). Bytes this library writes beyond that are in :func:`pool_extra_bytes`."""
     bh = w.B * w.H
     rd = bh * w.Nk * w.d * 2 * 2 + (bh * w.Nq * w.d * 2 if with_q else 0)
-    wr = bh * w.nkb * w.d * (4 + 4 + 4 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
-    wr += bh * w.Nk * w.d * 2   # fp16 copy of V
+    wr = bh * w.nkb * w.d * (4 + 4 + 2 + 2) + (bh * w.nqb * w.d * 4 if with_q else 0)
     if w.order >= 1:
         wr += bh * w.nkb * w.d * w.d * 2
     if w.order == 2:  # the global matrix and the covariance norms read the M table twice
         rd += 2 * bh * w.nkb * w.d * w.d * 2
         wr += bh * w.d * w.d * 6 + bh * w.nkb * 4
     return float(rd + wr)
+
+
+def pool_extra_bytes(w: W.Workload) -> dict:
+    """Bytes the pool writes beyond the method's tables: the fp16 copy of V (the operand
+    of the forward's exact value products) and the second (low) bf16 plane of the
+    centroids."""
+    bh = w.B * w.H
+    return {"v16": float(bh * w.Nk * w.d * 2), "kbar16_lo": float(bh * w.nkb * w.d * 2)}
 
 
 def route_work(w: W.Workload):
@@ -366,6 +378,293 @@ def run_reference(args, w):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+OTHER_CONFIGS = ("uniform-4k", "dit-21x30x52", "longvideo-41x30x52", "worldmodel-chunk")
+
+
+def keep_label(w: W.Workload) -> str:
+    if w.mode == "topk":
+        return f"top {w.rho[0]}/{w.rho[1]}"
+    if w.mode == "topk_cov":
+        return f"top {w.rho[0]}/{w.rho[1]}, covariance-aware"
+    if w.mode == "ear":
+        return f"top {w.rho[0]}/{w.rho[1]}, error-aware"
+    if w.mode == "mass":
+        return f"mass {w.tau}"
+    return "window+anchors" + (f", adaptive budget {w.budget}" if w.budget else "")
+
+
+def launches_per_step(w: W.Workload, splits: int) -> int:
+    """Kernels of one step: pool, route or mask, forward (+ the split merge); hybrid order
+    adds the two passes over M, error-aware routing its probe, clustering 2 x (7 + 8 iters)
+    k-means launches plus three gathers and the output scatter."""
+    n = 5 if w.order == 2 else 4 if w.mode == "ear" else 3
+    n += 1 if splits > 1 else 0
+    if w.clusters:
+        n += 2 * (7 + 8 * w.clusters[2]) + 4
+    return n
+
+
+class Session:
+    """One GPU rank: device, stream and the collective helpers of dist.py."""
+
+    def __init__(self):
+        import torch
+        from free_block_sparse_kv_b200 import dist as D
+        self.torch, self.D = torch, D
+        self.world, self.rank, local = D.env_ranks()
+        torch.cuda.set_device(local)
+        self.dev = torch.device("cuda", local)
+        D.init("nccl", device=self.dev)
+        self.stream = torch.cuda.current_stream(self.dev)
+        props = torch.cuda.get_device_properties(self.dev)
+        dev_id = str(getattr(props, "uuid", local))
+        if dev_id and not dev_id.startswith("GPU-") and len(dev_id) == 36:
+            dev_id = "GPU-" + dev_id
+        self.dev_id = dev_id
+
+    def barrier(self):
+        self.D.barrier()
+
+    def max(self, x: float) -> float:
+        return self.D.max_over_ranks(x, device=self.dev)
+
+
+class Bench:
+    """A workload set up on one rank: pinned host inputs, device inputs, the operator."""
+
+    def __init__(self, ses: Session, w: W.Workload, splits=None):
+        torch = ses.torch
+        from free_block_sparse_kv_b200 import attention as A
+        self.A, self.ses, self.w = A, ses, w
+        wr = ses.D.rank_workload(w, ses.rank)   # weak scaling: each rank its own problem
+        qb, kb, vb = W.full_inputs_bits(wr)
+        as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        self.q_h, self.k_h, self.v_h = (as_t(x).pin_memory() for x in (qb, kb, vb))
+        del qb, kb, vb
+        self.q, self.k, self.v = (x.to(ses.dev) for x in (self.q_h, self.k_h, self.v_h))
+        self.p = A.Problem(w.B, w.H, w.Nq, w.Nk, w.d, w.block, w.order)
+        geometry = dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
+                        n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0,
+                        budget=w.budget)
+        self.op = A.BlockSparseAttention(self.p, w.mode, rho=w.rho, tau=w.tau,
+                                         geometry=geometry if w.mode == "structured" else None,
+                                         out_dtype=torch.float32, device=ses.dev,
+                                         clusters=w.clusters or None, splits=splits)
+        self.cycle = w.steps if w.mode == "structured" else (0,)
+
+    def stage_step(self, s, ev):
+        """One step with events around each stage: (clustering), pool, mask/route,
+        forward, (output back to the query order)."""
+        A, w, op, p, st = self.A, self.w, self.op, self.p, self.ses.stream
+        use_q = w.mode != "structured"
+        ev[0].record(st)
+        qq, kk, vv, out = self.q, self.k, self.v, op.out
+        if w.clusters:
+            qq, kk, vv = op.cluster(self.q, self.k, self.v)
+            out = op.out_p
+        ev[5].record(st)
+        A.pool(qq if use_q else None, kk, vv, p, op.tables)
+        ev[1].record(st)
+        if w.mode == "structured":
+            A.structured_mask(p, op.kv_idx, op.kv_cnt, w.frame_tokens, w.n_frames, w.window,
+                              w.n_anchors, w.period, s, w.q_frame0, budget=w.budget)
+            ev[4].record(st)
+        else:
+            if w.mode == "ear":
+                A.ear_scores(kk, vv, p, op.tables, err_flag=op.err_flag)
+            ev[4].record(st)
+            A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
+        ev[2].record(st)
+        op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, qq, kk, vv, out)
+        ev[3].record(st)
+        if w.clusters:
+            A.permute_rows(op.out_p, op.cl_q.perm, op.out, gather=False)
+        ev[6].record(st)
+
+    def run(self, steps: int, warmup: int) -> dict:
+        """W untimed steps, then `steps` timed steps between barriers (max over ranks)."""
+        torch, ses = self.ses.torch, self.ses
+        for i in range(warmup):
+            self.op(self.q, self.k, self.v, step=self.cycle[i % len(self.cycle)])
+        torch.cuda.synchronize(ses.dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ses.barrier()
+        torch.cuda.synchronize(ses.dev)
+        with ClockSampler(ses.dev_id) as clocks:
+            start.record(ses.stream)
+            for i in range(steps):
+                self.stage_step(self.cycle[i % len(self.cycle)], evs[i])
+            end.record(ses.stream)
+            torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        self.op.check()
+        mean = lambda a, b: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+        per_call = [e[0].elapsed_time(e[6]) for e in evs]
+        r = dict(ms_step=ses.max(start.elapsed_time(end) / steps), per_call=per_call,
+                 pool=mean(5, 1), route=mean(1, 2), forward=mean(2, 3),
+                 probe=mean(1, 4) if self.w.mode == "ear" else None,
+                 cluster=(mean(0, 5), mean(3, 6)) if self.w.clusters else None,
+                 clocks=clocks.summary())
+        if self.w.mode == "structured":  # one entry per denoising step of the cycle
+            by_step = {}
+            for i in range(steps):
+                by_step.setdefault(self.cycle[i % len(self.cycle)], []).append(per_call[i])
+            r["by_step"] = {str(st): float(np.mean(v)) for st, v in sorted(by_step.items())}
+        return r
+
+    def secondary(self, steps: int):
+        """World model: the frames before the chunk form a KV cache whose pooled tables carry
+        over between chunks; only the chunk's own blocks are pooled (labelled row)."""
+        torch, ses, A, w, op, p = self.ses.torch, self.ses, self.A, self.w, self.op, self.p
+        j0 = kv_cached_start(w)
+        if not j0:
+            return None
+        q, k, v = self.q, self.k, self.v
+        A.pool(q, k, v, p, op.tables)           # the cache's tables, once
+        torch.cuda.synchronize(ses.dev)
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        ses.barrier()
+        torch.cuda.synchronize(ses.dev)
+        for i in range(steps):
+            e = ev2[i]
+            e[0].record(ses.stream)
+            A.pool(q, k, v, p, op.tables, kv_block_start=j0)
+            e[1].record(ses.stream)
+            A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
+            e[2].record(ses.stream)
+            op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, q, k, v, op.out)
+            e[3].record(ses.stream)
+        torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        ms2 = ses.max(float(np.mean([e[0].elapsed_time(e[3]) for e in ev2])))
+        m = lambda a, b: float(np.mean([e[a].elapsed_time(e[b]) for e in ev2]))
+        return {"label": f"KV cache pooled once: only the chunk's blocks {j0}..{w.nkb - 1} "
+                         f"pooled per call",
+                "value": ses.D.weak_scaling_value(w.dense_flops(), ses.world, ms2), "unit": UNIT,
+                "ms_per_step": ms2,
+                "stages_ms": {"pool": m(0, 1), "route": m(1, 2), "forward": m(2, 3)}}
+
+    def graph(self, steps: int):
+        """The same steps replayed from CUDA graphs (one per denoising step of the cycle)."""
+        torch, ses, op = self.ses.torch, self.ses, self.op
+        graphs = {st: op.capture(self.q, self.k, self.v, step=st) for st in sorted(set(self.cycle))}
+        for st in self.cycle:
+            graphs[st].replay()
+        torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(ses.stream)
+        for i in range(steps):
+            graphs[self.cycle[i % len(self.cycle)]].replay()
+        g1.record(ses.stream)
+        torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        gms = ses.max(g0.elapsed_time(g1) / steps)
+        del graphs
+        return {"ms_per_step": gms,
+                "value": ses.D.weak_scaling_value(self.w.dense_flops(), ses.world, gms),
+                "unit": UNIT, "graphs": len(set(self.cycle))}
+
+    def e2e(self, steps: int) -> dict:
+        """Through the public host-buffer call: per step, Q, K, V go from pinned host memory
+        to the device and the output comes back, overlapped with the compute range by range
+        of heads and, across steps, with the neighbouring steps' compute."""
+        torch, ses, op = self.ses.torch, self.ses, self.op
+        out_h = torch.empty(op.out.shape, dtype=op.out.dtype, pin_memory=True)
+        op.run_from_host(self.q_h, self.k_h, self.v_h, out_h, step=0)
+        torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(ses.stream)
+        for i in range(steps):
+            op.run_from_host(self.q_h, self.k_h, self.v_h, out_h,
+                             step=self.cycle[i % len(self.cycle)])
+        op.wait_host_copies()   # the last output copy ends inside the timed region
+        s1.record(ses.stream)
+        torch.cuda.synchronize(ses.dev)
+        ses.barrier()
+        e2e_ms = ses.max(s0.elapsed_time(s1) / steps)
+        h2d = sum(x.numel() * x.element_size() for x in (self.q_h, self.k_h, self.v_h))
+        d2h = out_h.numel() * out_h.element_size()
+        return {"value": ses.D.weak_scaling_value(self.w.dense_flops(), ses.world, e2e_ms),
+                "unit": UNIT, "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)}
+
+    def report(self, r: dict, pk: dict) -> dict:
+        """Per-call figures and roofline fractions of one measured workload."""
+        w, op, ses = self.w, self.op, self.ses
+        kv_idx, kv_cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
+        fl = executed_flops(w, kv_idx, kv_cnt)
+        fwd_s = r["forward"] / 1e3
+        achieved = fl["total"] / fwd_s / 1e12
+        kept = fl["exact"] / fwd_s / 1e12
+        pool_s = r["pool"] / 1e3
+        pb = pool_bytes(w, w.mode != "structured")
+        extra = pool_extra_bytes(w)
+        rb, rf = route_work(w)
+        route_s = r["route"] / 1e3
+        out = {
+            "ms_per_call": r["ms_step"],
+            "ms_per_call_median": float(np.median(r["per_call"])),
+            "value": ses.D.weak_scaling_value(w.dense_flops(), ses.world, r["ms_step"]),
+            "unit": UNIT,
+            "stages_ms": {"pool": r["pool"], "route" if w.mode != "structured" else "mask":
+                          r["route"], "forward": r["forward"]},
+            "roofline": {"kernel": "sparse_attn_forward", "bound": "tensor", "achieved": achieved,
+                         "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_sustained"],
+                         "frac_of_burst": achieved / pk["bf16"],
+                         "kept_only": {"achieved": kept, "frac": kept / pk["bf16_sustained"],
+                                       "frac_of_burst": kept / pk["bf16"]},
+                         "traffic": forward_traffic(w),
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                         "peak_kind": f"bf16 sustained ({pk['source']}); frac_of_burst against "
+                                      f"the burst peak {pk['bf16']}",
+                         "flops_per_launch": fl},
+            "pool_roofline": {"bound": "hbm", "bytes": pb, "achieved": pb / pool_s / 1e9,
+                              "peak": pk["hbm"], "unit": "GB/s",
+                              "frac": pb / pool_s / 1e9 / pk["hbm"],
+                              "extra_bytes": extra,
+                              "frac_with_extra": (pb + sum(extra.values())) / pool_s / 1e9
+                              / pk["hbm"]},
+            "route_roofline": {"bound": "latency", "bytes": rb, "achieved_gbs": rb / route_s / 1e9,
+                               "hbm_frac": rb / route_s / 1e9 / pk["hbm"], "fp32_flops": rf,
+                               "fp32_frac": rf / route_s / 1e12 / FP32_PEAK_TFLOPS,
+                               "fp32_peak_tflops": FP32_PEAK_TFLOPS},
+            "clocks": r["clocks"],
+            "forward_splits": op.last_splits,
+        }
+        if "by_step" in r:
+            out["ms_per_call_by_step"] = r["by_step"]
+        if r["cluster"] is not None:
+            out["stages_ms"]["cluster"], out["stages_ms"]["unpermute"] = r["cluster"]
+        if r["probe"] is not None:
+            # the probe's algorithmic work: logits and the value product, each
+            # 2 * nqb * Nk * d per head (the 2-piece splits are not counted)
+            ear_fl = 4.0 * w.B * w.H * w.nqb * w.Nk * w.d
+            out["stages_ms"]["ear_probe"] = r["probe"]
+            out["ear_roofline"] = {"kernel": "sparse_attn_ear_scores", "bound": "tensor",
+                                   "achieved": ear_fl / (r["probe"] / 1e3) / 1e12,
+                                   "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                                   "frac": ear_fl / (r["probe"] / 1e3) / 1e12 / pk["bf16_sustained"],
+                                   "peak_kind": f"bf16 sustained ({pk['source']})",
+                                   "flops_per_launch": ear_fl}
+        return out
+
+
+def workload_config(w: W.Workload, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "block": w.block, "order": w.order, "mode": w.mode, "keep": keep_label(w),
+            "output": "fp32",
+            "l2": "inputs exceed L2 (Q+K+V %.2f GB per GPU)" % (
+                (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2) / 1e9) if
+            w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2 > 126e6 else
+            "inputs fit in L2 (%.1f MB): latency-bound small case" % (
+                (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2) / 1e6),
+            "parallelism": f"weak: {world} independent problems, one per GPU"}
+
+
 def main():
     args = parse()
     w = W.WORKLOADS[args.workload]
@@ -375,252 +674,69 @@ def main():
         run_reference(args, w)
         return
 
-    import torch
-    from free_block_sparse_kv_b200 import attention as A
-    from free_block_sparse_kv_b200 import dist as D
-
-    world, rank, local = D.env_ranks()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    D.init("nccl", device=dev)
-    barrier = D.barrier
-    max_over_ranks = lambda x: D.max_over_ranks(x, device=dev)
-
-    wr = D.rank_workload(w, rank)   # weak scaling: each rank its own problem
-    qb, kb, vb = W.full_inputs_bits(wr)
-    as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-    q_h, k_h, v_h = (as_t(x).pin_memory() for x in (qb, kb, vb))
-    del qb, kb, vb
-    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
-    p = A.Problem(w.B, w.H, w.Nq, w.Nk, w.d, w.block, w.order)
-    geometry = dict(frame_tokens=w.frame_tokens, n_frames=w.n_frames, window=w.window,
-                    n_anchors=w.n_anchors, period=w.period, q_frame0=w.q_frame0, budget=w.budget)
-    op = A.BlockSparseAttention(p, w.mode, rho=w.rho, tau=w.tau,
-                                geometry=geometry if w.mode == "structured" else None,
-                                out_dtype=torch.float32, device=dev,
-                                clusters=w.clusters or None, splits=args.splits or None)
-    stream = torch.cuda.current_stream(dev)
-    steps_cycle = w.steps if w.mode == "structured" else (0,)
-
-    def stage_step(s, ev):
-        """One step with events around each stage: (clustering), pool, mask/route,
-        forward, (output back to the query order)."""
-        use_q = w.mode != "structured"
-        ev[0].record(stream)
-        qq, kk, vv, out = q, k, v, op.out
-        if w.clusters:
-            qq, kk, vv = op.cluster(q, k, v)
-            out = op.out_p
-        ev[5].record(stream)
-        A.pool(qq if use_q else None, kk, vv, p, op.tables)
-        ev[1].record(stream)
-        if w.mode == "structured":
-            A.structured_mask(p, op.kv_idx, op.kv_cnt, w.frame_tokens, w.n_frames, w.window,
-                              w.n_anchors, w.period, s, w.q_frame0, budget=w.budget)
-        else:
-            if w.mode == "ear":
-                A.ear_scores(kk, vv, p, op.tables, err_flag=op.err_flag)
-                ev[4].record(stream)
-            A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
-        ev[2].record(stream)
-        op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, qq, kk, vv, out)
-        ev[3].record(stream)
-        if w.clusters:
-            A.permute_rows(op.out_p, op.cl_q.perm, op.out, gather=False)
-        ev[6].record(stream)
-
-    for i in range(args.warmup):
-        op(q, k, v, step=steps_cycle[i % len(steps_cycle)])
-    torch.cuda.synchronize(dev)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    props = torch.cuda.get_device_properties(dev)
-    dev_id = str(getattr(props, "uuid", local))
-    if dev_id and not dev_id.startswith("GPU-") and len(dev_id) == 36:
-        dev_id = "GPU-" + dev_id
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev_id) as clocks:
-        start.record(stream)
-        for i in range(args.steps):
-            stage_step(steps_cycle[i % len(steps_cycle)], evs[i])
-        end.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier()
-    op.check()
-    ms_step = start.elapsed_time(end) / args.steps
-    ms_step_max = max_over_ranks(ms_step)
-    mean_ms = lambda a, b: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
-    per_call = [e[0].elapsed_time(e[6]) for e in evs]  # each timed step, start to end
-    stage_ms = [mean_ms(5, 1), mean_ms(1, 2), mean_ms(2, 3)]  # pool, route / mask, forward
-    cluster_ms = (mean_ms(0, 5), mean_ms(3, 6)) if w.clusters else None
-    # error-aware routing: the probe's share of the route stage (events 1 -> 4)
-    ear_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs])) if w.mode == "ear" else None
-
-    # The same steps replayed from CUDA graphs (one per denoising step of the cycle): no
-    # host work per launch. Reported beside the eager figure.
-    graph = None
-    if args.graphs:
-        graphs = {st: op.capture(q, k, v, step=st) for st in sorted(set(steps_cycle))}
-        for st in steps_cycle:
-            graphs[st].replay()
-        torch.cuda.synchronize(dev)
-        barrier()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for i in range(args.steps):
-            graphs[steps_cycle[i % len(steps_cycle)]].replay()
-        g1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        gms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
-        graph = {"ms_per_step": gms, "value": D.weak_scaling_value(w.dense_flops(), world, gms),
-                 "unit": UNIT, "graphs": len(graphs)}
-        del graphs
-
-    # World model: the frames before the chunk form a KV cache whose pooled tables carry
-    # over between chunks; only the chunk's own blocks are pooled (labelled secondary row).
-    secondary = None
-    j0 = kv_cached_start(w)
-    if j0:
-        A.pool(q, k, v, p, op.tables)           # the cache's tables, once
-        torch.cuda.synchronize(dev)
-        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-        barrier()
-        torch.cuda.synchronize(dev)
-        for i in range(args.steps):
-            e = ev2[i]
-            e[0].record(stream)
-            A.pool(q, k, v, p, op.tables, kv_block_start=j0)
-            e[1].record(stream)
-            A.route(p, op.tables, op.kv_idx, op.kv_cnt, w.mode, w.rho, w.tau)
-            e[2].record(stream)
-            op.forward_stage(p, op.tables, op.kv_idx, op.kv_cnt, q, k, v, op.out)
-            e[3].record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        ms2 = max_over_ranks(float(np.mean([e[0].elapsed_time(e[3]) for e in ev2])))
-        secondary = {"label": f"KV cache pooled once: only the chunk's blocks {j0}..{w.nkb - 1} "
-                              f"pooled per call",
-                     "value": D.weak_scaling_value(w.dense_flops(), world, ms2), "unit": UNIT,
-                     "ms_per_step": ms2,
-                     "stages_ms": {"pool": float(np.mean([e[0].elapsed_time(e[1]) for e in ev2])),
-                                   "route": float(np.mean([e[1].elapsed_time(e[2]) for e in ev2])),
-                                   "forward": float(np.mean([e[2].elapsed_time(e[3]) for e in ev2]))}}
-
-    # per-launch forward work for the lists of the last step
-    kv_idx, kv_cnt = op.kv_idx.cpu().numpy(), op.kv_cnt.cpu().numpy()
-    fl = executed_flops(w, kv_idx, kv_cnt)
+    ses = Session()
     pk = peaks()
-    fwd_s = stage_ms[2] / 1e3
-    achieved = fl["total"] / fwd_s / 1e12
-    value = D.weak_scaling_value(w.dense_flops(), world, ms_step_max)
+    b = Bench(ses, w, splits=args.splits or None)
+    r = b.run(args.steps, args.warmup)
+    graph = b.graph(args.steps) if args.graphs else None
+    secondary = b.secondary(args.steps)
+    rep = b.report(r, pk)
+    e2e = None if args.no_e2e else b.e2e(args.e2e_steps)
+    launches = launches_per_step(w, b.op.last_splits) * args.steps
+    del b
 
-    # end to end through the public API from pinned host buffers
-    e2e = None
-    if not args.no_e2e:
-        # through the public host-buffer call: per step, Q, K, V go from pinned host
-        # memory to the device and the output comes back, overlapped with the compute
-        # range by range of heads and, across steps, with the neighbouring steps' compute
-        out_h = torch.empty(op.out.shape, dtype=op.out.dtype, pin_memory=True)
-        op.run_from_host(q_h, k_h, v_h, out_h, step=0)
-        torch.cuda.synchronize(dev)
-        barrier()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for i in range(args.e2e_steps):
-            op.run_from_host(q_h, k_h, v_h, out_h, step=steps_cycle[i % len(steps_cycle)])
-        op.wait_host_copies()   # the last output copy ends inside the timed region
-        s1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps)
-        h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
-        d2h = out_h.numel() * out_h.element_size()
-        e2e = {"value": D.weak_scaling_value(w.dense_flops(), world, e2e_ms), "unit": UNIT,
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    # The other configurations of the benchmark set, each measured the same way in this
+    # run (one GPU only: every rank would otherwise generate every workload's inputs).
+    others = {}
+    if ses.world == 1 and not args.no_workloads and w.name == W.METRIC_WORKLOAD:
+        for name in OTHER_CONFIGS:
+            wo = W.WORKLOADS[name]
+            bo = Bench(ses, wo)
+            steps = max(args.steps, len(bo.cycle))
+            ro = bo.run(steps, max(args.warmup, 3))
+            entry = {"config": workload_config(wo, ses.world), "steps": steps,
+                     "warmup": max(args.warmup, 3), **bo.report(ro, pk)}
+            sec = bo.secondary(steps)
+            if sec is not None:
+                entry["secondary"] = sec
+            launches += launches_per_step(wo, bo.op.last_splits) * steps
+            others[name] = entry
+            del bo
+            ses.torch.cuda.empty_cache()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if ses.rank == 0 and ses.world == 1 and not args.no_cpu_baseline:
         res = time_oracle(w, args.cpu_seconds)
         cpu = {k: res[k] for k in ("value", "unit", "cores", "cpu_count", "blas", "kind", "sample")}
 
-    if rank == 0:
-        peak = pk["bf16_sustained"]
+    if ses.rank == 0:
+        value = ses.D.weak_scaling_value(w.dense_flops(), ses.world, r["ms_step"])
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
-                       "block": w.block, "order": w.order, "mode": w.mode,
-                       "keep": (f"top {w.rho[0]}/{w.rho[1]}" if w.mode == "topk" else
-                                f"top {w.rho[0]}/{w.rho[1]}, covariance-aware"
-                                if w.mode == "topk_cov" else
-                                f"top {w.rho[0]}/{w.rho[1]}, error-aware"
-                                if w.mode == "ear" else
-                                f"mass {w.tau}" if w.mode == "mass" else "window+anchors"),
-                       "output": "fp32",
-                       "l2": "inputs exceed L2 (Q+K+V %.2f GB per GPU)" % (
-                           (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2) / 1e9),
-                       "parallelism": f"weak: {world} independent problems, one per GPU"},
-            "pct_of_bf16_peak_dense_equiv": 100.0 * value / world / pk["bf16"],
-            "stages_ms": {"pool": stage_ms[0], "route" if w.mode != "structured" else "mask":
-                          stage_ms[1], "forward": stage_ms[2]},
-            "roofline": {"kernel": "sparse_attn_forward", "bound": "tensor",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": forward_traffic(w),
-                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                         "peak_kind": f"bf16 sustained ({pk['source']})",
-                         "flops_per_launch": fl},
-            "pool_roofline": {"bound": "hbm", "achieved": pool_bytes(w, w.mode != "structured")
-                              / (stage_ms[0] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s"},
-            "clocks": clocks.summary(),
-            "gpu_launches": ((5 if w.order == 2 else 4 if w.mode == "ear" else 3)
-                             + (1 if op.last_splits > 1 else 0)  # the merge of the splits
-                             + (2 * (7 + 8 * w.clusters[2]) + 4 if w.clusters else 0))
-                            * args.steps,
-            "forward_splits": op.last_splits,
-            "e2e": e2e,
-            "cpu_baseline": cpu,
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ses.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(w, ses.world),
+            "pct_of_bf16_peak_dense_equiv": 100.0 * value / ses.world / pk["bf16"],
+            "stages_ms": rep["stages_ms"], "roofline": rep["roofline"],
+            "pool_roofline": rep["pool_roofline"], "route_roofline": rep["route_roofline"],
+            "clocks": rep["clocks"], "gpu_launches": launches,
+            "forward_splits": rep["forward_splits"], "e2e": e2e, "cpu_baseline": cpu,
+            "ms_per_call_median": rep["ms_per_call_median"],
         }
-        line["pool_roofline"]["frac"] = line["pool_roofline"]["achieved"] / pk["hbm"]
-        line["ms_per_call_median"] = float(np.median(per_call))
-        if w.mode == "structured":  # one entry per denoising step of the cycle
-            by_step = {}
-            for i in range(args.steps):
-                by_step.setdefault(steps_cycle[i % len(steps_cycle)], []).append(per_call[i])
-            line["ms_per_call_by_step"] = {str(st): float(np.mean(v))
-                                           for st, v in sorted(by_step.items())}
-        rb, rf = route_work(w)
-        line["route_roofline"] = {"bound": "latency", "bytes": rb, "achieved_gbs":
-                                  rb / (stage_ms[1] / 1e3) / 1e9, "hbm_frac":
-                                  rb / (stage_ms[1] / 1e3) / 1e9 / pk["hbm"],
-                                  "fp32_flops": rf, "fp32_frac": rf / (stage_ms[1] / 1e3) / 1e12
-                                  / FP32_PEAK_TFLOPS, "fp32_peak_tflops": FP32_PEAK_TFLOPS}
+        for key in ("ms_per_call_by_step", "ear_roofline"):
+            if key in rep:
+                line[key] = rep[key]
         if secondary is not None:
             line["secondary"] = secondary
         if graph is not None:
             line["graph"] = graph
-        if cluster_ms is not None:
-            line["stages_ms"]["cluster"] = cluster_ms[0]
-            line["stages_ms"]["unpermute"] = cluster_ms[1]
+        if w.clusters:
             line["config"]["clusters"] = {"C_q": w.clusters[0], "C_k": w.clusters[1],
                                           "iters": w.clusters[2]}
-        if ear_ms is not None:
-            # the probe's algorithmic work: logits and the value product, each
-            # 2 * nqb * Nk * d per head (the 2-piece splits are not counted)
-            ear_fl = 4.0 * w.B * w.H * w.nqb * w.Nk * w.d
-            line["stages_ms"]["ear_probe"] = ear_ms
-            line["ear_roofline"] = {"kernel": "sparse_attn_ear_scores", "bound": "tensor",
-                                    "achieved": ear_fl / (ear_ms / 1e3) / 1e12,
-                                    "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                                    "peak_kind": f"bf16 sustained ({pk['source']})",
-                                    "flops_per_launch": ear_fl}
-            line["ear_roofline"]["frac"] = (line["ear_roofline"]["achieved"]
-                                            / pk["bf16_sustained"])
+        if others:
+            line["workloads"] = others
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if ses.world > 1:
         import torch.distributed as tdist
         tdist.destroy_process_group()
 

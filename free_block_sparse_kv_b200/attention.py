@@ -119,17 +119,18 @@ def _check_inputs(q, k, v):
             raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor [B,H,N,d]")
 
 
-def pool(q, k, v, p: Problem, t: Tables, stream=None, kv_block_start: int = 0):
+def pool(q, k, v, p: Problem, t: Tables, stream=None, kv_block_start: int = 0, err_flag=None):
     """Pooled tables; with order 2 also the global first-order matrix and the
     per-block covariance norms. kv_block_start > 0 pools only the KV blocks from there
-    on (a growing KV cache whose earlier blocks were pooled by an earlier call)."""
+    on (a growing KV cache whose earlier blocks were pooled by an earlier call).
+    err_flag (device int32) receives SA_FLAG_RANGE if an fp16 table value overflows."""
     if kv_block_start:
         C.sparse_attn_pool_incremental(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order,
                                        kv_block_start, t.qbar, t.kbar_t, t.vsum, t.kbar16,
-                                       t.vsum16, t.M, t.v16, stream)
+                                       t.vsum16, t.M, t.v16, err_flag, stream)
     else:
         C.sparse_attn_pool(q, k, v, p.B, p.H, p.Nq, p.Nk, p.d, p.block, p.order, t.qbar,
-                           t.kbar_t, t.vsum, t.kbar16, t.vsum16, t.M, t.v16, stream)
+                           t.kbar_t, t.vsum, t.kbar16, t.vsum16, t.M, t.v16, err_flag, stream)
     if p.order == 2:
         C.sparse_attn_hbar(t.M, p.B, p.H, p.nkb, p.d, t.hbar, t.hbar16, t.cov, stream)
 
@@ -292,7 +293,8 @@ class BlockSparseAttention:
             self._attend(p, t, idx, cnt, q, k, v, out, step, stream)
 
     def _attend(self, p, t, kv_idx, kv_cnt, q, k, v, out, step, stream):
-        pool(q if self.mode != "structured" else None, k, v, p, t, stream)
+        pool(q if self.mode != "structured" else None, k, v, p, t, stream,
+             err_flag=self.err_flag)
         if self.mode == "structured":
             g = self.geometry
             structured_mask(p, kv_idx, kv_cnt, g["frame_tokens"], g["n_frames"],
@@ -406,7 +408,14 @@ class BlockSparseAttention:
             torch.cuda.current_stream(self.out.device).wait_stream(self._d2h)
 
     def check(self):
-        """Raise if a bounded device wait of an earlier call gave up (synchronises)."""
+        """Raise if an earlier call failed on the device (synchronises): SA_ERR_RANGE when a
+        pooled fp16 table value did not fit (the output is then not valid), SA_ERR_TIMEOUT
+        when a bounded device wait gave up. The flag is sticky: it stays set until cleared
+        with ``err_flag.zero_()``."""
         flag = int(self.err_flag.item())
+        if flag & C.SA_FLAG_RANGE:
+            raise C.SparseAttnError(C.SA_ERR_RANGE, "a pooled fp16 table value (V copy, value "
+                                    "sum or M_j) does not fit in fp16 (|x| >= 65520); scale V "
+                                    f"down by a power of two (flag {flag:#x})")
         if flag:
             raise C.SparseAttnError(C.SA_ERR_TIMEOUT, f"device wait timed out (flag {flag:#x})")

@@ -98,7 +98,7 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Nq,
                      int Nk, int d, int block, int order, float* qbar, float* kbar_t, float* vsum,
                      uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
-                     void* stream) {
+                     int32_t* err_flag, void* stream) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
   SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
   const bool do_q = q != nullptr && Nq > 0;
@@ -117,9 +117,11 @@ int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
     SA_REQUIRE_PTR(q);
     SA_REQUIRE_PTR(qbar);
   }
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
   if (int rc = check_device()) return rc;
   sa::PoolArgs p{do_q ? q : nullptr, k, v, B, H, Nq, Nk, d, block, order,
-                 cdiv(Nq, block), cdiv(Nk, block), qbar, kbar_t, vsum, kbar16, vsum16, M, v16};
+                 cdiv(Nq, block), cdiv(Nk, block), qbar, kbar_t, vsum, kbar16, vsum16, M, v16,
+                 0, err_flag};
   return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
 }
 
@@ -127,7 +129,7 @@ int sparse_attn_pool_incremental(const uint16_t* q, const uint16_t* k, const uin
                                  int H, int Nq, int Nk, int d, int block, int order,
                                  int kv_block_start, float* qbar, float* kbar_t, float* vsum,
                                  uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
-                                 void* stream) {
+                                 int32_t* err_flag, void* stream) {
   if (int rc = check_shape(B, H, Nq, Nk, d, block)) return rc;
   SA_REQUIRE(order >= 0 && order <= 2, "order must be 0, 1 or 2");
   const int nkb = cdiv(Nk, block);
@@ -149,10 +151,11 @@ int sparse_attn_pool_incremental(const uint16_t* q, const uint16_t* k, const uin
     SA_REQUIRE_PTR(q);
     SA_REQUIRE_PTR(qbar);
   }
+  if (err_flag) SA_REQUIRE(((uintptr_t)err_flag & 3u) == 0, "err_flag must be 4-byte aligned");
   if (int rc = check_device()) return rc;
   sa::PoolArgs p{do_q ? q : nullptr, k, v, B, H, Nq, kv_block_start < nkb ? Nk : 0, d, block,
                  order, cdiv(Nq, block), nkb, qbar, kbar_t, vsum, kbar16, vsum16, M, v16,
-                 kv_block_start};
+                 kv_block_start, err_flag};
   return launched(sa::launch_pool(p, static_cast<cudaStream_t>(stream)), "pool launch");
 }
 

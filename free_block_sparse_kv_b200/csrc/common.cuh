@@ -21,6 +21,10 @@ SA_DEVI uint32_t smem_u32(const void* p) {
 SA_DEVI void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
 }
+// 4-byte async copy global -> shared (through L1); src_bytes 0 writes a zero.
+SA_DEVI void cp_async4(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
+}
 SA_DEVI void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 SA_DEVI void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }

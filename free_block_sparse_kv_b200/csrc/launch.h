@@ -12,6 +12,7 @@ struct PoolArgs {
   float *qbar, *kbar_t, *vsum;
   uint16_t *kbar16, *vsum16, *M, *v16;
   int j0 = 0;  // first KV block pooled (the tables of blocks < j0 are left as they are)
+  int32_t* err_flag = nullptr;  // SA_FLAG_RANGE when an fp16 value does not fit
 };
 
 struct RouteArgs {

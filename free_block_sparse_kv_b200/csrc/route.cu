@@ -7,20 +7,24 @@
 // Attention for Long Video Diffusion" §2 (A(t) = G u W(t), anchors shifted by
 // s mod T_per).
 //
-// Route kernel: one CTA of 8 warps per (batch*head, 8 query blocks).
-//   1. Scores s_ij = scale * qbar_i . kbar_j in fp32: thread j streams column j of
-//      the dim-major centroid table (coalesced), the 8 qbar rows are broadcast from
-//      shared memory.
+// Route kernel: one CTA of 8 warps per (batch*head, R query blocks), R = 16 (8 when a
+// row holds more than 1024 key blocks).
+//   1. Scores s_ij = scale * qbar_i . kbar_j in fp32 for the CTA's R rows. The head's
+//      dim-major centroid table streams through shared memory in chunks of a few
+//      dimensions (all key blocks of each; 4-byte cp.async, double-buffered, so many
+//      loads are in flight per thread); each thread accumulates an 8-row x MC-column
+//      tile with fp32 FMAs, the 8 rows' qbar values broadcast from shared memory.
+//      Every score is one fma chain over d = 0 .. D-1 in order.
 //   2. One warp per query block selects (select_row): a 32-step search over
 //      order-preserving score keys held in registers finds the threshold, ties at
 //      the threshold are taken in ascending block index, and the kept indices are
 //      written in ascending order with ballots.
 #include "common.cuh"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace sa {
 
-constexpr int kRouteRows = 8;      // query blocks per CTA (one warp each)
 constexpr int kRouteThreads = 256;
 
 
@@ -127,84 +131,129 @@ SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, 
   if (lane == 0) *cnt_out = min(off, cap);
 }
 
-template <int D, int SLOTS>
-__global__ void __launch_bounds__(kRouteThreads)
+// Shared-memory bytes of one route CTA: qbar block, two chunks of the centroid table,
+// the score rows.
+template <int D, int RG, int MC, int KD>
+constexpr size_t route_smem(int nkb) {
+  return (size_t)(D * 8 * RG + 2 * KD * (kRouteThreads / RG) * MC + 8 * RG * nkb) * 4;
+}
+
+template <int D, int SLOTS, int RG, int MC, int KD>
+__global__ void __launch_bounds__(kRouteThreads, SLOTS <= 32 ? 2 : 1)
 route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, int nqb, int nkb,
              int mode, int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
              int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov,
              const float* __restrict__ pre) {
+  constexpr int R = 8 * RG;                  // query blocks per CTA
+  constexpr int CT = kRouteThreads / RG;     // column threads per group of 8 rows
+  constexpr int NKP = CT * MC;               // key blocks per chunk row (padded)
+  constexpr int NCH = D / KD;                // chunks of KD dimensions
+  static_assert(D % KD == 0, "route chunks");
   extern __shared__ __align__(16) float rsm[];
-  float* qs = rsm;                         // [D][kRouteRows]
-  float* sc = rsm + D * kRouteRows;        // [kRouteRows][nkb] scores
+  float* qs = rsm;                           // [D][R]: qs[c * R + r] = qbar of row r, dim c
+  float* kc = qs + D * R;                    // [2][KD][NKP] chunks of the centroid table
+  float* sc = kc + 2 * KD * NKP;             // [R][nkb] scores
   const int tid = threadIdx.x;
   const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kRouteRows;
-  const int rows = min(kRouteRows, nqb - i0);
-
-  for (int x = tid; x < D * kRouteRows && !pre; x += kRouteThreads) {
-    const int r = x % kRouteRows, c = x / kRouteRows;
-    qs[x] = (r < rows) ? qbar[((size_t)bh * nqb + i0 + r) * D + c] : 0.f;
-  }
-  __syncthreads();
+  const int i0 = blockIdx.x * R;
+  const int rows = min(R, nqb - i0);
 
   if (pre) {
     // precomputed scores (error-aware routing): copy the rows, coalesced
     for (int r = 0; r < rows; ++r)
       for (int j = tid; j < nkb; j += kRouteThreads)
         sc[r * nkb + j] = pre[((size_t)bh * nqb + i0 + r) * nkb + j];
-  }
-  const float* kt = kbar_t + (size_t)bh * D * nkb;
-  for (int j = tid; j < nkb && !pre; j += kRouteThreads) {
-    float acc[kRouteRows];
-#pragma unroll
-    for (int r = 0; r < kRouteRows; ++r) acc[r] = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-      const float kv = kt[(size_t)c * nkb + j];
-      const float4 qa = *reinterpret_cast<const float4*>(qs + c * kRouteRows);
-      const float4 qb = *reinterpret_cast<const float4*>(qs + c * kRouteRows + 4);
-      acc[0] = fmaf(qa.x, kv, acc[0]);
-      acc[1] = fmaf(qa.y, kv, acc[1]);
-      acc[2] = fmaf(qa.z, kv, acc[2]);
-      acc[3] = fmaf(qa.w, kv, acc[3]);
-      acc[4] = fmaf(qb.x, kv, acc[4]);
-      acc[5] = fmaf(qb.y, kv, acc[5]);
-      acc[6] = fmaf(qb.z, kv, acc[6]);
-      acc[7] = fmaf(qb.w, kv, acc[7]);
+  } else {
+    const float* kt = kbar_t + (size_t)bh * D * nkb;
+    auto load_chunk = [&](int ch, int buf) {
+      float* dst = kc + buf * KD * NKP;
+      for (int x = tid; x < KD * NKP; x += kRouteThreads) {
+        const int k = x / NKP, j = x % NKP;
+        const bool ok = j < nkb;
+        cp_async4(smem_u32(dst + x), ok ? kt + (size_t)(ch * KD + k) * nkb + j : kt, ok ? 4 : 0);
+      }
+      cp_async_commit();
+    };
+    load_chunk(0, 0);
+    if (NCH > 1) load_chunk(1, 1);
+    for (int x = tid; x < D * R; x += kRouteThreads) {
+      const int r = x / D, c = x % D;   // coalesced along c
+      qs[c * R + r] = r < rows ? qbar[((size_t)bh * nqb + i0 + r) * D + c] : 0.f;
     }
-    // covariance-aware top-k: the log of block j's covariance norm joins every row's score
-    const float bias = cov ? logf(cov[(size_t)bh * nkb + j]) : 0.f;
+    const int rg = tid / CT, ct = tid % CT;   // a warp shares its group of 8 rows
+    // acc[r][m]: row r of the group, column ct + CT m
+    float acc[8][MC];
 #pragma unroll
-    for (int r = 0; r < kRouteRows; ++r) sc[r * nkb + j] = scale * acc[r] + bias;
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int m = 0; m < MC; ++m) acc[r][m] = 0.f;
+    for (int ch = 0; ch < NCH; ++ch) {
+      if (ch + 1 < NCH) cp_async_wait<1>(); else cp_async_wait<0>();
+      __syncthreads();  // chunk ch (and the qbar block) visible to every thread
+      const float* kb = kc + (ch & 1) * KD * NKP;
+#pragma unroll
+      for (int k = 0; k < KD; ++k) {
+        const int c = ch * KD + k;
+        const float4 q0 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8);
+        const float4 q1 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8 + 4);
+        const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int m = 0; m < MC; ++m) {
+          const float kv = kb[k * NKP + ct + CT * m];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) acc[r][m] = fmaf(qv[r], kv, acc[r][m]);
+        }
+      }
+      __syncthreads();  // every thread is done with this buffer before it is refilled
+      if (ch + 2 < NCH) load_chunk(ch + 2, ch & 1);
+    }
+#pragma unroll
+    for (int m = 0; m < MC; ++m) {
+      const int j = ct + CT * m;
+      if (j >= nkb) continue;
+      // covariance-aware top-k: the log of block j's covariance norm joins every row's score
+      const float bias = cov ? logf(cov[(size_t)bh * nkb + j]) : 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) sc[(rg * 8 + r) * nkb + j] = scale * acc[r][m] + bias;
+    }
   }
   __syncthreads();
 
   const int warp = tid / 32, lane = tid % 32;
-  if (warp >= rows) return;
-  select_row<SLOTS>(sc + warp * nkb, nkb, mode, keep, tau,
-                    kv_idx + ((size_t)bh * nqb + i0 + warp) * cap, kv_cnt + (size_t)bh * nqb + i0 + warp,
-                    cap, lane);
+  for (int r = warp; r < rows; r += kRouteThreads / 32)
+    select_row<SLOTS>(sc + r * nkb, nkb, mode, keep, tau,
+                      kv_idx + ((size_t)bh * nqb + i0 + r) * cap, kv_cnt + (size_t)bh * nqb + i0 + r,
+                      cap, lane);
 }
 
-template <int D, int SLOTS>
+template <int D, int SLOTS, int RG, int MC, int KD>
 static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
-  const size_t smem = (size_t)(D * kRouteRows + kRouteRows * p.nkb) * sizeof(float);
-  auto kern = route_kernel<D, SLOTS>;
+  const size_t smem = route_smem<D, RG, MC, KD>(p.nkb);
+  auto kern = route_kernel<D, SLOTS, RG, MC, KD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.nqb + kRouteRows - 1) / kRouteRows, p.B * p.H);
+  dim3 grid((p.nqb + 8 * RG - 1) / (8 * RG), p.B * p.H);
   kern<<<grid, kRouteThreads, smem, st>>>(p.qbar, p.kbar_t, p.nqb, p.nkb, p.mode, p.keep, p.tau,
                                           p.scale, p.kv_idx, p.kv_cnt, p.cap, p.cov, p.scores);
   return cudaGetLastError();
 }
 
+// Key slots per lane (select_row) and columns per thread (scoring) from nkb: up to 1024
+// key blocks, two groups of 8 rows share the columns (MC = ceil(nkb / 128)); beyond,
+// one group of 8 rows (MC = ceil(nkb / 256)). Chunks of 8 dimensions while the chunk
+// stays small, else 4.
 template <int D>
 static cudaError_t launch_route_d(const RouteArgs& p, cudaStream_t st) {
-  if (p.nkb <= 128) return launch_route_t<D, 4>(p, st);
-  if (p.nkb <= 256) return launch_route_t<D, 8>(p, st);
-  if (p.nkb <= 512) return launch_route_t<D, 16>(p, st);
-  if (p.nkb <= 1024) return launch_route_t<D, 32>(p, st);
-  if (p.nkb <= 2048) return launch_route_t<D, 64>(p, st);
+  const int n = p.nkb;
+  if (n <= 128) return launch_route_t<D, 4, 2, 1, 8>(p, st);
+  if (n <= 256) return launch_route_t<D, 8, 2, 2, 8>(p, st);
+  if (n <= 384) return launch_route_t<D, 12, 2, 3, 8>(p, st);
+  if (n <= 512) return launch_route_t<D, 16, 2, 4, 8>(p, st);
+  if (n <= 640) return launch_route_t<D, 20, 2, 5, 8>(p, st);
+  if (n <= 768) return launch_route_t<D, 24, 2, 6, 4>(p, st);
+  if (n <= 1024) return launch_route_t<D, 32, 2, 8, 4>(p, st);
+  if (n <= 1536) return launch_route_t<D, 48, 1, 6, 4>(p, st);
+  if (n <= 2048) return launch_route_t<D, 64, 1, 8, 4>(p, st);
   return cudaErrorInvalidValue;
 }
 

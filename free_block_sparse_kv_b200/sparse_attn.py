@@ -13,7 +13,8 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libsparse_attn.so")
 
-SA_OK, SA_ERR_INVALID, SA_ERR_LAUNCH, SA_ERR_TIMEOUT, SA_ERR_UNSUPPORTED = range(5)
+SA_OK, SA_ERR_INVALID, SA_ERR_LAUNCH, SA_ERR_TIMEOUT, SA_ERR_UNSUPPORTED, SA_ERR_RANGE = range(6)
+SA_FLAG_RANGE = 1 << 20   # err_flag bit: a pooled fp16 table value did not fit
 SA_ROUTE_TOPK, SA_ROUTE_MASS = 0, 1
 SA_OUT_F32, SA_OUT_BF16 = 0, 1
 
@@ -51,8 +52,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sparse_attn_last_error.restype = ctypes.c_char_p
     lib.sparse_attn_last_error.argtypes = []
     lib.sparse_attn_table_sizes.argtypes = [_I] * 7 + [ctypes.POINTER(ctypes.c_size_t)]
-    lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 7 + [_P]
-    lib.sparse_attn_pool_incremental.argtypes = [_P, _P, _P] + [_I] * 8 + [_P] * 7 + [_P]
+    lib.sparse_attn_pool.argtypes = [_P, _P, _P] + [_I] * 7 + [_P] * 8 + [_P]
+    lib.sparse_attn_pool_incremental.argtypes = [_P, _P, _P] + [_I] * 8 + [_P] * 8 + [_P]
     lib.sparse_attn_route.argtypes = [_P, _P] + [_I] * 8 + [_F, _F, _P, _P, _I, _P]
     lib.sparse_attn_route_cov.argtypes = [_P, _P, _P] + [_I] * 7 + [_F, _P, _P, _I, _P]
     lib.sparse_attn_hbar.argtypes = [_P] + [_I] * 4 + [_P, _P, _P, _P]
@@ -106,17 +107,19 @@ def sparse_attn_table_sizes(B, H, Nq, Nk, d, block, order):
 
 
 def sparse_attn_pool(q, k, v, B, H, Nq, Nk, d, block, order, qbar, kbar_t, vsum, kbar16, vsum16, M,
-                     v16, stream=None):
+                     v16, err_flag=None, stream=None):
     _check(load_library().sparse_attn_pool(
         _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, block, order, _ptr(qbar), _ptr(kbar_t),
-        _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _stream(stream)))
+        _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _ptr(err_flag),
+        _stream(stream)))
 
 
 def sparse_attn_pool_incremental(q, k, v, B, H, Nq, Nk, d, block, order, kv_block_start, qbar,
-                                 kbar_t, vsum, kbar16, vsum16, M, v16, stream=None):
+                                 kbar_t, vsum, kbar16, vsum16, M, v16, err_flag=None, stream=None):
     _check(load_library().sparse_attn_pool_incremental(
         _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, block, order, kv_block_start, _ptr(qbar),
-        _ptr(kbar_t), _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _stream(stream)))
+        _ptr(kbar_t), _ptr(vsum), _ptr(kbar16), _ptr(vsum16), _ptr(M), _ptr(v16), _ptr(err_flag),
+        _stream(stream)))
 
 
 def sparse_attn_route(qbar, kbar_t, B, H, nqb, nkb, d, mode, rho_num, rho_den, tau, scale, kv_idx,

@@ -50,8 +50,14 @@ enum {
   SA_ERR_INVALID = 1,      /* bad shape, null or misaligned pointer, capacity too small */
   SA_ERR_LAUNCH = 2,       /* a CUDA launch or runtime call failed */
   SA_ERR_TIMEOUT = 3,      /* a bounded device wait gave up (reported through err_flag) */
-  SA_ERR_UNSUPPORTED = 4   /* the current device is not sm_100 */
+  SA_ERR_UNSUPPORTED = 4,  /* the current device is not sm_100 */
+  SA_ERR_RANGE = 5         /* a pooled fp16 table value does not fit (reported through err_flag) */
 };
+
+/* Bit set in err_flag by the pool when a value of its fp16 outputs (V copy, value sums,
+ * M_j) would round to infinity (|x| >= 65520). The other bits of err_flag mark bounded
+ * device waits that gave up (SA_ERR_TIMEOUT). */
+#define SA_FLAG_RANGE (1 << 20)
 
 enum { SA_ROUTE_TOPK = 0, SA_ROUTE_MASS = 1 };
 enum { SA_OUT_F32 = 0, SA_OUT_BF16 = 1 };
@@ -88,18 +94,26 @@ int sparse_attn_table_sizes(int B, int H, int Nq, int Nk, int d, int block, int 
  *   M       [B,H,nkb,d,d] fp16  M_j[a][c] = sum_r (k_r[a] - kbar_j[a]) v_r[c],
  *                               a = key dim (rows), c = value dim; fp32 accumulate
  *   v16     [B,H,Nk,d]   fp16   V converted to fp16 (exact for |v| in the fp16
- *                               normal range; |v| must stay below 65504)
- * vsum16, M and v16 are IEEE fp16 (11-bit significand): the forward runs every
- * product that involves probabilities in fp16 with fp32 accumulation. Logits use
- * the bf16 Q against the bf16 K as given (kept tokens) or against both centroid
- * planes (skipped blocks).
- * Means of a partial last block use its true token count.
+ *                               normal range)
+ *   err_flag  optional device int32 (4-byte aligned): SA_FLAG_RANGE is ORed into it
+ *             when a value of vsum16, M or v16 does not fit in fp16 (|x| >= 65520; the
+ *             table then holds an infinity and the forward's output is not valid), other
+ *             bits when a bounded device wait gave up. NULL: nothing is reported.
+ * Precision departs from a bf16 table format on purpose: vsum16, M and v16 are IEEE
+ * fp16 (11-bit significand against bf16's 8), because the forward multiplies them by
+ * probabilities (also fp16) on the tensor cores, and bf16 probabilities would put up to
+ * ~2^-8 relative error on single dominant terms; fp16's narrower range is what
+ * err_flag guards. The centroids are two bf16 planes (hi + lo, ~16 significant bits)
+ * because they meet the bf16 queries in the centroid logits. Logits use the bf16 Q
+ * against the bf16 K as given (kept tokens) or against both centroid planes (skipped
+ * blocks). Means of a partial last block use its true token count.
+ * One launch (one persistent CTA per SM).
  */
 int sparse_attn_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int B, int H, int Nq, int Nk, int d, int block, int order,
                      float* qbar, float* kbar_t, float* vsum,
                      uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
-                     void* stream);
+                     int32_t* err_flag, void* stream);
 
 /*
  * Incremental pooling for a growing KV cache (an autoregressive world model attends a new
@@ -115,7 +129,7 @@ int sparse_attn_pool_incremental(const uint16_t* q, const uint16_t* k, const uin
                                  int B, int H, int Nq, int Nk, int d, int block, int order,
                                  int kv_block_start, float* qbar, float* kbar_t, float* vsum,
                                  uint16_t* kbar16, uint16_t* vsum16, uint16_t* M, uint16_t* v16,
-                                 void* stream);
+                                 int32_t* err_flag, void* stream);
 
 /*
  * Routing (PISA §2 top-k choice of the critical blocks; SVG-EAR §2 B pooled
@@ -327,8 +341,9 @@ int sparse_attn_wait_selftest(int32_t* err_flag, int rounds, int32_t* waited, vo
  * Ranges: probabilities enter the value products as fp16 at most 2^11 (relative to the
  * row's running maximum); with order 1 the operand scale * alpha * q_t is fp16 too, and
  * a row with |q| above 2^15 / (2^11 scale) (181 at d = 128) rescales its maximum earlier
- * so that the operand stays below 2^15. The pool's fp16 tables (V, value sums, M_j) must
- * hold values below 65504; nothing checks them.
+ * so that the operand stays below 2^15. The pool's fp16 tables (V, value sums, M_j) are
+ * checked by the pool (SA_FLAG_RANGE in its err_flag); given the same err_flag, a forward
+ * that starts after a range error finds the flag set and skips its work.
  */
 int sparse_attn_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v16,
                         const uint16_t* kbar16, const uint16_t* vsum16, const uint16_t* M,

@@ -56,11 +56,12 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 96, 64, 0),
         lambda: C.sparse_attn_table_sizes(1, 1, 64, 64, 64, 32, 0),
         lambda: C.sparse_attn_table_sizes(-1, 1, 64, 64, 64, 64, 0),
-        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 3, p, p, p, p, p, p, p, 0),
-        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, None, p, 0),
-        lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
-        lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, 0),
-        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, None, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 3, p, p, p, p, p, p, p, None, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 2, p, p, p, p, p, None, p, None, 0),
+        lambda: C.sparse_attn_pool(p, None, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, None, 0),
+        lambda: C.sparse_attn_pool(p, p + 8, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, None, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, None, None, 0),
+        lambda: C.sparse_attn_pool(p, p, p, 1, 1, 64, 64, 64, 64, 0, p, p, p, p, p, None, p, p + 2, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 3000, 64, 0, 1, 4, 0.9, 0.1, p, p, 750, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 0, 3, 2, 0.9, 0.1, p, p, 10, 0),
         lambda: C.sparse_attn_route(p, p, 1, 1, 4, 10, 64, 1, 1, 4, 1.5, 0.1, p, p, 10, 0),
@@ -86,9 +87,9 @@ def test_host_argument_checks(lib):
         lambda: C.sparse_attn_route_scores(None, 1, 1, 4, 10, 1, 4, p, p, 10, 0),
         lambda: C.sparse_attn_route_scores(p, 1, 1, 4, 0, 1, 4, p, p, 10, 0),
         lambda: C.sparse_attn_pool_incremental(p, p, p, 1, 1, 64, 640, 64, 64, 0, 11, p, p, p, p,
-                                               p, None, p, 0),
+                                               p, None, p, None, 0),
         lambda: C.sparse_attn_pool_incremental(p, p, p, 1, 1, 64, 640, 64, 64, 1, 2, p, p, p, p,
-                                               p, None, p, 0),
+                                               p, None, p, None, 0),
         lambda: C.sparse_attn_wait_selftest(p, 0, p, 0),
         lambda: C.sparse_attn_wait_selftest(None, 10, p, 0),
         lambda: C.sparse_attn_kmeans_sizes(1, 1, 64, 96, 4),

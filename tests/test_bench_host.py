@@ -47,9 +47,36 @@ def test_pool_bytes_closed_form():
     w = W.shrink(W.WORKLOADS["uniform-4k"], B=1, H=2, Nq=256, Nk=512, d=64, block=128, order=1)
     bh, nkb, nqb = 2, 4, 2
     rd = bh * 512 * 64 * 2 * 2 + bh * 256 * 64 * 2
-    wr = bh * nkb * 64 * 14 + bh * nqb * 64 * 4 + bh * 512 * 64 * 2 + bh * nkb * 64 * 64 * 2
+    # centroids and value sums: fp32 each plus one 16-bit copy each; query centroids fp32;
+    # M_j in 16 bits
+    wr = bh * nkb * 64 * 12 + bh * nqb * 64 * 4 + bh * nkb * 64 * 64 * 2
     assert bench.pool_bytes(w, True) == rd + wr
     assert bench.pool_bytes(w, False) == rd + wr - bh * 256 * 64 * 2 - bh * nqb * 64 * 4
+    # what the library writes beyond the method's tables: the fp16 copy of V and the low
+    # centroid plane
+    assert bench.pool_extra_bytes(w) == {"v16": bh * 512 * 64 * 2, "kbar16_lo": bh * nkb * 64 * 2}
+
+
+def test_pool_bytes_of_the_metric_workload():
+    """The 720p call moves 3.145 GB through the pool by the method's tables (K, V, Q read;
+    M_j 0.775 GB written); the fp16 copy of V adds 0.774 GB."""
+    w = W.WORKLOADS[W.METRIC_WORKLOAD]
+    assert abs(bench.pool_bytes(w, True) - 3.1448e9) < 1e6
+    assert abs(bench.pool_extra_bytes(w)["v16"] - 0.7741e9) < 1e6
+
+
+def test_reference_rows_per_step():
+    assert bench.reference_rows_per_step(0.01, 12.0, 20) == 48
+    assert bench.reference_rows_per_step(1.0, 12.0, 20) == 16
+    assert bench.reference_rows_per_step(1e-4, 10.0, 5) % 16 == 0
+
+
+def test_launch_counts():
+    assert bench.launches_per_step(W.WORKLOADS["dit720p-21x45x80"], 1) == 3
+    assert bench.launches_per_step(W.WORKLOADS["worldmodel-chunk"], 3) == 4
+    assert bench.launches_per_step(W.WORKLOADS["dit720p-hybrid-21x45x80"], 1) == 5
+    assert bench.launches_per_step(W.WORKLOADS["dit720p-ear-21x45x80"], 1) == 4
+    assert bench.launches_per_step(W.WORKLOADS["dit720p-kmeans-21x45x80"], 1) == 3 + 2 * 31 + 4
 
 
 def test_kv_cache_start_of_the_world_model_chunk():
