@@ -30,25 +30,80 @@ constexpr int kRouteThreads = 256;
 
 // One warp selects the kept blocks of one query block from its scores s[0..nkb).
 // Lane l holds blocks j = l + 32 i (i < SLOTS) as order-preserving 32-bit keys.
-//   1. MSB-first search over 32 key bits for the threshold key T:
-//        top-k: the largest T with #{key >= T} >= k;
-//        mass:  the largest T with sum_{key >= T} e^(s - max) >= tau * Z.
+//   1. The threshold key T:
+//        top-k: the largest T with #{key >= T} >= k, found one byte at a time (most
+//               significant first) from a 256-bin histogram of the keys that match the
+//               bytes found so far (warp-private bins in shared memory, integer counts);
+//        mass:  the largest T with sum_{key >= T} e^(s - max) >= tau * Z, by an MSB-first
+//               search over the 32 key bits (masses summed in one fixed order).
 //   2. Every block with key > T is kept; blocks with key == T (ties) are taken in
 //      ascending j until the count (top-k) or the mass (mass rule) is reached, so the
 //      order is (score descending, index ascending).
 //   3. Kept indices are written in ascending j with ballots.
-template <int SLOTS>
-SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, int32_t* out,
-                        int32_t* cnt_out, int cap, int lane) {
+template <int SLOTS, int MODE>
+SA_DEVI void select_row(const float* s, int nkb, int keep, float tau, int32_t* out,
+                        int32_t* cnt_out, int cap, int lane, int* hist) {
   uint32_t key[SLOTS];
-  float e[SLOTS];
+  float e[MODE == 1 ? SLOTS : 1];
 #pragma unroll
   for (int i = 0; i < SLOTS; ++i) {
     const int j = lane + 32 * i;
     key[i] = j < nkb ? float_key(s[j]) : 0u;  // 0 sorts below every real score
   }
   float goal = 0.f;
-  if (mode == 1) {
+  uint32_t T = 0;
+  int above = 0;        // top-k: keys strictly above T
+  float mabove = 0.f;   // mass: their mass
+  if constexpr (MODE == 0) {
+    uint32_t pmask = 0;
+    int need = keep;  // keys >= T still to be found among those matching the prefix
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < SLOTS; ++i)
+        if (lane + 32 * i < nkb && (key[i] & pmask) == T) atomicAdd(&hist[(key[i] >> shift) & 255], 1);
+      __syncwarp();
+      // lane l holds bins 255 - 8 l - t (t = 0..7), i.e. digits in descending order
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        cnt[t] = hist[255 - 8 * lane - t];
+        tot += cnt[t];
+      }
+      int incl = tot;  // inclusive scan over lanes (higher digits first)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int before = incl - tot;  // keys with a higher digit than this lane's bins
+      // the digit where the count from the top first reaches `need`
+      int found = -1, above_d = 0;
+      if (before < need && incl >= need) {
+        int acc = before;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (found < 0 && acc + cnt[t] >= need) {
+            found = 255 - 8 * lane - t;
+            above_d = acc;
+          }
+          acc += cnt[t];
+        }
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+      const int src = __ffs(who) - 1;
+      found = __shfl_sync(0xffffffffu, found, src);
+      above_d = __shfl_sync(0xffffffffu, above_d, src);
+      T |= (uint32_t)found << shift;
+      pmask |= 255u << shift;
+      need -= above_d;
+      above += above_d;
+      __syncwarp();  // the bins are read before the next pass clears them
+    }
+  } else {
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < SLOTS; ++i)
@@ -64,17 +119,8 @@ SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     goal = tau * z;
-  }
-  uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    if (mode == 0) {
-      int c = 0;
-#pragma unroll
-      for (int i = 0; i < SLOTS; ++i) c += key[i] >= cand;
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= keep) T = cand;
-    } else {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
       float m = 0.f;
 #pragma unroll
       for (int i = 0; i < SLOTS; ++i) m += key[i] >= cand ? e[i] : 0.f;
@@ -82,18 +128,12 @@ SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, 
       for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
       if (m >= goal) T = cand;
     }
-  }
-  // what the strictly larger keys already give
-  int above = 0;
-  float mabove = 0.f;
+    // what the strictly larger keys already give
 #pragma unroll
-  for (int i = 0; i < SLOTS; ++i) {
-    above += key[i] > T;
-    if (mode == 1) mabove += key[i] > T ? e[i] : 0.f;
-  }
-  above = __reduce_add_sync(0xffffffffu, above);
+    for (int i = 0; i < SLOTS; ++i) mabove += key[i] > T ? e[i] : 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mabove += __shfl_xor_sync(0xffffffffu, mabove, o);
+    for (int o = 16; o > 0; o >>= 1) mabove += __shfl_xor_sync(0xffffffffu, mabove, o);
+  }
   // walk the ties in ascending j; write every kept index in ascending j
   const unsigned lt = (1u << lane) - 1u;
   int off = 0, ties = 0;
@@ -104,7 +144,7 @@ SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, 
     const bool tie = key[i] == T && lane + 32 * i < nkb;
     const unsigned tb = __ballot_sync(0xffffffffu, tie);
     bool take_tie = false;
-    if (mode == 0) {
+    if constexpr (MODE == 0) {
       take_tie = tie && (ties + __popc(tb & lt)) < keep - above;
       ties += __popc(tb);
     } else {
@@ -131,28 +171,32 @@ SA_DEVI void select_row(const float* s, int nkb, int mode, int keep, float tau, 
   if (lane == 0) *cnt_out = min(off, cap);
 }
 
-// Shared-memory bytes of one route CTA: qbar block, two chunks of the centroid table,
-// the score rows.
+// Shared-memory bytes of one route CTA: qbar block, two chunks of the centroid table (rows
+// of NKP + 4 floats: a row is copied from the 16-byte boundary at or below its start),
+// the score rows, and a 256-bin histogram per warp for the top-k selection.
 template <int D, int RG, int MC, int KD>
 constexpr size_t route_smem(int nkb) {
-  return (size_t)(D * 8 * RG + 2 * KD * (kRouteThreads / RG) * MC + 8 * RG * nkb) * 4;
+  return (size_t)(D * 8 * RG + 2 * KD * ((kRouteThreads / RG) * MC + 4) + 8 * RG * nkb +
+                  (kRouteThreads / 32) * 256) * 4;
 }
 
-template <int D, int SLOTS, int RG, int MC, int KD>
+template <int D, int SLOTS, int RG, int MC, int KD, int MODE>
 __global__ void __launch_bounds__(kRouteThreads, SLOTS <= 32 ? 2 : 1)
 route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, int nqb, int nkb,
-             int mode, int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
+             int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
              int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov,
              const float* __restrict__ pre) {
   constexpr int R = 8 * RG;                  // query blocks per CTA
   constexpr int CT = kRouteThreads / RG;     // column threads per group of 8 rows
   constexpr int NKP = CT * MC;               // key blocks per chunk row (padded)
+  constexpr int NKS = NKP + 4;               // shared row stride (16-byte multiple)
   constexpr int NCH = D / KD;                // chunks of KD dimensions
-  static_assert(D % KD == 0, "route chunks");
+  static_assert(D % KD == 0 && NKP % 4 == 0, "route chunks");
   extern __shared__ __align__(16) float rsm[];
   float* qs = rsm;                           // [D][R]: qs[c * R + r] = qbar of row r, dim c
-  float* kc = qs + D * R;                    // [2][KD][NKP] chunks of the centroid table
-  float* sc = kc + 2 * KD * NKP;             // [R][nkb] scores
+  float* kc = qs + D * R;                    // [2][KD][NKS] chunks of the centroid table
+  float* sc = kc + 2 * KD * NKS;             // [R][nkb] scores
+  int* hist = reinterpret_cast<int*>(sc + R * nkb);  // [warps][256]
   const int tid = threadIdx.x;
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
@@ -165,12 +209,20 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
         sc[r * nkb + j] = pre[((size_t)bh * nqb + i0 + r) * nkb + j];
   } else {
     const float* kt = kbar_t + (size_t)bh * D * nkb;
+    // Row c of the table starts g = (bh D + c) nkb floats into kbar_t (16-byte aligned);
+    // it is copied in 16-byte pieces from the boundary at or below g, so element j of the
+    // row sits at (g & 3) + j in shared memory; the last piece stops at the row's end.
+    auto row_off = [&](int c) { return (int)(((size_t)bh * D + c) * nkb & 3u); };
     auto load_chunk = [&](int ch, int buf) {
-      float* dst = kc + buf * KD * NKP;
-      for (int x = tid; x < KD * NKP; x += kRouteThreads) {
-        const int k = x / NKP, j = x % NKP;
-        const bool ok = j < nkb;
-        cp_async4(smem_u32(dst + x), ok ? kt + (size_t)(ch * KD + k) * nkb + j : kt, ok ? 4 : 0);
+      float* dst = kc + buf * KD * NKS;
+      constexpr int PIECES = NKS / 4;
+      for (int x = tid; x < KD * PIECES; x += kRouteThreads) {
+        const int k = x / PIECES, q = x % PIECES;
+        const int c = ch * KD + k, o = row_off(c);
+        const int first = 4 * q - o;              // row element at the piece's start
+        const int bytes = max(0, min(16, (nkb - first) * 4));
+        const float* src = kt + (size_t)c * nkb + first;
+        cp_async16(smem_u32(dst + k * NKS + 4 * q), bytes > 0 ? src : kt, bytes);
       }
       cp_async_commit();
     };
@@ -190,16 +242,17 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
     for (int ch = 0; ch < NCH; ++ch) {
       if (ch + 1 < NCH) cp_async_wait<1>(); else cp_async_wait<0>();
       __syncthreads();  // chunk ch (and the qbar block) visible to every thread
-      const float* kb = kc + (ch & 1) * KD * NKP;
+      const float* kb = kc + (ch & 1) * KD * NKS;
 #pragma unroll
       for (int k = 0; k < KD; ++k) {
         const int c = ch * KD + k;
+        const float* krow = kb + k * NKS + row_off(c) + ct;
         const float4 q0 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8);
         const float4 q1 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8 + 4);
         const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
         for (int m = 0; m < MC; ++m) {
-          const float kv = kb[k * NKP + ct + CT * m];
+          const float kv = krow[CT * m];
 #pragma unroll
           for (int r = 0; r < 8; ++r) acc[r][m] = fmaf(qv[r], kv, acc[r][m]);
         }
@@ -221,20 +274,20 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
 
   const int warp = tid / 32, lane = tid % 32;
   for (int r = warp; r < rows; r += kRouteThreads / 32)
-    select_row<SLOTS>(sc + r * nkb, nkb, mode, keep, tau,
-                      kv_idx + ((size_t)bh * nqb + i0 + r) * cap, kv_cnt + (size_t)bh * nqb + i0 + r,
-                      cap, lane);
+    select_row<SLOTS, MODE>(sc + r * nkb, nkb, keep, tau,
+                            kv_idx + ((size_t)bh * nqb + i0 + r) * cap,
+                            kv_cnt + (size_t)bh * nqb + i0 + r, cap, lane, hist + warp * 256);
 }
 
 template <int D, int SLOTS, int RG, int MC, int KD>
 static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
   const size_t smem = route_smem<D, RG, MC, KD>(p.nkb);
-  auto kern = route_kernel<D, SLOTS, RG, MC, KD>;
+  auto kern = p.mode == 0 ? route_kernel<D, SLOTS, RG, MC, KD, 0> : route_kernel<D, SLOTS, RG, MC, KD, 1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nqb + 8 * RG - 1) / (8 * RG), p.B * p.H);
-  kern<<<grid, kRouteThreads, smem, st>>>(p.qbar, p.kbar_t, p.nqb, p.nkb, p.mode, p.keep, p.tau,
-                                          p.scale, p.kv_idx, p.kv_cnt, p.cap, p.cov, p.scores);
+  kern<<<grid, kRouteThreads, smem, st>>>(p.qbar, p.kbar_t, p.nqb, p.nkb, p.keep, p.tau, p.scale,
+                                          p.kv_idx, p.kv_cnt, p.cap, p.cov, p.scores);
   return cudaGetLastError();
 }
 
