@@ -322,7 +322,11 @@ int sparse_attn_wait_selftest(int32_t* err_flag, int rounds, int32_t* waited, vo
  *   D_t = sum_r e^(l_r - m)     + sum_j e^(c_j - m) n_j
  *   o_t = N_t / D_t
  *   q, k              [B,H,Nq,d] / [B,H,Nk,d] bf16, as for the pool
- *   v16, kbar16, vsum16  as written by the pool
+ *   v16, kbar16, vsum16  as written by the pool. The forward reads the pool's fp16 copy
+ *                     of V rather than V itself: the exact value products multiply fp16
+ *                     probabilities (bf16 ones would carry ~2^-8 relative error on a
+ *                     dominant term), and a tensor-core product takes one 16-bit type for
+ *                     both operands.
  *   M                 order 1: the pool's M table; order 2: hbar16 [B,H,d,d] from
  *                     sparse_attn_hbar; order 0: NULL
  *   kv_idx, kv_cnt    as written by routing or the structured mask: indices of
