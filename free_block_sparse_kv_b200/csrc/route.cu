@@ -10,11 +10,12 @@
 // Route kernel: one CTA of 8 warps per (batch*head, R query blocks), R = 16 (8 when a
 // row holds more than 1024 key blocks).
 //   1. Scores s_ij = scale * qbar_i . kbar_j in fp32 for the CTA's R rows. The head's
-//      dim-major centroid table streams through shared memory in chunks of a few
-//      dimensions (all key blocks of each; 4-byte cp.async, double-buffered, so many
-//      loads are in flight per thread); each thread accumulates an 8-row x MC-column
-//      tile with fp32 FMAs, the 8 rows' qbar values broadcast from shared memory.
-//      Every score is one fma chain over d = 0 .. D-1 in order.
+//      dim-major centroid table streams through shared memory in chunks of KD rows (KD
+//      dimensions, all key blocks of each): KD consecutive rows are one contiguous range
+//      that starts on a 16-byte boundary, copied with 16-byte cp.async into a double
+//      buffer; each thread accumulates an 8-row x MC-column tile with fp32 FMAs, the 8
+//      rows' qbar values broadcast from shared memory. Every score is one fma chain over
+//      d = 0 .. D-1 in order.
 //   2. One warp per query block selects (select_row): a 32-step search over
 //      order-preserving score keys held in registers finds the threshold, ties at
 //      the threshold are taken in ascending block index, and the kept indices are
@@ -171,14 +172,23 @@ SA_DEVI void select_row(const float* s, int nkb, int keep, float tau, int32_t* o
   if (lane == 0) *cnt_out = min(off, cap);
 }
 
-// Shared-memory bytes of one route CTA: qbar block, two chunks of the centroid table (rows
-// of NKP + 4 floats: a row is copied from the 16-byte boundary at or below its start),
-// the score rows, and a 256-bin histogram per warp for the top-k selection.
+// Shared-memory layout of one route CTA, in floats: the qbar block [D][R]; two chunk
+// buffers, each KD rows of the centroid table (KD * nkb floats, contiguous as in global
+// memory) and NKP - nkb spare floats that the column threads past nkb read (their
+// columns are never stored); the score rows [R][nkb], over the chunk buffers once the
+// scoring is done; a 256-bin histogram per warp for the top-k selection.
 template <int D, int RG, int MC, int KD>
-constexpr size_t route_smem(int nkb) {
-  return (size_t)(D * 8 * RG + 2 * KD * ((kRouteThreads / RG) * MC + 4) + 8 * RG * nkb +
-                  (kRouteThreads / 32) * 256) * 4;
-}
+struct RouteSmem {
+  static constexpr int R = 8 * RG, CT = kRouteThreads / RG, NKP = CT * MC;
+  static size_t __host__ __device__ buf(int nkb) { return ((size_t)KD * nkb + (NKP - nkb) + 3) & ~(size_t)3; }
+  static size_t __host__ __device__ chunks(int nkb) {
+    const size_t a = 2 * buf(nkb), b = (size_t)R * nkb;
+    return a > b ? a : b;
+  }
+  static size_t __host__ __device__ bytes(int nkb) {
+    return ((size_t)D * R + chunks(nkb) + (kRouteThreads / 32) * 256) * 4;
+  }
+};
 
 template <int D, int SLOTS, int RG, int MC, int KD, int MODE>
 __global__ void __launch_bounds__(kRouteThreads, SLOTS <= 32 ? 2 : 1)
@@ -186,17 +196,15 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
              int keep, float tau, float scale, int32_t* __restrict__ kv_idx,
              int32_t* __restrict__ kv_cnt, int cap, const float* __restrict__ cov,
              const float* __restrict__ pre) {
-  constexpr int R = 8 * RG;                  // query blocks per CTA
-  constexpr int CT = kRouteThreads / RG;     // column threads per group of 8 rows
-  constexpr int NKP = CT * MC;               // key blocks per chunk row (padded)
-  constexpr int NKS = NKP + 4;               // shared row stride (16-byte multiple)
+  using L = RouteSmem<D, RG, MC, KD>;
+  constexpr int R = L::R, CT = L::CT;
   constexpr int NCH = D / KD;                // chunks of KD dimensions
-  static_assert(D % KD == 0 && NKP % 4 == 0, "route chunks");
+  static_assert(D % KD == 0 && KD % 4 == 0, "a chunk is whole 16-byte pieces");
   extern __shared__ __align__(16) float rsm[];
   float* qs = rsm;                           // [D][R]: qs[c * R + r] = qbar of row r, dim c
-  float* kc = qs + D * R;                    // [2][KD][NKS] chunks of the centroid table
-  float* sc = kc + 2 * KD * NKS;             // [R][nkb] scores
-  int* hist = reinterpret_cast<int*>(sc + R * nkb);  // [warps][256]
+  float* kc = qs + D * R;                    // [2] chunk buffers
+  float* sc = kc;                            // [R][nkb] scores, once the chunks are done
+  int* hist = reinterpret_cast<int*>(kc + L::chunks(nkb));  // [warps][256]
   const int tid = threadIdx.x;
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
@@ -208,26 +216,18 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
       for (int j = tid; j < nkb; j += kRouteThreads)
         sc[r * nkb + j] = pre[((size_t)bh * nqb + i0 + r) * nkb + j];
   } else {
+    // Chunk ch: rows ch*KD .. ch*KD+KD-1 of the head's table, KD*nkb floats from element
+    // (bh*D + ch*KD)*nkb, a multiple of 4 (D and KD are), so a 16-byte aligned range.
     const float* kt = kbar_t + (size_t)bh * D * nkb;
-    // Row c of the table starts g = (bh D + c) nkb floats into kbar_t (16-byte aligned);
-    // it is copied in 16-byte pieces from the boundary at or below g, so element j of the
-    // row sits at (g & 3) + j in shared memory; the last piece stops at the row's end.
-    auto row_off = [&](int c) { return (int)(((size_t)bh * D + c) * nkb & 3u); };
-    auto load_chunk = [&](int ch, int buf) {
-      float* dst = kc + buf * KD * NKS;
-      constexpr int PIECES = NKS / 4;
-      for (int x = tid; x < KD * PIECES; x += kRouteThreads) {
-        const int k = x / PIECES, q = x % PIECES;
-        const int c = ch * KD + k, o = row_off(c);
-        const int first = 4 * q - o;              // row element at the piece's start
-        const int bytes = max(0, min(16, (nkb - first) * 4));
-        const float* src = kt + (size_t)c * nkb + first;
-        cp_async16(smem_u32(dst + k * NKS + 4 * q), bytes > 0 ? src : kt, bytes);
-      }
+    const size_t bs = L::buf(nkb);
+    const int pieces = KD * nkb / 4;
+    auto load_chunk = [&](int ch, int b) {
+      const float* src = kt + (size_t)ch * KD * nkb;
+      float* dst = kc + b * bs;
+      for (int x = tid; x < pieces; x += kRouteThreads) cp_async16(smem_u32(dst + 4 * x), src + 4 * x, 16);
       cp_async_commit();
     };
     load_chunk(0, 0);
-    if (NCH > 1) load_chunk(1, 1);
     for (int x = tid; x < D * R; x += kRouteThreads) {
       const int r = x / D, c = x % D;   // coalesced along c
       qs[c * R + r] = r < rows ? qbar[((size_t)bh * nqb + i0 + r) * D + c] : 0.f;
@@ -240,26 +240,25 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
 #pragma unroll
       for (int m = 0; m < MC; ++m) acc[r][m] = 0.f;
     for (int ch = 0; ch < NCH; ++ch) {
-      if (ch + 1 < NCH) cp_async_wait<1>(); else cp_async_wait<0>();
-      __syncthreads();  // chunk ch (and the qbar block) visible to every thread
-      const float* kb = kc + (ch & 1) * KD * NKS;
+      cp_async_wait<0>();
+      __syncthreads();  // chunk ch (and the qbar block) visible; chunk ch-1 read by every thread
+      if (ch + 1 < NCH) load_chunk(ch + 1, (ch + 1) & 1);  // into the buffer of chunk ch-1
+      const float* kb = kc + (ch & 1) * bs + ct;
 #pragma unroll
       for (int k = 0; k < KD; ++k) {
         const int c = ch * KD + k;
-        const float* krow = kb + k * NKS + row_off(c) + ct;
         const float4 q0 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8);
         const float4 q1 = *reinterpret_cast<const float4*>(qs + c * R + rg * 8 + 4);
         const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
         for (int m = 0; m < MC; ++m) {
-          const float kv = krow[CT * m];
+          const float kv = kb[k * nkb + CT * m];
 #pragma unroll
           for (int r = 0; r < 8; ++r) acc[r][m] = fmaf(qv[r], kv, acc[r][m]);
         }
       }
-      __syncthreads();  // every thread is done with this buffer before it is refilled
-      if (ch + 2 < NCH) load_chunk(ch + 2, ch & 1);
     }
+    __syncthreads();  // every chunk read before the scores overwrite the buffers
 #pragma unroll
     for (int m = 0; m < MC; ++m) {
       const int j = ct + CT * m;
@@ -281,7 +280,7 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
 
 template <int D, int SLOTS, int RG, int MC, int KD>
 static cudaError_t launch_route_t(const RouteArgs& p, cudaStream_t st) {
-  const size_t smem = route_smem<D, RG, MC, KD>(p.nkb);
+  const size_t smem = RouteSmem<D, RG, MC, KD>::bytes(p.nkb);
   auto kern = p.mode == 0 ? route_kernel<D, SLOTS, RG, MC, KD, 0> : route_kernel<D, SLOTS, RG, MC, KD, 1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
