@@ -211,10 +211,14 @@ route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar_t, i
   const int rows = min(R, nqb - i0);
 
   if (pre) {
-    // precomputed scores (error-aware routing): copy the rows, coalesced
-    for (int r = 0; r < rows; ++r)
-      for (int j = tid; j < nkb; j += kRouteThreads)
-        sc[r * nkb + j] = pre[((size_t)bh * nqb + i0 + r) * nkb + j];
+    // precomputed scores (error-aware routing): the CTA's rows are one contiguous range,
+    // copied with 4-byte cp.async (its start has no 16-byte alignment) so that every
+    // thread's loads are in flight at once
+    const float* src = pre + ((size_t)bh * nqb + i0) * nkb;
+    const int n = rows * nkb;
+    for (int x = tid; x < n; x += kRouteThreads) cp_async4(smem_u32(sc + x), src + x, 4);
+    cp_async_commit();
+    cp_async_wait<0>();
   } else {
     // Chunk ch: rows ch*KD .. ch*KD+KD-1 of the head's table, KD*nkb floats from element
     // (bh*D + ch*KD)*nkb, a multiple of 4 (D and KD are), so a 16-byte aligned range.
