@@ -16,10 +16,11 @@
 //      buffer; each thread accumulates an 8-row x MC-column tile with fp32 FMAs, the 8
 //      rows' qbar values broadcast from shared memory. Every score is one fma chain over
 //      d = 0 .. D-1 in order.
-//   2. One warp per query block selects (select_row): a 32-step search over
-//      order-preserving score keys held in registers finds the threshold, ties at
-//      the threshold are taken in ascending block index, and the kept indices are
-//      written in ascending order with ballots.
+//   2. One warp per query block selects (select_row) over order-preserving score keys
+//      held in registers: the threshold is found a byte at a time from warp histograms
+//      (top-k) or by a 32-step bit search on the covered mass (mass rule), ties at the
+//      threshold are taken in ascending block index, and the kept indices are written in
+//      ascending order with ballots.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
