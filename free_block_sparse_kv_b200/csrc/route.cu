@@ -83,7 +83,7 @@ SA_DEVI void select_row(const float* s, int nkb, int keep, float tau, int32_t* o
       }
       const int before = incl - tot;  // keys with a higher digit than this lane's bins
       // the digit where the count from the top first reaches `need`
-      int found = -1, above_d = 0;
+      int found = -1, above_d = 0, bucket = 0;
       if (before < need && incl >= need) {
         int acc = before;
 #pragma unroll
@@ -91,6 +91,7 @@ SA_DEVI void select_row(const float* s, int nkb, int keep, float tau, int32_t* o
           if (found < 0 && acc + cnt[t] >= need) {
             found = 255 - 8 * lane - t;
             above_d = acc;
+            bucket = cnt[t];
           }
           acc += cnt[t];
         }
@@ -99,11 +100,30 @@ SA_DEVI void select_row(const float* s, int nkb, int keep, float tau, int32_t* o
       const int src = __ffs(who) - 1;
       found = __shfl_sync(0xffffffffu, found, src);
       above_d = __shfl_sync(0xffffffffu, above_d, src);
+      bucket = __shfl_sync(0xffffffffu, bucket, src);
       T |= (uint32_t)found << shift;
       pmask |= 255u << shift;
       need -= above_d;
       above += above_d;
       __syncwarp();  // the bins are read before the next pass clears them
+      if (shift > 0 && (need == 1 || need == bucket)) {
+        // The rest follows without more passes: the `bucket` keys that match the prefix
+        // found so far hold the threshold. One still to find: it is their largest; all
+        // of them needed: it is their smallest, and those above it count as above T.
+        const bool top = need == 1;
+        uint32_t ext = top ? 0u : 0xffffffffu;
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i)
+          if (lane + 32 * i < nkb && (key[i] & pmask) == T) ext = top ? max(ext, key[i]) : min(ext, key[i]);
+        T = top ? __reduce_max_sync(0xffffffffu, ext) : __reduce_min_sync(0xffffffffu, ext);
+        if (!top) {
+          int eq = 0;
+#pragma unroll
+          for (int i = 0; i < SLOTS; ++i) eq += (lane + 32 * i < nkb && key[i] == T) ? 1 : 0;
+          above += bucket - (int)__reduce_add_sync(0xffffffffu, (unsigned)eq);
+        }
+        break;
+      }
     }
   } else {
     float mx = -INFINITY;
