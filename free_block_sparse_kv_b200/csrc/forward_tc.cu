@@ -953,6 +953,7 @@ template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ part, int nsplit,
                                                       long long rows, void* out, int out_dtype) {
   constexpr int V = D / 32;
+  static_assert(V == 2 || V == 4, "combine: d = 64 or 128");
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= rows) return;
@@ -968,20 +969,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       if (x.x == -INFINITY) continue;
       const float w = exp2f(x.x - M);
       L += w * x.y;
+      // a lane's V consecutive columns in one 16- (V = 4) or 8-byte load: rows of D floats
+      // in a 16-byte aligned buffer
       const float* o = part + ((size_t)sp * rows + row) * D + V * lane;
-#pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] += w * o[i];
+      if constexpr (V == 4) {
+        const float4 y = *reinterpret_cast<const float4*>(o);
+        acc[0] += w * y.x; acc[1] += w * y.y; acc[2] += w * y.z; acc[3] += w * y.w;
+      } else {
+        const float2 y = *reinterpret_cast<const float2*>(o);
+        acc[0] += w * y.x; acc[1] += w * y.y;
+      }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if (out_dtype == 0) {
     float* o = static_cast<float*>(out) + (size_t)row * D + V * lane;
-#pragma unroll
-    for (int i = 0; i < V; ++i) o[i] = acc[i] * inv;
+    if constexpr (V == 4) *reinterpret_cast<float4*>(o) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    else *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
   } else {
-    uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(out) + (size_t)row * D + V * lane);
-#pragma unroll
-    for (int i = 0; i < V / 2; ++i) o[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+    uint16_t* o = static_cast<uint16_t*>(out) + (size_t)row * D + V * lane;
+    if constexpr (V == 4) *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+    else *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[0] * inv, acc[1] * inv);
   }
 }
 
